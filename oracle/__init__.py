@@ -1,0 +1,27 @@
+"""fp64 CPU oracle for the causal sliding-window GQA attention block.
+
+TEST INFRASTRUCTURE, NOT PRODUCT CODE. Only the tests, ``__graft_entry__.smoke()``
+and the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import
+this package. The CUDA library never calls it and shares no code with it.
+
+Every function is the plain definition of one step of the attention block, as
+the nanochat and nanoGPT guides describe it, written out in float64 with numpy:
+no tiling, no online softmax, no fused passes. See ``attention.py``.
+"""
+from .attention import (  # noqa: F401
+    rms_norm,
+    rope_frequencies,
+    rope_angles,
+    rope,
+    rope_transpose,
+    row_positions,
+    prologue,
+    prologue_bwd,
+    visible,
+    attention_fwd,
+    attention_bwd,
+    attention_bwd_rows,
+    attention_bwd_keys,
+    decode,
+    useful_pairs,
+)

@@ -1,0 +1,397 @@
+"""Pins for the fp64 oracle: it is checked against things other than itself.
+
+  * a hand-worked two-token example (tests/golden/two_token_worked_example.json)
+  * a pure-Python brute force on tiny shapes (tests/brute.py)
+  * central finite differences of the whole block (prologue + attention)
+  * complex-number rotation (numpy complex exp) for RoPE
+  * closed forms and invariants: window >= T-1 is full causal, GQA equals MHA
+    with repeated KV heads, T = 1 and W = 0 return v, q = 0 gives the windowed
+    prefix mean of v with lse = ln(n), sum_j dK_j = 0, sum_j dV_j = sum_i dO_i
+  * torch's scaled_dot_product_attention and its autograd, in float64 on the CPU
+  * decode at position p equals row p of the forward pass
+The last test plants plausible mistakes in the oracle and shows a pin fails.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import oracle.attention as oa
+import workloads
+from tests import brute
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+def rnd(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def allclose(a, b, tol):
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    assert a.shape == b.shape, (a.shape, b.shape)
+    err = np.max(np.abs(a - b)) if a.size else 0.0
+    assert err <= tol, f"max abs err {err} > {tol}"
+
+
+# ---------------------------------------------------------------- checks
+# Each check raises AssertionError on failure; the planted-mistake test at the
+# bottom reuses them to show that they catch specific errors.
+
+def check_golden():
+    g = json.load(open(os.path.join(GOLDEN, "two_token_worked_example.json")))
+    i = g["inputs"]
+    q = np.array(i["q_raw"])[None, :, None, :]
+    k = np.array(i["k_raw"])[None, :, None, :]
+    v = np.array(i["v"])[None, :, None, :]
+    pos = oracle.row_positions(1, 2)
+    qh = oracle.prologue(q, pos, i["rope_base"], i["eps"])
+    kh = oracle.prologue(k, pos, i["rope_base"], i["eps"])
+    e = g["expected"]
+    allclose(qh[0, :, 0, :], e["q_hat"], 1e-12)
+    allclose(kh[0, :, 0, :], e["k_hat"], 1e-12)
+    o, lse = oracle.attention_fwd(qh, kh, v, i["window"], i["scale"])
+    allclose(o[0, :, 0, :], e["o"], 1e-12)
+    allclose(lse[0, 0, :], e["lse"], 1e-12)
+
+
+def check_brute(W, G, seed=0):
+    B, T, Hkv, D = 2, 9, 2, 8
+    Hq = Hkv * G
+    q, k = rnd((B, T, Hq, D), seed), rnd((B, T, Hkv, D), seed + 1)
+    v, do = rnd((B, T, Hkv, D), seed + 2), rnd((B, T, Hq, D), seed + 3)
+    offs = np.array([0, 5])
+    pos = oracle.row_positions(B, T, offs)
+    qh = oracle.prologue(q, pos, 10000.0, 1e-6)
+    kh = oracle.prologue(k, pos, 10000.0, 1e-6)
+    allclose(qh, brute.prologue(q, 10000.0, 1e-6, offs), 1e-12)
+    allclose(kh, brute.prologue(k, 10000.0, 1e-6, offs), 1e-12)
+    scale = 0.37
+    o, lse = oracle.attention_fwd(qh, kh, v, W, scale)
+    bo, blse = brute.attention(qh, kh, v, W, scale)
+    allclose(o, bo, 1e-12)
+    allclose(lse, blse, 1e-12)
+    dq, dk, dv = oracle.attention_bwd(qh, kh, v, do, W, scale)
+    bq, bk, bv = brute.attention_grads(qh, kh, v, do, W, scale)
+    allclose(dq, bq, 1e-12)
+    allclose(dk, bk, 1e-12)
+    allclose(dv, bv, 1e-12)
+
+
+def _block_loss(q, k, v, do, W, scale, pos, base, eps):
+    qh = oracle.prologue(q, pos, base, eps)
+    kh = oracle.prologue(k, pos, base, eps)
+    o, _ = oracle.attention_fwd(qh, kh, v, W, scale)
+    return float(np.sum(do * o))
+
+
+def check_finite_differences(W=2, seed=3):
+    B, T, Hq, Hkv, D = 1, 6, 4, 2, 4
+    base, eps, scale = 10000.0, 1e-6, 0.8
+    q, k = rnd((B, T, Hq, D), seed), rnd((B, T, Hkv, D), seed + 1)
+    v, do = rnd((B, T, Hkv, D), seed + 2), rnd((B, T, Hq, D), seed + 3)
+    pos = oracle.row_positions(B, T, [3])
+    qh = oracle.prologue(q, pos, base, eps)
+    kh = oracle.prologue(k, pos, base, eps)
+    dqh, dkh, dv = oracle.attention_bwd(qh, kh, v, do, W, scale)
+    dq = oracle.prologue_bwd(q, dqh, pos, base, eps)
+    dk = oracle.prologue_bwd(k, dkh, pos, base, eps)
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args = dict(q=q, k=k, v=v)
+            args[name] = xp
+            lp = _block_loss(args["q"], args["k"], args["v"], do, W, scale, pos, base, eps)
+            args[name] = xm
+            lm = _block_loss(args["q"], args["k"], args["v"], do, W, scale, pos, base, eps)
+            fd[idx] = (lp - lm) / (2 * h)
+        rel = np.linalg.norm(fd - g) / np.linalg.norm(g)
+        assert rel <= 1e-6, f"d{name}: finite-difference rel err {rel}"
+
+
+def check_rope_complex(seed=4):
+    """Half-split RoPE is z_j * exp(i phi_j) with z_j = x_j + i x_{j+D/2}."""
+    B, T, H, D = 2, 7, 3, 16
+    x = rnd((B, T, H, D), seed)
+    pos = oracle.row_positions(B, T, [0, 1000])
+    y = oracle.rope(x, pos, 10000.0)
+    z = x[..., : D // 2] + 1j * x[..., D // 2:]
+    j = np.arange(D // 2)
+    phi = pos[:, :, None, None] * (10000.0 ** (-2.0 * j / D))
+    w = z * np.exp(1j * phi)
+    allclose(y[..., : D // 2], w.real, 1e-12)
+    allclose(y[..., D // 2:], w.imag, 1e-12)
+
+
+def check_window_full_causal(seed=5):
+    B, T, Hq, Hkv, D = 1, 12, 2, 1, 8
+    q, k, v = rnd((B, T, Hq, D), seed), rnd((B, T, Hkv, D), seed + 1), rnd((B, T, Hkv, D), seed + 2)
+    ref, lref = oracle.attention_fwd(q, k, v, -1, 0.5)
+    for W in (T - 1, T, 10 * T):
+        o, l = oracle.attention_fwd(q, k, v, W, 0.5)
+        allclose(o, ref, 0.0)
+        allclose(l, lref, 0.0)
+    o, _ = oracle.attention_fwd(q, k, v, T - 2, 0.5)
+    assert np.max(np.abs(o - ref)) > 1e-6, "W = T-2 must drop the (T-1, 0) pair"
+    # with q = 0 every visible key weighs the same, so lse = ln(#keys) = ln(W + 1) once i >= W
+    _, l0 = oracle.attention_fwd(np.zeros_like(q), k, v, 3, 0.5)
+    allclose(l0[0, 0, 3:], np.full(T - 3, math.log(4)), 1e-12)
+
+
+def check_gqa_repeat(seed=6):
+    B, T, Hkv, G, D = 2, 10, 2, 3, 8
+    Hq = Hkv * G
+    q, k = rnd((B, T, Hq, D), seed), rnd((B, T, Hkv, D), seed + 1)
+    v, do = rnd((B, T, Hkv, D), seed + 2), rnd((B, T, Hq, D), seed + 3)
+    kr, vr = np.repeat(k, G, axis=2), np.repeat(v, G, axis=2)
+    W = 4
+    o, l = oracle.attention_fwd(q, k, v, W, 0.3)
+    om, lm = oracle.attention_fwd(q, kr, vr, W, 0.3)
+    allclose(o, om, 1e-13)
+    allclose(l, lm, 1e-13)
+    dq, dk, dv = oracle.attention_bwd(q, k, v, do, W, 0.3)
+    dqm, dkm, dvm = oracle.attention_bwd(q, kr, vr, do, W, 0.3)
+    allclose(dq, dqm, 1e-13)
+    allclose(dk, dkm.reshape(B, T, Hkv, G, D).sum(3), 1e-12)
+    allclose(dv, dvm.reshape(B, T, Hkv, G, D).sum(3), 1e-12)
+
+
+def check_special_cases(seed=7):
+    B, T, Hq, Hkv, D = 2, 9, 4, 2, 8
+    q, k, v = rnd((B, T, Hq, D), seed), rnd((B, T, Hkv, D), seed + 1), rnd((B, T, Hkv, D), seed + 2)
+    vq = np.repeat(v, 2, axis=2)
+    o, l = oracle.attention_fwd(q, k, v, 0, 0.7)            # W = 0: self only
+    allclose(o, vq, 1e-14)
+    o, l = oracle.attention_fwd(q[:, :1], k[:, :1], v[:, :1], -1, 0.7)   # T = 1
+    allclose(o, vq[:, :1], 1e-14)
+    for W in (-1, 3):                                      # q = 0: uniform weights
+        o, l = oracle.attention_fwd(np.zeros_like(q), k, v, W, 0.7)
+        for i in range(T):
+            lo = 0 if W < 0 else max(0, i - W)
+            allclose(o[:, i], vq[:, lo:i + 1].mean(axis=1), 1e-13)
+            allclose(l[:, :, i], np.full((B, Hq), math.log(i + 1 - lo)), 1e-13)
+    # identical keys: scores are constant along each row, so dq must vanish
+    ksame = np.broadcast_to(k[:, :1], k.shape).copy()
+    dq, _, _ = oracle.attention_bwd(q, ksame, v, rnd((B, T, Hq, D), 9), 3, 0.7)
+    allclose(dq, np.zeros_like(dq), 1e-12)
+
+
+def check_bwd_invariants(seed=8):
+    B, T, Hkv, G, D = 2, 11, 2, 2, 8
+    Hq = Hkv * G
+    q, k = rnd((B, T, Hq, D), seed), rnd((B, T, Hkv, D), seed + 1)
+    v, do = rnd((B, T, Hkv, D), seed + 2), rnd((B, T, Hq, D), seed + 3)
+    dq, dk, dv = oracle.attention_bwd(q, k, v, do, 3, 0.6)
+    # rows of P sum to one  =>  sum_j dV_j = sum over the group's heads of sum_i dO_i
+    allclose(dv.sum(axis=1), do.reshape(B, T, Hkv, G, D).sum(axis=(1, 3)), 1e-12)
+    # rows of dS sum to zero  =>  sum_j dK_j = 0
+    allclose(dk.sum(axis=1), np.zeros((B, Hkv, D)), 1e-12)
+
+
+def check_sdpa(seed=9):
+    """torch's scaled_dot_product_attention (float64, CPU) and its autograd."""
+    B, T, Hkv, G, D = 2, 13, 2, 2, 16
+    Hq = Hkv * G
+    q, k = rnd((B, T, Hq, D), seed), rnd((B, T, Hkv, D), seed + 1)
+    v, do = rnd((B, T, Hkv, D), seed + 2), rnd((B, T, Hq, D), seed + 3)
+    for W in (-1, 0, 4):
+        i = torch.arange(T)
+        mask = (i[None, :] <= i[:, None])
+        if W >= 0:
+            mask &= (i[:, None] - i[None, :]) <= W
+        tq, tk, tv = (torch.tensor(a).transpose(1, 2).requires_grad_(True) for a in (q, k, v))
+        o = torch.nn.functional.scaled_dot_product_attention(
+            tq, tk, tv, attn_mask=mask, scale=0.45, enable_gqa=True)
+        o.backward(torch.tensor(do).transpose(1, 2))
+        ro, _ = oracle.attention_fwd(q, k, v, W, 0.45)
+        allclose(ro, o.detach().transpose(1, 2).numpy(), 1e-12)
+        dq, dk, dv = oracle.attention_bwd(q, k, v, do, W, 0.45)
+        allclose(dq, tq.grad.transpose(1, 2).numpy(), 1e-12)
+        allclose(dk, tk.grad.transpose(1, 2).numpy(), 1e-12)
+        allclose(dv, tv.grad.transpose(1, 2).numpy(), 1e-12)
+
+
+def check_decode_row(seed=10):
+    B, Tmax, Hq, Hkv, D = 3, 20, 4, 2, 8
+    kc, vc = rnd((B, Tmax, Hkv, D), seed), rnd((B, Tmax, Hkv, D), seed + 1)
+    qall = rnd((B, Tmax, Hq, D), seed + 2)
+    pos = np.array([0, 7, 19])
+    for W in (-1, 3):
+        o_full, l_full = oracle.attention_fwd(qall, kc, vc, W, 0.5)
+        qd = np.stack([qall[b, pos[b]] for b in range(B)])[:, None]
+        o, l, _, _ = oracle.decode(qd, kc, vc, pos, W, 0.5,
+                                   k_new=kc[np.arange(B), pos][:, None],
+                                   v_new=vc[np.arange(B), pos][:, None])
+        for b in range(B):
+            allclose(o[b, 0], o_full[b, pos[b]], 1e-13)
+            allclose(l[b], l_full[b, :, pos[b]], 1e-13)
+
+
+# ---------------------------------------------------------------- tests
+def test_golden_two_token():
+    check_golden()
+
+
+@pytest.mark.parametrize("W", [-1, 0, 1, 3])
+@pytest.mark.parametrize("G", [1, 2])
+def test_brute_force(W, G):
+    check_brute(W, G)
+
+
+@pytest.mark.parametrize("W", [-1, 2])
+def test_finite_differences(W):
+    check_finite_differences(W)
+
+
+def test_rope_is_complex_rotation():
+    check_rope_complex()
+
+
+def test_rope_and_norm_closed_forms():
+    x = rnd((2, 5, 3, 32), 11)
+    p0 = np.zeros((2, 5), np.int64)
+    allclose(oracle.rope(x, p0, 10000.0), x, 0.0)                       # p = 0 is identity
+    pos = oracle.row_positions(2, 5, [3, 900])
+    y = oracle.rope(x, pos, 10000.0)
+    allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), 1e-12)   # orthogonal
+    allclose(oracle.rope_transpose(y, pos, 10000.0), x, 1e-12)          # transpose inverts
+    # relative position: <R_p a, R_s b> depends only on p - s
+    a, b = x[0, 0, 0], x[1, 1, 1]
+    def rot(vec, p):
+        return oracle.rope(vec[None, None, None], np.array([[p]]), 10000.0)[0, 0, 0]
+    allclose(rot(a, 5) @ rot(b, 2), rot(a, 103) @ rot(b, 100), 1e-12)
+    # norm: unit RMS up to eps, scale invariance, exact eps term, commutes with rope
+    n = oracle.rms_norm(x, 0.0)
+    allclose(np.sqrt(np.mean(n * n, -1)), np.ones(n.shape[:-1]), 1e-12)
+    allclose(oracle.rms_norm(7.5 * x, 0.0), n, 1e-12)
+    u = x / np.sqrt(np.mean(x * x, -1, keepdims=True))                 # mean(u^2) = 1
+    allclose(oracle.rms_norm(u, 0.5), u / math.sqrt(1.5), 1e-12)
+    allclose(oracle.rope(oracle.rms_norm(x, 1e-6), pos, 1e4),
+             oracle.rms_norm(oracle.rope(x, pos, 1e4), 1e-6), 1e-12)
+    allclose(oracle.rms_norm(np.zeros((1, 1, 1, 8)), 1e-6), np.zeros((1, 1, 1, 8)), 0.0)
+
+
+def test_window_ge_T_is_full_causal():
+    check_window_full_causal()
+
+
+def test_gqa_equals_mha_with_repeated_kv():
+    check_gqa_repeat()
+
+
+def test_special_cases():
+    check_special_cases()
+
+
+def test_backward_invariants():
+    check_bwd_invariants()
+
+
+def test_matches_torch_sdpa_fp64():
+    check_sdpa()
+
+
+def test_decode_equals_forward_row():
+    check_decode_row()
+
+
+def test_sampled_backward_matches_full():
+    B, T, Hq, Hkv, D = 2, 40, 4, 2, 8
+    q, k = rnd((B, T, Hq, D), 12), rnd((B, T, Hkv, D), 13)
+    v, do = rnd((B, T, Hkv, D), 14), rnd((B, T, Hq, D), 15)
+    for W in (-1, 6):
+        dq, dk, dv = oracle.attention_bwd(q, k, v, do, W, 0.4)
+        rows = np.array([0, 5, 17, 39])
+        allclose(oracle.attention_bwd_rows(q, k, v, do, W, 0.4, rows), dq[:, rows], 1e-12)
+        sk, sv = oracle.attention_bwd_keys(q, k, v, do, W, 0.4, rows)
+        allclose(sk, dk[:, rows], 1e-12)
+        allclose(sv, dv[:, rows], 1e-12)
+        o, l = oracle.attention_fwd(q, k, v, W, 0.4)
+        so, sl = oracle.attention_fwd(q, k, v, W, 0.4, rows=rows)
+        allclose(so, o[:, rows], 1e-13)
+        allclose(sl, l[:, :, rows], 1e-13)
+
+
+def test_visible_pair_count():
+    for T, W in ((256, 128), (2048, 1024), (2048, 2048), (2048, 512), (8192, 2048), (8192, -1), (5, 0), (1, -1)):
+        assert workloads.visible_pairs(T, W) == oracle.useful_pairs(T, W)
+
+
+# ---------------------------------------------------------------- planted mistakes
+def _rope_wrong_sign(x, positions, base):
+    return oa.rope_transpose(x, positions, base)
+
+
+def _rope_interleaved(x, positions, base):
+    """Pairs (2j, 2j+1) instead of (j, j + D/2)."""
+    x = np.asarray(x, np.float64)
+    D = x.shape[-1]
+    phi = oa.rope_angles(positions, D, base)[:, :, None, :]
+    c, s = np.cos(phi), np.sin(phi)
+    y = np.empty_like(x)
+    y[..., 0::2] = x[..., 0::2] * c - x[..., 1::2] * s
+    y[..., 1::2] = x[..., 0::2] * s + x[..., 1::2] * c
+    return y
+
+
+def _visible_off_by_one(i, j, window):
+    i, j = np.asarray(i), np.asarray(j)
+    ok = j <= i
+    if window >= 0:
+        ok = ok & ((i - j) < window)
+    return ok
+
+
+def _group_modulo(q, k):
+    return q.shape[2] // k.shape[2]
+
+
+def _row_grads_no_delta(q, k, v, dout, b, h, G, window, scale, rows):
+    P, _ = oa._probabilities(q, k, b, h, G, window, scale, rows)
+    dP = dout[b, rows, h, :] @ v[b, :, h // G, :].T
+    return P, P * dP
+
+
+def _prologue_bwd_no_projection(x, dy, positions, base, eps):
+    x = np.asarray(x, np.float64)
+    r = np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    return oa.rope_transpose(dy, positions, base) / r
+
+
+@pytest.mark.parametrize("name,attr,bad,check", [
+    ("rope rotates the wrong way", "rope", _rope_wrong_sign, check_rope_complex),
+    ("rope pairs interleaved", "rope", _rope_interleaved, check_rope_complex),
+    ("window holds W keys, not W+1", "visible", _visible_off_by_one, check_window_full_causal),
+    ("softmax backward drops Delta", "_row_grads", _row_grads_no_delta, check_sdpa),
+    ("prologue backward drops the norm projection", "prologue_bwd", _prologue_bwd_no_projection,
+     check_finite_differences),
+])
+def test_pins_catch_planted_mistakes(monkeypatch, name, attr, bad, check):
+    monkeypatch.setattr(oa, attr, bad)
+    monkeypatch.setattr(oracle, attr, bad, raising=False)
+    with pytest.raises(AssertionError):
+        check()
+
+
+def test_pins_catch_wrong_gqa_mapping(monkeypatch):
+    """Query head h must read KV head h // G; reading h % Hkv breaks GQA == repeated MHA."""
+    def probs_modulo(q, k, b, h, G, window, scale, rows):
+        T = k.shape[1]
+        Hkv = k.shape[2]
+        S = scale * (q[b, rows, h, :] @ k[b, :, h % Hkv, :].T)
+        S = np.where(oa.visible(rows[:, None], np.arange(T)[None, :], window), S, -np.inf)
+        m = S.max(axis=1, keepdims=True)
+        E = np.exp(S - m)
+        return E / E.sum(axis=1, keepdims=True), (m + np.log(E.sum(axis=1, keepdims=True)))[:, 0]
+    monkeypatch.setattr(oa, "_probabilities", probs_modulo)
+    with pytest.raises(AssertionError):
+        check_gqa_repeat()
