@@ -1,0 +1,351 @@
+// C ABI of the causal sliding-window GQA attention library (see cswa_attn.h):
+// argument checks, TMA tensor-map encoding and kernel launches. Nothing here
+// allocates device memory; every launch is asynchronous on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "cswa_attn.h"
+#include "bwd.cuh"
+#include "decode.cuh"
+#include "fwd.cuh"
+#include "prologue.cuh"
+
+using namespace cswa;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// BTHD bf16 tensor as a 4-D tensor map (D, H, T, B); box = 64 x 1 x 128 x 1
+// (one 128-row, 128-byte-wide panel), 128-byte swizzle, zero fill past T.
+bool encode_bthd(CUtensorMap* m, const void* base, int B, int T, int H, int D) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool dims_ok(int B, int T, int Hq, int Hkv) {
+  return B >= 1 && T >= 1 && Hq >= 1 && Hkv >= 1 && Hq % Hkv == 0 && (long long)B * T * Hq < (1ll << 40);
+}
+inline bool scale_ok(float s) { return std::isfinite(s) && s > 0.f; }
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+inline attn_status_t launched() { return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH; }
+
+constexpr float kLog2e = 1.4426950408889634f;
+inline int tiles128(int T) { return (T + 127) / 128; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+template <int D>
+bool set_smem_attrs() {
+  // once per process and head dim; cudaFuncSetAttribute is per-function, device-independent here
+  static bool ok = [] {
+    bool r = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  FwdLayout<D>::kBytes) == cudaSuccess;
+    r = r && cudaFuncSetAttribute(attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  BwdLayout<D>::kBytes) == cudaSuccess;
+    return r;
+  }();
+  return ok;
+}
+
+template <int D, bool kBwd>
+attn_status_t launch_rope(const RopeParams& p, cudaStream_t st) {
+  const long long rows = p.rows[0] + p.rows[1];
+  constexpr int kRowsPerBlock = 256 / (D / 8);
+  const long long blocks = (rows + kRowsPerBlock - 1) / kRowsPerBlock;
+  if (blocks > 0x7fffffffll) return ATTN_ERR_INVALID_ARG;
+  rope_qknorm_kernel<D, kBwd><<<(unsigned)blocks, 256, 0, st>>>(p);
+  return launched();
+}
+
+attn_status_t rope_common(const void* x0, const void* x1, const void* dy0, const void* dy1, void* y0, void* y1,
+                          const int32_t* pos, int B, int T, int Hq, int Hkv, int D, float base, float eps,
+                          void* stream, bool bwd) {
+  if (!dims_ok(B, T, Hq, Hkv) || !(base > 1.f) || !std::isfinite(base) || !(eps >= 0.f) || !std::isfinite(eps))
+    return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!x0 && !x1) return ATTN_ERR_INVALID_ARG;
+  if ((x0 && (!y0 || !aligned16(x0) || !aligned16(y0) || (bwd && (!dy0 || !aligned16(dy0))))) ||
+      (x1 && (!y1 || !aligned16(x1) || !aligned16(y1) || (bwd && (!dy1 || !aligned16(dy1))))))
+    return ATTN_ERR_INVALID_ARG;
+  RopeParams p{};
+  p.x[0] = static_cast<const __nv_bfloat16*>(x0);
+  p.x[1] = static_cast<const __nv_bfloat16*>(x1);
+  p.dy[0] = static_cast<const __nv_bfloat16*>(dy0);
+  p.dy[1] = static_cast<const __nv_bfloat16*>(dy1);
+  p.y[0] = static_cast<__nv_bfloat16*>(y0);
+  p.y[1] = static_cast<__nv_bfloat16*>(y1);
+  p.pos = pos;
+  p.rows[0] = x0 ? (long long)B * T * Hq : 0;
+  p.rows[1] = x1 ? (long long)B * T * Hkv : 0;
+  p.T = T;
+  p.H[0] = Hq;
+  p.H[1] = Hkv;
+  p.eps = eps;
+  p.log2_base = std::log2((double)base);
+  cudaStream_t st = as_stream(stream);
+  if (D == 64) return bwd ? launch_rope<64, true>(p, st) : launch_rope<64, false>(p, st);
+  return bwd ? launch_rope<128, true>(p, st) : launch_rope<128, false>(p, st);
+}
+
+template <int D>
+attn_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T, int Hq,
+                         int Hkv, int window, float scale, cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  if (!encode_bthd(&tq, q, B, T, Hq, D) || !encode_bthd(&tk, k, B, T, Hkv, D) || !encode_bthd(&tv, v, B, T, Hkv, D))
+    return ATTN_ERR_LAUNCH;
+  if (!set_smem_attrs<D>()) return ATTN_ERR_LAUNCH;
+  FwdParams p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.T = T;
+  p.Hq = Hq;
+  p.G = Hq / Hkv;
+  p.window = (window >= T) ? -1 : window;
+  p.scale_log2 = scale * kLog2e;
+  p.nq_tiles = tiles128(T);
+  p.n_pairs = (p.nq_tiles + 1) / 2;
+  dim3 grid(Hq, B, p.n_pairs);
+  attn_fwd_kernel<D><<<grid, 384, FwdLayout<D>::kBytes, st>>>(tq, tk, tv, p);
+  return launched();
+}
+
+struct BwdWorkspace {
+  float* dq_acc;
+  float* lse2;
+  float* delta;
+};
+BwdWorkspace carve_bwd(void* ws, int B, int T, int Hq, int D) {
+  const int Tpad = tiles128(T) * 128;
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  BwdWorkspace w;
+  w.dq_acc = reinterpret_cast<float*>(p);
+  p += align256((size_t)B * T * Hq * D * 4);
+  w.lse2 = reinterpret_cast<float*>(p);
+  p += align256((size_t)B * Hq * Tpad * 4);
+  w.delta = reinterpret_cast<float*>(p);
+  return w;
+}
+
+template <int D>
+attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                         const float* lse, void* dq, void* dk, void* dv, void* ws, int B, int T, int Hq, int Hkv,
+                         int window, float scale, cudaStream_t st) {
+  CUtensorMap tq, tk, tv, tdo;
+  if (!encode_bthd(&tq, q, B, T, Hq, D) || !encode_bthd(&tk, k, B, T, Hkv, D) ||
+      !encode_bthd(&tv, v, B, T, Hkv, D) || !encode_bthd(&tdo, dO, B, T, Hq, D))
+    return ATTN_ERR_LAUNCH;
+  if (!set_smem_attrs<D>()) return ATTN_ERR_LAUNCH;
+  const int Tpad = tiles128(T) * 128;
+  BwdWorkspace w = carve_bwd(ws, B, T, Hq, D);
+  {
+    const long long threads = (long long)B * Tpad * Hq * (D / 8);
+    attn_bwd_prep_kernel<D><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, w.lse2, w.delta,
+        w.dq_acc, B, T, Tpad, Hq);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  }
+  BwdParams p{};
+  p.lse2 = w.lse2;
+  p.delta = w.delta;
+  p.dq_acc = w.dq_acc;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.T = T;
+  p.Tpad = Tpad;
+  p.Hq = Hq;
+  p.G = Hq / Hkv;
+  p.window = (window >= T) ? -1 : window;
+  p.n_tiles = tiles128(T);
+  p.scale = scale;
+  p.scale_log2 = scale * kLog2e;
+  dim3 grid(Hkv, B, p.n_tiles);
+  attn_bwd_kernel<D><<<grid, 384, BwdLayout<D>::kBytes, st>>>(tq, tk, tv, tdo, p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  const long long n8 = (long long)B * T * Hq * D / 8;
+  attn_bwd_dq_cast_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(w.dq_acc, static_cast<__nv_bfloat16*>(dq),
+                                                                       n8);
+  return launched();
+}
+
+template <int D, int GMAX>
+attn_status_t launch_decode(const DecodeParams& p, int B, cudaStream_t st) {
+  dim3 g1(p.n_chunks, p.Hkv, B);
+  decode_chunk_kernel<D, GMAX><<<g1, 128, 0, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  dim3 g2(p.Hq, B);
+  decode_combine_kernel<D><<<g2, D, 0, st>>>(p);
+  return launched();
+}
+
+int decode_chunks(int Tmax, int window) {
+  const int span = (window < 0 || window >= Tmax) ? Tmax : window + 1;
+  return (span + kDecodeChunk - 1) / kDecodeChunk;
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_rope_qknorm(const void* q, const void* k, void* q_out, void* k_out, const int32_t* pos, int B,
+                               int T, int Hq, int Hkv, int D, float rope_base, float eps, void* stream) {
+  return rope_common(q, k, nullptr, nullptr, q_out, k_out, pos, B, T, Hq, Hkv, D, rope_base, eps, stream, false);
+}
+
+attn_status_t attn_rope_qknorm_bwd(const void* q, const void* k, const void* dq_hat, const void* dk_hat, void* dq,
+                                   void* dk, const int32_t* pos, int B, int T, int Hq, int Hkv, int D,
+                                   float rope_base, float eps, void* stream) {
+  return rope_common(q, k, dq_hat, dk_hat, dq, dk, pos, B, T, Hq, Hkv, D, rope_base, eps, stream, true);
+}
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T, int Hq,
+                       int Hkv, int D, int window, float scale, void* stream) {
+  if (!dims_ok(B, T, Hq, Hkv) || !scale_ok(scale)) return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o || !lse || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      !aligned16(lse))
+    return ATTN_ERR_INVALID_ARG;
+  if ((long long)B * Hq > 65535ll * 65535ll || Hq > 0x7fffffff || tiles128(T) > 2 * 65535) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  return D == 64 ? launch_fwd<64>(q, k, v, o, lse, B, T, Hq, Hkv, window, scale, st)
+                 : launch_fwd<128>(q, k, v, o, lse, B, T, Hq, Hkv, window, scale, st);
+}
+
+size_t attn_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D) {
+  if (!dims_ok(B, T, Hq, Hkv) || (D != 64 && D != 128)) return 0;
+  const size_t Tpad = (size_t)tiles128(T) * 128;
+  return align256((size_t)B * T * Hq * D * 4) + 2 * align256((size_t)B * Hq * Tpad * 4);
+}
+
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                       void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int T, int Hq, int Hkv,
+                       int D, int window, float scale, void* stream) {
+  if (!dims_ok(B, T, Hq, Hkv) || !scale_ok(scale)) return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, k, v, o, dO, lse, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return ATTN_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      ws_bytes < attn_bwd_workspace_bytes(B, T, Hq, Hkv, D))
+    return ATTN_ERR_INVALID_ARG;
+  if (Hkv > 65535 || B > 65535 || tiles128(T) > 65535) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  return D == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, workspace, B, T, Hq, Hkv, window, scale, st)
+                 : launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, workspace, B, T, Hq, Hkv, window, scale, st);
+}
+
+size_t attn_decode_workspace_bytes(int B, int Hq, int D, int Tmax, int window) {
+  if (B < 1 || Hq < 1 || Tmax < 1 || (D != 64 && D != 128)) return 0;
+  return (size_t)B * Hq * decode_chunks(Tmax, window) * (D + 2) * 4;
+}
+
+attn_status_t attn_decode(const void* q, void* kcache, void* vcache, const void* k_new, const void* v_new,
+                          const int32_t* pos, void* o, float* lse, int B, int Tmax, int Hq, int Hkv, int D, int window,
+                          float scale, void* workspace, size_t ws_bytes, void* stream) {
+  if (!dims_ok(B, Tmax, Hq, Hkv) || !scale_ok(scale)) return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G > 8) return ATTN_ERR_UNSUPPORTED;
+  if (!q || !kcache || !vcache || !pos || !o || !workspace || (k_new == nullptr) != (v_new == nullptr))
+    return ATTN_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, kcache, vcache, o, workspace};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return ATTN_ERR_INVALID_ARG;
+  if ((k_new && !aligned16(k_new)) || (v_new && !aligned16(v_new)) || (reinterpret_cast<uintptr_t>(pos) & 3u) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return ATTN_ERR_INVALID_ARG;
+  if (ws_bytes < attn_decode_workspace_bytes(B, Hq, D, Tmax, window) || Hkv > 65535 || B > 65535 || Hq > 65535)
+    return ATTN_ERR_INVALID_ARG;
+  DecodeParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.kc = static_cast<__nv_bfloat16*>(kcache);
+  p.vc = static_cast<__nv_bfloat16*>(vcache);
+  p.kn = static_cast<const __nv_bfloat16*>(k_new);
+  p.vn = static_cast<const __nv_bfloat16*>(v_new);
+  p.pos = pos;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.ws = static_cast<float*>(workspace);
+  p.Tmax = Tmax;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = G;
+  p.window = window;
+  p.n_chunks = decode_chunks(Tmax, window);
+  p.scale_log2 = scale * kLog2e;
+  cudaStream_t st = as_stream(stream);
+  const int gm = G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : 8;
+  if (D == 64) {
+    switch (gm) {
+      case 1: return launch_decode<64, 1>(p, B, st);
+      case 2: return launch_decode<64, 2>(p, B, st);
+      case 4: return launch_decode<64, 4>(p, B, st);
+      default: return launch_decode<64, 8>(p, B, st);
+    }
+  }
+  switch (gm) {
+    case 1: return launch_decode<128, 1>(p, B, st);
+    case 2: return launch_decode<128, 2>(p, B, st);
+    case 4: return launch_decode<128, 4>(p, B, st);
+    default: return launch_decode<128, 8>(p, B, st);
+  }
+}
+
+attn_status_t attn_get_status(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return ATTN_ERR_LAUNCH;
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return ATTN_ERR_LAUNCH;
+  if (v && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_LAUNCH;
+  if (v & (kStatusTimeout | kStatusLayout)) return ATTN_ERR_TIMEOUT;
+  if (v & kStatusBadPosition) return ATTN_ERR_DEVICE;
+  return ATTN_OK;
+}
+
+const char* attn_status_string(attn_status_t s) {
+  switch (s) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported head dim or device";
+    case ATTN_ERR_LAUNCH: return "CUDA launch or tensor-map encode failed";
+    case ATTN_ERR_TIMEOUT: return "a device-side wait timed out";
+    case ATTN_ERR_DEVICE: return "a device-side range check failed (decode position out of range)";
+  }
+  return "unknown status";
+}
+
+int attn_device_supported(void) {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return 0;
+  return (major == 10 && minor == 0) ? 1 : 0;
+}
+
+}  // extern "C"

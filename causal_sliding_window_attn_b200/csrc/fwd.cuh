@@ -1,0 +1,314 @@
+// attn_fwd: causal sliding-window GQA attention forward on tcgen05 / TMEM.
+//
+// Computes, per (batch b, query head h, query row i), over the visible keys
+// j (j <= i and, for window W >= 0, i - j <= W) of KV head h / G:
+//   o_i = softmax_j(scale * <q_i, k_j>) v_j,   lse_i = log sum_j exp(scale * <q_i, k_j>)
+// (nanochat Admin & Developer Guide, 3 "Sliding-window attention" and 6 "Attention:
+// FA3 with SDPA Fallback"; nanoGPT Administrator & Developer Guide, 8
+// "CausalSelfAttention", manual path).
+//
+// One CTA owns two 128-row query tiles ("slots") of one (b, h): tiles 2p and
+// 2p+1. It walks the union of their key-tile ranges inside the causal/window
+// band; key tiles outside the band are never loaded.
+//   warp 0      TMA producer: Q once, then K/V tiles into a 2-stage ring
+//   warp 1      MMA issuer (one thread): S_s = Q_s K^T (SS), O_s += P_s V (TS)
+//   warp 2      TMEM allocator
+//   warps 4-7   softmax + epilogue for slot 0 (thread = query row)
+//   warps 8-11  softmax + epilogue for slot 1
+// TMEM (512 columns): S0 | S1 | O0 | O1. P_s (bf16) overwrites the first half
+// of S_s in place and feeds the PV product straight from tensor memory.
+// Softmax runs in the log2 domain; the running max is only moved (and O
+// rescaled) when it grows by more than 2^8, which leaves the result exact.
+#pragma once
+#include "ptx.cuh"
+
+namespace cswa {
+
+struct FwdParams {
+  __nv_bfloat16* o;
+  float* lse;
+  int T, Hq, G, window;
+  float scale_log2;  // scale * log2(e)
+  int nq_tiles;
+  int n_pairs;
+};
+
+template <int D>
+struct FwdLayout {
+  static constexpr int kTile = 128 * D * 2;  // bytes of one 128-row bf16 tile
+  static constexpr int kPanels = D / 64;     // 128-byte-wide panels per tile
+  static constexpr int kQ0 = 0, kQ1 = kTile, kK0 = 2 * kTile, kV0 = 4 * kTile;
+  static constexpr int kBar = 6 * kTile;
+  static constexpr int kBytes = kBar + 256 + 1024;  // + barriers + alignment slack
+  static constexpr uint32_t kTmemCols = 512;
+};
+
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+__global__ void __launch_bounds__(384, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using L = FwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* v_full = bars + 3;    // [2]
+  uint64_t* kv_empty = bars + 5;  // [2]
+  uint64_t* s_full = bars + 7;    // [2]
+  uint64_t* p_full = bars + 9;    // [2]
+  uint64_t* pv_done = bars + 11;  // [2]
+  uint64_t* final_bar = bars + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 15);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int pair = p.n_pairs - 1 - blockIdx.z;  // heaviest tiles first
+  const int hk = h / p.G;
+  const int W = p.window;
+
+  int qt[2], lo[2], hi[2];
+  bool has[2];
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    qt[s] = 2 * pair + s;
+    has[s] = qt[s] < p.nq_tiles;
+    hi[s] = qt[s];
+    lo[s] = (W < 0) ? 0 : max(0, qt[s] * 128 - W) / 128;
+  }
+  const int t_lo = lo[0];
+  const int t_hi = has[1] ? hi[1] : hi[0];
+
+  if (warp == 0 && lane == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 128);
+      mbar_init(&pv_done[s], 1);
+    }
+    mbar_init(final_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS[2] = {tmem, tmem + 128};
+  const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ[2] = {sbase + L::kQ0, sbase + L::kQ1};
+  const uint32_t sK[2] = {sbase + L::kK0, sbase + L::kK0 + L::kTile};
+  const uint32_t sV[2] = {sbase + L::kV0, sbase + L::kV0 + L::kTile};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(q_full, (has[1] ? 2 : 1) * L::kTile);
+      for (int s = 0; s < 2; ++s)
+        if (has[s])
+          for (int pn = 0; pn < L::kPanels; ++pn)
+            tma_load_4d(smem + (s ? L::kQ1 : L::kQ0) + pn * 16384, &tm_q, q_full, pn * 64, h, qt[s] * 128, b);
+      int n = 0, last_issue[2] = {-1, -1};
+      for (int t = t_lo; t <= t_hi; ++t, ++n) {
+        const int st = n & 1;
+        const uint32_t ph = (n >> 1) & 1;
+        if (!mbar_wait(&kv_empty[st], ph ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&k_full[st], L::kTile);
+        for (int pn = 0; pn < L::kPanels; ++pn)
+          tma_load_4d(smem + L::kK0 + st * L::kTile + pn * 16384, &tm_k, &k_full[st], pn * 64, hk, t * 128, b);
+        mbar_arrive_expect_tx(&v_full[st], L::kTile);
+        for (int pn = 0; pn < L::kPanels; ++pn)
+          tma_load_4d(smem + L::kV0 + st * L::kTile + pn * 16384, &tm_v, &v_full[st], pn * 64, hk, t * 128, b);
+        last_issue[st] = n;
+      }
+      if (*abort_flag) {
+        // never leave with copies in flight: wait (bounded) for the last load of each stage
+        for (int st = 0; st < 2; ++st)
+          if (last_issue[st] >= 0) {
+            volatile int dummy = 0;
+            mbar_wait(&k_full[st], (last_issue[st] >> 1) & 1, &dummy);
+            mbar_wait(&v_full[st], (last_issue[st] >> 1) & 1, &dummy);
+          }
+        volatile int dummy = 0;
+        mbar_wait(q_full, 0, &dummy);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idO = idesc_bf16(128, D, false, true);
+      int cnt[2] = {0, 0};
+      bool ok = mbar_wait(q_full, 0, abort_flag);
+      tc_fence_after();
+      int n = 0;
+      for (int t = t_lo; ok && t <= t_hi; ++t, ++n) {
+        const int st = n & 1;
+        const uint32_t ph = (n >> 1) & 1;
+        if (!(ok = mbar_wait(&k_full[st], ph, abort_flag))) break;
+        tc_fence_after();
+        for (int s = 0; s < 2; ++s) {
+          if (!(has[s] && lo[s] <= t && t <= hi[s])) continue;
+          // P_s of the previous tile lives where S_s goes: wait until PV has read it
+          if (cnt[s] > 0 && !(ok = mbar_wait(&pv_done[s], (cnt[s] - 1) & 1, abort_flag))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_ss(tS[s], sdesc_sw128(sQ[s] + off, 16, 1024), sdesc_sw128(sK[st] + off, 16, 1024), idS,
+                   kk > 0);
+          }
+          mma_commit(&s_full[s]);
+        }
+        if (!ok) break;
+        if (!(ok = mbar_wait(&v_full[st], ph, abort_flag))) break;
+        tc_fence_after();
+        for (int s = 0; s < 2; ++s) {
+          if (!(has[s] && lo[s] <= t && t <= hi[s])) continue;
+          if (!(ok = mbar_wait(&p_full[s], cnt[s] & 1, abort_flag))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tO[s], tS[s] + kk * 8, sdesc_sw128(sV[st] + kk * 2048, 16384, 1024), idO,
+                   (cnt[s] > 0 || kk > 0));
+          mma_commit(&pv_done[s]);
+          ++cnt[s];
+        }
+        mma_commit(&kv_empty[st]);
+      }
+      // every MMA issued above has finished before TMEM is released
+      mma_commit(final_bar);
+      volatile int dummy = 0;
+      mbar_wait(final_bar, 0, &dummy);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax
+    const int s = (warp - 4) >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    if (has[s]) {
+      const int q0 = qt[s] * 128;
+      const int i = q0 + row;
+      const float sl2 = p.scale_log2;
+      float m_run = -INFINITY, l_run = 0.f;
+      int cnt = 0;
+      bool ok = true;
+      for (int t = lo[s]; t <= hi[s]; ++t, ++cnt) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[s], cnt & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t r[128];
+        tmem_ld32(tS[s] + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(tS[s] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_ld32(tS[s] + lane_off + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
+        tmem_ld32(tS[s] + lane_off + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
+        tmem_ld_wait();
+        const int k0 = t * 128;
+        const bool full = (k0 + 127 <= q0) && (W < 0 || q0 + 127 - k0 <= W);
+        float mx = -INFINITY;
+        if (full) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(r[c]));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            const int j = k0 + c;
+            const bool vis = (j <= i) && (W < 0 || i - j <= W);
+            if (!vis) r[c] = __float_as_uint(-INFINITY);
+            mx = fmaxf(mx, __uint_as_float(r[c]));
+          }
+        }
+        const float m_tile = mx * sl2;
+        bool rescale = false;
+        float factor = 1.f;
+        if (cnt == 0) {
+          m_run = m_tile;
+        } else if (m_tile > m_run + kRescaleThreshold) {
+          factor = ex2_approx(m_run - m_tile);
+          m_run = m_tile;
+          l_run *= factor;
+          rescale = true;
+        }
+        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+        float lsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * c]), sl2, -m_use));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * c + 1]), sl2, -m_use));
+          lsum += p0 + p1;
+          r[c] = pack_bf16x2(p0, p1);
+        }
+        l_run += lsum;
+        tmem_st32(tS[s] + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_st32(tS[s] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        // rescale only when some row of the warp needs it (O is stable: the MMA
+        // warp waited for the previous PV before issuing this tile's S)
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO[s] + lane_off + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+            tmem_st32(tO[s] + lane_off + c * 32, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[s]);
+      }
+      // ---------------------------------------------------------- epilogue
+      if (ok && cnt > 0) ok = mbar_wait(&pv_done[s], (cnt - 1) & 1, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+      if (ok) {
+        // tcgen05.ld is warp-collective: every lane loads, only rows < T store
+        const bool store = i < p.T;
+        const float inv_l = 1.f / l_run;
+        __nv_bfloat16* dst = p.o + ((size_t)((size_t)b * p.T + i) * p.Hq + h) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO[s] + lane_off + c * 32, o);
+          tmem_ld_wait();
+          uint4 v[4];
+          uint32_t* pv = reinterpret_cast<uint32_t*>(v);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pv[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+          if (store) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) d4[e] = v[e];
+          }
+        }
+        if (store) p.lse[((size_t)b * p.Hq + h) * p.T + i] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+}  // namespace cswa

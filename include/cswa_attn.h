@@ -1,0 +1,139 @@
+/*
+ * cswa_attn.h -- C ABI of the B200 (sm_100a) causal sliding-window GQA attention block.
+ *
+ * The operation is the causal self-attention of the nanochat GPT: queries and
+ * keys RMS-normalised (no weight) and rotated by RoPE, grouped-query heads
+ * (Hkv <= Hq, query head h reads KV head h / (Hq/Hkv)), and a per-layer causal
+ * sliding window (nanochat Admin & Developer Guide, 3 "The GPT Model
+ * (Internals)" and its "Sliding-window attention" part; 6 "Attention: FA3 with
+ * SDPA Fallback"; 7 "KV cache"), with the plain softmax attention of the
+ * nanoGPT Administrator & Developer Guide, 8 "CausalSelfAttention".
+ *
+ * Conventions shared by every call
+ *   - Tensors are device memory owned by the caller. The library never
+ *     allocates: where a call needs scratch space, the caller passes a
+ *     workspace of at least the size the matching *_workspace_bytes() returns.
+ *   - bf16 tensors are stored as raw 16-bit words, in BTHD layout: (B, T, H, D)
+ *     contiguous, D fastest. Every tensor pointer must be 16-byte aligned.
+ *   - D (head dim) is 64 or 128. Hq % Hkv == 0. B, T >= 1.
+ *   - window W >= 0: key j is visible from query i iff 0 <= i - j <= W
+ *     (W + 1 keys including the query itself; FlashAttention's (left=W,
+ *     right=0)). W < 0: plain causal, no window. W >= T - 1 equals W < 0.
+ *   - scale multiplies q.k (1/sqrt(D) for plain attention; nanochat's QK gain
+ *     is folded in here). It must be finite and > 0.
+ *   - lse is the natural-log log-sum-exp of the scaled scores, fp32.
+ *   - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls are asynchronous: they enqueue kernels and return.
+ *   - Argument errors are reported synchronously, before anything is
+ *     enqueued, and leave every output untouched. Errors found on the device
+ *     (a wait that timed out, a decode position out of range) are recorded in a
+ *     per-device status word that attn_get_status() returns and clears.
+ *   - Calls on different streams may run concurrently; they share nothing but
+ *     the status word.
+ */
+#ifndef CSWA_ATTN_H
+#define CSWA_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, Hq % Hkv != 0, bad scale */
+  ATTN_ERR_UNSUPPORTED = 2, /* head dim other than 64/128, or not an sm_100 device */
+  ATTN_ERR_LAUNCH = 3,      /* a CUDA launch or tensor-map encode failed */
+  ATTN_ERR_TIMEOUT = 4,     /* a device-side wait gave up (reported by attn_get_status) */
+  ATTN_ERR_DEVICE = 5       /* a device-side range check failed (reported by attn_get_status) */
+} attn_status_t;
+
+/*
+ * attn_rope_qknorm -- the fused prologue (nanochat Admin & Developer Guide, 3):
+ *   for every row x (D values) of q (B,T,Hq,D) and of k (B,T,Hkv,D):
+ *     xh = x / sqrt(mean(x^2) + eps)
+ *     (y_j, y_{j+D/2}) = rotation of (xh_j, xh_{j+D/2}) by phi_j = p * rope_base^(-2j/D)
+ *   with p = t + (pos ? pos[b] : 0). v is not touched.
+ * q/k may be null (then q_out/k_out are ignored), not both. q_out may equal q
+ * and k_out may equal k (in place). pos: optional int32 device array (B).
+ * eps >= 0, rope_base > 1.
+ */
+attn_status_t attn_rope_qknorm(const void* q, const void* k, void* q_out, void* k_out, const int32_t* pos,
+                               int B, int T, int Hq, int Hkv, int D, float rope_base, float eps, void* stream);
+
+/*
+ * attn_rope_qknorm_bwd -- gradient of the prologue: given the raw q, k and the
+ * gradients dq_hat, dk_hat with respect to its outputs, writes
+ *   dx = (g - xh (g . xh) / D) / r,   r = sqrt(mean(x^2) + eps),
+ * where g is dx_hat rotated by -phi. Same shapes, nullability and aliasing
+ * rules as attn_rope_qknorm (dq may equal dq_hat).
+ */
+attn_status_t attn_rope_qknorm_bwd(const void* q, const void* k, const void* dq_hat, const void* dk_hat,
+                                   void* dq, void* dk, const int32_t* pos, int B, int T, int Hq, int Hkv,
+                                   int D, float rope_base, float eps, void* stream);
+
+/*
+ * attn_fwd -- o = softmax(scale * q k^T restricted to the causal window) v.
+ *   q (B,T,Hq,D), k and v (B,T,Hkv,D) bf16 -> o (B,T,Hq,D) bf16, lse (B,Hq,T) fp32.
+ * o and lse must not overlap the inputs. tcgen05 tensor cores, fp32 accumulation.
+ */
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T,
+                       int Hq, int Hkv, int D, int window, float scale, void* stream);
+
+/* Bytes of workspace attn_bwd needs: an fp32 dQ accumulator (B,T,Hq,D) and
+ * the per-row fp32 dot products Delta_i = dO_i . o_i (B,Hq,T), each 256-byte aligned. */
+size_t attn_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D);
+
+/*
+ * attn_bwd -- gradients of sum(dO * o) for o = attn_fwd(q, k, v):
+ *   Delta_i = dO_i . o_i,  P = exp(scale q k^T - lse),  dV = P^T dO,
+ *   dS = P * (dO V^T - Delta),  dQ = scale dS K,  dK = scale dS^T Q,
+ * with dK, dV summed over the Hq/Hkv query heads of each KV head.
+ * Inputs: q, k, v, o, dO (bf16) and lse (fp32) exactly as attn_fwd produced
+ * them. Outputs dq (B,T,Hq,D), dk, dv (B,T,Hkv,D) bf16, fully overwritten.
+ * workspace: device memory of ws_bytes >= attn_bwd_workspace_bytes(...).
+ */
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                       const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B,
+                       int T, int Hq, int Hkv, int D, int window, float scale, void* stream);
+
+/* Bytes of workspace attn_decode needs (fp32 split-K partials). */
+size_t attn_decode_workspace_bytes(int B, int Hq, int D, int Tmax, int window);
+
+/*
+ * attn_decode -- one new token per sequence against its KV cache
+ * (nanochat Admin & Developer Guide, 7 "KV cache"; 6: decode slices the window).
+ *   q (B,1,Hq,D) bf16, already through the prologue at position pos[b].
+ *   kcache, vcache (B,Tmax,Hkv,D) bf16; pos int32 (B): entries already in
+ *   each cache = the new token's position, 0 <= pos[b] < Tmax.
+ *   k_new, v_new (B,1,Hkv,D) or both null: when given they are written into
+ *   the caches at pos[b] (in place) and attended to; when null the caches must
+ *   already hold the new token's entry at pos[b].
+ *   The token attends to keys [max(0, pos[b] - window), pos[b]].
+ *   o (B,1,Hq,D) bf16; lse (B,Hq) fp32 or null.
+ * Hq/Hkv <= 8 (ATTN_ERR_UNSUPPORTED above). A pos[b] out of range leaves NaN
+ * in that row's outputs and raises ATTN_ERR_DEVICE in the status word.
+ * Memory-bound split-K over key chunks.
+ */
+attn_status_t attn_decode(const void* q, void* kcache, void* vcache, const void* k_new, const void* v_new,
+                          const int32_t* pos, void* o, float* lse, int B, int Tmax, int Hq, int Hkv, int D,
+                          int window, float scale, void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then returns and clears the device status word of the
+ * current device: ATTN_OK, ATTN_ERR_TIMEOUT or ATTN_ERR_DEVICE (or
+ * ATTN_ERR_LAUNCH if a CUDA error is pending). */
+attn_status_t attn_get_status(void* stream);
+
+/* Static description of a status code. */
+const char* attn_status_string(attn_status_t status);
+
+/* 1 when the current device is an sm_100 part this library was built for, else 0. */
+int attn_device_supported(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSWA_ATTN_H */

@@ -1,0 +1,55 @@
+"""Shared helpers for the GPU parity tests: tolerances, error metrics, GPU runners.
+
+Tolerances (outputs: max-abs 1e-2 and relative L2 5e-3; gradients dQ/dK/dV:
+relative L2 1e-2) are the acceptance bar for the attention block; lse gets
+1e-3 absolute.
+"""
+import numpy as np
+import torch
+
+OUT_MAX_ABS = 1e-2
+OUT_REL_L2 = 5e-3
+GRAD_REL_L2 = 1e-2
+LSE_MAX_ABS = 1e-3
+ROPE_BASE = 10000.0
+EPS = 1e-6
+
+
+def f64(t):
+    """bf16/fp32 tensor -> float64 numpy (exact widening)."""
+    return t.detach().to(torch.float32).cpu().numpy().astype(np.float64)
+
+
+def rel_l2(a, ref):
+    a, ref = np.asarray(a, np.float64), np.asarray(ref, np.float64)
+    return float(np.linalg.norm(a - ref) / max(np.linalg.norm(ref), 1e-300))
+
+
+def max_abs(a, ref):
+    return float(np.max(np.abs(np.asarray(a, np.float64) - np.asarray(ref, np.float64))))
+
+
+def check_out(name, a, ref, max_abs_tol=OUT_MAX_ABS, rel_tol=OUT_REL_L2):
+    ma, rl = max_abs(a, ref), rel_l2(a, ref)
+    assert np.all(np.isfinite(a)), f"{name}: non-finite values"
+    assert ma <= max_abs_tol and rl <= rel_tol, f"{name}: max-abs {ma:.3e} rel-L2 {rl:.3e} (max|ref| {np.max(np.abs(ref)):.2f})"
+    return ma, rl
+
+
+def check_grad(name, a, ref, rel_tol=GRAD_REL_L2):
+    rl = rel_l2(a, ref)
+    assert np.all(np.isfinite(a)), f"{name}: non-finite values"
+    assert rl <= rel_tol, f"{name}: rel-L2 {rl:.3e}"
+    return rl
+
+
+def run_block(cswa, q, k, v, do, window, scale):
+    """prologue -> fwd -> bwd -> prologue bwd on the GPU; returns a dict of CUDA tensors."""
+    q, k, v, do = (t.cuda() for t in (q, k, v, do))
+    qh, kh = cswa.attn_rope_qknorm(q, k, rope_base=ROPE_BASE, eps=EPS)
+    o, lse = cswa.attn_fwd(qh, kh, v, window, scale)
+    dqh, dkh, dv = cswa.attn_bwd(qh, kh, v, o, do, lse, window, scale)
+    dq, dk = cswa.attn_rope_qknorm_bwd(q, k, dqh, dkh, rope_base=ROPE_BASE, eps=EPS)
+    torch.cuda.synchronize()
+    assert cswa.attn_get_status() == 0
+    return dict(qh=qh, kh=kh, o=o, lse=lse, dqh=dqh, dkh=dkh, dv=dv, dq=dq, dk=dk)

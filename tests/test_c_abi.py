@@ -1,0 +1,117 @@
+"""CPU-side checks of the C ABI: the library builds, loads without a GPU, exports
+every entry point include/cswa_attn.h declares, sizes workspaces, and rejects
+bad arguments before touching the device (so none of these calls needs a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "cswa_attn.h")
+
+INVALID, UNSUPPORTED = 1, 2
+
+
+@pytest.fixture(scope="module")
+def L():
+    from causal_sliding_window_attn_b200 import build
+    build.build()
+    import causal_sliding_window_attn_b200 as m
+    return m.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_symbols_exported(L):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in cswa_attn.h but not exported"
+
+
+def test_status_strings(L):
+    for s in range(6):
+        assert L.attn_status_string(s)
+    assert b"unknown" in L.attn_status_string(99)
+
+
+def test_bwd_workspace_size(L):
+    B, T, Hq, Hkv, D = 8, 2048, 10, 10, 128
+    dq = B * T * Hq * D * 4
+    rows = B * Hq * 2048 * 4
+    assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D) == dq + 2 * rows
+    # ragged T pads the per-row arrays to whole 128-row tiles
+    n = L.attn_bwd_workspace_bytes(1, 130, 2, 1, 64)
+    assert n == ((130 * 2 * 64 * 4 + 255) // 256) * 256 + 2 * ((2 * 256 * 4 + 255) // 256) * 256
+    assert L.attn_bwd_workspace_bytes(1, 16, 3, 2, 128) == 0     # Hq % Hkv != 0
+    assert L.attn_bwd_workspace_bytes(1, 16, 2, 2, 96) == 0      # head dim
+
+
+def test_decode_workspace_size(L):
+    # 1025 visible keys at most -> 9 chunks of 128
+    assert L.attn_decode_workspace_bytes(32, 10, 128, 2176, 1024) == 32 * 10 * 9 * 130 * 4
+    assert L.attn_decode_workspace_bytes(2, 4, 64, 300, -1) == 2 * 4 * 3 * 66 * 4
+
+
+P = ctypes.c_void_p(0x10000)      # a 16-byte aligned stand-in; never dereferenced
+MIS = ctypes.c_void_p(0x10008)    # misaligned stand-in
+
+
+def test_fwd_rejects_bad_args(L):
+    ok = [P, P, P, P, P, 1, 128, 4, 2, 128, 64, ctypes.c_float(0.1), None]
+    def call(**ch):
+        a = list(ok)
+        for i, v in ch.items():
+            a[int(i[1:])] = v
+        return L.attn_fwd(*a)
+    assert call(a9=96) == UNSUPPORTED                 # head dim
+    assert call(a8=3) == INVALID                      # Hq % Hkv
+    assert call(a5=0) == INVALID                      # B
+    assert call(a6=0) == INVALID                      # T
+    assert call(a11=ctypes.c_float(0.0)) == INVALID   # scale
+    assert call(a11=ctypes.c_float(float("nan"))) == INVALID
+    assert call(a0=None) == INVALID                   # null q
+    assert call(a3=MIS) == INVALID                    # misaligned o
+
+
+def test_bwd_rejects_bad_args(L):
+    ws = L.attn_bwd_workspace_bytes(1, 128, 4, 2, 128)
+    base = [P] * 9 + [P, ws, 1, 128, 4, 2, 128, 64, ctypes.c_float(0.1), None]
+    def call(i, v):
+        a = list(base)
+        a[i] = v
+        return L.attn_bwd(*a)
+    assert call(10, ws - 1) == INVALID                # workspace too small
+    assert call(9, ctypes.c_void_p(0x10010)) == INVALID  # workspace not 256-aligned
+    assert call(6, None) == INVALID                   # null dq
+    assert call(15, 96) == UNSUPPORTED                # head dim
+
+
+def test_rope_rejects_bad_args(L):
+    f = ctypes.c_float
+    assert L.attn_rope_qknorm(None, None, None, None, None, 1, 4, 2, 2, 128, f(1e4), f(1e-6), None) == INVALID
+    assert L.attn_rope_qknorm(P, None, P, None, None, 1, 4, 2, 2, 128, f(1.0), f(1e-6), None) == INVALID
+    assert L.attn_rope_qknorm(P, None, P, None, None, 1, 4, 2, 2, 128, f(1e4), f(-1.0), None) == INVALID
+    assert L.attn_rope_qknorm(P, None, MIS, None, None, 1, 4, 2, 2, 128, f(1e4), f(1e-6), None) == INVALID
+    assert L.attn_rope_qknorm(P, P, P, P, None, 1, 4, 2, 2, 32, f(1e4), f(1e-6), None) == UNSUPPORTED
+
+
+def test_decode_rejects_bad_args(L):
+    ws = L.attn_decode_workspace_bytes(2, 4, 128, 64, -1)
+    base = [P, P, P, None, None, P, P, P, 2, 64, 4, 2, 128, -1, ctypes.c_float(0.1), P, ws, None]
+    def call(i, v):
+        a = list(base)
+        a[i] = v
+        return L.attn_decode(*a)
+    assert call(16, ws - 4) == INVALID
+    assert call(3, P) == INVALID                      # k_new without v_new
+    assert call(10, 5) == INVALID                     # Hq % Hkv
+    a = list(base)
+    a[10], a[11] = 18, 2                              # G = 9 > 8
+    a[16] = L.attn_decode_workspace_bytes(2, 18, 128, 64, -1)
+    assert L.attn_decode(*a) == UNSUPPORTED

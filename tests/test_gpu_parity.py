@@ -1,0 +1,207 @@
+"""GPU parity: every call of the C ABI against the fp64 oracle, element by element.
+
+Small cases span several 128-row tiles and a ragged tail; two levels each:
+  kernel-only  the oracle's attention run on the exact bf16 q_hat / k_hat the GPU
+               prologue produced (isolates the attention kernels)
+  end-to-end   the oracle's own fp64 prologue from the raw bf16 q, k
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests.parity import (EPS, LSE_MAX_ABS, ROPE_BASE, check_grad, check_out, f64, max_abs, run_block)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def cswa():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import causal_sliding_window_attn_b200 as m
+    m.lib()
+    assert m.lib().attn_device_supported() == 1, "not an sm_100 device"
+    return m
+
+
+CASES = [
+    # B, T, Hq, Hkv, D, window
+    (1, 256, 4, 2, 64, 128),     # the tiny correctness configuration
+    (2, 700, 4, 2, 128, 200),    # ragged tail, window not a tile multiple
+    (1, 300, 2, 2, 128, -1),     # full causal, ragged
+    (1, 513, 4, 4, 128, 256),    # window = 2 tiles, one row past a tile
+    (1, 129, 3, 1, 64, 0),       # self only, G = 3
+    (2, 1, 2, 1, 128, -1),       # T = 1
+    (1, 640, 8, 2, 128, 1000),   # window >= T: plain causal
+    (1, 384, 2, 1, 128, 127),    # window one short of a tile
+]
+
+
+def _ids(c):
+    return "B{}_T{}_Hq{}_Hkv{}_D{}_W{}".format(*c)
+
+
+@pytest.mark.parametrize("case", CASES, ids=_ids)
+def test_block_matches_oracle(cswa, case):
+    B, T, Hq, Hkv, D, W = case
+    scale = workloads.default_scale(D)
+    q, k, v, do = workloads.training_inputs(B, T, Hq, Hkv, D, seed=100 + T)
+    g = run_block(cswa, q, k, v, do, W, scale)
+    pos = oracle.row_positions(B, T)
+    qf, kf, vf, dof = f64(q), f64(k), f64(v), f64(do)
+
+    # prologue
+    qh_ref = oracle.prologue(qf, pos, ROPE_BASE, EPS)
+    kh_ref = oracle.prologue(kf, pos, ROPE_BASE, EPS)
+    check_out("q_hat", f64(g["qh"]), qh_ref)
+    check_out("k_hat", f64(g["kh"]), kh_ref)
+
+    # forward, kernel-only
+    qh, kh = f64(g["qh"]), f64(g["kh"])
+    o_ref, lse_ref = oracle.attention_fwd(qh, kh, vf, W, scale)
+    check_out("o (kernel)", f64(g["o"]), o_ref)
+    assert max_abs(f64(g["lse"]), lse_ref) <= LSE_MAX_ABS
+    # forward, end-to-end
+    o_e2e, _ = oracle.attention_fwd(qh_ref, kh_ref, vf, W, scale)
+    check_out("o (end-to-end)", f64(g["o"]), o_e2e)
+
+    # backward, kernel-only
+    dq_ref, dk_ref, dv_ref = oracle.attention_bwd(qh, kh, vf, dof, W, scale)
+    check_grad("dq_hat", f64(g["dqh"]), dq_ref)
+    check_grad("dk_hat", f64(g["dkh"]), dk_ref)
+    check_grad("dv", f64(g["dv"]), dv_ref)
+    # backward through the prologue, end-to-end from the raw inputs
+    dqe, dke, dve = oracle.attention_bwd(qh_ref, kh_ref, vf, dof, W, scale)
+    check_grad("dq (end-to-end)", f64(g["dq"]), oracle.prologue_bwd(qf, dqe, pos, ROPE_BASE, EPS))
+    check_grad("dk (end-to-end)", f64(g["dk"]), oracle.prologue_bwd(kf, dke, pos, ROPE_BASE, EPS))
+    check_grad("dv (end-to-end)", f64(g["dv"]), dve)
+
+
+def test_prologue_positions_and_inplace(cswa):
+    """Per-row position offsets (decode / chunked prefill) and in-place operation."""
+    B, T, Hq, Hkv, D = 3, 5, 4, 2, 128
+    q, k, _, dy = workloads.training_inputs(B, T, Hq, Hkv, D, seed=7)
+    pos = torch.tensor([0, 777, 8000], dtype=torch.int32)
+    qd, kd, dyd = q.cuda(), k.cuda(), dy.cuda()
+    qh, kh = cswa.attn_rope_qknorm(qd, kd, pos=pos.cuda())
+    positions = oracle.row_positions(B, T, pos.numpy())
+    check_out("q_hat", f64(qh), oracle.prologue(f64(q), positions, ROPE_BASE, EPS))
+    check_out("k_hat", f64(kh), oracle.prologue(f64(k), positions, ROPE_BASE, EPS))
+    q2 = qd.clone()
+    cswa.attn_rope_qknorm(q2, None, q_out=q2, pos=pos.cuda())
+    assert torch.equal(q2, qh)
+    dq, _ = cswa.attn_rope_qknorm_bwd(qd, None, dyd, None, pos=pos.cuda())
+    check_grad("dq", f64(dq), oracle.prologue_bwd(f64(q), f64(dy), positions, ROPE_BASE, EPS))
+
+
+def test_window_ge_T_is_causal_on_gpu(cswa):
+    B, T, Hq, Hkv, D = 1, 400, 2, 1, 128
+    q, k, v, _ = workloads.training_inputs(B, T, Hq, Hkv, D, seed=11)
+    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    ref, lref = cswa.attn_fwd(q, k, v, -1)
+    for W in (T - 1, T, 5000):
+        o, l = cswa.attn_fwd(q, k, v, W)
+        assert torch.equal(o, ref) and torch.equal(l, lref)
+    o, _ = cswa.attn_fwd(q, k, v, T - 2)
+    assert not torch.equal(o, ref)
+
+
+def test_gqa_matches_repeated_kv_on_gpu(cswa):
+    B, T, Hkv, G, D = 1, 300, 2, 4, 128
+    q, k, v, do = workloads.training_inputs(B, T, Hkv * G, Hkv, D, seed=12)
+    q, k, v, do = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    kr, vr = k.repeat_interleave(G, dim=2).contiguous(), v.repeat_interleave(G, dim=2).contiguous()
+    o, l = cswa.attn_fwd(q, k, v, 100)
+    om, lm = cswa.attn_fwd(q, kr, vr, 100)
+    assert torch.equal(o, om) and torch.equal(l, lm)
+    dq, dk, dv = cswa.attn_bwd(q, k, v, o, do, l, 100)
+    dqm, dkm, dvm = cswa.attn_bwd(q, kr, vr, om, do, lm, 100)
+    check_grad("dq", f64(dq), f64(dqm), 2e-3)
+    check_grad("dk", f64(dk), f64(dkm).reshape(B, T, Hkv, G, D).sum(3), 5e-3)
+    check_grad("dv", f64(dv), f64(dvm).reshape(B, T, Hkv, G, D).sum(3), 5e-3)
+
+
+def test_T1_W0_return_v(cswa):
+    B, T, Hq, Hkv, D = 2, 200, 4, 2, 64
+    q, k, v, _ = workloads.training_inputs(B, T, Hq, Hkv, D, seed=13)
+    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    o, _ = cswa.attn_fwd(q, k, v, 0)
+    assert torch.equal(o, v.repeat_interleave(2, dim=2))
+    o, _ = cswa.attn_fwd(q[:, :1].contiguous(), k[:, :1].contiguous(), v[:, :1].contiguous(), -1)
+    assert torch.equal(o, v[:, :1].repeat_interleave(2, dim=2))
+
+
+def _decode_case(cswa, B, Tmax, Hq, Hkv, D, W, pos, seed, append):
+    g = torch.Generator().manual_seed(seed)
+    kraw = torch.randn((B, Tmax, Hkv, D), generator=g).to(torch.bfloat16).cuda()
+    vc = torch.randn((B, Tmax, Hkv, D), generator=g).to(torch.bfloat16).cuda()
+    qraw = torch.randn((B, 1, Hq, D), generator=g).to(torch.bfloat16).cuda()
+    knraw = torch.randn((B, 1, Hkv, D), generator=g).to(torch.bfloat16).cuda()
+    vn = torch.randn((B, 1, Hkv, D), generator=g).to(torch.bfloat16).cuda()
+    kc, _ = cswa.attn_rope_qknorm(None, kraw)
+    posd = torch.tensor(pos, dtype=torch.int32).cuda()
+    qd, kn = cswa.attn_rope_qknorm(qraw, knraw, pos=posd)
+    # slots past each sequence's position hold NaN: they must never be read
+    for b, p in enumerate(pos):
+        kc[b, p + (1 if not append else 0):] = float("nan")
+        vc[b, p + (1 if not append else 0):] = float("nan")
+    if not append:
+        for b, p in enumerate(pos):
+            kc[b, p] = kn[b, 0]
+            vc[b, p] = vn[b, 0]
+    kc_before, vc_before = kc.clone(), vc.clone()
+    o, lse = cswa.attn_decode(qd, kc, vc, posd, W, k_new=kn if append else None, v_new=vn if append else None)
+    torch.cuda.synchronize()
+    assert cswa.attn_get_status() == 0
+    o_ref, lse_ref, kc_ref, vc_ref = oracle.decode(f64(qd), np.nan_to_num(f64(kc_before)),
+                                                   np.nan_to_num(f64(vc_before)), np.array(pos), W,
+                                                   workloads.default_scale(D),
+                                                   k_new=f64(kn) if append else None,
+                                                   v_new=f64(vn) if append else None)
+    check_out("decode o", f64(o), o_ref)
+    assert max_abs(f64(lse), lse_ref) <= LSE_MAX_ABS
+    if append:
+        for b, p in enumerate(pos):
+            assert torch.equal(kc[b, p], kn[b, 0]) and torch.equal(vc[b, p], vn[b, 0])
+        # nothing else in the caches changed
+        mask = torch.ones(B, Tmax, dtype=torch.bool)
+        for b, p in enumerate(pos):
+            mask[b, p] = False
+        assert torch.equal(kc[mask.cuda()].nan_to_num(7.0), kc_before[mask.cuda()].nan_to_num(7.0))
+    return o
+
+
+@pytest.mark.parametrize("append", [True, False])
+@pytest.mark.parametrize("W", [100, -1, 0])
+def test_decode_small(cswa, W, append):
+    _decode_case(cswa, 4, 300, 4, 2, 128, W, [0, 150, 299, 37], seed=21, append=append)
+
+
+def test_decode_d64_gqa8(cswa):
+    _decode_case(cswa, 2, 700, 8, 1, 64, 300, [650, 5], seed=22, append=True)
+
+
+def test_decode_equals_forward_row(cswa):
+    """Decode at position p equals row p of attn_fwd on the same sequence."""
+    B, T, Hq, Hkv, D, W = 1, 520, 4, 2, 128, 200
+    q, k, v, _ = workloads.training_inputs(B, T, Hq, Hkv, D, seed=23)
+    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    qh, kh = cswa.attn_rope_qknorm(q, k)
+    o, lse = cswa.attn_fwd(qh, kh, v, W)
+    for p in (0, 127, 128, 519):
+        posd = torch.tensor([p], dtype=torch.int32).cuda()
+        od, ld = cswa.attn_decode(qh[:, p:p + 1].contiguous(), kh.clone(), v.clone(), posd, W)
+        assert max_abs(f64(od[0, 0]), f64(o[0, p])) <= 1e-2
+        assert max_abs(f64(ld[0]), f64(lse[0, :, p])) <= 1e-3
+
+
+def test_decode_bad_position_is_reported(cswa):
+    B, Tmax, H, D = 2, 64, 2, 128
+    q = torch.zeros((B, 1, H, D), dtype=torch.bfloat16).cuda()
+    kc = torch.zeros((B, Tmax, H, D), dtype=torch.bfloat16).cuda()
+    pos = torch.tensor([3, Tmax], dtype=torch.int32).cuda()
+    o, lse = cswa.attn_decode(q, kc, kc.clone(), pos, -1)
+    assert cswa.attn_get_status() == 5  # ATTN_ERR_DEVICE
+    assert torch.isnan(o[1].float()).all() and torch.isfinite(o[0].float()).all()
+    assert cswa.attn_get_status() == 0  # cleared
