@@ -1,0 +1,458 @@
+"""Benchmark of the causal sliding-window GQA attention block on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cswa|reference]
+
+One step is the whole hot path on one batch: for each layer of the nanochat-d20
+shaped pair (B=8, T=2048, Hq=Hkv=10, D=128; a short layer with window 1024 and
+a long layer with window 2048 = full causal) it runs the RoPE + QK-norm
+prologue, attention forward, attention backward and the prologue backward.
+`value` is useful fwd+bwd TFLOP/s: 12*D per visible (query, key) pair (the
+pages' 3 x forward convention), masked work and recompute not counted. The
+KV-cache decode workload (32 sequences, lengths U[512, 2048], window 1024) is
+timed in the same run and reported under "decode" as HBM GB/s.
+
+Under torchrun each rank runs its own batch (weak scaling, no collective on
+the data path); times are the max over ranks. `--impl reference` times the
+fp64 CPU oracle on a bounded sample of the same workload instead.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+import workloads  # noqa: E402
+
+METRIC = "attention fwd+bwd TFLOP/s (useful FLOPs) & % bf16 peak; decode HBM GB/s"
+WORKLOAD = ("nanochat-d20 attention layer pair, fwd+bwd incl. RoPE+QK-norm prologue: B=8 T=2048 Hq=Hkv=10 "
+            "D=128 bf16, windows 1024 (short layer) and 2048 (long layer)")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ distributed
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def shard_seed(base_seed, rank):
+    """Each rank draws its own batch: the global batch is world x B sequences."""
+    return base_seed + 1000 * rank
+
+
+# ------------------------------------------------------------------ FLOPs / bytes
+def layer_useful_flops(B, T, Hq, D, W):
+    n = B * Hq * workloads.visible_pairs(T, W)
+    return 4.0 * D * n, 8.0 * D * n
+
+
+def decode_bytes(lengths, Hq, Hkv, D, W):
+    """Algorithmic HBM bytes of one decode step: the visible K and V rows, q, o,
+    lse, the new k/v read and appended, and pos."""
+    B = len(lengths)
+    n = sum(min(int(p), W) + 1 if W >= 0 else int(p) + 1 for p in lengths)
+    return (n * Hkv * D * 2 * 2 + B * Hq * D * 2 * 2 + B * Hq * 4 + 2 * B * Hkv * D * 2 * 2 + B * 4)
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons every 200 ms while running."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.rows = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                     timeout=5).stdout.strip()
+                if out:
+                    self.rows.append([x.strip() for x in out.split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        self._t.join(timeout=10)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if len(r) > 5 + i and r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+# ------------------------------------------------------------------ GPU arm
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "causal_sliding_window_attn_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel):
+    """dram bytes per launch from the committed ncu summary, if the kernel sources are unchanged."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel)
+    if not d or d.get("csrc_sha") != kernel_source_sha():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+def flush_l2(buf):
+    buf.add_(1)
+
+
+def run_gpu(args, rank, world, local):
+    import causal_sliding_window_attn_b200 as cswa
+    cswa.lib()
+    dev = torch.device("cuda", local)
+    c = workloads.CONFIGS["d20"]
+    B, T, Hq, Hkv, D = c["B"], c["T"], c["Hq"], c["Hkv"], c["D"]
+    windows = c["windows"]
+    scale = workloads.default_scale(D)
+    q, k, v, do = (t.to(dev) for t in workloads.training_inputs(B, T, Hq, Hkv, D, shard_seed(c["seed"], rank)))
+    # per-layer buffers (all outputs preallocated; the library allocates nothing)
+    L = []
+    for W in windows:
+        L.append(dict(W=W, qh=torch.empty_like(q), kh=torch.empty_like(k), o=torch.empty_like(q),
+                      lse=torch.empty((B, Hq, T), device=dev, dtype=torch.float32),
+                      dqh=torch.empty_like(q), dkh=torch.empty_like(k), dv=torch.empty_like(v),
+                      dq=torch.empty_like(q), dk=torch.empty_like(k),
+                      ws=torch.empty(cswa.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D), device=dev,
+                                     dtype=torch.uint8)))
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    per_op = {"prologue": 0.0, "fwd": 0.0, "bwd": 0.0, "prologue_bwd": 0.0}
+    bwd_ms = [0.0, 0.0]
+
+    def step(record):
+        for li, l in enumerate(L):
+            e = [ev() for _ in range(5)] if record else None
+            if record:
+                e[0].record()
+            cswa.attn_rope_qknorm(q, k, l["qh"], l["kh"])
+            if record:
+                e[1].record()
+            cswa.attn_fwd(l["qh"], l["kh"], v, l["W"], scale, o=l["o"], lse=l["lse"])
+            if record:
+                e[2].record()
+            cswa.attn_bwd(l["qh"], l["kh"], v, l["o"], do, l["lse"], l["W"], scale, dq=l["dqh"], dk=l["dkh"],
+                          dv=l["dv"], workspace=l["ws"])
+            if record:
+                e[3].record()
+            cswa.attn_rope_qknorm_bwd(q, k, l["dqh"], l["dkh"], l["dq"], l["dk"])
+            if record:
+                e[4].record()
+                l["events"] = l.get("events", []) + [e]
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    assert cswa.attn_get_status() == 0
+    for l in L:
+        l["events"] = []
+    barrier(world)
+    torch.cuda.synchronize()
+    t0, t1 = ev(), ev()
+    with ClockSampler(local) as clocks:
+        t0.record()
+        for _ in range(args.steps):
+            step(True)
+        t1.record()
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_total = t0.elapsed_time(t1)
+    for li, l in enumerate(L):
+        for e in l["events"]:
+            per_op["prologue"] += e[0].elapsed_time(e[1])
+            per_op["fwd"] += e[1].elapsed_time(e[2])
+            bwd_ms[li] += e[2].elapsed_time(e[3])
+            per_op["prologue_bwd"] += e[3].elapsed_time(e[4])
+    per_op["bwd"] = sum(bwd_ms)
+    status = cswa.attn_get_status()
+    assert status == 0, f"device status {status}"
+
+    ms_step = max_over_ranks(ms_total / args.steps, world)
+    flops_f = sum(layer_useful_flops(B, T, Hq, D, W)[0] for W in windows)
+    flops_b = sum(layer_useful_flops(B, T, Hq, D, W)[1] for W in windows)
+    value = world * (flops_f + flops_b) / (ms_step * 1e-3) / 1e12
+
+    pk, pk_src = peaks()
+    peak_sus = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    peak_burst = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    bwd_avg_ms = per_op["bwd"] / (2 * args.steps)
+    bwd_tflops = flops_b / 2 / (bwd_avg_ms * 1e-3) / 1e12
+    fwd_avg_ms = per_op["fwd"] / (2 * args.steps)
+    traffic = ncu_traffic("attn_bwd_kernel")
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 activations of the d20 shapes)",
+        "config": {"workload": WORKLOAD, "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world}",
+                   "l2": "no flush: each layer's inputs (q,k,v,dO: 168 MB) exceed the 126 MB L2"},
+        "pct_bf16_peak": {"of_sustained": round(value / world / peak_sus, 4),
+                          "of_burst": round(value / world / peak_burst, 4), "peaks": pk_src},
+        "breakdown_ms_per_step": {k2: round(v2 / args.steps, 4) for k2, v2 in per_op.items()},
+        "fwd_tflops": round(flops_f / 2 / (fwd_avg_ms * 1e-3) / 1e12, 1),
+        "bwd_tflops": round(bwd_tflops, 1),
+        "bwd_tflops_fa_convention": round(bwd_tflops * 10 / 8, 1),
+        "roofline": {"kernel": "attn_bwd call (prep + main + dq cast launches), both layers", "bound": "tensor",
+                     "achieved": round(bwd_tflops, 1), "peak": peak_sus, "unit": "TFLOP/s",
+                     "frac": round(bwd_tflops / peak_sus, 4),
+                     "peak_kind": f"bf16 sustained ({pk_src}); burst {peak_burst}",
+                     "traffic": traffic,
+                     "algorithmic_flops_per_launch": flops_b / 2},
+        "gpu_launches": 12 * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and not args.no_decode:
+        result["decode"] = run_decode(cswa, dev, args, pk, pk_src)
+    if not args.no_e2e:
+        result["e2e"] = run_e2e(cswa, dev, args, q, k, v, do, L, scale, world, flops_f + flops_b)
+    return result
+
+
+def run_decode(cswa, dev, args, pk, pk_src):
+    c = workloads.DECODE
+    B, Hq, Hkv, D, Tmax, W = c["B"], c["Hq"], c["Hkv"], c["D"], c["Tmax"], c["window"]
+    lengths, kraw, vc, qraw, knraw, vn = workloads.decode_inputs(**c)
+    kraw, vc, qraw, knraw, vn = (t.to(dev) for t in (kraw, vc, qraw, knraw, vn))
+    pos = lengths.to(dev)
+    _, kc = cswa.attn_rope_qknorm(None, kraw)
+    qd, kn = cswa.attn_rope_qknorm(qraw, knraw, pos=pos)
+    o = torch.empty_like(qd)
+    lse = torch.empty((B, Hq), device=dev, dtype=torch.float32)
+    ws = torch.empty(cswa.attn_decode_workspace_bytes(B, Hq, D, Tmax, W), device=dev, dtype=torch.uint8)
+    flush = torch.empty(256 * 1024 * 1024 // 4, device=dev, dtype=torch.float32)
+    reps = max(20, args.steps)
+    times = []
+    for i in range(5 + reps):
+        flush_l2(flush)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        cswa.attn_decode(qd, kc, vc, pos, W, k_new=kn, v_new=vn, o=o, lse=lse, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 5:
+            times.append(e0.elapsed_time(e1))
+    assert cswa.attn_get_status() == 0
+    ms = statistics.median(times)
+    nbytes = decode_bytes(lengths.tolist(), Hq, Hkv, D, W)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    hbm = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    return {"workload": "KV-cache decode: 32 sequences, lengths U[512,2048] (seed 4), Hq=Hkv=10, D=128, "
+                        "Tmax=2176, window 1024, append of the new k/v",
+            "us_per_step": round(ms * 1e3, 2), "us_p10": round(np.percentile(times, 10) * 1e3, 2),
+            "us_p90": round(np.percentile(times, 90) * 1e3, 2), "value": round(gbs, 1), "unit": "GB/s",
+            "l2": "flushed (256 MB write) before every call", "gpu_launches_per_step": 2,
+            "roofline": {"kernel": "attn_decode (chunk + combine)", "bound": "hbm", "achieved": round(gbs, 1),
+                         "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                         "traffic": ncu_traffic("decode_chunk_kernel"), "algorithmic_bytes": nbytes,
+                         "peak_kind": pk_src}}
+
+
+def run_e2e(cswa, dev, args, q, k, v, do, L, scale, world, flops):
+    """The same step through the public API with pinned HOST buffers: inputs copied
+    to the device and the layer outputs (o, dq, dk, dv) copied back every step."""
+    hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+    outs = []
+    for l in L:
+        outs.append([(l[n], torch.empty(l[n].shape, dtype=l[n].dtype, pin_memory=True))
+                     for n in ("o", "dq", "dk", "dv")])
+    B, T, Hq, D = q.shape
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+    d2h = sum(h.numel() * h.element_size() for lst in outs for _, h in lst)
+
+    def step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        do.copy_(hdo, non_blocking=True)
+        for l in L:
+            cswa.attn_rope_qknorm(q, k, l["qh"], l["kh"])
+            cswa.attn_fwd(l["qh"], l["kh"], v, l["W"], scale, o=l["o"], lse=l["lse"])
+            cswa.attn_bwd(l["qh"], l["kh"], v, l["o"], do, l["lse"], l["W"], scale, dq=l["dqh"], dk=l["dkh"],
+                          dv=l["dv"], workspace=l["ws"])
+            cswa.attn_rope_qknorm_bwd(q, k, l["dqh"], l["dkh"], l["dq"], l["dk"])
+        for lst in outs:
+            for d, h in lst:
+                h.copy_(d, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    steps = max(5, args.steps // 4)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    return {"value": round(world * flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 3),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "how": "pinned host q,k,v,dO -> device, both layers fwd+bwd, o/dq/dk/dv -> pinned host"}
+
+
+# ------------------------------------------------------------------ CPU (oracle) arm
+def oracle_sample(seconds_budget, seed_offset=0):
+    """Times the fp64 oracle on (batch, head) units of the d20 pair until the budget
+    is spent: per unit, prologue + forward + backward + prologue backward of one
+    head of one sequence, for both layers. Returns (TFLOP/s, description, cores)."""
+    import oracle
+    c = workloads.CONFIGS["d20"]
+    B, T, Hq, Hkv, D = c["B"], c["T"], c["Hq"], c["Hkv"], c["D"]
+    scale = workloads.default_scale(D)
+    q, k, v, do = workloads.training_inputs(1, T, Hq, Hkv, D, c["seed"] + seed_offset)
+    pos = oracle.row_positions(1, T)
+    flops, units = 0.0, 0
+    t0 = time.perf_counter()
+    h = 0
+    while True:
+        hs = slice(h % Hq, h % Hq + 1)
+        qf, kf, vf, dof = (t[:, :, hs].float().numpy().astype(np.float64) for t in (q, k, v, do))
+        for W in c["windows"]:
+            qh = oracle.prologue(qf, pos, workloads.ROPE_BASE, workloads.EPS)
+            kh = oracle.prologue(kf, pos, workloads.ROPE_BASE, workloads.EPS)
+            oracle.attention_fwd(qh, kh, vf, W, scale)
+            dqh, dkh, _ = oracle.attention_bwd(qh, kh, vf, dof, W, scale)
+            oracle.prologue_bwd(qf, dqh, pos, workloads.ROPE_BASE, workloads.EPS)
+            oracle.prologue_bwd(kf, dkh, pos, workloads.ROPE_BASE, workloads.EPS)
+            flops += 12.0 * D * workloads.visible_pairs(T, W)
+        units += 1
+        h += 1
+        if time.perf_counter() - t0 >= seconds_budget:
+            break
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    desc = (f"{units} (sequence, head) units of the d20 layer pair (both windows), fp64 numpy oracle, "
+            f"{dt:.1f} s")
+    return flops / dt / 1e12, desc, cores
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(budget)
+    vals = []
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        v, desc, cores = oracle_sample(budget, seed_offset=0)
+        vals.append(v)
+    wall = time.perf_counter() - t0
+    value = statistics.median(vals)
+    ms = 12.0 * 128 * sum(workloads.visible_pairs(2048, W) for W in (1024, 2048)) * 80 / (value * 1e12) * 1e3
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": 8, "seq_len": 2048, "parallelism": "cpu"},
+            "cpu_baseline": {"kind": "oracle", "value": value, "unit": "TFLOP/s", "cores": cores,
+                             "sample": desc + f" per step; {args.steps} steps in {wall:.1f} s"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="cswa", choices=["cswa", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the cpu_baseline oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, rank, world)
+        else:
+            if args.warmup < 3:
+                raise SystemExit("timing rules need at least 3 warm-up steps")
+            res = run_gpu(args, rank, world, local)
+            if rank == 0 and not args.no_cpu_baseline:
+                v, desc, cores = oracle_sample(args.cpu_seconds)
+                res["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                       "sample": desc}
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

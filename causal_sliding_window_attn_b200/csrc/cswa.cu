@@ -88,7 +88,9 @@ attn_status_t launch_rope(const RopeParams& p, cudaStream_t st) {
 attn_status_t rope_common(const void* x0, const void* x1, const void* dy0, const void* dy1, void* y0, void* y1,
                           const int32_t* pos, int B, int T, int Hq, int Hkv, int D, float base, float eps,
                           void* stream, bool bwd) {
-  if (!dims_ok(B, T, Hq, Hkv) || !(base > 1.f) || !std::isfinite(base) || !(eps >= 0.f) || !std::isfinite(eps))
+  // the prologue treats q and k rows alike: no Hq/Hkv relation is needed here
+  if (B < 1 || T < 1 || (x0 && Hq < 1) || (x1 && Hkv < 1) || (long long)B * T * (Hq + Hkv) >= (1ll << 40) ||
+      !(base > 1.f) || !std::isfinite(base) || !(eps >= 0.f) || !std::isfinite(eps))
     return ATTN_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
   if (!x0 && !x1) return ATTN_ERR_INVALID_ARG;

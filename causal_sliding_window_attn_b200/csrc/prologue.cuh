@@ -11,8 +11,8 @@
 //
 // HBM-bound elementwise work: D/8 lanes own one row, 16 bytes each (one
 // vector load per operand), the pair partner j + D/2 is a shuffle away. The
-// angle p * omega_j is formed and reduced modulo 2*pi in fp64 so that the
-// fp32 sin/cos see an exact argument even at positions of several thousand.
+// angle p * omega_j is reduced modulo 2*pi exactly in 64-bit fixed point, so
+// the fp32 sin/cos see a small, accurate argument at any position.
 #pragma once
 #include "ptx.cuh"
 
@@ -29,22 +29,25 @@ struct RopeParams {
   double log2_base;
 };
 
+// The angle of pair j at position p, in turns, is p * u_j with u_j = omega_j / (2 pi).
+// u_j is held as a 64-bit fixed-point fraction U_j = u_j * 2^64, so that
+// p * U_j mod 2^64 is the exact fractional part of p * u_j (to 2^-53 of u_j,
+// from the fp64 value it was built from) for any 32-bit position; its top 32
+// bits, read as a signed number, give the reduced angle in [-pi, pi).
 template <int D>
-__device__ __forceinline__ void rope_row_angles(const RopeParams& p, const double* omega, int seg, long long r,
-                                                int lane_in_row, float (&c)[8], float (&s)[8]) {
+__device__ __forceinline__ void rope_row_angles(const RopeParams& p, const unsigned long long* turns, int seg,
+                                                long long r, int lane_in_row, float (&c)[8], float (&s)[8]) {
   const long long bt = r / p.H[seg];
   const int t = (int)(bt % p.T);
   const int b = (int)(bt / p.T);
-  const double pos = (double)(t + (p.pos ? p.pos[b] : 0));
+  const unsigned long long pos = (unsigned long long)(unsigned)(t + (p.pos ? p.pos[b] : 0));
   constexpr int kHalfLanes = D / 16;
   const int j0 = (lane_in_row % kHalfLanes) * 8;  // first pair index of this lane
-  constexpr double kTwoPi = 6.283185307179586476925286766559;
-  constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
-    const double phi = pos * omega[j0 + u];
-    const double red = fma(-rint(phi * kInvTwoPi), kTwoPi, phi);
-    sincosf((float)red, &s[u], &c[u]);
+    const unsigned long long frac = pos * turns[j0 + u];
+    const float ang = (float)(int)(unsigned)(frac >> 32) * 1.4629180792671596e-09f;  // 2 pi / 2^32
+    __sincosf(ang, &s[u], &c[u]);
   }
 }
 
@@ -64,9 +67,12 @@ __global__ void __launch_bounds__(256) rope_qknorm_kernel(const RopeParams p) {
   const long long r = active ? (seg ? row - p.rows[0] : row) : 0;
   const bool second_half = lr >= kLanesPerRow / 2;
 
-  // omega_j = base^(-2j/D), one fp64 table per block
-  __shared__ double omega[D / 2];
-  for (int j = threadIdx.x; j < D / 2; j += blockDim.x) omega[j] = exp2(-2.0 * (double)j / (double)D * p.log2_base);
+  // U_j = (base^(-2j/D) / (2 pi)) * 2^64, one table per block
+  __shared__ unsigned long long turns[D / 2];
+  for (int j = threadIdx.x; j < D / 2; j += blockDim.x) {
+    const double u = exp2(-2.0 * (double)j / (double)D * p.log2_base) * 0.15915494309189533576888376337251;
+    turns[j] = (unsigned long long)(u * 18446744073709551616.0);
+  }
   __syncthreads();
 
   float x[8], g[8];
@@ -102,7 +108,7 @@ __global__ void __launch_bounds__(256) rope_qknorm_kernel(const RopeParams p) {
 
   float c[8], s[8];
   if (active) {
-    rope_row_angles<D>(p, omega, seg, r, lr, c, s);
+    rope_row_angles<D>(p, turns, seg, r, lr, c, s);
   } else {
 #pragma unroll
     for (int u = 0; u < 8; ++u) c[u] = 1.f, s[u] = 0.f;

@@ -1,0 +1,97 @@
+"""GPU parity at the full workload sizes, in the launch configuration bench.py times.
+
+The oracle cannot expand every row at these sizes, so it checks sampled
+outputs it can compute one by one: whole query rows of o / lse / dq (rows at
+tile edges, window edges and the ends, plus random ones) for every batch and
+head, and dk / dv at clusters of keys (every query row that sees them is
+expanded). The prologue and its backward are checked on a batch slice.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests.parity import (EPS, LSE_MAX_ABS, ROPE_BASE, check_bf16, check_grad, check_out, f64, max_abs,
+                          run_block)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def cswa():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import causal_sliding_window_attn_b200 as m
+    m.lib()
+    return m
+
+
+def sample_rows(T, W, seed):
+    fixed = {0, 1, 127, 128, 129, T // 2 - 1, T // 2, T - 129, T - 128, T - 2, T - 1}
+    if W >= 0:
+        fixed |= {W - 1, W, W + 1, W + 127, W + 128}
+    rng = np.random.default_rng(seed)
+    rows = fixed | set(rng.integers(0, T, 16).tolist())
+    return np.array(sorted(r for r in rows if 0 <= r < T))
+
+
+@pytest.mark.parametrize("name,W", [("d20", 1024), ("d20", 2048), ("gqa", 512), ("long", 2048), ("long", -1)])
+def test_fullsize_sampled(cswa, name, W):
+    c = workloads.CONFIGS[name]
+    B, T, Hq, Hkv, D = c["B"], c["T"], c["Hq"], c["Hkv"], c["D"]
+    scale = workloads.default_scale(D)
+    q, k, v, do = workloads.config_inputs(name)
+    g = run_block(cswa, q, k, v, do, W, scale)
+    qh, kh = f64(g["qh"]), f64(g["kh"])
+    vf, dof = f64(v), f64(do)
+
+    rows = sample_rows(T, W, seed=T + W)
+    o_ref, lse_ref = oracle.attention_fwd(qh, kh, vf, W, scale, rows=rows)
+    check_out(f"{name} o rows", f64(g["o"])[:, rows], o_ref)
+    assert max_abs(f64(g["lse"])[:, :, rows], lse_ref) <= LSE_MAX_ABS
+
+    bs = [0, B - 1] if B > 1 else [0]
+    dq_ref = oracle.attention_bwd_rows(qh[bs], kh[bs], vf[bs], dof[bs], W, scale, rows)
+    check_grad(f"{name} dq_hat rows", f64(g["dqh"])[bs][:, rows], dq_ref)
+
+    clusters = [np.arange(T - 12, T)]
+    clusters.append(np.arange(100, 104) if W >= 0 else np.arange(T - 300, T - 296))
+    for keys in clusters:
+        dk_ref, dv_ref = oracle.attention_bwd_keys(qh[:1], kh[:1], vf[:1], dof[:1], W, scale, keys)
+        check_grad(f"{name} dk_hat keys {keys[0]}..", f64(g["dkh"])[:1, keys], dk_ref)
+        check_grad(f"{name} dv keys {keys[0]}..", f64(g["dv"])[:1, keys], dv_ref)
+
+    # prologue forward and backward on one batch row
+    pos = oracle.row_positions(1, T)
+    check_bf16("q_hat", qh[:1], oracle.prologue(f64(q[:1]), pos, ROPE_BASE, EPS))
+    check_bf16("k_hat", kh[:1], oracle.prologue(f64(k[:1]), pos, ROPE_BASE, EPS))
+    check_grad("dq (prologue bwd)", f64(g["dq"][:1]), oracle.prologue_bwd(f64(q[:1]), f64(g["dqh"][:1]), pos,
+                                                                           ROPE_BASE, EPS))
+    check_grad("dk (prologue bwd)", f64(g["dk"][:1]), oracle.prologue_bwd(f64(k[:1]), f64(g["dkh"][:1]), pos,
+                                                                           ROPE_BASE, EPS))
+
+
+def test_fullsize_decode(cswa):
+    c = workloads.DECODE
+    B, Hq, Hkv, D, Tmax, W = c["B"], c["Hq"], c["Hkv"], c["D"], c["Tmax"], c["window"]
+    lengths, kraw, vc, qraw, knraw, vn = workloads.decode_inputs(**c)
+    kraw, vc, qraw, knraw, vn = (t.cuda() for t in (kraw, vc, qraw, knraw, vn))
+    pos = lengths.cuda()
+    _, kc = cswa.attn_rope_qknorm(None, kraw)
+    qd, kn = cswa.attn_rope_qknorm(qraw, knraw, pos=pos)
+    kc0, vc0 = kc.clone(), vc.clone()
+    o, lse = cswa.attn_decode(qd, kc, vc, pos, W, k_new=kn, v_new=vn)
+    torch.cuda.synchronize()
+    assert cswa.attn_get_status() == 0
+    o_ref, lse_ref, _, _ = oracle.decode(f64(qd), f64(kc0), f64(vc0), lengths.numpy(), W,
+                                         workloads.default_scale(D), k_new=f64(kn), v_new=f64(vn))
+    check_out("decode o", f64(o), o_ref)
+    assert max_abs(f64(lse), lse_ref) <= LSE_MAX_ABS
+    # end-to-end: the oracle's own prologue of the raw cache and query
+    L = lengths.numpy()
+    kc_e2e = oracle.prologue(f64(kraw), oracle.row_positions(B, Tmax), ROPE_BASE, EPS)
+    q_e2e = oracle.prologue(f64(qraw), oracle.row_positions(B, 1, L), ROPE_BASE, EPS)
+    kn_e2e = oracle.prologue(f64(knraw), oracle.row_positions(B, 1, L), ROPE_BASE, EPS)
+    o_e2e, _, _, _ = oracle.decode(q_e2e, kc_e2e, f64(vc0), L, W, workloads.default_scale(D), k_new=kn_e2e,
+                                   v_new=f64(vn))
+    check_out("decode o (end-to-end)", f64(o), o_e2e, max_abs_tol=2e-2)
