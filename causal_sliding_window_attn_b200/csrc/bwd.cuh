@@ -14,20 +14,23 @@
 //                rows get P = 0), and zeroes the fp32 dQ accumulator.
 //   bwd_main     one CTA per (128-key tile, KV head, batch). K and V stay in
 //                shared memory; the CTA walks every (query head of the group,
-//                128-row query tile) that sees the key tile. Per step:
-//                  S^T  = K Q^T        (SS)   -> TMEM cols [0,128)
-//                  dP^T = V dO^T       (SS)   -> TMEM cols [128,256)
-//                  P^T  = exp2(S^T*c - lse)   written back as bf16 into [0,64)
-//                  dV  += P^T dO       (TS)   -> TMEM (persistent)
-//                  dS^T = P^T (dP^T - Delta)  bf16 into shared memory
-//                  dK  += dS^T Q       (SS)   -> TMEM (persistent)
-//                  dQ   = dS K         (SS, dS read MN-major) -> TMEM [128,128+D)
-//                and dQ is added to the fp32 accumulator with vector atomics.
-//                dK, dV are complete in the CTA (the whole group is walked here),
-//                so they are written once, as bf16, with no atomics.
-//   bwd_dq_cast  the fp32 dQ accumulator -> bf16 dq.
+//                64-row query sub-tile) that sees the key tile. Per step:
+//                  S^T  = K Q^T         (SS)  -> TMEM [0,64)
+//                  dP^T = V dO^T        (SS)  -> TMEM [64,128)
+//                  P^T  = exp2(S^T c - lse)     bf16 back into TMEM [0,32)
+//                  dV  += P^T dO        (TS)  -> TMEM [128,128+D)
+//                  dS^T = P^T (dP^T - Delta)    bf16 into shared memory
+//                  dK  += dS^T Q        (SS)  -> TMEM [128+D,128+2D)
+//                  dQ^T = K^T dS^T      (SS, both MN-major) -> TMEM [384,448) or [448,512)
+//                dQ^T is double-buffered in TMEM; a drain warpgroup moves it
+//                to a shared-memory staging tile and adds it to the fp32
+//                accumulator with one TMA reduce-add per step, off the
+//                critical path of the tensor pipe.
+//                dK, dV are complete in the CTA (the whole group is walked
+//                here), so they are written once, as bf16, with no atomics.
+//   bwd_dq_cast  the fp32 dQ accumulator (B, Hq, Tpad, D) -> bf16 dq (B, T, Hq, D).
 // Warp roles in bwd_main: 0 TMA, 1 MMA issuer, 2 TMEM allocator,
-// 4-7 P/dS (thread = key row), 8-11 dQ drain (thread = query row).
+// 4-7 P/dS + dK epilogue (thread = key row), 8-11 dQ drain + dV epilogue.
 #pragma once
 #include "ptx.cuh"
 
@@ -36,10 +39,9 @@ namespace cswa {
 struct BwdParams {
   const float* lse2;   // (B, Hq, Tpad): lse * log2(e), +inf on padded rows
   const float* delta;  // (B, Hq, Tpad)
-  float* dq_acc;       // (B, T, Hq, D)
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
-  int T, Tpad, Hq, G, window, n_tiles;
+  int T, Tpad, Hq, G, window, n_kv_tiles, n_q_tiles;  // q tiles of 64 rows
   float scale, scale_log2;
 };
 
@@ -50,16 +52,43 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+// 2-D tiled reduce-add shared -> global (fp32 add in L2), bulk-group completion.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* m, const void* src, int c0, int c1) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void named_barrier_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 
 template <int D>
 struct BwdLayout {
-  static constexpr int kTile = 128 * D * 2;
-  static constexpr int kPanels = D / 64;
-  static constexpr int kK = 0, kV = kTile, kQ = 2 * kTile, kDO = 4 * kTile, kDS = 6 * kTile;
-  static constexpr int kStat = kDS + 32768;  // lse2[2][128], delta[2][128]
-  static constexpr int kBar = kStat + 2048;
+  static constexpr int kKV = 128 * D * 2;       // K or V tile: 128 rows
+  static constexpr int kQT = 64 * D * 2;        // Q or dO tile: 64 rows
+  static constexpr int kPanelKV = 128 * 128;    // one 64-column panel of a 128-row tile
+  static constexpr int kPanelQ = 64 * 128;      // one 64-column panel of a 64-row tile
+  static constexpr int kK = 0;
+  static constexpr int kZero = kK + kKV;        // D = 64: zero panel after K (pads K^T to M = 128)
+  static constexpr int kV = kZero + (D == 64 ? kPanelKV : 0);
+  static constexpr int kQ = kV + kKV;           // [2]
+  static constexpr int kDO = kQ + 2 * kQT;      // [2]
+  static constexpr int kDS = kDO + 2 * kQT;     // dS^T: 128 keys x 64 queries bf16 = 16 KB
+  static constexpr int kStage = kDS + 16384;    // dQ staging [2]: 64 x D fp32
+  static constexpr int kStageBytes = 64 * D * 4;
+  static constexpr int kStat = kStage + 2 * kStageBytes;  // lse2[2][64], delta[2][64]
+  static constexpr int kBar = kStat + 1024;
   static constexpr int kUsed = kBar + 256;
-  static constexpr int kBytes = (kUsed + 1024 <= 232448) ? kUsed + 1024 : 232448;
+  static constexpr int kBytes = kUsed + 1024;
+  static_assert(kBytes <= 232448, "shared memory budget");
   static constexpr uint32_t kTmemCols = 512;
 };
 
@@ -67,16 +96,10 @@ template <int D>
 __global__ void __launch_bounds__(384, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const BwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using L = BwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  // The layout needs a 1024-byte aligned base; report (never corrupt) if the
-  // runtime placed dynamic shared memory so that the aligned layout overflows.
-  if ((smem - smem_raw) + L::kUsed > L::kBytes) {
-    if (threadIdx.x == 0) atomicOr(&g_status, kStatusLayout);
-    return;
-  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* kv_full = bars + 0;
   uint64_t* qd_full = bars + 1;   // [2]
@@ -86,35 +109,41 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* p_full = bars + 7;
   uint64_t* ds_full = bars + 8;
   uint64_t* dv_done = bars + 9;
-  uint64_t* dq_full = bars + 10;
-  uint64_t* dq_free = bars + 11;
-  uint64_t* final_bar = bars + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 14);
-  float* s_lse = reinterpret_cast<float*>(smem + L::kStat);          // [2][128]
-  float* s_delta = reinterpret_cast<float*>(smem + L::kStat + 1024);  // [2][128]
+  uint64_t* dq_full = bars + 10;  // [2]
+  uint64_t* dq_free = bars + 12;  // [2]
+  uint64_t* final_bar = bars + 14;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 16);
+  float* s_lse = reinterpret_cast<float*>(smem + L::kStat);         // [2][64]
+  float* s_delta = reinterpret_cast<float*>(smem + L::kStat + 512);  // [2][64]
 
   const int warp = warp_id(), lane = lane_id();
   const int hk = blockIdx.x, b = blockIdx.y, n = blockIdx.z;
   const int W = p.window, G = p.G;
   const int k0 = n * 128;
-  const int m_hi = (W < 0) ? p.n_tiles - 1 : min(p.n_tiles - 1, (k0 + 127 + W) / 128);
-  const int m_cnt = m_hi - n + 1;
+  const int m_lo = 2 * n;
+  const int m_hi = (W < 0) ? p.n_q_tiles - 1 : min(p.n_q_tiles - 1, (k0 + 127 + W) / 64);
+  const int m_cnt = m_hi - m_lo + 1;
   const int n_iters = G * m_cnt;
 
+  if (D == 64) {
+    for (int i = threadIdx.x; i < L::kPanelKV / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(smem + L::kZero)[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
   if (warp == 0 && lane == 0) {
     mbar_init(kv_full, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&qd_full[s], 1);
       mbar_init(&qd_empty[s], 1);
+      mbar_init(&dq_full[s], 1);
+      mbar_init(&dq_free[s], 128);
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
     mbar_init(p_full, 128);
     mbar_init(ds_full, 128);
     mbar_init(dv_done, 1);
-    mbar_init(dq_full, 1);
-    mbar_init(dq_free, 128);
     mbar_init(final_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -127,10 +156,14 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 128, tdV = tmem + 256, tdK = tmem + 256 + D;
+  const uint32_t tS = tmem, tdP = tmem + 64, tdV = tmem + 128, tdK = tmem + 128 + D;
+  const uint32_t tdQ[2] = {tmem + 384, tmem + 448};
 
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sK = sbase + L::kK, sV = sbase + L::kV, sDS = sbase + L::kDS;
+
+  auto iter_head = [&](int it) { return hk * G + it / m_cnt; };
+  auto iter_q0 = [&](int it) { return (m_lo + it % m_cnt) * 64; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -139,26 +172,24 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
-      mbar_arrive_expect_tx(kv_full, 2 * L::kTile);
-      for (int pn = 0; pn < L::kPanels; ++pn) {
-        tma_load_4d(smem + L::kK + pn * 16384, &tm_k, kv_full, pn * 64, hk, k0, b);
-        tma_load_4d(smem + L::kV + pn * 16384, &tm_v, kv_full, pn * 64, hk, k0, b);
+      mbar_arrive_expect_tx(kv_full, 2 * L::kKV);
+      for (int pn = 0; pn < D / 64; ++pn) {
+        tma_load_4d(smem + L::kK + pn * L::kPanelKV, &tm_k, kv_full, pn * 64, hk, k0, b);
+        tma_load_4d(smem + L::kV + pn * L::kPanelKV, &tm_v, kv_full, pn * 64, hk, k0, b);
       }
       int last_issue[2] = {-1, -1};
       for (int it = 0; it < n_iters; ++it) {
         const int st = it & 1;
-        const int g = it / m_cnt, m = n + it % m_cnt;
-        const int h = hk * G + g;
+        const int h = iter_head(it), q0 = iter_q0(it);
         if (!mbar_wait(&qd_empty[st], ((it >> 1) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&qd_full[st], 2 * L::kTile + 1024);
-        for (int pn = 0; pn < L::kPanels; ++pn) {
-          tma_load_4d(smem + L::kQ + st * L::kTile + pn * 16384, &tm_q, &qd_full[st], pn * 64, h, m * 128, b);
-          tma_load_4d(smem + L::kDO + st * L::kTile + pn * 16384, &tm_do, &qd_full[st], pn * 64, h, m * 128,
-                      b);
+        mbar_arrive_expect_tx(&qd_full[st], 2 * L::kQT + 512);
+        for (int pn = 0; pn < D / 64; ++pn) {
+          tma_load_4d(smem + L::kQ + st * L::kQT + pn * L::kPanelQ, &tm_q, &qd_full[st], pn * 64, h, q0, b);
+          tma_load_4d(smem + L::kDO + st * L::kQT + pn * L::kPanelQ, &tm_do, &qd_full[st], pn * 64, h, q0, b);
         }
-        const size_t row0 = ((size_t)b * p.Hq + h) * p.Tpad + (size_t)m * 128;
-        bulk_load(s_lse + st * 128, p.lse2 + row0, 512, &qd_full[st]);
-        bulk_load(s_delta + st * 128, p.delta + row0, 512, &qd_full[st]);
+        const size_t row0 = ((size_t)b * p.Hq + h) * p.Tpad + q0;
+        bulk_load(s_lse + st * 64, p.lse2 + row0, 256, &qd_full[st]);
+        bulk_load(s_delta + st * 64, p.delta + row0, 256, &qd_full[st]);
         last_issue[st] = it;
       }
       if (*abort_flag) {
@@ -171,50 +202,63 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idSP = idesc_bf16(128, 128, false, false);  // S^T, dP^T
-      constexpr uint32_t idKV = idesc_bf16(128, D, false, true);     // dV (TS), dK: B MN-major
-      constexpr uint32_t idQ = idesc_bf16(128, D, true, true);       // dQ: A and B MN-major
-      bool ok = mbar_wait(kv_full, 0, abort_flag);
+      constexpr uint32_t idSP = idesc_bf16(128, 64, false, false);  // S^T, dP^T
+      constexpr uint32_t idKV = idesc_bf16(128, D, false, true);    // dV (TS), dK: B MN-major
+      constexpr uint32_t idQ = idesc_bf16(128, 64, true, true);     // dQ^T: A, B MN-major
+      auto issue_S = [&](int st) {
+        const uint32_t sQ = sbase + L::kQ + st * L::kQT;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tS, sdesc_sw128(sK + (kk >> 2) * L::kPanelKV + (kk & 3) * 32, 16, 1024),
+                 sdesc_sw128(sQ + (kk >> 2) * L::kPanelQ + (kk & 3) * 32, 16, 1024), idSP, kk > 0);
+        mma_commit(s_full);
+      };
+      auto issue_dP = [&](int st) {
+        const uint32_t sDO = sbase + L::kDO + st * L::kQT;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tdP, sdesc_sw128(sV + (kk >> 2) * L::kPanelKV + (kk & 3) * 32, 16, 1024),
+                 sdesc_sw128(sDO + (kk >> 2) * L::kPanelQ + (kk & 3) * 32, 16, 1024), idSP, kk > 0);
+        mma_commit(dp_full);
+      };
+      bool ok = mbar_wait(kv_full, 0, abort_flag) && mbar_wait(&qd_full[0], 0, abort_flag);
+      tc_fence_after();
+      if (ok && n_iters > 0) {
+        issue_S(0);
+        issue_dP(0);
+      }
       for (int it = 0; ok && it < n_iters; ++it) {
         const int st = it & 1;
-        const uint32_t sQ = sbase + L::kQ + st * L::kTile, sDO = sbase + L::kDO + st * L::kTile;
-        if (!(ok = mbar_wait(&qd_full[st], (it >> 1) & 1, abort_flag))) break;
-        if (it > 0 && !(ok = mbar_wait(dv_done, (it - 1) & 1, abort_flag))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), idSP, kk > 0);
-        }
-        mma_commit(s_full);
-        if (it > 0 && !(ok = mbar_wait(dq_free, (it - 1) & 1, abort_flag))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tdP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sDO + off, 16, 1024), idSP, kk > 0);
-        }
-        mma_commit(dp_full);
+        const uint32_t sQ = sbase + L::kQ + st * L::kQT, sDO = sbase + L::kDO + st * L::kQT;
         if (!(ok = mbar_wait(p_full, it & 1, abort_flag))) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tdV, tS + kk * 8, sdesc_sw128(sDO + kk * 2048, 16384, 1024), idKV, (it > 0 || kk > 0));
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tdV, tS + kk * 8, sdesc_sw128(sDO + kk * 2048, L::kPanelQ, 1024), idKV, (it > 0 || kk > 0));
         mma_commit(dv_done);
+        if (it + 1 < n_iters) {
+          // S^T of the next step overwrites P^T: wait until dV has read it
+          if (!(ok = mbar_wait(&qd_full[st ^ 1], ((it + 1) >> 1) & 1, abort_flag))) break;
+          if (!(ok = mbar_wait(dv_done, it & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_S(st ^ 1);
+        }
         if (!(ok = mbar_wait(ds_full, it & 1, abort_flag))) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tdK, sdesc_sw128(sDS + off, 16, 1024), sdesc_sw128(sQ + kk * 2048, 16384, 1024), idKV,
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(tdK, sdesc_sw128(sDS + kk * 32, 16, 1024), sdesc_sw128(sQ + kk * 2048, L::kPanelQ, 1024), idKV,
                  (it > 0 || kk > 0));
-        }
+        if (it >= 2 && !(ok = mbar_wait(&dq_free[st], ((it - 2) >> 1) & 1, abort_flag))) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tdQ, sdesc_sw128(sDS + kk * 2048, 16384, 1024), sdesc_sw128(sK + kk * 2048, 16384, 1024), idQ,
-                 kk > 0);
-        mma_commit(dq_full);
+          mma_ss(tdQ[st], sdesc_sw128(sK + kk * 2048, L::kPanelKV, 1024), sdesc_sw128(sDS + kk * 2048, 16, 1024),
+                 idQ, kk > 0);
+        mma_commit(&dq_full[st]);
         mma_commit(&qd_empty[st]);
+        // dP^T of the next step: the P/dS warps read this step's dP^T before ds_full
+        if (it + 1 < n_iters) issue_dP(st ^ 1);
       }
       mma_commit(final_bar);
       volatile int dummy = 0;
@@ -231,61 +275,57 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
     for (int it = 0; it < n_iters; ++it) {
       const int st = it & 1;
-      const int q0 = (n + it % m_cnt) * 128;
-      const float* lse_s = s_lse + st * 128;
-      const float* dl_s = s_delta + st * 128;
+      const int q0 = iter_q0(it);
+      const float* lse_s = s_lse + st * 64;
+      const float* dl_s = s_delta + st * 64;
       ok = __all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[128];
+      uint32_t sr[64];
       tmem_ld32(tS + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
       tmem_ld32(tS + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld32(tS + lane_off + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-      tmem_ld32(tS + lane_off + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
       tmem_ld_wait();
-      const bool full = (k0 + 127 <= q0) && (W < 0 || q0 + 127 - k0 <= W);
+      const bool full = (k0 + 127 <= q0) && (W < 0 || q0 + 63 - k0 <= W);
+      const int c_lo = j - q0;                       // query q0 + c sees key j iff c >= c_lo
+      const int c_hi = (W < 0) ? 63 : j + W - q0;    //   and c <= c_hi
       // P^T row in place as packed bf16 pairs; the same bf16 P feeds dV (TMEM) and dS
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const int i = q0 + 2 * c;
-        const bool v0 = full || ((j <= i) && (W < 0 || i - j <= W));
-        const bool v1 = full || ((j <= i + 1) && (W < 0 || i + 1 - j <= W));
-        const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(sr[2 * c]), sl2, -lse_s[2 * c])) : 0.f;
-        const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -lse_s[2 * c + 1])) : 0.f;
+      for (int c = 0; c < 32; ++c) {
+        const int c0 = 2 * c, c1 = 2 * c + 1;
+        const bool v0 = full || (c0 >= c_lo && c0 <= c_hi);
+        const bool v1 = full || (c1 >= c_lo && c1 <= c_hi);
+        const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(sr[c0]), sl2, -lse_s[c0])) : 0.f;
+        const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(sr[c1]), sl2, -lse_s[c1])) : 0.f;
         sr[c] = pack_bf16x2(p0, p1);
       }
-      tmem_st32(tS + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_st32(tS + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_st32(tS + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full);
 
       ok = __all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, abort_flag));
-      if (ok && it > 0) ok = __all_sync(0xffffffffu, mbar_wait(dq_full, (it - 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
+      uint32_t dp[64];
+      tmem_ld32(tdP + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+      tmem_ld32(tdP + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+      tmem_ld_wait();
+      // dS^T of the previous step must have been consumed by dK and dQ
+      if (it > 0) ok = __all_sync(0xffffffffu, mbar_wait(&dq_full[st ^ 1], ((it - 1) >> 1) & 1, abort_flag));
+      if (!ok) break;
+      uint32_t w[32];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t dp[32];
-        tmem_ld32(tdP + lane_off + cc * 32, dp);
-        tmem_ld_wait();
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c0 = cc * 32 + 2 * e;
-          const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sr[cc * 16 + e]));
-          const float d0 = pp.x * (__uint_as_float(dp[2 * e]) - dl_s[c0]);
-          const float d1 = pp.y * (__uint_as_float(dp[2 * e + 1]) - dl_s[c0 + 1]);
-          w[e] = pack_bf16x2(d0, d1);
-        }
-        // queries cc*32 .. cc*32+31 = 4 16-byte chunks of panel cc/2, chunks (cc&1)*4 ..
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const uint32_t chunk = (cc & 1) * 4 + u;
-          uint4* dst = reinterpret_cast<uint4*>(ds_row + (cc >> 1) * 16384 + ((chunk ^ (r & 7)) << 4));
-          *dst = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-        }
+      for (int e = 0; e < 32; ++e) {
+        const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sr[e]));
+        const float d0 = pp.x * (__uint_as_float(dp[2 * e]) - dl_s[2 * e]);
+        const float d1 = pp.y * (__uint_as_float(dp[2 * e + 1]) - dl_s[2 * e + 1]);
+        w[e] = pack_bf16x2(d0, d1);
       }
+      // row r of the dS^T panel: 8 chunks of 16 bytes, 128-byte swizzle
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        *reinterpret_cast<uint4*>(ds_row + ((u ^ (r & 7)) << 4)) =
+            make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(ds_full);
@@ -312,41 +352,45 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
   } else if (warp >= 8) {
-    // ------------------------------------------------------------ dQ drain (thread = query row)
+    // ------------------------------------------------------------ dQ drain (thread = head-dim index)
     const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;
+    const int dd = quarter * 32 + lane;  // d index of this thread's TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const bool leader = (warp == 8 && lane == 0);
     bool ok = true;
     for (int it = 0; it < n_iters; ++it) {
-      const int g = it / m_cnt;
-      const int i = (n + it % m_cnt) * 128 + row;
-      const int h = hk * G + g;
-      ok = __all_sync(0xffffffffu, mbar_wait(dq_full, it & 1, abort_flag));
+      const int st = it & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&dq_full[st], (it >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      float* dst = p.dq_acc + ((size_t)((size_t)b * p.T + i) * p.Hq + h) * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tdQ + lane_off + c * 32, o);
-        tmem_ld_wait();
-        if (i < p.T) {
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            float4 v = make_float4(__uint_as_float(o[4 * u]) * p.scale, __uint_as_float(o[4 * u + 1]) * p.scale,
-                                   __uint_as_float(o[4 * u + 2]) * p.scale, __uint_as_float(o[4 * u + 3]) * p.scale);
-            atomicAdd(reinterpret_cast<float4*>(dst + c * 32 + 4 * u), v);
-          }
-        }
-      }
+      uint32_t v[64];
+      tmem_ld32(tdQ[st] + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_ld32(tdQ[st] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(dq_free);
+      mbar_arrive(&dq_free[st]);
+      // the reduce that last read this staging buffer (two steps ago) must be done reading
+      if (leader) bulk_wait_read<1>();
+      named_barrier_sync(1, 128);
+      float* stage = reinterpret_cast<float*>(smem + L::kStage + st * L::kStageBytes);
+      if (dd < D) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) stage[c * D + dd] = __uint_as_float(v[c]) * p.scale;
+      }
+      fence_proxy_async_smem();
+      named_barrier_sync(1, 128);
+      if (leader) {
+        const int row = (int)(((size_t)b * p.Hq + iter_head(it)) * p.Tpad + iter_q0(it));
+        tma_reduce_add_2d(&tm_dq, stage, 0, row);
+        bulk_commit();
+      }
     }
+    if (leader) bulk_wait_all();
     // ---------------------------------------------------------- dV epilogue (thread = key row)
     ok = __all_sync(0xffffffffu, ok && mbar_wait(final_bar, 0, abort_flag));
     tc_fence_after();
     if (ok) {
-      const int j = k0 + row;
+      const int j = k0 + dd;
       __nv_bfloat16* dst = p.dv + ((size_t)((size_t)b * p.T + j) * (p.Hq / G) + hk) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
@@ -373,7 +417,7 @@ __global__ void __launch_bounds__(384, 1)
 }
 
 // Delta_i = dO_i . o_i and lse_i * log2(e) into the padded (B, Hq, Tpad) workspace
-// arrays, and zeroes the dQ accumulator row: D/8 lanes per (b, t, h) row.
+// arrays, and zeroes the padded dQ accumulator row: D/8 lanes per (b, t, h) row.
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16* o, const __nv_bfloat16* dout,
                                                              const float* lse, float* lse2, float* delta,
@@ -401,7 +445,9 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16*
       const float2 a = __bfloat1622float2(o2[u]), c = __bfloat1622float2(g2[u]);
       dsum = fmaf(a.x, c.x, fmaf(a.y, c.y, dsum));
     }
-    float4* z = reinterpret_cast<float4*>(dq_acc + off);
+  }
+  if (active) {
+    float4* z = reinterpret_cast<float4*>(dq_acc + (((size_t)b * Hq + h) * Tpad + t) * D + lr * 8);
     z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
     z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
@@ -414,11 +460,19 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16*
   }
 }
 
-__global__ void __launch_bounds__(256) attn_bwd_dq_cast_kernel(const float* acc, __nv_bfloat16* dq, long long n8) {
+// dq (B, T, Hq, D) bf16 <- dq_acc (B, Hq, Tpad, D) fp32; one thread per 8 values.
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_dq_cast_kernel(const float* acc, __nv_bfloat16* dq, int T, int Tpad,
+                                                                int Hq, long long n8) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n8) return;
-  const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
-  const float4 c = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+  const int d8 = (int)(i % (D / 8));
+  const long long row = i / (D / 8);  // (b, t, h) of the output
+  const int h = (int)(row % Hq);
+  const long long bt = row / Hq;
+  const int t = (int)(bt % T), b = (int)(bt / T);
+  const float4* src = reinterpret_cast<const float4*>(acc + (((size_t)b * Hq + h) * Tpad + t) * D + d8 * 8);
+  const float4 a = src[0], c = src[1];
   reinterpret_cast<uint4*>(dq)[i] =
       make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(c.x, c.y), pack_bf16x2(c.z, c.w));
 }

@@ -36,17 +36,31 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// BTHD bf16 tensor as a 4-D tensor map (D, H, T, B); box = 64 x 1 x 128 x 1
-// (one 128-row, 128-byte-wide panel), 128-byte swizzle, zero fill past T.
-bool encode_bthd(CUtensorMap* m, const void* base, int B, int T, int H, int D) {
+// BTHD bf16 tensor as a 4-D tensor map (D, H, T, B); box = 64 x 1 x rows x 1
+// (one rows-high, 128-byte-wide panel), 128-byte swizzle, zero fill past T.
+bool encode_bthd(CUtensorMap* m, const void* base, int B, int T, int H, int D, int rows = 128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
   const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
-  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Row-major fp32 matrix (rows, cols) as a 2-D tensor map with a (64 x cols) box,
+// no swizzle: the dQ accumulator, target of TMA reduce-adds.
+bool encode_f32_rows(CUtensorMap* m, const void* base, long long rows, int cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+  const cuuint32_t box[2] = {(cuuint32_t)cols, 64};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -76,10 +90,8 @@ bool set_smem_attrs() {
 }
 
 template <int D, bool kBwd>
-attn_status_t launch_rope(const RopeParams& p, cudaStream_t st) {
-  const long long rows = p.rows[0] + p.rows[1];
-  constexpr int kRowsPerBlock = 256 / (D / 8);
-  const long long blocks = (rows + kRowsPerBlock - 1) / kRowsPerBlock;
+attn_status_t launch_rope(const RopeParams& p, long long n_pos, cudaStream_t st) {
+  const long long blocks = (n_pos + kPosPerBlock - 1) / kPosPerBlock;
   if (blocks > 0x7fffffffll) return ATTN_ERR_INVALID_ARG;
   rope_qknorm_kernel<D, kBwd><<<(unsigned)blocks, 256, 0, st>>>(p);
   return launched();
@@ -113,8 +125,9 @@ attn_status_t rope_common(const void* x0, const void* x1, const void* dy0, const
   p.eps = eps;
   p.log2_base = std::log2((double)base);
   cudaStream_t st = as_stream(stream);
-  if (D == 64) return bwd ? launch_rope<64, true>(p, st) : launch_rope<64, false>(p, st);
-  return bwd ? launch_rope<128, true>(p, st) : launch_rope<128, false>(p, st);
+  const long long n_pos = (long long)B * T;
+  if (D == 64) return bwd ? launch_rope<64, true>(p, n_pos, st) : launch_rope<64, false>(p, n_pos, st);
+  return bwd ? launch_rope<128, true>(p, n_pos, st) : launch_rope<128, false>(p, n_pos, st);
 }
 
 template <int D>
@@ -140,16 +153,16 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, f
 }
 
 struct BwdWorkspace {
-  float* dq_acc;
-  float* lse2;
-  float* delta;
+  float* dq_acc;  // (B, Hq, Tpad, D)
+  float* lse2;    // (B, Hq, Tpad)
+  float* delta;   // (B, Hq, Tpad)
 };
 BwdWorkspace carve_bwd(void* ws, int B, int T, int Hq, int D) {
-  const int Tpad = tiles128(T) * 128;
+  const size_t Tpad = (size_t)tiles128(T) * 128;
   uint8_t* p = static_cast<uint8_t*>(ws);
   BwdWorkspace w;
   w.dq_acc = reinterpret_cast<float*>(p);
-  p += align256((size_t)B * T * Hq * D * 4);
+  p += align256((size_t)B * Hq * Tpad * D * 4);
   w.lse2 = reinterpret_cast<float*>(p);
   p += align256((size_t)B * Hq * Tpad * 4);
   w.delta = reinterpret_cast<float*>(p);
@@ -160,13 +173,14 @@ template <int D>
 attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                          const float* lse, void* dq, void* dk, void* dv, void* ws, int B, int T, int Hq, int Hkv,
                          int window, float scale, cudaStream_t st) {
-  CUtensorMap tq, tk, tv, tdo;
-  if (!encode_bthd(&tq, q, B, T, Hq, D) || !encode_bthd(&tk, k, B, T, Hkv, D) ||
-      !encode_bthd(&tv, v, B, T, Hkv, D) || !encode_bthd(&tdo, dO, B, T, Hq, D))
-    return ATTN_ERR_LAUNCH;
-  if (!set_smem_attrs<D>()) return ATTN_ERR_LAUNCH;
   const int Tpad = tiles128(T) * 128;
   BwdWorkspace w = carve_bwd(ws, B, T, Hq, D);
+  CUtensorMap tq, tk, tv, tdo, tdq;
+  if (!encode_bthd(&tq, q, B, T, Hq, D, 64) || !encode_bthd(&tk, k, B, T, Hkv, D) ||
+      !encode_bthd(&tv, v, B, T, Hkv, D) || !encode_bthd(&tdo, dO, B, T, Hq, D, 64) ||
+      !encode_f32_rows(&tdq, w.dq_acc, (long long)B * Hq * Tpad, D))
+    return ATTN_ERR_LAUNCH;
+  if (!set_smem_attrs<D>()) return ATTN_ERR_LAUNCH;
   {
     const long long threads = (long long)B * Tpad * Hq * (D / 8);
     attn_bwd_prep_kernel<D><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
@@ -177,7 +191,6 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
   BwdParams p{};
   p.lse2 = w.lse2;
   p.delta = w.delta;
-  p.dq_acc = w.dq_acc;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.T = T;
@@ -185,15 +198,16 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
   p.Hq = Hq;
   p.G = Hq / Hkv;
   p.window = (window >= T) ? -1 : window;
-  p.n_tiles = tiles128(T);
+  p.n_kv_tiles = tiles128(T);
+  p.n_q_tiles = (T + 63) / 64;
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
-  dim3 grid(Hkv, B, p.n_tiles);
-  attn_bwd_kernel<D><<<grid, 384, BwdLayout<D>::kBytes, st>>>(tq, tk, tv, tdo, p);
+  dim3 grid(Hkv, B, p.n_kv_tiles);
+  attn_bwd_kernel<D><<<grid, 384, BwdLayout<D>::kBytes, st>>>(tq, tk, tv, tdo, tdq, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
   const long long n8 = (long long)B * T * Hq * D / 8;
-  attn_bwd_dq_cast_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(w.dq_acc, static_cast<__nv_bfloat16*>(dq),
-                                                                       n8);
+  attn_bwd_dq_cast_kernel<D><<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(
+      w.dq_acc, static_cast<__nv_bfloat16*>(dq), T, Tpad, Hq, n8);
   return launched();
 }
 
@@ -243,7 +257,7 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
 size_t attn_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D) {
   if (!dims_ok(B, T, Hq, Hkv) || (D != 64 && D != 128)) return 0;
   const size_t Tpad = (size_t)tiles128(T) * 128;
-  return align256((size_t)B * T * Hq * D * 4) + 2 * align256((size_t)B * Hq * Tpad * 4);
+  return align256((size_t)B * Hq * Tpad * D * 4) + 2 * align256((size_t)B * Hq * Tpad * 4);
 }
 
 attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,

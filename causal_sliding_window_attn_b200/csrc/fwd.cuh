@@ -221,19 +221,25 @@ __global__ void __launch_bounds__(384, 1)
         tmem_ld_wait();
         const int k0 = t * 128;
         const bool full = (k0 + 127 <= q0) && (W < 0 || q0 + 127 - k0 <= W);
-        float mx = -INFINITY;
+        // 8 independent max chains instead of one 128-long dependent chain
+        float mx8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
         if (full) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(r[c]));
+          for (int c = 0; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(r[c]));
         } else {
+          // visible columns of this row: [c_lo, c_hi] (empty when c_lo > c_hi)
+          const int c_hi = i - k0;
+          const int c_lo = (W < 0) ? -1 : i - W - k0;
 #pragma unroll
           for (int c = 0; c < 128; ++c) {
-            const int j = k0 + c;
-            const bool vis = (j <= i) && (W < 0 || i - j <= W);
-            if (!vis) r[c] = __float_as_uint(-INFINITY);
-            mx = fmaxf(mx, __uint_as_float(r[c]));
+            if (c > c_hi || c < c_lo) r[c] = __float_as_uint(-INFINITY);
+            mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(r[c]));
           }
         }
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float m_tile = mx * sl2;
         bool rescale = false;
         float factor = 1.f;
@@ -246,15 +252,17 @@ __global__ void __launch_bounds__(384, 1)
           rescale = true;
         }
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-        float lsum = 0.f;
+        float ls8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) ls8[u] = 0.f;
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * c]), sl2, -m_use));
           const float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * c + 1]), sl2, -m_use));
-          lsum += p0 + p1;
+          ls8[c & 7] += p0 + p1;
           r[c] = pack_bf16x2(p0, p1);
         }
-        l_run += lsum;
+        l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
         tmem_st32(tS[s] + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
         tmem_st32(tS[s] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
         // rescale only when some row of the warp needs it (O is stable: the MMA

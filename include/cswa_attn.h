@@ -82,8 +82,9 @@ attn_status_t attn_rope_qknorm_bwd(const void* q, const void* k, const void* dq_
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T,
                        int Hq, int Hkv, int D, int window, float scale, void* stream);
 
-/* Bytes of workspace attn_bwd needs: an fp32 dQ accumulator (B,T,Hq,D) and
- * the per-row fp32 dot products Delta_i = dO_i . o_i (B,Hq,T), each 256-byte aligned. */
+/* Bytes of workspace attn_bwd needs: an fp32 dQ accumulator (B,Hq,Tpad,D), the
+ * per-row lse*log2(e) and Delta_i = dO_i . o_i (B,Hq,Tpad), Tpad = T rounded up
+ * to a multiple of 128, each part 256-byte aligned. */
 size_t attn_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D);
 
 /*

@@ -42,12 +42,12 @@ def test_status_strings(L):
 
 def test_bwd_workspace_size(L):
     B, T, Hq, Hkv, D = 8, 2048, 10, 10, 128
-    dq = B * T * Hq * D * 4
+    dq = B * Hq * 2048 * D * 4
     rows = B * Hq * 2048 * 4
     assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D) == dq + 2 * rows
     # ragged T pads the per-row arrays to whole 128-row tiles
     n = L.attn_bwd_workspace_bytes(1, 130, 2, 1, 64)
-    assert n == ((130 * 2 * 64 * 4 + 255) // 256) * 256 + 2 * ((2 * 256 * 4 + 255) // 256) * 256
+    assert n == 2 * 256 * 64 * 4 + 2 * 2 * 256 * 4
     assert L.attn_bwd_workspace_bytes(1, 16, 3, 2, 128) == 0     # Hq % Hkv != 0
     assert L.attn_bwd_workspace_bytes(1, 16, 2, 2, 96) == 0      # head dim
 
