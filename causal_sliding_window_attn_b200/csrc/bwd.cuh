@@ -15,17 +15,18 @@
 //   bwd_main     one CTA per (128-key tile, KV head, batch). K and V stay in
 //                shared memory; the CTA walks every (query head of the group,
 //                64-row query sub-tile) that sees the key tile. Per step:
-//                  S^T  = K Q^T         (SS)  -> TMEM [0,64)
-//                  dP^T = V dO^T        (SS)  -> TMEM [64,128)
-//                  P^T  = exp2(S^T c - lse)     bf16 back into TMEM [0,32)
-//                  dV  += P^T dO        (TS)  -> TMEM [128,128+D)
+//                  S^T  = K Q^T         (SS)  -> TMEM [0,64) / [64,128), alternating
+//                  dP^T = V dO^T        (SS)  -> TMEM [128,192)
+//                  P^T  = exp2(S^T c - lse)     bf16 back over its S^T
+//                  dV  += P^T dO        (TS)  -> TMEM [256,256+D)
 //                  dS^T = P^T (dP^T - Delta)    bf16 into shared memory
-//                  dK  += dS^T Q        (SS)  -> TMEM [128+D,128+2D)
-//                  dQ^T = K^T dS^T      (SS, both MN-major) -> TMEM [384,448) or [448,512)
-//                dQ^T is double-buffered in TMEM; a drain warpgroup moves it
-//                to a shared-memory staging tile and adds it to the fp32
-//                accumulator with one TMA reduce-add per step, off the
-//                critical path of the tensor pipe.
+//                  dK  += dS^T Q        (SS)  -> TMEM [256+D,256+2D)
+//                  dQ^T = K^T dS^T      (SS, both MN-major) -> TMEM [192,256)
+//                S^T/P^T alternate between two TMEM buffers, so the next
+//                step's S^T is issued right behind this step's dV. A drain
+//                warpgroup moves dQ^T to a shared-memory staging tile and adds
+//                it to the fp32 accumulator with one TMA reduce-add per step,
+//                off the critical path of the tensor pipe.
 //                dK, dV are complete in the CTA (the whole group is walked
 //                here), so they are written once, as bf16, with no atomics.
 //   bwd_dq_cast  the fp32 dQ accumulator (B, Hq, Tpad, D) -> bf16 dq (B, T, Hq, D).
@@ -104,16 +105,16 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* kv_full = bars + 0;
   uint64_t* qd_full = bars + 1;   // [2]
   uint64_t* qd_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;
-  uint64_t* dp_full = bars + 6;
-  uint64_t* p_full = bars + 7;
-  uint64_t* ds_full = bars + 8;
-  uint64_t* dv_done = bars + 9;
-  uint64_t* dq_full = bars + 10;  // [2]
-  uint64_t* dq_free = bars + 12;  // [2]
-  uint64_t* final_bar = bars + 14;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 16);
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* p_full = bars + 7;    // [2]
+  uint64_t* dv_done = bars + 9;   // [2]
+  uint64_t* dp_full = bars + 11;
+  uint64_t* ds_full = bars + 12;
+  uint64_t* dq_full = bars + 13;
+  uint64_t* dq_free = bars + 14;
+  uint64_t* final_bar = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 17);
   float* s_lse = reinterpret_cast<float*>(smem + L::kStat);         // [2][64]
   float* s_delta = reinterpret_cast<float*>(smem + L::kStat + 512);  // [2][64]
 
@@ -136,14 +137,14 @@ __global__ void __launch_bounds__(384, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&qd_full[s], 1);
       mbar_init(&qd_empty[s], 1);
-      mbar_init(&dq_full[s], 1);
-      mbar_init(&dq_free[s], 128);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 128);
+      mbar_init(&dv_done[s], 1);
     }
-    mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_full, 128);
     mbar_init(ds_full, 128);
-    mbar_init(dv_done, 1);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, 128);
     mbar_init(final_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -156,8 +157,8 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tdP = tmem + 64, tdV = tmem + 128, tdK = tmem + 128 + D;
-  const uint32_t tdQ[2] = {tmem + 384, tmem + 448};
+  const uint32_t tS[2] = {tmem, tmem + 64};
+  const uint32_t tdP = tmem + 128, tdQ = tmem + 192, tdV = tmem + 256, tdK = tmem + 256 + D;
 
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sK = sbase + L::kK, sV = sbase + L::kV, sDS = sbase + L::kDS;
@@ -205,16 +206,17 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t idSP = idesc_bf16(128, 64, false, false);  // S^T, dP^T
       constexpr uint32_t idKV = idesc_bf16(128, D, false, true);    // dV (TS), dK: B MN-major
       constexpr uint32_t idQ = idesc_bf16(128, 64, true, true);     // dQ^T: A, B MN-major
-      auto issue_S = [&](int st) {
-        const uint32_t sQ = sbase + L::kQ + st * L::kQT;
+      // step it uses Q/dO stage it & 1 and S^T/P^T buffer it & 1
+      auto issue_S = [&](int it) {
+        const uint32_t sQ = sbase + L::kQ + (it & 1) * L::kQT;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tS, sdesc_sw128(sK + (kk >> 2) * L::kPanelKV + (kk & 3) * 32, 16, 1024),
+          mma_ss(tS[it & 1], sdesc_sw128(sK + (kk >> 2) * L::kPanelKV + (kk & 3) * 32, 16, 1024),
                  sdesc_sw128(sQ + (kk >> 2) * L::kPanelQ + (kk & 3) * 32, 16, 1024), idSP, kk > 0);
-        mma_commit(s_full);
+        mma_commit(&s_full[it & 1]);
       };
-      auto issue_dP = [&](int st) {
-        const uint32_t sDO = sbase + L::kDO + st * L::kQT;
+      auto issue_dP = [&](int it) {
+        const uint32_t sDO = sbase + L::kDO + (it & 1) * L::kQT;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tdP, sdesc_sw128(sV + (kk >> 2) * L::kPanelKV + (kk & 3) * 32, 16, 1024),
@@ -230,18 +232,18 @@ __global__ void __launch_bounds__(384, 1)
       for (int it = 0; ok && it < n_iters; ++it) {
         const int st = it & 1;
         const uint32_t sQ = sbase + L::kQ + st * L::kQT, sDO = sbase + L::kDO + st * L::kQT;
-        if (!(ok = mbar_wait(p_full, it & 1, abort_flag))) break;
+        if (!(ok = mbar_wait(&p_full[st], (it >> 1) & 1, abort_flag))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tdV, tS + kk * 8, sdesc_sw128(sDO + kk * 2048, L::kPanelQ, 1024), idKV, (it > 0 || kk > 0));
-        mma_commit(dv_done);
+          mma_ts(tdV, tS[st] + kk * 8, sdesc_sw128(sDO + kk * 2048, L::kPanelQ, 1024), idKV, (it > 0 || kk > 0));
+        mma_commit(&dv_done[st]);
         if (it + 1 < n_iters) {
-          // S^T of the next step overwrites P^T: wait until dV has read it
+          // the other S^T/P^T buffer was last read by dV of step it - 1
           if (!(ok = mbar_wait(&qd_full[st ^ 1], ((it + 1) >> 1) & 1, abort_flag))) break;
-          if (!(ok = mbar_wait(dv_done, it & 1, abort_flag))) break;
+          if (it >= 1 && !(ok = mbar_wait(&dv_done[st ^ 1], ((it - 1) >> 1) & 1, abort_flag))) break;
           tc_fence_after();
-          issue_S(st ^ 1);
+          issue_S(it + 1);
         }
         if (!(ok = mbar_wait(ds_full, it & 1, abort_flag))) break;
         tc_fence_after();
@@ -249,16 +251,17 @@ __global__ void __launch_bounds__(384, 1)
         for (int kk = 0; kk < 4; ++kk)
           mma_ss(tdK, sdesc_sw128(sDS + kk * 32, 16, 1024), sdesc_sw128(sQ + kk * 2048, L::kPanelQ, 1024), idKV,
                  (it > 0 || kk > 0));
-        if (it >= 2 && !(ok = mbar_wait(&dq_free[st], ((it - 2) >> 1) & 1, abort_flag))) break;
+        // dQ^T of the previous step must have left TMEM
+        if (it >= 1 && !(ok = mbar_wait(dq_free, (it - 1) & 1, abort_flag))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tdQ[st], sdesc_sw128(sK + kk * 2048, L::kPanelKV, 1024), sdesc_sw128(sDS + kk * 2048, 16, 1024),
-                 idQ, kk > 0);
-        mma_commit(&dq_full[st]);
+          mma_ss(tdQ, sdesc_sw128(sK + kk * 2048, L::kPanelKV, 1024), sdesc_sw128(sDS + kk * 2048, 16, 1024), idQ,
+                 kk > 0);
+        mma_commit(dq_full);
         mma_commit(&qd_empty[st]);
         // dP^T of the next step: the P/dS warps read this step's dP^T before ds_full
-        if (it + 1 < n_iters) issue_dP(st ^ 1);
+        if (it + 1 < n_iters) issue_dP(it + 1);
       }
       mma_commit(final_bar);
       volatile int dummy = 0;
@@ -278,12 +281,12 @@ __global__ void __launch_bounds__(384, 1)
       const int q0 = iter_q0(it);
       const float* lse_s = s_lse + st * 64;
       const float* dl_s = s_delta + st * 64;
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[st], (it >> 1) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       uint32_t sr[64];
-      tmem_ld32(tS + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tS + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tS[st] + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tS[st] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_ld_wait();
       const bool full = (k0 + 127 <= q0) && (W < 0 || q0 + 63 - k0 <= W);
       const int c_lo = j - q0;                       // query q0 + c sees key j iff c >= c_lo
@@ -298,34 +301,37 @@ __global__ void __launch_bounds__(384, 1)
         const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(sr[c1]), sl2, -lse_s[c1])) : 0.f;
         sr[c] = pack_bf16x2(p0, p1);
       }
-      tmem_st32(tS + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_st32(tS[st] + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[st]);
 
       ok = __all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t dp[64];
-      tmem_ld32(tdP + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-      tmem_ld32(tdP + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
-      tmem_ld_wait();
       // dS^T of the previous step must have been consumed by dK and dQ
-      if (it > 0) ok = __all_sync(0xffffffffu, mbar_wait(&dq_full[st ^ 1], ((it - 1) >> 1) & 1, abort_flag));
+      if (it > 0) ok = __all_sync(0xffffffffu, mbar_wait(dq_full, (it - 1) & 1, abort_flag));
       if (!ok) break;
-      uint32_t w[32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sr[e]));
-        const float d0 = pp.x * (__uint_as_float(dp[2 * e]) - dl_s[2 * e]);
-        const float d1 = pp.y * (__uint_as_float(dp[2 * e + 1]) - dl_s[2 * e + 1]);
-        w[e] = pack_bf16x2(d0, d1);
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t dp[32];
+        tmem_ld32(tdP + lane_off + hf * 32, dp);
+        tmem_ld_wait();
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c0 = hf * 32 + 2 * e;
+          const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sr[hf * 16 + e]));
+          const float d0 = pp.x * (__uint_as_float(dp[2 * e]) - dl_s[c0]);
+          const float d1 = pp.y * (__uint_as_float(dp[2 * e + 1]) - dl_s[c0 + 1]);
+          w[e] = pack_bf16x2(d0, d1);
+        }
+        // row r of the dS^T panel: chunks 4*hf .. 4*hf+3 of 16 bytes, 128-byte swizzle
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          *reinterpret_cast<uint4*>(ds_row + (((4 * hf + u) ^ (r & 7)) << 4)) =
+              make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
       }
-      // row r of the dS^T panel: 8 chunks of 16 bytes, 128-byte swizzle
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        *reinterpret_cast<uint4*>(ds_row + ((u ^ (r & 7)) << 4)) =
-            make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(ds_full);
@@ -360,15 +366,15 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
     for (int it = 0; it < n_iters; ++it) {
       const int st = it & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&dq_full[st], (it >> 1) & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait(dq_full, it & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       uint32_t v[64];
-      tmem_ld32(tdQ[st] + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_ld32(tdQ[st] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      tmem_ld32(tdQ + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_ld32(tdQ + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(&dq_free[st]);
+      mbar_arrive(dq_free);
       // the reduce that last read this staging buffer (two steps ago) must be done reading
       if (leader) bulk_wait_read<1>();
       named_barrier_sync(1, 128);
