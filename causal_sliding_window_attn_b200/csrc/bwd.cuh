@@ -182,7 +182,9 @@ __global__ void __launch_bounds__(384, 1)
       for (int it = 0; it < n_iters; ++it) {
         const int st = it & 1;
         const int h = iter_head(it), q0 = iter_q0(it);
+        CSWA_MARK(3, it, 0);
         if (!mbar_wait(&qd_empty[st], ((it >> 1) & 1) ^ 1, abort_flag)) break;
+        CSWA_MARK(3, it, 1);
         mbar_arrive_expect_tx(&qd_full[st], 2 * L::kQT + 512);
         for (int pn = 0; pn < D / 64; ++pn) {
           tma_load_4d(smem + L::kQ + st * L::kQT + pn * L::kPanelQ, &tm_q, &qd_full[st], pn * 64, h, q0, b);
@@ -206,21 +208,28 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t idSP = idesc_bf16(128, 64, false, false);  // S^T, dP^T
       constexpr uint32_t idKV = idesc_bf16(128, D, false, true);    // dV (TS), dK: B MN-major
       constexpr uint32_t idQ = idesc_bf16(128, 64, true, true);     // dQ^T: A, B MN-major
+      // Descriptors are built once; a step only adds (byte offset >> 4) to the start field.
+      const uint64_t dK_kmaj = sdesc_sw128(sK, 16, 1024), dV_kmaj = sdesc_sw128(sV, 16, 1024);
+      const uint64_t dK_mn = sdesc_sw128(sK, L::kPanelKV, 1024);
+      const uint64_t dQ_kmaj = sdesc_sw128(sbase + L::kQ, 16, 1024), dDO_kmaj = sdesc_sw128(sbase + L::kDO, 16, 1024);
+      const uint64_t dQ_mn = sdesc_sw128(sbase + L::kQ, L::kPanelQ, 1024);
+      const uint64_t dDO_mn = sdesc_sw128(sbase + L::kDO, L::kPanelQ, 1024);
+      const uint64_t dDS_kmaj = sdesc_sw128(sDS, 16, 1024), dDS_mn = sdesc_sw128(sDS, 16, 1024);
       // step it uses Q/dO stage it & 1 and S^T/P^T buffer it & 1
       auto issue_S = [&](int it) {
-        const uint32_t sQ = sbase + L::kQ + (it & 1) * L::kQT;
+        const uint32_t qoff = (it & 1) * L::kQT;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tS[it & 1], sdesc_sw128(sK + (kk >> 2) * L::kPanelKV + (kk & 3) * 32, 16, 1024),
-                 sdesc_sw128(sQ + (kk >> 2) * L::kPanelQ + (kk & 3) * 32, 16, 1024), idSP, kk > 0);
+          mma_ss(tS[it & 1], dK_kmaj + (((kk >> 2) * L::kPanelKV + (kk & 3) * 32) >> 4),
+                 dQ_kmaj + ((qoff + (kk >> 2) * L::kPanelQ + (kk & 3) * 32) >> 4), idSP, kk > 0);
         mma_commit(&s_full[it & 1]);
       };
       auto issue_dP = [&](int it) {
-        const uint32_t sDO = sbase + L::kDO + (it & 1) * L::kQT;
+        const uint32_t qoff = (it & 1) * L::kQT;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tdP, sdesc_sw128(sV + (kk >> 2) * L::kPanelKV + (kk & 3) * 32, 16, 1024),
-                 sdesc_sw128(sDO + (kk >> 2) * L::kPanelQ + (kk & 3) * 32, 16, 1024), idSP, kk > 0);
+          mma_ss(tdP, dV_kmaj + (((kk >> 2) * L::kPanelKV + (kk & 3) * 32) >> 4),
+                 dDO_kmaj + ((qoff + (kk >> 2) * L::kPanelQ + (kk & 3) * 32) >> 4), idSP, kk > 0);
         mma_commit(dp_full);
       };
       bool ok = mbar_wait(kv_full, 0, abort_flag) && mbar_wait(&qd_full[0], 0, abort_flag);
@@ -231,12 +240,14 @@ __global__ void __launch_bounds__(384, 1)
       }
       for (int it = 0; ok && it < n_iters; ++it) {
         const int st = it & 1;
-        const uint32_t sQ = sbase + L::kQ + st * L::kQT, sDO = sbase + L::kDO + st * L::kQT;
+        const uint32_t qoff = st * L::kQT;
+        CSWA_MARK(0, it, 0);
         if (!(ok = mbar_wait(&p_full[st], (it >> 1) & 1, abort_flag))) break;
+        CSWA_MARK(0, it, 1);
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tdV, tS[st] + kk * 8, sdesc_sw128(sDO + kk * 2048, L::kPanelQ, 1024), idKV, (it > 0 || kk > 0));
+          mma_ts(tdV, tS[st] + kk * 8, dDO_mn + ((qoff + kk * 2048) >> 4), idKV, (it > 0 || kk > 0));
         mma_commit(&dv_done[st]);
         if (it + 1 < n_iters) {
           // the other S^T/P^T buffer was last read by dV of step it - 1
@@ -244,20 +255,21 @@ __global__ void __launch_bounds__(384, 1)
           if (it >= 1 && !(ok = mbar_wait(&dv_done[st ^ 1], ((it - 1) >> 1) & 1, abort_flag))) break;
           tc_fence_after();
           issue_S(it + 1);
+          CSWA_MARK(0, it, 2);
         }
         if (!(ok = mbar_wait(ds_full, it & 1, abort_flag))) break;
+        CSWA_MARK(0, it, 3);
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tdK, sdesc_sw128(sDS + kk * 32, 16, 1024), sdesc_sw128(sQ + kk * 2048, L::kPanelQ, 1024), idKV,
-                 (it > 0 || kk > 0));
+          mma_ss(tdK, dDS_kmaj + ((kk * 32) >> 4), dQ_mn + ((qoff + kk * 2048) >> 4), idKV, (it > 0 || kk > 0));
         // dQ^T of the previous step must have left TMEM
         if (it >= 1 && !(ok = mbar_wait(dq_free, (it - 1) & 1, abort_flag))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tdQ, sdesc_sw128(sK + kk * 2048, L::kPanelKV, 1024), sdesc_sw128(sDS + kk * 2048, 16, 1024), idQ,
-                 kk > 0);
+          mma_ss(tdQ, dK_mn + ((kk * 2048) >> 4), dDS_mn + ((kk * 2048) >> 4), idQ, kk > 0);
+        CSWA_MARK(0, it, 4);
         mma_commit(dq_full);
         mma_commit(&qd_empty[st]);
         // dP^T of the next step: the P/dS warps read this step's dP^T before ds_full
@@ -281,36 +293,50 @@ __global__ void __launch_bounds__(384, 1)
       const int q0 = iter_q0(it);
       const float* lse_s = s_lse + st * 64;
       const float* dl_s = s_delta + st * 64;
+      if (warp == 4 && lane == 0) CSWA_MARK(1, it, 0);
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[st], (it >> 1) & 1, abort_flag));
+      if (warp == 4 && lane == 0) CSWA_MARK(1, it, 1);
       if (!ok) break;
       tc_fence_after();
       uint32_t sr[64];
       tmem_ld32(tS[st] + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
       tmem_ld32(tS[st] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_ld_wait();
+      if (warp == 4 && lane == 0) CSWA_MARK(1, it, 6);
       const bool full = (k0 + 127 <= q0) && (W < 0 || q0 + 63 - k0 <= W);
       const int c_lo = j - q0;                       // query q0 + c sees key j iff c >= c_lo
       const int c_hi = (W < 0) ? 63 : j + W - q0;    //   and c <= c_hi
-      // P^T row in place as packed bf16 pairs; the same bf16 P feeds dV (TMEM) and dS
+      // P^T row in place as packed bf16 pairs; the same bf16 P feeds dV (TMEM) and dS.
+      // Masked entries get exponent -inf (ex2 -> 0): no branch around the exponential.
+      const float4* lse4 = reinterpret_cast<const float4*>(lse_s);
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const int c0 = 2 * c, c1 = 2 * c + 1;
-        const bool v0 = full || (c0 >= c_lo && c0 <= c_hi);
-        const bool v1 = full || (c1 >= c_lo && c1 <= c_hi);
-        const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(sr[c0]), sl2, -lse_s[c0])) : 0.f;
-        const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(sr[c1]), sl2, -lse_s[c1])) : 0.f;
-        sr[c] = pack_bf16x2(p0, p1);
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 l = lse4[c4];
+        const float lv[4] = {l.x, l.y, l.z, l.w};
+        float pv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = 4 * c4 + u;
+          const bool vis = full || (c >= c_lo && c <= c_hi);
+          pv[u] = ex2_approx(vis ? fmaf(__uint_as_float(sr[c]), sl2, -lv[u]) : -INFINITY);
+        }
+        sr[2 * c4] = pack_bf16x2(pv[0], pv[1]);
+        sr[2 * c4 + 1] = pack_bf16x2(pv[2], pv[3]);
       }
+      if (warp == 4 && lane == 0) CSWA_MARK(1, it, 7);
       tmem_st32(tS[st] + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[st]);
+      if (warp == 4 && lane == 0) CSWA_MARK(1, it, 2);
 
       ok = __all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, abort_flag));
+      if (warp == 4 && lane == 0) CSWA_MARK(1, it, 3);
       if (!ok) break;
       tc_fence_after();
       // dS^T of the previous step must have been consumed by dK and dQ
       if (it > 0) ok = __all_sync(0xffffffffu, mbar_wait(dq_full, (it - 1) & 1, abort_flag));
+      if (warp == 4 && lane == 0) CSWA_MARK(1, it, 4);
       if (!ok) break;
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
@@ -318,13 +344,16 @@ __global__ void __launch_bounds__(384, 1)
         tmem_ld32(tdP + lane_off + hf * 32, dp);
         tmem_ld_wait();
         uint32_t w[16];
+        const float4* dl4 = reinterpret_cast<const float4*>(dl_s + hf * 32);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c0 = hf * 32 + 2 * e;
-          const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sr[hf * 16 + e]));
-          const float d0 = pp.x * (__uint_as_float(dp[2 * e]) - dl_s[c0]);
-          const float d1 = pp.y * (__uint_as_float(dp[2 * e + 1]) - dl_s[c0 + 1]);
-          w[e] = pack_bf16x2(d0, d1);
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 dl = dl4[e4];
+          const float2 p0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sr[hf * 16 + 2 * e4]));
+          const float2 p1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sr[hf * 16 + 2 * e4 + 1]));
+          w[2 * e4] = pack_bf16x2(p0.x * (__uint_as_float(dp[4 * e4]) - dl.x),
+                                  p0.y * (__uint_as_float(dp[4 * e4 + 1]) - dl.y));
+          w[2 * e4 + 1] = pack_bf16x2(p1.x * (__uint_as_float(dp[4 * e4 + 2]) - dl.z),
+                                      p1.y * (__uint_as_float(dp[4 * e4 + 3]) - dl.w));
         }
         // row r of the dS^T panel: chunks 4*hf .. 4*hf+3 of 16 bytes, 128-byte swizzle
 #pragma unroll
@@ -335,6 +364,7 @@ __global__ void __launch_bounds__(384, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(ds_full);
+      if (warp == 4 && lane == 0) CSWA_MARK(1, it, 5);
     }
     // ---------------------------------------------------------- dK epilogue
     ok = __all_sync(0xffffffffu, ok && mbar_wait(final_bar, 0, abort_flag));
@@ -366,7 +396,9 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
     for (int it = 0; it < n_iters; ++it) {
       const int st = it & 1;
+      if (leader) CSWA_MARK(2, it, 0);
       ok = __all_sync(0xffffffffu, mbar_wait(dq_full, it & 1, abort_flag));
+      if (leader) CSWA_MARK(2, it, 1);
       if (!ok) break;
       tc_fence_after();
       uint32_t v[64];
@@ -389,6 +421,7 @@ __global__ void __launch_bounds__(384, 1)
         const int row = (int)(((size_t)b * p.Hq + iter_head(it)) * p.Tpad + iter_q0(it));
         tma_reduce_add_2d(&tm_dq, stage, 0, row);
         bulk_commit();
+        CSWA_MARK(2, it, 2);
       }
     }
     if (leader) bulk_wait_all();

@@ -153,6 +153,10 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idO = idesc_bf16(128, D, false, true);
+      // descriptors built once; each MMA adds (byte offset >> 4) to the start field
+      const uint64_t dQ0 = sdesc_sw128(sQ[0], 16, 1024), dQ1 = sdesc_sw128(sQ[1], 16, 1024);
+      const uint64_t dK0 = sdesc_sw128(sK[0], 16, 1024);
+      const uint64_t dV0 = sdesc_sw128(sV[0], 16384, 1024);
       int cnt[2] = {0, 0};
       bool ok = mbar_wait(q_full, 0, abort_flag);
       tc_fence_after();
@@ -170,8 +174,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_ss(tS[s], sdesc_sw128(sQ[s] + off, 16, 1024), sdesc_sw128(sK[st] + off, 16, 1024), idS,
-                   kk > 0);
+            mma_ss(tS[s], (s ? dQ1 : dQ0) + (off >> 4), dK0 + ((st * L::kTile + off) >> 4), idS, kk > 0);
           }
           mma_commit(&s_full[s]);
         }
@@ -184,8 +187,7 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tO[s], tS[s] + kk * 8, sdesc_sw128(sV[st] + kk * 2048, 16384, 1024), idO,
-                   (cnt[s] > 0 || kk > 0));
+            mma_ts(tO[s], tS[s] + kk * 8, dV0 + ((st * L::kTile + kk * 2048) >> 4), idO, (cnt[s] > 0 || kk > 0));
           mma_commit(&pv_done[s]);
           ++cnt[s];
         }

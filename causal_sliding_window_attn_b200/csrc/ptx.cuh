@@ -15,6 +15,21 @@ enum : unsigned { kStatusTimeout = 1u, kStatusBadPosition = 2u, kStatusLayout = 
 __device__ unsigned int g_status;
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
 
+// Pipeline trace marks: compiled out unless CSWA_TRACE is defined (profiling
+// builds record clock64() per (CTA, role, step, tag) for the first CTAs).
+#ifdef CSWA_TRACE
+__device__ unsigned long long g_trace[64 * 4 * 64 * 8];
+#define CSWA_MARK(role, it, tag)                                                                      \
+  do {                                                                                                \
+    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z < 64 && (it) < 64)                           \
+      g_trace[((blockIdx.z * 4 + (role)) * 64 + (it)) * 8 + (tag)] = clock64();                       \
+  } while (0)
+#else
+#define CSWA_MARK(role, it, tag) \
+  do {                           \
+  } while (0)
+#endif
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
