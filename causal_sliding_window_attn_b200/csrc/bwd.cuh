@@ -307,21 +307,33 @@ __global__ void __launch_bounds__(384, 1)
       const int c_lo = j - q0;                       // query q0 + c sees key j iff c >= c_lo
       const int c_hi = (W < 0) ? 63 : j + W - q0;    //   and c <= c_hi
       // P^T row in place as packed bf16 pairs; the same bf16 P feeds dV (TMEM) and dS.
-      // Masked entries get exponent -inf (ex2 -> 0): no branch around the exponential.
+      // Masked entries get exponent -inf (ex2 -> 0): no branch around the exponential;
+      // tiles inside the band skip the mask (a warp-uniform branch).
       const float4* lse4 = reinterpret_cast<const float4*>(lse_s);
+      if (full) {
 #pragma unroll
-      for (int c4 = 0; c4 < 16; ++c4) {
-        const float4 l = lse4[c4];
-        const float lv[4] = {l.x, l.y, l.z, l.w};
-        float pv[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int c = 4 * c4 + u;
-          const bool vis = full || (c >= c_lo && c <= c_hi);
-          pv[u] = ex2_approx(vis ? fmaf(__uint_as_float(sr[c]), sl2, -lv[u]) : -INFINITY);
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 l = lse4[c4];
+          sr[2 * c4] = pack_bf16x2(ex2_approx(fmaf(__uint_as_float(sr[4 * c4]), sl2, -l.x)),
+                                   ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 1]), sl2, -l.y)));
+          sr[2 * c4 + 1] = pack_bf16x2(ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 2]), sl2, -l.z)),
+                                       ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 3]), sl2, -l.w)));
         }
-        sr[2 * c4] = pack_bf16x2(pv[0], pv[1]);
-        sr[2 * c4 + 1] = pack_bf16x2(pv[2], pv[3]);
+      } else {
+#pragma unroll
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 l = lse4[c4];
+          const float lv[4] = {l.x, l.y, l.z, l.w};
+          float pv[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int c = 4 * c4 + u;
+            const bool vis = (c >= c_lo) & (c <= c_hi);
+            pv[u] = ex2_approx(vis ? fmaf(__uint_as_float(sr[c]), sl2, -lv[u]) : -INFINITY);
+          }
+          sr[2 * c4] = pack_bf16x2(pv[0], pv[1]);
+          sr[2 * c4 + 1] = pack_bf16x2(pv[2], pv[3]);
+        }
       }
       if (warp == 4 && lane == 0) CSWA_MARK(1, it, 7);
       tmem_st32(tS[st] + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));

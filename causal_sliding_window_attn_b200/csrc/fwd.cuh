@@ -236,7 +236,8 @@ __global__ void __launch_bounds__(384, 1)
           const int c_lo = (W < 0) ? -1 : i - W - k0;
 #pragma unroll
           for (int c = 0; c < 128; ++c) {
-            if (c > c_hi || c < c_lo) r[c] = __float_as_uint(-INFINITY);
+            const bool vis = (c <= c_hi) & (c >= c_lo);
+            r[c] = vis ? r[c] : __float_as_uint(-INFINITY);
             mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(r[c]));
           }
         }
