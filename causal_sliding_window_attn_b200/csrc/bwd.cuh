@@ -14,19 +14,18 @@
 //                rows get P = 0), and zeroes the fp32 dQ accumulator.
 //   bwd_main     one CTA per (128-key tile, KV head, batch). K and V stay in
 //                shared memory; the CTA walks every (query head of the group,
-//                64-row query sub-tile) that sees the key tile. Per step:
-//                  S^T  = K Q^T         (SS)  -> TMEM [0,64) / [64,128), alternating
-//                  dP^T = V dO^T        (SS)  -> TMEM [128,192)
-//                  P^T  = exp2(S^T c - lse)     bf16 back over its S^T
+//                128-row query tile) that sees the key tile. Per step, all
+//                MMAs M = 128, N = 128 (the shape the tensor pipe runs at full
+//                rate), TMEM regions R0, R1 of 128 columns each:
+//                  S^T  = K Q^T         (SS)  -> R0
+//                  P^T  = exp2(S^T c - lse)     bf16 back into R0
 //                  dV  += P^T dO        (TS)  -> TMEM [256,256+D)
+//                  dP^T = V dO^T        (SS)  -> R1
 //                  dS^T = P^T (dP^T - Delta)    bf16 into shared memory
 //                  dK  += dS^T Q        (SS)  -> TMEM [256+D,256+2D)
-//                  dQ^T = K^T dS^T      (SS, both MN-major) -> TMEM [192,256)
-//                S^T/P^T alternate between two TMEM buffers, so the next
-//                step's S^T is issued right behind this step's dV. A drain
-//                warpgroup moves dQ^T to a shared-memory staging tile and adds
-//                it to the fp32 accumulator with one TMA reduce-add per step,
-//                off the critical path of the tensor pipe.
+//                  dQ^T = K^T dS^T      (SS, both MN-major) -> R1
+//                A drain warpgroup reads dQ^T out of TMEM and adds it to the
+//                fp32 accumulator with 128-byte coalesced reductions.
 //                dK, dV are complete in the CTA (the whole group is walked
 //                here), so they are written once, as bf16, with no atomics.
 //   bwd_dq_cast  the fp32 dQ accumulator (B, Hq, Tpad, D) -> bf16 dq (B, T, Hq, D).
@@ -42,7 +41,7 @@ struct BwdParams {
   const float* delta;  // (B, Hq, Tpad)
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
-  int T, Tpad, Hq, G, window, n_kv_tiles, n_q_tiles;  // q tiles of 64 rows
+  int T, Tpad, Hq, G, window, n_kv_tiles, n_q_tiles;  // tiles of 128 rows
   float scale, scale_log2;
 };
 
@@ -73,23 +72,19 @@ __device__ __forceinline__ void named_barrier_sync(int id, int count) {
 
 template <int D>
 struct BwdLayout {
-  static constexpr int kKV = 128 * D * 2;       // K or V tile: 128 rows
-  static constexpr int kQT = 64 * D * 2;        // Q or dO tile: 64 rows
-  static constexpr int kPanelKV = 128 * 128;    // one 64-column panel of a 128-row tile
-  static constexpr int kPanelQ = 64 * 128;      // one 64-column panel of a 64-row tile
+  static constexpr int kTile = 128 * D * 2;   // one 128-row bf16 tile (K, V, Q or dO)
+  static constexpr int kPanel = 128 * 128;    // one 64-column panel of a 128-row tile
   static constexpr int kK = 0;
-  static constexpr int kZero = kK + kKV;        // D = 64: zero panel after K (pads K^T to M = 128)
-  static constexpr int kV = kZero + (D == 64 ? kPanelKV : 0);
-  static constexpr int kQ = kV + kKV;           // [2]
-  static constexpr int kDO = kQ + 2 * kQT;      // [2]
-  static constexpr int kDS = kDO + 2 * kQT;     // dS^T: 128 keys x 64 queries bf16 = 16 KB
-  static constexpr int kStage = kDS + 16384;    // dQ staging [2]: 64 x D fp32
-  static constexpr int kStageBytes = 64 * D * 4;
-  static constexpr int kStat = kStage + 2 * kStageBytes;  // lse2[2][64], delta[2][64]
-  static constexpr int kBar = kStat + 1024;
+  static constexpr int kZero = kK + kTile;    // D = 64: zero panel after K (pads K^T to M = 128)
+  static constexpr int kV = kZero + (D == 64 ? kPanel : 0);
+  static constexpr int kQ = kV + kTile;       // [2]
+  static constexpr int kDO = kQ + 2 * kTile;  // [2]
+  static constexpr int kDS = kDO + 2 * kTile; // dS^T: 128 keys x 128 queries bf16, 2 panels
+  static constexpr int kStat = kDS + 2 * kPanel;  // lse2[2][128], delta[2][128]
+  static constexpr int kBar = kStat + 2048;
   static constexpr int kUsed = kBar + 256;
-  static constexpr int kBytes = kUsed + 1024;
-  static_assert(kBytes <= 232448, "shared memory budget");
+  static constexpr int kBytes = (kUsed + 1024 <= 232448) ? kUsed + 1024 : 232448;
+  static_assert(kUsed <= 232448, "shared memory budget");
   static constexpr uint32_t kTmemCols = 512;
 };
 
@@ -97,38 +92,42 @@ template <int D>
 __global__ void __launch_bounds__(384, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+                    float* __restrict__ dq_acc, const BwdParams p) {
   using L = BwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // the layout needs a 1024-byte aligned base: report (never overrun) if the slack is too small
+  if ((smem - smem_raw) + L::kUsed > L::kBytes) {
+    if (threadIdx.x == 0) atomicOr(&g_status, kStatusLayout);
+    return;
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* kv_full = bars + 0;
   uint64_t* qd_full = bars + 1;   // [2]
   uint64_t* qd_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;    // [2]
-  uint64_t* p_full = bars + 7;    // [2]
-  uint64_t* dv_done = bars + 9;   // [2]
-  uint64_t* dp_full = bars + 11;
-  uint64_t* ds_full = bars + 12;
-  uint64_t* dq_full = bars + 13;
-  uint64_t* dq_free = bars + 14;
-  uint64_t* final_bar = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 17);
-  float* s_lse = reinterpret_cast<float*>(smem + L::kStat);         // [2][64]
-  float* s_delta = reinterpret_cast<float*>(smem + L::kStat + 512);  // [2][64]
+  uint64_t* s_full = bars + 5;
+  uint64_t* p_full = bars + 6;
+  uint64_t* dv_done = bars + 7;
+  uint64_t* dp_full = bars + 8;
+  uint64_t* ds_full = bars + 9;
+  uint64_t* dq_full = bars + 10;
+  uint64_t* dq_free = bars + 11;
+  uint64_t* final_bar = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 14);
+  float* s_lse = reinterpret_cast<float*>(smem + L::kStat);           // [2][128]
+  float* s_delta = reinterpret_cast<float*>(smem + L::kStat + 1024);  // [2][128]
 
   const int warp = warp_id(), lane = lane_id();
   const int hk = blockIdx.x, b = blockIdx.y, n = blockIdx.z;
   const int W = p.window, G = p.G;
   const int k0 = n * 128;
-  const int m_lo = 2 * n;
-  const int m_hi = (W < 0) ? p.n_q_tiles - 1 : min(p.n_q_tiles - 1, (k0 + 127 + W) / 64);
-  const int m_cnt = m_hi - m_lo + 1;
+  const int m_hi = (W < 0) ? p.n_q_tiles - 1 : min(p.n_q_tiles - 1, (k0 + 127 + W) / 128);
+  const int m_cnt = m_hi - n + 1;
   const int n_iters = G * m_cnt;
 
   if (D == 64) {
-    for (int i = threadIdx.x; i < L::kPanelKV / 16; i += blockDim.x)
+    for (int i = threadIdx.x; i < L::kPanel / 16; i += blockDim.x)
       reinterpret_cast<uint4*>(smem + L::kZero)[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
   }
@@ -137,10 +136,10 @@ __global__ void __launch_bounds__(384, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&qd_full[s], 1);
       mbar_init(&qd_empty[s], 1);
-      mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
-      mbar_init(&dv_done[s], 1);
     }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(dv_done, 1);
     mbar_init(dp_full, 1);
     mbar_init(ds_full, 128);
     mbar_init(dq_full, 1);
@@ -157,14 +156,12 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS[2] = {tmem, tmem + 64};
-  const uint32_t tdP = tmem + 128, tdQ = tmem + 192, tdV = tmem + 256, tdK = tmem + 256 + D;
+  // R0: S^T, then P^T (bf16) in its first 64 columns; R1: dP^T, then dQ^T
+  const uint32_t tR0 = tmem, tR1 = tmem + 128, tdV = tmem + 256, tdK = tmem + 256 + D;
 
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t sK = sbase + L::kK, sV = sbase + L::kV, sDS = sbase + L::kDS;
-
   auto iter_head = [&](int it) { return hk * G + it / m_cnt; };
-  auto iter_q0 = [&](int it) { return (m_lo + it % m_cnt) * 64; };
+  auto iter_q0 = [&](int it) { return (n + it % m_cnt) * 128; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -173,10 +170,10 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
-      mbar_arrive_expect_tx(kv_full, 2 * L::kKV);
+      mbar_arrive_expect_tx(kv_full, 2 * L::kTile);
       for (int pn = 0; pn < D / 64; ++pn) {
-        tma_load_4d(smem + L::kK + pn * L::kPanelKV, &tm_k, kv_full, pn * 64, hk, k0, b);
-        tma_load_4d(smem + L::kV + pn * L::kPanelKV, &tm_v, kv_full, pn * 64, hk, k0, b);
+        tma_load_4d(smem + L::kK + pn * L::kPanel, &tm_k, kv_full, pn * 64, hk, k0, b);
+        tma_load_4d(smem + L::kV + pn * L::kPanel, &tm_v, kv_full, pn * 64, hk, k0, b);
       }
       int last_issue[2] = {-1, -1};
       for (int it = 0; it < n_iters; ++it) {
@@ -185,14 +182,14 @@ __global__ void __launch_bounds__(384, 1)
         CSWA_MARK(3, it, 0);
         if (!mbar_wait(&qd_empty[st], ((it >> 1) & 1) ^ 1, abort_flag)) break;
         CSWA_MARK(3, it, 1);
-        mbar_arrive_expect_tx(&qd_full[st], 2 * L::kQT + 512);
+        mbar_arrive_expect_tx(&qd_full[st], 2 * L::kTile + 1024);
         for (int pn = 0; pn < D / 64; ++pn) {
-          tma_load_4d(smem + L::kQ + st * L::kQT + pn * L::kPanelQ, &tm_q, &qd_full[st], pn * 64, h, q0, b);
-          tma_load_4d(smem + L::kDO + st * L::kQT + pn * L::kPanelQ, &tm_do, &qd_full[st], pn * 64, h, q0, b);
+          tma_load_4d(smem + L::kQ + st * L::kTile + pn * L::kPanel, &tm_q, &qd_full[st], pn * 64, h, q0, b);
+          tma_load_4d(smem + L::kDO + st * L::kTile + pn * L::kPanel, &tm_do, &qd_full[st], pn * 64, h, q0, b);
         }
         const size_t row0 = ((size_t)b * p.Hq + h) * p.Tpad + q0;
-        bulk_load(s_lse + st * 64, p.lse2 + row0, 256, &qd_full[st]);
-        bulk_load(s_delta + st * 64, p.delta + row0, 256, &qd_full[st]);
+        bulk_load(s_lse + st * 128, p.lse2 + row0, 512, &qd_full[st]);
+        bulk_load(s_delta + st * 128, p.delta + row0, 512, &qd_full[st]);
         last_issue[st] = it;
       }
       if (*abort_flag) {
@@ -205,31 +202,34 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idSP = idesc_bf16(128, 64, false, false);  // S^T, dP^T
-      constexpr uint32_t idKV = idesc_bf16(128, D, false, true);    // dV (TS), dK: B MN-major
-      constexpr uint32_t idQ = idesc_bf16(128, 64, true, true);     // dQ^T: A, B MN-major
-      // Descriptors are built once; a step only adds (byte offset >> 4) to the start field.
-      const uint64_t dK_kmaj = sdesc_sw128(sK, 16, 1024), dV_kmaj = sdesc_sw128(sV, 16, 1024);
-      const uint64_t dK_mn = sdesc_sw128(sK, L::kPanelKV, 1024);
-      const uint64_t dQ_kmaj = sdesc_sw128(sbase + L::kQ, 16, 1024), dDO_kmaj = sdesc_sw128(sbase + L::kDO, 16, 1024);
-      const uint64_t dQ_mn = sdesc_sw128(sbase + L::kQ, L::kPanelQ, 1024);
-      const uint64_t dDO_mn = sdesc_sw128(sbase + L::kDO, L::kPanelQ, 1024);
-      const uint64_t dDS_kmaj = sdesc_sw128(sDS, 16, 1024), dDS_mn = sdesc_sw128(sDS, 16, 1024);
-      // step it uses Q/dO stage it & 1 and S^T/P^T buffer it & 1
+      constexpr uint32_t idSP = idesc_bf16(128, 128, false, false);  // S^T, dP^T
+      constexpr uint32_t idKV = idesc_bf16(128, D, false, true);     // dV (TS), dK: B MN-major
+      constexpr uint32_t idQ = idesc_bf16(128, 128, true, true);     // dQ^T: A and B MN-major
+      // Descriptors are built once; an MMA only adds (byte offset >> 4) to the start field.
+      const uint64_t dK_k = sdesc_sw128(sbase + L::kK, 16, 1024), dV_k = sdesc_sw128(sbase + L::kV, 16, 1024);
+      const uint64_t dK_mn = sdesc_sw128(sbase + L::kK, L::kPanel, 1024);
+      const uint64_t dQ_k = sdesc_sw128(sbase + L::kQ, 16, 1024), dDO_k = sdesc_sw128(sbase + L::kDO, 16, 1024);
+      const uint64_t dQ_mn = sdesc_sw128(sbase + L::kQ, L::kPanel, 1024);
+      const uint64_t dDO_mn = sdesc_sw128(sbase + L::kDO, L::kPanel, 1024);
+      const uint64_t dDS_k = sdesc_sw128(sbase + L::kDS, 16, 1024);
+      const uint64_t dDS_mn = sdesc_sw128(sbase + L::kDS, L::kPanel, 1024);
+      // step it reads Q/dO stage it & 1
       auto issue_S = [&](int it) {
-        const uint32_t qoff = (it & 1) * L::kQT;
+        const uint32_t qo = (it & 1) * L::kTile;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tS[it & 1], dK_kmaj + (((kk >> 2) * L::kPanelKV + (kk & 3) * 32) >> 4),
-                 dQ_kmaj + ((qoff + (kk >> 2) * L::kPanelQ + (kk & 3) * 32) >> 4), idSP, kk > 0);
-        mma_commit(&s_full[it & 1]);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kPanel + (kk & 3) * 32;
+          mma_ss(tR0, dK_k + (off >> 4), dQ_k + ((qo + off) >> 4), idSP, kk > 0);
+        }
+        mma_commit(s_full);
       };
       auto issue_dP = [&](int it) {
-        const uint32_t qoff = (it & 1) * L::kQT;
+        const uint32_t qo = (it & 1) * L::kTile;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tdP, dV_kmaj + (((kk >> 2) * L::kPanelKV + (kk & 3) * 32) >> 4),
-                 dDO_kmaj + ((qoff + (kk >> 2) * L::kPanelQ + (kk & 3) * 32) >> 4), idSP, kk > 0);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kPanel + (kk & 3) * 32;
+          mma_ss(tR1, dV_k + (off >> 4), dDO_k + ((qo + off) >> 4), idSP, kk > 0);
+        }
         mma_commit(dp_full);
       };
       bool ok = mbar_wait(kv_full, 0, abort_flag) && mbar_wait(&qd_full[0], 0, abort_flag);
@@ -240,19 +240,19 @@ __global__ void __launch_bounds__(384, 1)
       }
       for (int it = 0; ok && it < n_iters; ++it) {
         const int st = it & 1;
-        const uint32_t qoff = st * L::kQT;
+        const uint32_t qo = st * L::kTile;
         CSWA_MARK(0, it, 0);
-        if (!(ok = mbar_wait(&p_full[st], (it >> 1) & 1, abort_flag))) break;
+        if (!(ok = mbar_wait(p_full, it & 1, abort_flag))) break;
         CSWA_MARK(0, it, 1);
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tdV, tS[st] + kk * 8, dDO_mn + ((qoff + kk * 2048) >> 4), idKV, (it > 0 || kk > 0));
-        mma_commit(&dv_done[st]);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tdV, tR0 + kk * 8, dDO_mn + ((qo + kk * 2048) >> 4), idKV, (it > 0 || kk > 0));
+        mma_commit(dv_done);
         if (it + 1 < n_iters) {
-          // the other S^T/P^T buffer was last read by dV of step it - 1
+          // S^T of the next step overwrites P^T: wait until dV has read it
           if (!(ok = mbar_wait(&qd_full[st ^ 1], ((it + 1) >> 1) & 1, abort_flag))) break;
-          if (it >= 1 && !(ok = mbar_wait(&dv_done[st ^ 1], ((it - 1) >> 1) & 1, abort_flag))) break;
+          if (!(ok = mbar_wait(dv_done, it & 1, abort_flag))) break;
           tc_fence_after();
           issue_S(it + 1);
           CSWA_MARK(0, it, 2);
@@ -261,19 +261,22 @@ __global__ void __launch_bounds__(384, 1)
         CSWA_MARK(0, it, 3);
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tdK, dDS_kmaj + ((kk * 32) >> 4), dQ_mn + ((qoff + kk * 2048) >> 4), idKV, (it > 0 || kk > 0));
-        // dQ^T of the previous step must have left TMEM
-        if (it >= 1 && !(ok = mbar_wait(dq_free, (it - 1) & 1, abort_flag))) break;
-        tc_fence_after();
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tdK, dDS_k + (((kk >> 2) * L::kPanel + (kk & 3) * 32) >> 4), dQ_mn + ((qo + kk * 2048) >> 4),
+                 idKV, (it > 0 || kk > 0));
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tdQ, dK_mn + ((kk * 2048) >> 4), dDS_mn + ((kk * 2048) >> 4), idQ, kk > 0);
+          mma_ss(tR1, dK_mn + ((kk * 2048) >> 4), dDS_mn + ((kk * 2048) >> 4), idQ, kk > 0);
         CSWA_MARK(0, it, 4);
         mma_commit(dq_full);
         mma_commit(&qd_empty[st]);
-        // dP^T of the next step: the P/dS warps read this step's dP^T before ds_full
-        if (it + 1 < n_iters) issue_dP(it + 1);
+        if (it + 1 < n_iters) {
+          // dP^T of the next step goes where dQ^T is: wait until the drain has read it
+          if (!(ok = mbar_wait(dq_free, it & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_dP(it + 1);
+          CSWA_MARK(0, it, 5);
+        }
       }
       mma_commit(final_bar);
       volatile int dummy = 0;
@@ -291,28 +294,27 @@ __global__ void __launch_bounds__(384, 1)
     for (int it = 0; it < n_iters; ++it) {
       const int st = it & 1;
       const int q0 = iter_q0(it);
-      const float* lse_s = s_lse + st * 64;
-      const float* dl_s = s_delta + st * 64;
+      const float* lse_s = s_lse + st * 128;
+      const float* dl_s = s_delta + st * 128;
       if (warp == 4 && lane == 0) CSWA_MARK(1, it, 0);
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[st], (it >> 1) & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag));
       if (warp == 4 && lane == 0) CSWA_MARK(1, it, 1);
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld32(tS[st] + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tS[st] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      uint32_t sr[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tR0 + lane_off + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
       tmem_ld_wait();
-      if (warp == 4 && lane == 0) CSWA_MARK(1, it, 6);
-      const bool full = (k0 + 127 <= q0) && (W < 0 || q0 + 63 - k0 <= W);
+      const bool full = (k0 + 127 <= q0) && (W < 0 || q0 + 127 - k0 <= W);
       const int c_lo = j - q0;                       // query q0 + c sees key j iff c >= c_lo
-      const int c_hi = (W < 0) ? 63 : j + W - q0;    //   and c <= c_hi
-      // P^T row in place as packed bf16 pairs; the same bf16 P feeds dV (TMEM) and dS.
+      const int c_hi = (W < 0) ? 127 : j + W - q0;   //   and c <= c_hi
+      // P^T row in place as packed bf16 pairs (the same bf16 P feeds dV and dS).
       // Masked entries get exponent -inf (ex2 -> 0): no branch around the exponential;
       // tiles inside the band skip the mask (a warp-uniform branch).
       const float4* lse4 = reinterpret_cast<const float4*>(lse_s);
       if (full) {
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
+        for (int c4 = 0; c4 < 32; ++c4) {
           const float4 l = lse4[c4];
           sr[2 * c4] = pack_bf16x2(ex2_approx(fmaf(__uint_as_float(sr[4 * c4]), sl2, -l.x)),
                                    ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 1]), sl2, -l.y)));
@@ -321,7 +323,7 @@ __global__ void __launch_bounds__(384, 1)
         }
       } else {
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
+        for (int c4 = 0; c4 < 32; ++c4) {
           const float4 l = lse4[c4];
           const float lv[4] = {l.x, l.y, l.z, l.w};
           float pv[4];
@@ -335,43 +337,45 @@ __global__ void __launch_bounds__(384, 1)
           sr[2 * c4 + 1] = pack_bf16x2(pv[2], pv[3]);
         }
       }
-      if (warp == 4 && lane == 0) CSWA_MARK(1, it, 7);
-      tmem_st32(tS[st] + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      if (warp == 4 && lane == 0) CSWA_MARK(1, it, 6);
+      tmem_st32(tR0 + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_st32(tR0 + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&p_full[st]);
+      mbar_arrive(p_full);
       if (warp == 4 && lane == 0) CSWA_MARK(1, it, 2);
 
       ok = __all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, abort_flag));
       if (warp == 4 && lane == 0) CSWA_MARK(1, it, 3);
-      if (!ok) break;
-      tc_fence_after();
-      // dS^T of the previous step must have been consumed by dK and dQ
-      if (it > 0) ok = __all_sync(0xffffffffu, mbar_wait(dq_full, (it - 1) & 1, abort_flag));
+      // dS^T of the previous step must have been consumed by dK and dQ^T
+      if (ok && it > 0) ok = __all_sync(0xffffffffu, mbar_wait(dq_full, (it - 1) & 1, abort_flag));
       if (warp == 4 && lane == 0) CSWA_MARK(1, it, 4);
       if (!ok) break;
+      tc_fence_after();
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
+      for (int cc = 0; cc < 4; ++cc) {
         uint32_t dp[32];
-        tmem_ld32(tdP + lane_off + hf * 32, dp);
+        tmem_ld32(tR1 + lane_off + cc * 32, dp);
         tmem_ld_wait();
+        const float4* dl4 = reinterpret_cast<const float4*>(dl_s + cc * 32);
         uint32_t w[16];
-        const float4* dl4 = reinterpret_cast<const float4*>(dl_s + hf * 32);
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
           const float4 dl = dl4[e4];
-          const float2 p0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sr[hf * 16 + 2 * e4]));
-          const float2 p1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sr[hf * 16 + 2 * e4 + 1]));
+          const float2 p0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sr[cc * 16 + 2 * e4]));
+          const float2 p1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sr[cc * 16 + 2 * e4 + 1]));
           w[2 * e4] = pack_bf16x2(p0.x * (__uint_as_float(dp[4 * e4]) - dl.x),
                                   p0.y * (__uint_as_float(dp[4 * e4 + 1]) - dl.y));
           w[2 * e4 + 1] = pack_bf16x2(p1.x * (__uint_as_float(dp[4 * e4 + 2]) - dl.z),
                                       p1.y * (__uint_as_float(dp[4 * e4 + 3]) - dl.w));
         }
-        // row r of the dS^T panel: chunks 4*hf .. 4*hf+3 of 16 bytes, 128-byte swizzle
+        // queries cc*32 .. cc*32+31 = 16-byte chunks (cc&1)*4 .. +3 of panel cc/2, 128-byte swizzle
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          *reinterpret_cast<uint4*>(ds_row + (((4 * hf + u) ^ (r & 7)) << 4)) =
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t chunk = (cc & 1) * 4 + u;
+          *reinterpret_cast<uint4*>(ds_row + (cc >> 1) * L::kPanel + ((chunk ^ (r & 7)) << 4)) =
               make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        }
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -404,39 +408,28 @@ __global__ void __launch_bounds__(384, 1)
     const int quarter = warp & 3;
     const int dd = quarter * 32 + lane;  // d index of this thread's TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const bool leader = (warp == 8 && lane == 0);
     bool ok = true;
     for (int it = 0; it < n_iters; ++it) {
-      const int st = it & 1;
-      if (leader) CSWA_MARK(2, it, 0);
+      if (warp == 8 && lane == 0) CSWA_MARK(2, it, 0);
       ok = __all_sync(0xffffffffu, mbar_wait(dq_full, it & 1, abort_flag));
-      if (leader) CSWA_MARK(2, it, 1);
+      if (warp == 8 && lane == 0) CSWA_MARK(2, it, 1);
       if (!ok) break;
       tc_fence_after();
-      uint32_t v[64];
-      tmem_ld32(tdQ + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_ld32(tdQ + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      uint32_t v[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tR1 + lane_off + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(dq_free);
-      // the reduce that last read this staging buffer (two steps ago) must be done reading
-      if (leader) bulk_wait_read<1>();
-      named_barrier_sync(1, 128);
-      float* stage = reinterpret_cast<float*>(smem + L::kStage + st * L::kStageBytes);
+      // dQ[q0 + c][dd] += scale * dQ^T[dd][c]: a warp covers 32 consecutive d, one
+      // 128-byte coalesced fp32 reduction per instruction
       if (dd < D) {
+        float* dst = dq_acc + (((size_t)b * p.Hq + iter_head(it)) * p.Tpad + iter_q0(it)) * D + dd;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) stage[c * D + dd] = __uint_as_float(v[c]) * p.scale;
+        for (int c = 0; c < 128; ++c) atomicAdd(dst + (size_t)c * D, __uint_as_float(v[c]) * p.scale);
       }
-      fence_proxy_async_smem();
-      named_barrier_sync(1, 128);
-      if (leader) {
-        const int row = (int)(((size_t)b * p.Hq + iter_head(it)) * p.Tpad + iter_q0(it));
-        tma_reduce_add_2d(&tm_dq, stage, 0, row);
-        bulk_commit();
-        CSWA_MARK(2, it, 2);
-      }
+      if (warp == 8 && lane == 0) CSWA_MARK(2, it, 2);
     }
-    if (leader) bulk_wait_all();
     // ---------------------------------------------------------- dV epilogue (thread = key row)
     ok = __all_sync(0xffffffffu, ok && mbar_wait(final_bar, 0, abort_flag));
     tc_fence_after();

@@ -50,20 +50,6 @@ bool encode_bthd(CUtensorMap* m, const void* base, int B, int T, int H, int D, i
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Row-major fp32 matrix (rows, cols) as a 2-D tensor map with a (64 x cols) box,
-// no swizzle: the dQ accumulator, target of TMA reduce-adds.
-bool encode_f32_rows(CUtensorMap* m, const void* base, long long rows, int cols) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
-  const cuuint32_t box[2] = {(cuuint32_t)cols, 64};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool dims_ok(int B, int T, int Hq, int Hkv) {
   return B >= 1 && T >= 1 && Hq >= 1 && Hkv >= 1 && Hq % Hkv == 0 && (long long)B * T * Hq < (1ll << 40);
@@ -175,10 +161,9 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
                          int window, float scale, cudaStream_t st) {
   const int Tpad = tiles128(T) * 128;
   BwdWorkspace w = carve_bwd(ws, B, T, Hq, D);
-  CUtensorMap tq, tk, tv, tdo, tdq;
-  if (!encode_bthd(&tq, q, B, T, Hq, D, 64) || !encode_bthd(&tk, k, B, T, Hkv, D) ||
-      !encode_bthd(&tv, v, B, T, Hkv, D) || !encode_bthd(&tdo, dO, B, T, Hq, D, 64) ||
-      !encode_f32_rows(&tdq, w.dq_acc, (long long)B * Hq * Tpad, D))
+  CUtensorMap tq, tk, tv, tdo;
+  if (!encode_bthd(&tq, q, B, T, Hq, D) || !encode_bthd(&tk, k, B, T, Hkv, D) ||
+      !encode_bthd(&tv, v, B, T, Hkv, D) || !encode_bthd(&tdo, dO, B, T, Hq, D))
     return ATTN_ERR_LAUNCH;
   if (!set_smem_attrs<D>()) return ATTN_ERR_LAUNCH;
   {
@@ -199,11 +184,11 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
   p.G = Hq / Hkv;
   p.window = (window >= T) ? -1 : window;
   p.n_kv_tiles = tiles128(T);
-  p.n_q_tiles = (T + 63) / 64;
+  p.n_q_tiles = tiles128(T);
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
   dim3 grid(Hkv, B, p.n_kv_tiles);
-  attn_bwd_kernel<D><<<grid, 384, BwdLayout<D>::kBytes, st>>>(tq, tk, tv, tdo, tdq, p);
+  attn_bwd_kernel<D><<<grid, 384, BwdLayout<D>::kBytes, st>>>(tq, tk, tv, tdo, w.dq_acc, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
   const long long n8 = (long long)B * T * Hq * D / 8;
   attn_bwd_dq_cast_kernel<D><<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(
