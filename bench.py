@@ -182,7 +182,7 @@ def run_gpu(args, rank, world, local):
                       lse=torch.empty((B, Hq, T), device=dev, dtype=torch.float32),
                       dqh=torch.empty_like(q), dkh=torch.empty_like(k), dv=torch.empty_like(v),
                       dq=torch.empty_like(q), dk=torch.empty_like(k),
-                      ws=torch.empty(cswa.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D), device=dev,
+                      ws=torch.empty(cswa.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, W), device=dev,
                                      dtype=torch.uint8)))
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     per_op = {"prologue": 0.0, "fwd": 0.0, "bwd": 0.0, "prologue_bwd": 0.0}
@@ -265,7 +265,7 @@ def run_gpu(args, rank, world, local):
                      "peak_kind": f"bf16 sustained ({pk_src}); burst {peak_burst}",
                      "traffic": traffic,
                      "algorithmic_flops_per_launch": flops_b / 2},
-        "gpu_launches": 12 * args.steps,
+        "gpu_launches": 12 * args.steps,  # per layer: prologue, fwd, bwd prep/main/dq, prologue bwd
         "clocks": clocks.summary(),
     }
     if rank == 0 and not args.no_decode:

@@ -36,7 +36,7 @@ _SIGS = {
     "attn_rope_qknorm": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _f, _vp]),
     "attn_rope_qknorm_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _f, _vp]),
     "attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp]),
-    "attn_bwd_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
+    "attn_bwd_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "attn_bwd": (_i, [_vp] * 9 + [_vp, _sz, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "attn_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "attn_decode": (_i, [_vp] * 8 + [_i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
@@ -147,8 +147,8 @@ def attn_fwd(q, k, v, window=-1, scale=None, o=None, lse=None, stream=None):
     return o, lse
 
 
-def attn_bwd_workspace_bytes(B, T, Hq, Hkv, D):
-    return int(lib().attn_bwd_workspace_bytes(B, T, Hq, Hkv, D))
+def attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, window=-1):
+    return int(lib().attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, int(window)))
 
 
 def attn_bwd(q, k, v, o, dout, lse, window=-1, scale=None, dq=None, dk=None, dv=None, workspace=None,
@@ -161,7 +161,7 @@ def attn_bwd(q, k, v, o, dout, lse, window=-1, scale=None, dq=None, dk=None, dv=
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    nbytes = attn_bwd_workspace_bytes(B, T, Hq, Hkv, D)
+    nbytes = attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, window)
     if workspace is None:
         workspace = torch.empty(nbytes, device=q.device, dtype=torch.uint8)
     _check("attn_bwd", lib().attn_bwd(

@@ -50,6 +50,20 @@ bool encode_bthd(CUtensorMap* m, const void* base, int B, int T, int H, int D, i
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The stored dS^T tiles: a (rows, 128) bf16 matrix, box = 64 columns x 128 rows,
+// 128-byte swizzle (the shared-memory layout of one 64-query panel).
+bool encode_ds_tiles(CUtensorMap* m, const void* base, long long rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {256};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool dims_ok(int B, int T, int Hq, int Hkv) {
   return B >= 1 && T >= 1 && Hq >= 1 && Hkv >= 1 && Hq % Hkv == 0 && (long long)B * T * Hq < (1ll << 40);
@@ -139,38 +153,59 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, f
 }
 
 struct BwdWorkspace {
-  float* dq_acc;  // (B, Hq, Tpad, D)
-  float* lse2;    // (B, Hq, Tpad)
-  float* delta;   // (B, Hq, Tpad)
+  float* lse2;            // (B, Hq, Tpad)
+  float* delta;           // (B, Hq, Tpad)
+  __nv_bfloat16* ds;      // stored dS^T tiles, 128 x 128 each
+  long long tiles_per_bh;
+  int span;
 };
-BwdWorkspace carve_bwd(void* ws, int B, int T, int Hq, int D) {
-  const size_t Tpad = (size_t)tiles128(T) * 128;
-  uint8_t* p = static_cast<uint8_t*>(ws);
+int eff_window(int window, int T) { return (window >= T) ? -1 : window; }
+BwdWorkspace carve_bwd(void* ws, int B, int T, int Hq, int window) {
+  const int nt = tiles128(T);
+  const size_t Tpad = (size_t)nt * 128;
   BwdWorkspace w;
-  w.dq_acc = reinterpret_cast<float*>(p);
-  p += align256((size_t)B * Hq * Tpad * D * 4);
+  w.span = bwd_span(nt, eff_window(window, T));
+  w.tiles_per_bh = ds_tiles_before(nt, nt, w.span);
+  uint8_t* p = static_cast<uint8_t*>(ws);
   w.lse2 = reinterpret_cast<float*>(p);
   p += align256((size_t)B * Hq * Tpad * 4);
   w.delta = reinterpret_cast<float*>(p);
+  p += align256((size_t)B * Hq * Tpad * 4);
+  w.ds = reinterpret_cast<__nv_bfloat16*>(p);
   return w;
+}
+size_t bwd_ws_bytes(int B, int T, int Hq, int window) {
+  const int nt = tiles128(T);
+  const size_t Tpad = (size_t)nt * 128;
+  const long long tiles = ds_tiles_before(nt, nt, bwd_span(nt, eff_window(window, T)));
+  return 2 * align256((size_t)B * Hq * Tpad * 4) + (size_t)B * Hq * tiles * 32768;
+}
+
+template <int D>
+bool set_dq_attr() {
+  static bool ok = cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        DqLayout<D>::kBytes) == cudaSuccess;
+  return ok;
 }
 
 template <int D>
 attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                          const float* lse, void* dq, void* dk, void* dv, void* ws, int B, int T, int Hq, int Hkv,
                          int window, float scale, cudaStream_t st) {
-  const int Tpad = tiles128(T) * 128;
-  BwdWorkspace w = carve_bwd(ws, B, T, Hq, D);
-  CUtensorMap tq, tk, tv, tdo;
+  const int nt = tiles128(T);
+  const int Tpad = nt * 128;
+  BwdWorkspace w = carve_bwd(ws, B, T, Hq, window);
+  CUtensorMap tq, tk, tv, tdo, tds;
   if (!encode_bthd(&tq, q, B, T, Hq, D) || !encode_bthd(&tk, k, B, T, Hkv, D) ||
-      !encode_bthd(&tv, v, B, T, Hkv, D) || !encode_bthd(&tdo, dO, B, T, Hq, D))
+      !encode_bthd(&tv, v, B, T, Hkv, D) || !encode_bthd(&tdo, dO, B, T, Hq, D) ||
+      !encode_ds_tiles(&tds, w.ds, (long long)B * Hq * w.tiles_per_bh * 128))
     return ATTN_ERR_LAUNCH;
-  if (!set_smem_attrs<D>()) return ATTN_ERR_LAUNCH;
+  if (!set_smem_attrs<D>() || !set_dq_attr<D>()) return ATTN_ERR_LAUNCH;
   {
     const long long threads = (long long)B * Tpad * Hq * (D / 8);
     attn_bwd_prep_kernel<D><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, w.lse2, w.delta,
-        w.dq_acc, B, T, Tpad, Hq);
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, w.lse2, w.delta, B, T,
+        Tpad, Hq);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
   }
   BwdParams p{};
@@ -178,21 +213,20 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
   p.delta = w.delta;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.dq = static_cast<__nv_bfloat16*>(dq);
   p.T = T;
   p.Tpad = Tpad;
   p.Hq = Hq;
   p.G = Hq / Hkv;
-  p.window = (window >= T) ? -1 : window;
-  p.n_kv_tiles = tiles128(T);
-  p.n_q_tiles = tiles128(T);
+  p.window = eff_window(window, T);
+  p.n_tiles = nt;
+  p.span = w.span;
+  p.tiles_per_bh = w.tiles_per_bh;
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
-  dim3 grid(Hkv, B, p.n_kv_tiles);
-  attn_bwd_kernel<D><<<grid, 384, BwdLayout<D>::kBytes, st>>>(tq, tk, tv, tdo, w.dq_acc, p);
+  attn_bwd_kernel<D><<<dim3(Hkv, B, nt), 384, BwdLayout<D>::kBytes, st>>>(tq, tk, tv, tdo, tds, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
-  const long long n8 = (long long)B * T * Hq * D / 8;
-  attn_bwd_dq_cast_kernel<D><<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(
-      w.dq_acc, static_cast<__nv_bfloat16*>(dq), T, Tpad, Hq, n8);
+  attn_bwd_dq_kernel<D><<<dim3(Hq, B, nt), 256, DqLayout<D>::kBytes, st>>>(tk, tds, p);
   return launched();
 }
 
@@ -239,10 +273,9 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
                  : launch_fwd<128>(q, k, v, o, lse, B, T, Hq, Hkv, window, scale, st);
 }
 
-size_t attn_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D) {
+size_t attn_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int window) {
   if (!dims_ok(B, T, Hq, Hkv) || (D != 64 && D != 128)) return 0;
-  const size_t Tpad = (size_t)tiles128(T) * 128;
-  return align256((size_t)B * Hq * Tpad * D * 4) + 2 * align256((size_t)B * Hq * Tpad * 4);
+  return bwd_ws_bytes(B, T, Hq, window);
 }
 
 attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
@@ -254,9 +287,12 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
   for (const void* ptr : ptrs)
     if (!ptr || !aligned16(ptr)) return ATTN_ERR_INVALID_ARG;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
-      ws_bytes < attn_bwd_workspace_bytes(B, T, Hq, Hkv, D))
+      ws_bytes < attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, window))
     return ATTN_ERR_INVALID_ARG;
-  if (Hkv > 65535 || B > 65535 || tiles128(T) > 65535) return ATTN_ERR_INVALID_ARG;
+  if (Hq > 65535 || B > 65535 || tiles128(T) > 65535) return ATTN_ERR_INVALID_ARG;
+  if ((long long)B * Hq * ds_tiles_before(tiles128(T), tiles128(T), bwd_span(tiles128(T), eff_window(window, T))) *
+          128 >= (1ll << 31))
+    return ATTN_ERR_UNSUPPORTED;  // stored dS^T rows are addressed with 32-bit TMA coordinates
   cudaStream_t st = as_stream(stream);
   return D == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, workspace, B, T, Hq, Hkv, window, scale, st)
                  : launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, workspace, B, T, Hq, Hkv, window, scale, st);

@@ -82,10 +82,12 @@ attn_status_t attn_rope_qknorm_bwd(const void* q, const void* k, const void* dq_
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T,
                        int Hq, int Hkv, int D, int window, float scale, void* stream);
 
-/* Bytes of workspace attn_bwd needs: an fp32 dQ accumulator (B,Hq,Tpad,D), the
- * per-row lse*log2(e) and Delta_i = dO_i . o_i (B,Hq,Tpad), Tpad = T rounded up
- * to a multiple of 128, each part 256-byte aligned. */
-size_t attn_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D);
+/* Bytes of workspace attn_bwd needs for this window: the per-row lse*log2(e) and
+ * Delta_i = dO_i . o_i (fp32, (B,Hq,Tpad), Tpad = T rounded up to a multiple of 128)
+ * and the bf16 dS^T tiles (128 x 128) of every (query tile, key tile) pair inside
+ * the causal window, kept between the main backward kernel and the dQ kernel:
+ * about B*Hq*T*min(T, W+128)*2 bytes for window W (B*Hq*T^2 without a window). */
+size_t attn_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int window);
 
 /*
  * attn_bwd -- gradients of sum(dO * o) for o = attn_fwd(q, k, v):
@@ -94,7 +96,9 @@ size_t attn_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D);
  * with dK, dV summed over the Hq/Hkv query heads of each KV head.
  * Inputs: q, k, v, o, dO (bf16) and lse (fp32) exactly as attn_fwd produced
  * them. Outputs dq (B,T,Hq,D), dk, dv (B,T,Hkv,D) bf16, fully overwritten.
- * workspace: device memory of ws_bytes >= attn_bwd_workspace_bytes(...).
+ * workspace: device memory, 256-byte aligned, of ws_bytes >=
+ * attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, window). Calls whose stored dS^T
+ * tiles would exceed 2^31 rows return ATTN_ERR_UNSUPPORTED.
  */
 attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                        const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B,

@@ -41,15 +41,20 @@ def test_status_strings(L):
 
 
 def test_bwd_workspace_size(L):
+    # lse*log2e and Delta (fp32, padded to 128-row tiles) + one 32 KB dS^T tile per
+    # (key tile, query tile) pair inside the window
     B, T, Hq, Hkv, D = 8, 2048, 10, 10, 128
-    dq = B * Hq * 2048 * D * 4
     rows = B * Hq * 2048 * 4
-    assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D) == dq + 2 * rows
-    # ragged T pads the per-row arrays to whole 128-row tiles
-    n = L.attn_bwd_workspace_bytes(1, 130, 2, 1, 64)
-    assert n == 2 * 256 * 64 * 4 + 2 * 2 * 256 * 4
-    assert L.attn_bwd_workspace_bytes(1, 16, 3, 2, 128) == 0     # Hq % Hkv != 0
-    assert L.attn_bwd_workspace_bytes(1, 16, 2, 2, 96) == 0      # head dim
+    # window 1024: key tile n sees min(16 - n, 9) query tiles -> 7*9 + (9+8+...+1) = 108
+    assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, 1024) == 2 * rows + B * Hq * 108 * 32768
+    # no window: the 16*17/2 = 136 tiles of the lower triangle; window >= T - 1 is the same
+    full = 2 * rows + B * Hq * 136 * 32768
+    assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, -1) == full
+    assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, 2048) == full
+    # ragged T pads the per-row arrays to whole 128-row tiles; window 0 keeps the diagonal only
+    assert L.attn_bwd_workspace_bytes(1, 130, 2, 1, 64, 0) == 2 * 2048 + 2 * 2 * 32768
+    assert L.attn_bwd_workspace_bytes(1, 16, 3, 2, 128, -1) == 0     # Hq % Hkv != 0
+    assert L.attn_bwd_workspace_bytes(1, 16, 2, 2, 96, -1) == 0      # head dim
 
 
 def test_decode_workspace_size(L):
@@ -80,7 +85,7 @@ def test_fwd_rejects_bad_args(L):
 
 
 def test_bwd_rejects_bad_args(L):
-    ws = L.attn_bwd_workspace_bytes(1, 128, 4, 2, 128)
+    ws = L.attn_bwd_workspace_bytes(1, 128, 4, 2, 128, 64)
     base = [P] * 9 + [P, ws, 1, 128, 4, 2, 128, 64, ctypes.c_float(0.1), None]
     def call(i, v):
         a = list(base)
