@@ -305,6 +305,7 @@ __global__ void __launch_bounds__(384, 1)
       const long long base = ((long long)b * p.Hq) * p.tiles_per_bh + ds_tiles_before(n, p.n_tiles, p.span);
       for (int it = 0; it < n_iters; ++it) {
         if (!mbar_wait(ds_full, it & 1, abort_flag)) break;
+        CSWA_MARK(3, it, 2);
         const int h = iter_head(it);
         const long long tile = base + (long long)h * p.tiles_per_bh + it % m_cnt;
         const int row = (int)(tile * 128);
@@ -312,13 +313,14 @@ __global__ void __launch_bounds__(384, 1)
         tma_store_2d(&tm_ds, smem + L::kDS + L::kPanel, 64, row);
         bulk_commit();
         bulk_wait_read<0>();
+        CSWA_MARK(3, it, 3);
         mbar_arrive(ds_free);
       }
       bulk_wait_all();
     }
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------ P and dS (thread = key row)
-    // warps 4-7 take query columns 0-63, warps 8-11 columns 64-127
+    // warps 4-7 take query columns 0-63, warps 8-11 columns 64-127 (warp 2 only allocates TMEM)
     const int half = (warp >= 8) ? 1 : 0;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
@@ -327,6 +329,7 @@ __global__ void __launch_bounds__(384, 1)
     const float sl2 = p.scale_log2;
     uint8_t* ds_row = smem + L::kDS + half * L::kPanel + r * 128;
     const bool tracer = (warp == 4 && lane == 0);
+    const bool tracer1 = (warp == 8 && lane == 0);
     bool ok = true;
     for (int it = 0; it < n_iters; ++it) {
       const int st = it & 1;
@@ -334,14 +337,27 @@ __global__ void __launch_bounds__(384, 1)
       const float* lse_s = s_lse + st * 128 + 64 * half;
       const float* dl_s = s_delta + st * 128 + 64 * half;
       if (tracer) CSWA_MARK(1, it, 0);
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag));
+      if (tracer1) CSWA_MARK(2, it, 0);
+      // the lse/Delta rows of this stage come from a bulk copy: acquire them from its
+      // own barrier (completion of S^T alone does not order that copy before our reads)
+      ok = __all_sync(0xffffffffu, mbar_wait(&qd_full[st], (it >> 1) & 1, abort_flag) &&
+                                       mbar_wait(s_full, it & 1, abort_flag));
       if (tracer) CSWA_MARK(1, it, 1);
+      if (tracer1) CSWA_MARK(2, it, 1);
       if (!ok) break;
       tc_fence_after();
       uint32_t sr[64];
       tmem_ld32(tR0 + lane_off + 64 * half + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
       tmem_ld32(tR0 + lane_off + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_ld_wait();
+      // debug dump layout: [it][half][r][kind][64]
+#define DBG_SLOT(kind, c) ((((it * 2 + half) * 128 + r) * 5 + (kind)) * 64 + (c))
+      if (it < 3) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) CSWA_DUMP(DBG_SLOT(0, c), __uint_as_float(sr[c]));
+#pragma unroll
+        for (int c = 0; c < 64; ++c) CSWA_DUMP(DBG_SLOT(1, c), lse_s[c]);
+      }
       const bool full = (k0 + 127 <= q0) && (W < 0 || q0 + 63 - k0 <= W);
       const int c_lo = j - q0;                      // query q0 + c sees key j iff c >= c_lo
       const int c_hi = (W < 0) ? 63 : j + W - q0;   //   and c <= c_hi
@@ -375,6 +391,7 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       if (tracer) CSWA_MARK(1, it, 6);
+      if (tracer1) CSWA_MARK(2, it, 6);
       // P^T of this warpgroup's 64 queries goes over the first half of its own S^T
       // columns (64*half .. 64*half+31), which only this warpgroup has read
       tmem_st32(tR0 + lane_off + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
@@ -382,12 +399,15 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before();
       mbar_arrive(p_full);
       if (tracer) CSWA_MARK(1, it, 2);
+      if (tracer1) CSWA_MARK(2, it, 2);
 
       ok = __all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, abort_flag));
       if (tracer) CSWA_MARK(1, it, 3);
+      if (tracer1) CSWA_MARK(2, it, 3);
       // dS^T of the previous step must have been read by dK and by its TMA store
       if (ok && it > 0) ok = __all_sync(0xffffffffu, mbar_wait(ds_free, (it - 1) & 1, abort_flag));
       if (tracer) CSWA_MARK(1, it, 4);
+      if (tracer1) CSWA_MARK(2, it, 4);
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
@@ -396,6 +416,18 @@ __global__ void __launch_bounds__(384, 1)
         tmem_ld32(tR1 + lane_off + 64 * half + cc * 32, dp);
         tmem_ld_wait();
         const float4* dl4 = reinterpret_cast<const float4*>(dl_s + cc * 32);
+        if (it < 3) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) CSWA_DUMP(DBG_SLOT(2, cc * 32 + e), __uint_as_float(dp[e]));
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sr[cc * 16 + e]));
+            CSWA_DUMP(DBG_SLOT(3, cc * 32 + 2 * e), pp.x);
+            CSWA_DUMP(DBG_SLOT(3, cc * 32 + 2 * e + 1), pp.y);
+          }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) CSWA_DUMP(DBG_SLOT(4, cc * 32 + e), dl_s[cc * 32 + e]);
+        }
         uint32_t w[16];
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
@@ -419,6 +451,7 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before();
       mbar_arrive(ds_full);
       if (tracer) CSWA_MARK(1, it, 5);
+      if (tracer1) CSWA_MARK(2, it, 5);
     }
     // ---------------------------------------------------------- dK (warps 4-7) / dV (8-11) epilogue
     ok = __all_sync(0xffffffffu, ok && mbar_wait(final_bar, 0, abort_flag));

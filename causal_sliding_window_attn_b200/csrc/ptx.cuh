@@ -24,7 +24,16 @@ __device__ unsigned long long g_trace[64 * 4 * 64 * 8];
     if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z < 64 && (it) < 64)                           \
       g_trace[((blockIdx.z * 4 + (role)) * 64 + (it)) * 8 + (tag)] = clock64();                       \
   } while (0)
+// value dumps for debugging builds: g_dbg[slot] = v (first CTA only)
+__device__ float g_dbg[1 << 20];
+#define CSWA_DUMP(slot, v)                                                                              \
+  do {                                                                                                \
+    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (slot) < (1 << 20)) g_dbg[slot] = (v); \
+  } while (0)
 #else
+#define CSWA_DUMP(slot, v) \
+  do {                     \
+  } while (0)
 #define CSWA_MARK(role, it, tag) \
   do {                           \
   } while (0)
