@@ -40,6 +40,7 @@ _SIGS = {
     "attn_bwd": (_i, [_vp] * 9 + [_vp, _sz, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "attn_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "attn_decode": (_i, [_vp] * 8 + [_i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
+    "attn_decode_noalloc": (_i, [_vp] * 8 + [_i, _i, _i, _i, _i, _i, _f, _vp]),
     "attn_get_status": (_i, [_vp]),
     "attn_status_string": (ctypes.c_char_p, [_i]),
     "attn_device_supported": (_i, []),

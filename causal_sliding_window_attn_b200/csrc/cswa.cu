@@ -245,6 +245,32 @@ int decode_chunks(int Tmax, int window) {
   return (span + kDecodeChunk - 1) / kDecodeChunk;
 }
 
+// ---------------------------------------------------------------- no-allocation decode
+// Scratch for attn_decode_noalloc: the split-K partials live in this file-scope
+// device array instead of a caller-provided workspace. Every GPU that loads the
+// library holds it (kNoAllocScratchFloats * 4 bytes) until the process exits.
+constexpr size_t kNoAllocScratchFloats = size_t(1) << 20;  // 4 MiB
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+
+// The device address of g_noalloc_scratch, looked up once per device with that
+// device current (host code only sees a stand-in symbol, never the address).
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+attn_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_LAUNCH;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return ATTN_ERR_LAUNCH;
+    g_noalloc_addr[dev] = ptr;
+  }
+  *out = g_noalloc_addr[dev];
+  return ATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -353,6 +379,22 @@ attn_status_t attn_decode(const void* q, void* kcache, void* vcache, const void*
     case 4: return launch_decode<128, 4>(p, B, st);
     default: return launch_decode<128, 8>(p, B, st);
   }
+}
+
+// attn_decode without a workspace argument: the split-K partials go to the
+// library's own device scratch (see cswa_attn.h for who needs this and the limits).
+attn_status_t attn_decode_noalloc(const void* q, void* kcache, void* vcache, const void* k_new, const void* v_new,
+                                  const int32_t* pos, void* o, float* lse, int B, int Tmax, int Hq, int Hkv, int D,
+                                  int window, float scale, void* stream) {
+  const size_t need = attn_decode_workspace_bytes(B, Hq, D, Tmax, window);
+  if (need == 0) return ATTN_ERR_INVALID_ARG;
+  if (need > kNoAllocScratchFloats * sizeof(float)) return ATTN_ERR_INVALID_ARG;  // beyond the fixed scratch
+  void* scratch = nullptr;
+  const attn_status_t st = noalloc_scratch(&scratch);
+  if (st != ATTN_OK) return st;
+  // every partial the combine step reads is written earlier in the same call: nothing to clear
+  return attn_decode(q, kcache, vcache, k_new, v_new, pos, o, lse, B, Tmax, Hq, Hkv, D, window, scale, scratch, need,
+                     stream);
 }
 
 attn_status_t attn_get_status(void* stream) {

@@ -126,6 +126,37 @@ attn_status_t attn_decode(const void* q, void* kcache, void* vcache, const void*
                           const int32_t* pos, void* o, float* lse, int B, int Tmax, int Hq, int Hkv, int D,
                           int window, float scale, void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * attn_decode_noalloc -- attn_decode for callers that cannot allocate device memory.
+ * (This entry point has no counterpart on the pages: it is a packaging variant.)
+ *
+ * Some callers have no way to hand this library a workspace: code that runs
+ * inside a framework whose allocator it cannot reach, a serving loop that is
+ * not allowed to allocate once it has started, or a host program linked only
+ * against this C ABI. This call computes exactly what attn_decode computes
+ * (same arguments minus the workspace) but keeps the split-K partials in a
+ * fixed scratch array that the library itself holds in device memory.
+ *
+ *   - Limit: the partials of one call, attn_decode_workspace_bytes(B, Hq, D,
+ *     Tmax, window), must fit in the fixed 4 MiB scratch (4194304 bytes; e.g.
+ *     32 sequences x 16 query heads at window 1024 and D = 128 need 2.4 MB).
+ *     Larger calls return ATTN_ERR_INVALID_ARG and enqueue nothing.
+ *   - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ *     The scratch is a file-scope __device__ array, so every GPU that loads the
+ *     library holds those 4 MiB until the process exits.
+ *   - The first call on a device looks the scratch's device address up (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - All calls on a device share the one scratch, which keeps the last call's
+ *     contents. Calls whose kernels overlap on the GPU (different streams, no
+ *     ordering between them) race on it and give undefined results; calls on
+ *     one stream are safe. No part of it needs to start at zero: every partial
+ *     a call reads is written earlier in that same call.
+ */
+attn_status_t attn_decode_noalloc(const void* q, void* kcache, void* vcache, const void* k_new, const void* v_new,
+                                  const int32_t* pos, void* o, float* lse, int B, int Tmax, int Hq, int Hkv, int D,
+                                  int window, float scale, void* stream);
+
 /* Synchronises `stream`, then returns and clears the device status word of the
  * current device: ATTN_OK, ATTN_ERR_TIMEOUT or ATTN_ERR_DEVICE (or
  * ATTN_ERR_LAUNCH if a CUDA error is pending). */
