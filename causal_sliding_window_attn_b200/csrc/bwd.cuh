@@ -9,43 +9,53 @@
 // dK and dV of a KV head summed over its G = Hq/Hkv query heads.
 //
 // Three kernels:
-//   bwd_prep     Delta_i and lse_i * log2(e) per row into the workspace
-//                (padded to 128-row tiles with Delta = 0, lse = +inf so padded
-//                rows get P = 0).
+//   bwd_prep     per query row, -lse_i/scale and -Delta_i as bf16 hi + lo pairs,
+//                laid out as one extra K = 16 step of an MMA (padded rows: a
+//                large negative lse term, so P = 0 there).
 //   bwd_main     one CTA per (128-key tile, KV head, batch). K and V stay in
 //                shared memory; the CTA walks every (query head of the group,
-//                128-row query tile) that sees the key tile. Per step, all
-//                MMAs M = 128, N = 128 (the shape the tensor pipe runs at full
-//                rate), TMEM regions R0, R1 of 128 columns each:
-//                  S^T  = K Q^T         (SS)  -> R0
-//                  P^T  = exp2(S^T c - lse)     bf16 back over the S^T it came from
-//                  dV  += P^T dO        (TS)  -> TMEM [256,256+D)
-//                  dP^T = V dO^T        (SS)  -> R1
-//                  dS^T = P^T (dP^T - Delta)    bf16 into shared memory
-//                  dK  += dS^T Q        (SS)  -> TMEM [256+D,256+2D)
-//                and the dS^T tile goes to the workspace with one TMA store.
-//                Two warpgroups split the elementwise work by query columns.
-//                dK, dV are complete in the CTA (the whole group is walked
-//                here), so they are written once, as bf16, with no atomics.
+//                128-row query tile) that sees the key tile, with Q and dO in
+//                rings of 3 and 2 stages. Per step, all MMAs M = 128, N = 128 (the
+//                shape the tensor pipe runs at full rate), TMEM regions R0, R1 of
+//                128 columns each:
+//                  S^T' = K Q^T - lse/scale     (SS, + extension step) -> R0
+//                  P^T  = exp2(c S^T')          bf16 pairs written over R0
+//                  dV  += P^T dO                (TS: A from TMEM) -> [256,256+D)
+//                  dP^T'= V dO^T - Delta        (SS, + extension step) -> R1
+//                  dS^T = P^T dP^T'             bf16 pairs written over R1
+//                  dK  += dS^T Q                (TS) -> [256+D,256+2D)
+//                The extension step adds the per-query terms inside the MMA, so
+//                the elementwise warps read no per-column statistics at all.
+//                The MMA warp issues dV(it) + S^T(it+1) and dK(it) + dP^T(it+1)
+//                as bursts, so S^T and dP^T of the next step are computed while
+//                the elementwise warps work on this one. dS^T leaves as bf16
+//                tiles for bwd_dq (plain 512-byte coalesced stores). dK, dV are
+//                complete in the CTA (the whole group is walked here), so they
+//                are written once, as bf16, with no atomics.
 //   bwd_dq       one CTA per (128-row query tile, query head, batch):
 //                dQ = scale * sum over key tiles of dS K, accumulated in TMEM
-//                from the stored dS^T tiles and K tiles, written once as bf16.
-// Splitting dQ out keeps the per-step fp32 reductions of dQ out of the main
-// kernel's load/store pipe, which its elementwise warps need.
-// Warp roles in bwd_main: 0 TMA, 1 MMA issuer, 2 TMEM allocator, 3 dS store,
-// 4-7 and 8-11 P/dS (thread = key row; columns 0-63 and 64-127), then the
-// dK and dV epilogues.
+//                from the stored dS^T tiles (one bulk copy each) and K tiles,
+//                written once as bf16.
+// Splitting dQ out keeps fp32 dQ reductions out of the main kernel, whose
+// TMEM (512 columns) and shared memory are fully used.
+// Warp roles in bwd_main: 0 TMA (K, V, Q ring), 1 MMA issuer (whole warp, one
+// elected lane issues), 2 TMEM allocator, 3 TMA (dO ring), 4-7 and 8-11 P/dS
+// (thread = key row; query columns 0-63 and 64-127), then the dK and dV epilogues.
 #pragma once
 #include "ptx.cuh"
 
 namespace cswa {
 
 struct BwdParams {
-  const float* lse2;   // (B, Hq, Tpad): lse * log2(e), +inf on padded rows
-  const float* delta;  // (B, Hq, Tpad)
+  // per (batch, query head, 128-row query tile): 512 bytes holding -lse/scale and
+  // -Delta of the tile's rows as bf16 hi + lo pairs, laid out as the extra K = 16 step
+  // of the S^T and dP^T MMAs reads them (see attn_bwd_prep_kernel)
+  const uint8_t* ext_lse;
+  const uint8_t* ext_delta;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   __nv_bfloat16* dq;
+  __nv_bfloat16* ds;   // stored dS^T tiles: 128 key rows x 128 query columns each, row-major
   int T, Tpad, Hq, G, window, n_tiles, span;  // tiles of 128 rows; span = query tiles per key tile
   long long tiles_per_bh;                     // stored dS^T tiles per (batch, query head)
   float scale, scale_log2;
@@ -56,6 +66,14 @@ struct BwdParams {
 // one (batch, head) are stored key tile by key tile; this is where key tile n starts.
 __host__ __device__ inline int bwd_span(int n_tiles, int window) {
   return window < 0 ? n_tiles : min(n_tiles, (127 + window) / 128 + 1);
+}
+// Byte offset, inside one stored 32 KB dS^T tile, of the 16-byte unit holding
+// queries 8u .. 8u+7 (u in 0..15) of key row r: 8 KB per 32 keys, 512 bytes per 8
+// queries, 16 bytes per key. A warp of 32 key rows thus writes 512 contiguous bytes
+// per unit index, and the tile is the no-swizzle MN-major operand layout of the dQ
+// MMA (core matrices of 8 keys x 8 queries: 128 bytes along K, 512 bytes along M).
+__host__ __device__ inline uint32_t ds_unit_offset(int r, int u) {
+  return (uint32_t)((r >> 5) * 8192 + u * 512 + (r & 31) * 16);
 }
 __host__ __device__ inline long long ds_tiles_before(int n, int n_tiles, int span) {
   const int a = max(0, n_tiles - span);  // key tiles whose whole span fits
@@ -71,49 +89,21 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
-// 2-D tiled reduce-add shared -> global (fp32 add in L2), bulk-group completion.
-__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* m, const void* src, int c0, int c1) {
-  asm volatile(
-      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(m)),
-      "r"(smem_u32(src)), "r"(c0), "r"(c1)
-      : "memory");
-}
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int c0, int c1) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                   reinterpret_cast<uint64_t>(m)),
-               "r"(smem_u32(src)), "r"(c0), "r"(c1)
-               : "memory");
-}
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uint64_t* bar, int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::
-          "r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void named_barrier_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 template <int D>
 struct BwdLayout {
+  static constexpr int kQStages = 3, kDOStages = 2;
   static constexpr int kTile = 128 * D * 2;   // one 128-row bf16 tile (K, V, Q or dO)
   static constexpr int kPanel = 128 * 128;    // one 64-column panel of a 128-row tile
   static constexpr int kK = 0;
   static constexpr int kV = kK + kTile;
-  static constexpr int kQ = kV + kTile;       // [2]
-  static constexpr int kDO = kQ + 2 * kTile;  // [2]
-  static constexpr int kDS = kDO + 2 * kTile; // dS^T: 128 keys x 128 queries bf16, 2 panels
-  static constexpr int kStat = kDS + 2 * kPanel;  // lse2[2][128], delta[2][128]
-  static constexpr int kBar = kStat + 2048;
-  static constexpr int kUsed = kBar + 256;
+  static constexpr int kQ = kV + kTile;                    // [kQStages]
+  static constexpr int kDO = kQ + kQStages * kTile;        // [kDOStages]
+  // per-row extension slots (512 bytes, see the prep kernel) of the Q stages, then of
+  // the dO stages, then the constant key-side extension (a core of ones, a core of zeros)
+  static constexpr int kExt = kDO + kDOStages * kTile;
+  static constexpr int kExtOnes = kExt + (kQStages + kDOStages) * 512;
+  static constexpr int kBar = kExtOnes + 256;
+  static constexpr int kUsed = kBar + 192;
   static constexpr int kBytes = (kUsed + 1024 <= 232448) ? kUsed + 1024 : 232448;
   static_assert(kUsed <= 232448, "shared memory budget");
   static constexpr uint32_t kTmemCols = 512;
@@ -123,8 +113,9 @@ template <int D>
 __global__ void __launch_bounds__(384, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const __grid_constant__ CUtensorMap tm_ds, const BwdParams p) {
+                    const BwdParams p) {
   using L = BwdLayout<D>;
+  constexpr int QS = L::kQStages, DS = L::kDOStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // the layout needs a 1024-byte aligned base: report (never overrun) if the slack is too small
@@ -134,22 +125,25 @@ __global__ void __launch_bounds__(384, 1)
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* kv_full = bars + 0;
-  uint64_t* qd_full = bars + 1;   // [2]
-  uint64_t* qd_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;
-  uint64_t* p_full = bars + 6;
-  uint64_t* dv_done = bars + 7;
-  uint64_t* dp_full = bars + 8;
-  uint64_t* ds_full = bars + 9;
-  uint64_t* ds_free = bars + 10;
-  uint64_t* final_bar = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 13);
-  float* s_lse = reinterpret_cast<float*>(smem + L::kStat);           // [2][128]
-  float* s_delta = reinterpret_cast<float*>(smem + L::kStat + 1024);  // [2][128]
+  uint64_t* q_full = bars + 1;                 // [QS]
+  uint64_t* q_empty = q_full + QS;             // [QS]  dK has read the Q tile
+  uint64_t* do_full = q_empty + QS;            // [DS]
+  uint64_t* do_empty = do_full + DS;           // [DS]  dV has read the dO tile
+  uint64_t* s_full = do_empty + DS;            // S^T in TMEM
+  uint64_t* p_full = s_full + 1;               // P^T written over S^T
+  uint64_t* dp_full = p_full + 1;              // dP^T in TMEM
+  uint64_t* ds_full = dp_full + 1;             // dS^T written over dP^T
+  uint64_t* final_bar = ds_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(final_bar + 2);
+#ifdef CSWA_TRACE
+  uint64_t* trace_bar = final_bar + 3;  // [4] completion of dV, S, dK, dP groups (profiling builds)
+#endif
 
   const int warp = warp_id(), lane = lane_id();
-  const int hk = blockIdx.x, b = blockIdx.y, n = blockIdx.z;
+  // key tiles of one (b, KV head) are adjacent in launch order, so the CTAs that read
+  // the same Q/dO tiles run together and share them through L2
+  const int n = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int W = p.window, G = p.G;
   const int k0 = n * 128;
   const int m_cnt = min(p.n_tiles - n, p.span);
@@ -157,17 +151,22 @@ __global__ void __launch_bounds__(384, 1)
 
   if (warp == 0 && lane == 0) {
     mbar_init(kv_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&qd_full[s], 1);
-      mbar_init(&qd_empty[s], 1);
+    for (int s = 0; s < QS; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+    }
+    for (int s = 0; s < DS; ++s) {
+      mbar_init(&do_full[s], 1);
+      mbar_init(&do_empty[s], 1);
     }
     mbar_init(s_full, 1);
     mbar_init(p_full, 256);
-    mbar_init(dv_done, 1);
     mbar_init(dp_full, 1);
     mbar_init(ds_full, 256);
-    mbar_init(ds_free, 2);  // dK has read dS^T (MMA commit) + the TMA store has read it
     mbar_init(final_bar, 1);
+#ifdef CSWA_TRACE
+    for (int i = 0; i < 4; ++i) mbar_init(&trace_bar[i], 1);
+#endif
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -176,148 +175,180 @@ __global__ void __launch_bounds__(384, 1)
     tmem_relinquish();
     tc_fence_before();
   }
+  if (warp == 3) {
+    // Extension slots start at zero (an MMA reads up to 96 bytes past a slot, into
+    // the next one or the constant cores, always multiplied by zero: those bytes must
+    // hold finite values even before the first copy lands). The constant key-side
+    // cores: rows of (1, 1, 0, 0, 0, 0, 0, 0), then zeros.
+    uint32_t* e = reinterpret_cast<uint32_t*>(smem + L::kExt);
+    for (int i = lane; i < (L::kExtOnes - L::kExt) / 4; i += 32) e[i] = 0u;
+    uint32_t* ones = reinterpret_cast<uint32_t*>(smem + L::kExtOnes);
+    for (int i = lane; i < 64; i += 32) ones[i] = (i < 32 && (i & 3) == 0) ? 0x3F803F80u : 0u;
+    fence_proxy_async_smem();
+  }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // R0: S^T, then P^T (bf16) in columns 0-31 and 64-95; R1: dP^T
+  // S^T (P^T packed over it), dP^T (dS^T packed over it), dV, dK
   const uint32_t tR0 = tmem, tR1 = tmem + 128, tdV = tmem + 256, tdK = tmem + 256 + D;
 
   const uint32_t sbase = smem_u32(smem);
   auto iter_head = [&](int it) { return hk * G + it / m_cnt; };
   auto iter_q0 = [&](int it) { return (n + it % m_cnt) * 128; };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || warp == 3) {
+    // ------------------------------------------------------------ producers
+    // warp 0: K, V and the Q ring; warp 3: the dO ring (its stages free up at a
+    // different point of the step, so it waits on its own). Each stage also takes
+    // the 512-byte row extension of its tile: -lse/scale with Q, -Delta with dO.
     if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      tma_prefetch_desc(&tm_do);
-      mbar_arrive_expect_tx(kv_full, 2 * L::kTile);
-      for (int pn = 0; pn < D / 64; ++pn) {
-        tma_load_4d(smem + L::kK + pn * L::kPanel, &tm_k, kv_full, pn * 64, hk, k0, b);
-        tma_load_4d(smem + L::kV + pn * L::kPanel, &tm_v, kv_full, pn * 64, hk, k0, b);
-      }
-      int last_issue[2] = {-1, -1};
-      for (int it = 0; it < n_iters; ++it) {
-        const int st = it & 1;
-        const int h = iter_head(it), q0 = iter_q0(it);
-        CSWA_MARK(3, it, 0);
-        if (!mbar_wait(&qd_empty[st], ((it >> 1) & 1) ^ 1, abort_flag)) break;
-        CSWA_MARK(3, it, 1);
-        mbar_arrive_expect_tx(&qd_full[st], 2 * L::kTile + 1024);
+      const bool qside = (warp == 0);
+      const int nst = qside ? QS : DS;
+      int last_issue[3] = {-1, -1, -1};
+      if (qside) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        mbar_arrive_expect_tx(kv_full, 2 * L::kTile);
         for (int pn = 0; pn < D / 64; ++pn) {
-          tma_load_4d(smem + L::kQ + st * L::kTile + pn * L::kPanel, &tm_q, &qd_full[st], pn * 64, h, q0, b);
-          tma_load_4d(smem + L::kDO + st * L::kTile + pn * L::kPanel, &tm_do, &qd_full[st], pn * 64, h, q0, b);
+          tma_load_4d(smem + L::kK + pn * L::kPanel, &tm_k, kv_full, pn * 64, hk, k0, b);
+          tma_load_4d(smem + L::kV + pn * L::kPanel, &tm_v, kv_full, pn * 64, hk, k0, b);
         }
-        const size_t row0 = ((size_t)b * p.Hq + h) * p.Tpad + q0;
-        bulk_load(s_lse + st * 128, p.lse2 + row0, 512, &qd_full[st]);
-        bulk_load(s_delta + st * 128, p.delta + row0, 512, &qd_full[st]);
+      } else {
+        tma_prefetch_desc(&tm_do);
+      }
+      uint64_t* full = qside ? q_full : do_full;
+      uint64_t* empty = qside ? q_empty : do_empty;
+      const CUtensorMap* tm = qside ? &tm_q : &tm_do;
+      const int base = qside ? L::kQ : L::kDO;
+      const uint8_t* ext = qside ? p.ext_lse : p.ext_delta;
+      uint8_t* ext_slot = smem + L::kExt + (qside ? 0 : QS * 512);
+      for (int it = 0; it < n_iters; ++it) {
+        const int st = it % nst;
+        const int h = iter_head(it), q0 = iter_q0(it);
+        if (qside) CSWA_MARK(3, it, 0);
+        if (!mbar_wait(&empty[st], ((it / nst) & 1) ^ 1, abort_flag)) break;
+        if (qside) CSWA_MARK(3, it, 1);
+        mbar_arrive_expect_tx(&full[st], L::kTile + 512);
+        for (int pn = 0; pn < D / 64; ++pn)
+          tma_load_4d(smem + base + st * L::kTile + pn * L::kPanel, tm, &full[st], pn * 64, h, q0, b);
+        bulk_load(ext_slot + st * 512, ext + (((size_t)b * p.Hq + h) * p.n_tiles + q0 / 128) * 512, 512, &full[st]);
         last_issue[st] = it;
       }
       if (*abort_flag) {
+        // let every copy in flight land before the CTA's shared memory is released
         volatile int dummy = 0;
-        for (int st = 0; st < 2; ++st)
-          if (last_issue[st] >= 0) mbar_wait(&qd_full[st], (last_issue[st] >> 1) & 1, &dummy);
-        mbar_wait(kv_full, 0, &dummy);
+        for (int s = 0; s < nst; ++s)
+          if (last_issue[s] >= 0) mbar_wait(&full[s], (last_issue[s] / nst) & 1, &dummy);
+        if (qside) mbar_wait(kv_full, 0, &dummy);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idSP = idesc_bf16(128, 128, false, false);  // S^T, dP^T
-      constexpr uint32_t idKV = idesc_bf16(128, D, false, true);     // dV (TS), dK: B MN-major
-      // Descriptors are built once; an MMA only adds (byte offset >> 4) to the start field.
-      const uint64_t dK_k = sdesc_sw128(sbase + L::kK, 16, 1024), dV_k = sdesc_sw128(sbase + L::kV, 16, 1024);
-      const uint64_t dQ_k = sdesc_sw128(sbase + L::kQ, 16, 1024), dDO_k = sdesc_sw128(sbase + L::kDO, 16, 1024);
-      const uint64_t dQ_mn = sdesc_sw128(sbase + L::kQ, L::kPanel, 1024);
-      const uint64_t dDO_mn = sdesc_sw128(sbase + L::kDO, L::kPanel, 1024);
-      const uint64_t dDS_k = sdesc_sw128(sbase + L::kDS, 16, 1024);
-      // step it reads Q/dO stage it & 1
-      auto issue_S = [&](int it) {
-        const uint32_t qo = (it & 1) * L::kTile;
+    // The whole warp runs the loop (descriptors stay warp-uniform); one elected lane
+    // issues the MMAs and commits.
+    const uint32_t leader = elect_one();
+    constexpr uint32_t idSP = idesc_bf16(128, 128, false, false);  // S^T, dP^T
+    constexpr uint32_t idKV = idesc_bf16(128, D, false, true);     // dV, dK: A from TMEM, B MN-major
+    // Descriptors are built once; an MMA only adds (byte offset >> 4) to the start field.
+    const uint64_t dK_k = sdesc_sw128(sbase + L::kK, 16, 1024), dV_k = sdesc_sw128(sbase + L::kV, 16, 1024);
+    const uint64_t dQ_k = sdesc_sw128(sbase + L::kQ, 16, 1024), dDO_k = sdesc_sw128(sbase + L::kDO, 16, 1024);
+    const uint64_t dQ_mn = sdesc_sw128(sbase + L::kQ, L::kPanel, 1024);
+    const uint64_t dDO_mn = sdesc_sw128(sbase + L::kDO, L::kPanel, 1024);
+    // The extra K = 16 step: A = rows of (1, 1, 0, ..., 0) for every key (one core
+    // repeated along M: stride 0; the second K core is the zero core), B = the slot's
+    // (hi, lo) rows, MN-major, 32 bytes per 8 queries. B's K rows 2..15 are multiplied
+    // by zeros (the second K core repeats the first: stride 0).
+    constexpr uint32_t idX = idesc_bf16(128, 128, false, true);
+    const uint64_t dOnes = sdesc_noswz(sbase + L::kExtOnes, 128, 0);
+    const uint64_t dX = sdesc_noswz(sbase + L::kExt, 0, 32);
+    // S^T' = K Q^T - lse/scale and dP^T' = V dO^T - Delta: A = K or V, B = Q or dO, both
+    // K-major over d, then the extension step with slot xslot
+    auto issue_R = [&](uint32_t dst, uint64_t dA, uint64_t dB, uint32_t boff, int xslot, uint64_t* done) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kPanel + (kk & 3) * 32;
-          mma_ss(tR0, dK_k + (off >> 4), dQ_k + ((qo + off) >> 4), idSP, kk > 0);
-        }
-        mma_commit(s_full);
-      };
-      auto issue_dP = [&](int it) {
-        const uint32_t qo = (it & 1) * L::kTile;
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * L::kPanel + (kk & 3) * 32;
+        mma_ss(dst, dA + (off >> 4), dB + ((boff + off) >> 4), idSP, kk > 0, leader);
+      }
+      mma_ss(dst, dOnes, dX + ((xslot * 512) >> 4), idX, 1, leader);
+      mma_commit(done, leader);
+    };
+    // dV += P^T dO and dK += dS^T Q: A = the bf16 pairs packed over S^T / dP^T (queries
+    // 0-63 in columns 0-31, 64-127 in columns 64-95), B = dO or Q, MN-major
+    auto issue_acc = [&](uint32_t dst, uint32_t a_tmem, uint64_t dB, uint32_t boff, bool first) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kPanel + (kk & 3) * 32;
-          mma_ss(tR1, dV_k + (off >> 4), dDO_k + ((qo + off) >> 4), idSP, kk > 0);
-        }
-        mma_commit(dp_full);
-      };
-      bool ok = mbar_wait(kv_full, 0, abort_flag) && mbar_wait(&qd_full[0], 0, abort_flag);
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ts(dst, a_tmem + (kk >> 2) * 64 + (kk & 3) * 8, dB + ((boff + kk * 2048) >> 4), idKV,
+               (!first || kk > 0), leader);
+    };
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+    };
+    bool ok = wait_all(kv_full, 0) && wait_all(&q_full[0], 0);
+    tc_fence_after();
+    if (ok) issue_R(tR0, dK_k, dQ_k, 0, 0, s_full);
+    ok = ok && wait_all(&do_full[0], 0);
+    tc_fence_after();
+    if (ok) issue_R(tR1, dV_k, dDO_k, 0, QS, dp_full);
+    const bool tracer = (lane == 0);
+    (void)tracer;
+    // Each step issues two bursts, each preceded by all of its waits (a barrier wait
+    // between two groups would let the tensor pipe run dry): dV(it) + S^T(it+1) once
+    // P^T(it) is written, dK(it) + dP^T(it+1) once dS^T(it) is written.
+    for (int it = 0; ok && it < n_iters; ++it) {
+      const int qs = it % QS, ds = it % DS;
+      const int q1 = (it + 1) % QS, d1 = (it + 1) % DS;
+      const bool more = it + 1 < n_iters;
+      if (tracer) CSWA_MARK(0, it, 0);
+      if (more && !(ok = wait_all(&q_full[q1], ((it + 1) / QS) & 1))) break;
+      if (!(ok = wait_all(p_full, it & 1))) break;
+      if (tracer) CSWA_MARK(0, it, 1);
       tc_fence_after();
-      if (ok && n_iters > 0) {
-        issue_S(0);
-        issue_dP(0);
-      }
-      for (int it = 0; ok && it < n_iters; ++it) {
-        const int st = it & 1;
-        const uint32_t qo = st * L::kTile;
-        CSWA_MARK(0, it, 0);
-        if (!(ok = mbar_wait(p_full, it & 1, abort_flag))) break;
-        CSWA_MARK(0, it, 1);
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // P^T of queries 16kk..16kk+15: columns 64*(kk/4) + 8*(kk%4)
-          mma_ts(tdV, tR0 + (kk >> 2) * 64 + (kk & 3) * 8, dDO_mn + ((qo + kk * 2048) >> 4), idKV,
-                 (it > 0 || kk > 0));
-        mma_commit(dv_done);
-        if (it + 1 < n_iters) {
-          // S^T of the next step overwrites P^T: wait until dV has read it
-          if (!(ok = mbar_wait(&qd_full[st ^ 1], ((it + 1) >> 1) & 1, abort_flag))) break;
-          if (!(ok = mbar_wait(dv_done, it & 1, abort_flag))) break;
-          tc_fence_after();
-          issue_S(it + 1);
-          CSWA_MARK(0, it, 2);
-        }
-        if (!(ok = mbar_wait(ds_full, it & 1, abort_flag))) break;
-        CSWA_MARK(0, it, 3);
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tdK, dDS_k + (((kk >> 2) * L::kPanel + (kk & 3) * 32) >> 4), dQ_mn + ((qo + kk * 2048) >> 4),
-                 idKV, (it > 0 || kk > 0));
-        mma_commit(ds_free);
-        mma_commit(&qd_empty[st]);
-        CSWA_MARK(0, it, 4);
-        // dP^T of the next step: the P/dS warps read this step's dP^T before ds_full
-        if (it + 1 < n_iters) {
-          issue_dP(it + 1);
-          CSWA_MARK(0, it, 5);
-        }
-      }
-      mma_commit(final_bar);
-      volatile int dummy = 0;
-      mbar_wait(final_bar, 0, &dummy);
+      issue_acc(tdV, tR0, dDO_mn, ds * L::kTile, it == 0);
+      mma_commit(&do_empty[ds], leader);
+#ifdef CSWA_TRACE
+      mma_commit(&trace_bar[0], leader);
+#endif
+      if (tracer) CSWA_MARK(0, it, 2);
+      // S^T(it+1) overwrites P^T(it) only after dV(it) has read it: MMAs run in issue order
+      if (more) issue_R(tR0, dK_k, dQ_k, q1 * L::kTile, q1, s_full);
+#ifdef CSWA_TRACE
+      if (more) mma_commit(&trace_bar[1], leader);
+#endif
+      if (tracer) CSWA_MARK(0, it, 4);
+      if (more && !(ok = wait_all(&do_full[d1], ((it + 1) / DS) & 1))) break;
+      if (!(ok = wait_all(ds_full, it & 1))) break;
+      if (tracer) CSWA_MARK(0, it, 5);
+      tc_fence_after();
+      issue_acc(tdK, tR1, dQ_mn, qs * L::kTile, it == 0);
+      mma_commit(&q_empty[qs], leader);
+#ifdef CSWA_TRACE
+      mma_commit(&trace_bar[2], leader);
+#endif
+      if (tracer) CSWA_MARK(0, it, 6);
+      if (more) issue_R(tR1, dV_k, dDO_k, d1 * L::kTile, QS + d1, dp_full);
+#ifdef CSWA_TRACE
+      if (more) mma_commit(&trace_bar[3], leader);
+#endif
+      if (tracer) CSWA_MARK(0, it, 7);
     }
-  } else if (warp == 3) {
-    // ------------------------------------------------------------ dS^T tile store
+    mma_commit(final_bar, leader);
+    volatile int dummy = 0;
+    mbar_wait(final_bar, 0, &dummy);
+  } else if (warp == 2) {
+#ifdef CSWA_TRACE
+    // profiling builds: the TMEM allocator warp records when each MMA group completes
     if (lane == 0) {
-      tma_prefetch_desc(&tm_ds);
-      const long long base = ((long long)b * p.Hq) * p.tiles_per_bh + ds_tiles_before(n, p.n_tiles, p.span);
-      for (int it = 0; it < n_iters; ++it) {
-        if (!mbar_wait(ds_full, it & 1, abort_flag)) break;
-        CSWA_MARK(3, it, 2);
-        const int h = iter_head(it);
-        const long long tile = base + (long long)h * p.tiles_per_bh + it % m_cnt;
-        const int row = (int)(tile * 128);
-        tma_store_2d(&tm_ds, smem + L::kDS, 0, row);
-        tma_store_2d(&tm_ds, smem + L::kDS + L::kPanel, 64, row);
-        bulk_commit();
-        bulk_wait_read<0>();
-        CSWA_MARK(3, it, 3);
-        mbar_arrive(ds_free);
+      volatile int own_abort = 0;
+      for (int it = 0; it < n_iters && !own_abort; ++it) {
+        for (int g = 0; g < 4 && !own_abort; ++g) {
+          if ((g == 1 || g == 3) && it + 1 >= n_iters) continue;
+          if (!mbar_wait(&trace_bar[g], it & 1, &own_abort)) break;
+          CSWA_MARK(3, it, 4 + g);
+        }
       }
-      bulk_wait_all();
     }
+#endif
   } else if (warp >= 4) {
     // ------------------------------------------------------------ P and dS (thread = key row)
     // warps 4-7 take query columns 0-63, warps 8-11 columns 64-127 (warp 2 only allocates TMEM)
@@ -326,132 +357,98 @@ __global__ void __launch_bounds__(384, 1)
     const int r = quarter * 32 + lane;
     const int j = k0 + r;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t cols = lane_off + 64 * half;  // this thread's S^T / dP^T columns
     const float sl2 = p.scale_log2;
-    uint8_t* ds_row = smem + L::kDS + half * L::kPanel + r * 128;
-    const bool tracer = (warp == 4 && lane == 0);
-    const bool tracer1 = (warp == 8 && lane == 0);
+    // row r of the stored dS^T tile, this warpgroup's 64 queries
+    const long long tile0 = ((long long)b * p.Hq) * p.tiles_per_bh + ds_tiles_before(n, p.n_tiles, p.span);
+    const bool tracer = ((warp == 4 || warp == 8) && lane == 0);
+    const int trole = 1 + half;
+    (void)tracer;
+    (void)trole;
     bool ok = true;
     for (int it = 0; it < n_iters; ++it) {
-      const int st = it & 1;
       const int q0 = iter_q0(it) + 64 * half;  // first query of this thread's columns
-      const float* lse_s = s_lse + st * 128 + 64 * half;
-      const float* dl_s = s_delta + st * 128 + 64 * half;
-      if (tracer) CSWA_MARK(1, it, 0);
-      if (tracer1) CSWA_MARK(2, it, 0);
-      // the lse/Delta rows of this stage come from a bulk copy: acquire them from its
-      // own barrier (completion of S^T alone does not order that copy before our reads)
-      ok = __all_sync(0xffffffffu, mbar_wait(&qd_full[st], (it >> 1) & 1, abort_flag) &&
-                                       mbar_wait(s_full, it & 1, abort_flag));
-      if (tracer) CSWA_MARK(1, it, 1);
-      if (tracer1) CSWA_MARK(2, it, 1);
+      if (tracer) CSWA_MARK(trole, it, 0);
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag));
+      if (tracer) CSWA_MARK(trole, it, 1);
       if (!ok) break;
       tc_fence_after();
       uint32_t sr[64];
-      tmem_ld32(tR0 + lane_off + 64 * half + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tR0 + lane_off + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tR0 + cols + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tR0 + cols + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_ld_wait();
-      // debug dump layout: [it][half][r][kind][64]
-#define DBG_SLOT(kind, c) ((((it * 2 + half) * 128 + r) * 5 + (kind)) * 64 + (c))
-      if (it < 3) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) CSWA_DUMP(DBG_SLOT(0, c), __uint_as_float(sr[c]));
-#pragma unroll
-        for (int c = 0; c < 64; ++c) CSWA_DUMP(DBG_SLOT(1, c), lse_s[c]);
-      }
+      if (tracer) CSWA_MARK(trole, it, 2);
       const bool full = (k0 + 127 <= q0) && (W < 0 || q0 + 63 - k0 <= W);
       const int c_lo = j - q0;                      // query q0 + c sees key j iff c >= c_lo
       const int c_hi = (W < 0) ? 63 : j + W - q0;   //   and c <= c_hi
-      // P^T in place as packed bf16 pairs (the same bf16 P feeds dV and dS).
-      // Masked entries get exponent -inf (ex2 -> 0): no branch around the exponential;
+      // P = exp2(scale log2e (S - lse/scale)): the MMA has already added -lse/scale, so
+      // one packed multiply per two columns; masked entries are set to 0 after the exp2,
       // tiles inside the band skip the mask (a warp-uniform branch).
-      const float4* lse4 = reinterpret_cast<const float4*>(lse_s);
-      if (full) {
+      const float2 sl2v = make_float2(sl2, sl2);
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
-          const float4 l = lse4[c4];
-          sr[2 * c4] = pack_bf16x2(ex2_approx(fmaf(__uint_as_float(sr[4 * c4]), sl2, -l.x)),
-                                   ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 1]), sl2, -l.y)));
-          sr[2 * c4 + 1] = pack_bf16x2(ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 2]), sl2, -l.z)),
-                                       ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 3]), sl2, -l.w)));
-        }
-      } else {
+      for (int c2 = 0; c2 < 32; ++c2) {
+        const float2 e = __fmul2_rn(make_float2(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1])), sl2v);
+        float y[2] = {ex2_approx(e.x), ex2_approx(e.y)};
+        if (!full) {
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
-          const float4 l = lse4[c4];
-          const float lv[4] = {l.x, l.y, l.z, l.w};
-          float pv[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int c = 4 * c4 + u;
-            const bool vis = (c >= c_lo) & (c <= c_hi);
-            pv[u] = ex2_approx(vis ? fmaf(__uint_as_float(sr[c]), sl2, -lv[u]) : -INFINITY);
+          for (int u = 0; u < 2; ++u) {
+            const int c = 2 * c2 + u;
+            y[u] = ((c >= c_lo) & (c <= c_hi)) ? y[u] : 0.f;
           }
-          sr[2 * c4] = pack_bf16x2(pv[0], pv[1]);
-          sr[2 * c4 + 1] = pack_bf16x2(pv[2], pv[3]);
         }
+        sr[2 * c2] = __float_as_uint(y[0]);
+        sr[2 * c2 + 1] = __float_as_uint(y[1]);
       }
-      if (tracer) CSWA_MARK(1, it, 6);
-      if (tracer1) CSWA_MARK(2, it, 6);
-      // P^T of this warpgroup's 64 queries goes over the first half of its own S^T
-      // columns (64*half .. 64*half+31), which only this warpgroup has read
-      tmem_st32(tR0 + lane_off + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      const float* pf = reinterpret_cast<const float*>(sr);
+      if (tracer) CSWA_MARK(trole, it, 3);
+      {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pf[2 * c], pf[2 * c + 1]);
+        tmem_st32(tR0 + cols, pk);  // over this thread's own (already read) S^T columns
+      }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full);
-      if (tracer) CSWA_MARK(1, it, 2);
-      if (tracer1) CSWA_MARK(2, it, 2);
+      if (tracer) CSWA_MARK(trole, it, 4);
 
       ok = __all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, abort_flag));
-      if (tracer) CSWA_MARK(1, it, 3);
-      if (tracer1) CSWA_MARK(2, it, 3);
-      // dS^T of the previous step must have been read by dK and by its TMA store
-      if (ok && it > 0) ok = __all_sync(0xffffffffu, mbar_wait(ds_free, (it - 1) & 1, abort_flag));
-      if (tracer) CSWA_MARK(1, it, 4);
-      if (tracer1) CSWA_MARK(2, it, 4);
       if (!ok) break;
+      if (tracer) CSWA_MARK(trole, it, 5);
       tc_fence_after();
+      // dS = P * (dP - Delta): the MMA has already subtracted Delta; one packed multiply
+      // per two columns, 32 columns at a time
+      uint32_t dsk[32];
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
+      for (int hc = 0; hc < 2; ++hc) {
         uint32_t dp[32];
-        tmem_ld32(tR1 + lane_off + 64 * half + cc * 32, dp);
+        tmem_ld32(tR1 + cols + 32 * hc, dp);
         tmem_ld_wait();
-        const float4* dl4 = reinterpret_cast<const float4*>(dl_s + cc * 32);
-        if (it < 3) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) CSWA_DUMP(DBG_SLOT(2, cc * 32 + e), __uint_as_float(dp[e]));
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float2 pp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sr[cc * 16 + e]));
-            CSWA_DUMP(DBG_SLOT(3, cc * 32 + 2 * e), pp.x);
-            CSWA_DUMP(DBG_SLOT(3, cc * 32 + 2 * e + 1), pp.y);
-          }
-#pragma unroll
-          for (int e = 0; e < 32; ++e) CSWA_DUMP(DBG_SLOT(4, cc * 32 + e), dl_s[cc * 32 + e]);
-        }
-        uint32_t w[16];
-#pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const float4 dl = dl4[e4];
-          const float2 p0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sr[cc * 16 + 2 * e4]));
-          const float2 p1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sr[cc * 16 + 2 * e4 + 1]));
-          w[2 * e4] = pack_bf16x2(p0.x * (__uint_as_float(dp[4 * e4]) - dl.x),
-                                  p0.y * (__uint_as_float(dp[4 * e4 + 1]) - dl.y));
-          w[2 * e4 + 1] = pack_bf16x2(p1.x * (__uint_as_float(dp[4 * e4 + 2]) - dl.z),
-                                      p1.y * (__uint_as_float(dp[4 * e4 + 3]) - dl.w));
-        }
-        // this warpgroup's panel, queries cc*32 .. cc*32+31 = 16-byte chunks cc*4 .. cc*4+3
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const uint32_t chunk = cc * 4 + u;
-          *reinterpret_cast<uint4*>(ds_row + ((chunk ^ (r & 7)) << 4)) =
-              make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        for (int c2 = 0; c2 < 16; ++c2) {
+          const int c = 32 * hc + 2 * c2;
+          const float2 d = __fmul2_rn(make_float2(pf[c], pf[c + 1]),
+                                      make_float2(__uint_as_float(dp[2 * c2]), __uint_as_float(dp[2 * c2 + 1])));
+          dsk[c / 2] = pack_bf16x2(d.x, d.y);
         }
       }
-      fence_proxy_async_smem();
+      if (tracer) CSWA_MARK(trole, it, 6);
+      tmem_st32(tR1 + cols, dsk);  // over this thread's own (already read) dP^T columns
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(ds_full);
-      if (tracer) CSWA_MARK(1, it, 5);
-      if (tracer1) CSWA_MARK(2, it, 5);
+      if (tracer) CSWA_MARK(trole, it, 7);
+      // dS^T of this warp's 32 keys x 64 queries into the workspace tile the dQ kernel
+      // reads (after the arrive: dK need not wait for these stores), as 16-byte units
+      // (8 queries of one key) ordered so that every warp store covers 512 contiguous
+      // bytes (see ds_unit_offset)
+      {
+        const long long tile = tile0 + (long long)iter_head(it) * p.tiles_per_bh + it % m_cnt;
+        uint8_t* dst = reinterpret_cast<uint8_t*>(p.ds) + (size_t)tile * 32768 + ds_unit_offset(r, 8 * half);
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+          *reinterpret_cast<uint4*>(dst + g * 512) = make_uint4(dsk[4 * g], dsk[4 * g + 1], dsk[4 * g + 2], dsk[4 * g + 3]);
+      }
     }
     // ---------------------------------------------------------- dK (warps 4-7) / dV (8-11) epilogue
     ok = __all_sync(0xffffffffu, ok && mbar_wait(final_bar, 0, abort_flag));
@@ -500,8 +497,7 @@ struct DqLayout {
 
 template <int D>
 __global__ void __launch_bounds__(256, 1)
-    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_ds,
-                       const BwdParams p) {
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const BwdParams p) {
   using L = DqLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -513,7 +509,8 @@ __global__ void __launch_bounds__(256, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * L::kStages + 2);
 
   const int warp = warp_id(), lane = lane_id();
-  const int h = blockIdx.x, b = blockIdx.y, m = blockIdx.z;
+  // query tiles of one (b, h) are adjacent in launch order (they share K tiles in L2)
+  const int m = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int hk = h / p.G;
   // key tiles n whose query range [n, n + span - 1] holds m
   const int n_lo = max(0, m - p.span + 1);
@@ -542,7 +539,6 @@ __global__ void __launch_bounds__(256, 1)
   if (warp == 0) {
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_ds);
       int last_issue[L::kStages];
       for (int s = 0; s < L::kStages; ++s) last_issue[s] = -1;
       for (int i = 0; i < steps; ++i) {
@@ -550,10 +546,9 @@ __global__ void __launch_bounds__(256, 1)
         const int n = n_lo + i;
         if (!mbar_wait(&empty[st], ((i / L::kStages) & 1) ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(&full[st], L::kDS + L::kK);
-        const int row = (int)((bh_base + ds_tiles_before(n, p.n_tiles, p.span) + (m - n)) * 128);
+        const long long tile = bh_base + ds_tiles_before(n, p.n_tiles, p.span) + (m - n);
         uint8_t* dst = smem + st * L::kStage;
-        tma_load_2d(dst, &tm_ds, &full[st], 0, row);
-        tma_load_2d(dst + 16384, &tm_ds, &full[st], 64, row);
+        bulk_load(dst, reinterpret_cast<const uint8_t*>(p.ds) + (size_t)tile * L::kDS, L::kDS, &full[st]);
         for (int pn = 0; pn < D / 64; ++pn)
           tma_load_4d(dst + L::kDS + pn * 16384, &tm_k, &full[st], pn * 64, hk, n * 128, b);
         last_issue[st] = i;
@@ -573,9 +568,12 @@ __global__ void __launch_bounds__(256, 1)
         if (!(ok = mbar_wait(&full[st], (i / L::kStages) & 1, abort_flag))) break;
         tc_fence_after();
         const uint32_t sds = sbase + st * L::kStage, sk = sds + L::kDS;
-        const uint64_t da = sdesc_sw128(sds, 16384, 1024), db = sdesc_sw128(sk, 16384, 1024);
+        // A = dS (M = queries, K = keys) in the stored unit order: 128 bytes between
+        // core matrices along K, 512 along M; 16 keys per MMA = (kk / 2) * 8 KB + (kk & 1) * 256
+        const uint64_t da = sdesc_noswz(sds, 128, 512), db = sdesc_sw128(sk, 16384, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ss(tmem, da + ((kk * 2048) >> 4), db + ((kk * 2048) >> 4), id, (i > 0 || kk > 0));
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem, da + ((ds_unit_offset(16 * kk, 0)) >> 4), db + ((kk * 2048) >> 4), id, (i > 0 || kk > 0));
         mma_commit(&empty[st]);
       }
       mma_commit(done);
@@ -615,12 +613,20 @@ __global__ void __launch_bounds__(256, 1)
   }
 }
 
-// Delta_i = dO_i . o_i and lse_i * log2(e) into the padded (B, Hq, Tpad) workspace
-// arrays: D/8 lanes per (b, t, h) row.
+// Row extensions of the S^T and dP^T MMAs. For each query row i (padded to 128-row
+// tiles) x = -lse_i / scale and y = -Delta_i = -(dO_i . o_i) are split into bf16
+// pairs hi + lo (hi = bf16(x), lo = bf16(x - hi): together 16 significant bits), so
+// that one extra K = 16 MMA step against key-side rows (1, 1, 0, ...) adds x (or y)
+// to every entry of query column i in fp32. Padded rows get x = -1e30 (finite: the
+// MMA also multiplies these bytes by zero; exp2 of it is 0) and y = 0.
+// Per (batch, head, query tile) 512 bytes: for each group g of 8 rows, 16 bytes of
+// the 8 hi values then 16 bytes of the 8 lo values (the MN-major no-swizzle layout:
+// one core row per K index). D/8 lanes per (b, t, h) row.
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16* o, const __nv_bfloat16* dout,
-                                                             const float* lse, float* lse2, float* delta, int B,
-                                                             int T, int Tpad, int Hq) {
+                                                             const float* lse, uint8_t* ext_lse,
+                                                             uint8_t* ext_delta, int B, int T, int Tpad, int Hq,
+                                                             float inv_scale) {
   constexpr int LK = D / 8;
   const long long rows = (long long)B * Tpad * Hq;
   const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -648,9 +654,16 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16*
 #pragma unroll
   for (int s = LK / 2; s >= 1; s >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, s);
   if (active && lr == 0) {
-    const size_t so = ((size_t)b * Hq + h) * Tpad + t;
-    delta[so] = real ? dsum : 0.f;
-    lse2[so] = real ? lse[((size_t)b * Hq + h) * T + t] * 1.4426950408889634f : INFINITY;
+    // clamped to stay finite in bf16 (a huge 1/scale must not turn x into -inf)
+    const float x = real ? fminf(fmaxf(-lse[((size_t)b * Hq + h) * T + t] * inv_scale, -3.0e38f), 3.0e38f) : -1e30f;
+    const float y = real ? -dsum : 0.f;
+    const int i = t & 127;
+    const size_t at = (((size_t)b * Hq + h) * (Tpad / 128) + t / 128) * 512 + (i >> 3) * 32 + (i & 7) * 2;
+    const __nv_bfloat16 xh = __float2bfloat16_rn(x), yh = __float2bfloat16_rn(y);
+    *reinterpret_cast<__nv_bfloat16*>(ext_lse + at) = xh;
+    *reinterpret_cast<__nv_bfloat16*>(ext_lse + at + 16) = __float2bfloat16_rn(x - __bfloat162float(xh));
+    *reinterpret_cast<__nv_bfloat16*>(ext_delta + at) = yh;
+    *reinterpret_cast<__nv_bfloat16*>(ext_delta + at + 16) = __float2bfloat16_rn(y - __bfloat162float(yh));
   }
 }
 

@@ -52,18 +52,6 @@ bool encode_bthd(CUtensorMap* m, const void* base, int B, int T, int H, int D, i
 
 // The stored dS^T tiles: a (rows, 128) bf16 matrix, box = 64 columns x 128 rows,
 // 128-byte swizzle (the shared-memory layout of one 64-query panel).
-bool encode_ds_tiles(CUtensorMap* m, const void* base, long long rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {128, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {256};
-  const cuuint32_t box[2] = {64, 128};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool dims_ok(int B, int T, int Hq, int Hkv) {
   return B >= 1 && T >= 1 && Hq >= 1 && Hkv >= 1 && Hq % Hkv == 0 && (long long)B * T * Hq < (1ll << 40);
@@ -153,8 +141,8 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, f
 }
 
 struct BwdWorkspace {
-  float* lse2;            // (B, Hq, Tpad)
-  float* delta;           // (B, Hq, Tpad)
+  uint8_t* ext_lse;       // (B, Hq, Tpad / 128) x 512 bytes
+  uint8_t* ext_delta;     // (B, Hq, Tpad / 128) x 512 bytes
   __nv_bfloat16* ds;      // stored dS^T tiles, 128 x 128 each
   long long tiles_per_bh;
   int span;
@@ -167,9 +155,9 @@ BwdWorkspace carve_bwd(void* ws, int B, int T, int Hq, int window) {
   w.span = bwd_span(nt, eff_window(window, T));
   w.tiles_per_bh = ds_tiles_before(nt, nt, w.span);
   uint8_t* p = static_cast<uint8_t*>(ws);
-  w.lse2 = reinterpret_cast<float*>(p);
+  w.ext_lse = p;
   p += align256((size_t)B * Hq * Tpad * 4);
-  w.delta = reinterpret_cast<float*>(p);
+  w.ext_delta = p;
   p += align256((size_t)B * Hq * Tpad * 4);
   w.ds = reinterpret_cast<__nv_bfloat16*>(p);
   return w;
@@ -195,25 +183,25 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
   const int nt = tiles128(T);
   const int Tpad = nt * 128;
   BwdWorkspace w = carve_bwd(ws, B, T, Hq, window);
-  CUtensorMap tq, tk, tv, tdo, tds;
+  CUtensorMap tq, tk, tv, tdo;
   if (!encode_bthd(&tq, q, B, T, Hq, D) || !encode_bthd(&tk, k, B, T, Hkv, D) ||
-      !encode_bthd(&tv, v, B, T, Hkv, D) || !encode_bthd(&tdo, dO, B, T, Hq, D) ||
-      !encode_ds_tiles(&tds, w.ds, (long long)B * Hq * w.tiles_per_bh * 128))
+      !encode_bthd(&tv, v, B, T, Hkv, D) || !encode_bthd(&tdo, dO, B, T, Hq, D))
     return ATTN_ERR_LAUNCH;
   if (!set_smem_attrs<D>() || !set_dq_attr<D>()) return ATTN_ERR_LAUNCH;
   {
     const long long threads = (long long)B * Tpad * Hq * (D / 8);
     attn_bwd_prep_kernel<D><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, w.lse2, w.delta, B, T,
-        Tpad, Hq);
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, w.ext_lse, w.ext_delta, B, T,
+        Tpad, Hq, 1.f / scale);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
   }
   BwdParams p{};
-  p.lse2 = w.lse2;
-  p.delta = w.delta;
+  p.ext_lse = w.ext_lse;
+  p.ext_delta = w.ext_delta;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.ds = w.ds;
   p.T = T;
   p.Tpad = Tpad;
   p.Hq = Hq;
@@ -224,9 +212,9 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
   p.tiles_per_bh = w.tiles_per_bh;
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
-  attn_bwd_kernel<D><<<dim3(Hkv, B, nt), 384, BwdLayout<D>::kBytes, st>>>(tq, tk, tv, tdo, tds, p);
+  attn_bwd_kernel<D><<<dim3(nt, Hkv, B), 384, BwdLayout<D>::kBytes, st>>>(tq, tk, tv, tdo, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
-  attn_bwd_dq_kernel<D><<<dim3(Hq, B, nt), 256, DqLayout<D>::kBytes, st>>>(tk, tds, p);
+  attn_bwd_dq_kernel<D><<<dim3(nt, Hq, B), 256, DqLayout<D>::kBytes, st>>>(tk, p);
   return launched();
 }
 
@@ -293,7 +281,7 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
   if (!q || !k || !v || !o || !lse || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
       !aligned16(lse))
     return ATTN_ERR_INVALID_ARG;
-  if ((long long)B * Hq > 65535ll * 65535ll || Hq > 0x7fffffff || tiles128(T) > 2 * 65535) return ATTN_ERR_INVALID_ARG;
+  if (B > 65535 || Hq > 65535) return ATTN_ERR_INVALID_ARG;
   cudaStream_t st = as_stream(stream);
   return D == 64 ? launch_fwd<64>(q, k, v, o, lse, B, T, Hq, Hkv, window, scale, st)
                  : launch_fwd<128>(q, k, v, o, lse, B, T, Hq, Hkv, window, scale, st);

@@ -104,13 +104,11 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS[2] = {tmem, tmem + 128};
-  const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+  // TMEM columns of slot s: S_s at 128*s, O_s at 256 + D*s
+  auto tS = [&](int s) { return tmem + 128u * s; };
+  auto tO = [&](int s) { return tmem + 256u + (uint32_t)D * s; };
 
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t sQ[2] = {sbase + L::kQ0, sbase + L::kQ1};
-  const uint32_t sK[2] = {sbase + L::kK0, sbase + L::kK0 + L::kTile};
-  const uint32_t sV[2] = {sbase + L::kV0, sbase + L::kV0 + L::kTile};
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -154,9 +152,9 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idO = idesc_bf16(128, D, false, true);
       // descriptors built once; each MMA adds (byte offset >> 4) to the start field
-      const uint64_t dQ0 = sdesc_sw128(sQ[0], 16, 1024), dQ1 = sdesc_sw128(sQ[1], 16, 1024);
-      const uint64_t dK0 = sdesc_sw128(sK[0], 16, 1024);
-      const uint64_t dV0 = sdesc_sw128(sV[0], 16384, 1024);
+      const uint64_t dQ0 = sdesc_sw128(sbase + L::kQ0, 16, 1024), dQ1 = sdesc_sw128(sbase + L::kQ1, 16, 1024);
+      const uint64_t dK0 = sdesc_sw128(sbase + L::kK0, 16, 1024);
+      const uint64_t dV0 = sdesc_sw128(sbase + L::kV0, 16384, 1024);
       int cnt[2] = {0, 0};
       bool ok = mbar_wait(q_full, 0, abort_flag);
       tc_fence_after();
@@ -174,7 +172,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_ss(tS[s], (s ? dQ1 : dQ0) + (off >> 4), dK0 + ((st * L::kTile + off) >> 4), idS, kk > 0);
+            mma_ss(tS(s), (s ? dQ1 : dQ0) + (off >> 4), dK0 + ((st * L::kTile + off) >> 4), idS, kk > 0);
           }
           mma_commit(&s_full[s]);
         }
@@ -187,7 +185,7 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tO[s], tS[s] + kk * 8, dV0 + ((st * L::kTile + kk * 2048) >> 4), idO, (cnt[s] > 0 || kk > 0));
+            mma_ts(tO(s), tS(s) + kk * 8, dV0 + ((st * L::kTile + kk * 2048) >> 4), idO, (cnt[s] > 0 || kk > 0));
           mma_commit(&pv_done[s]);
           ++cnt[s];
         }
@@ -204,33 +202,32 @@ __global__ void __launch_bounds__(384, 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    if (has[s]) {
-      const int q0 = qt[s] * 128;
+    const int my_qt = 2 * pair + s;
+    const int my_hi = my_qt;
+    const int my_lo = (W < 0) ? 0 : max(0, my_qt * 128 - W) / 128;
+    const uint32_t tSs = tS(s) + lane_off, tOs = tO(s) + lane_off;
+    if (my_qt < p.nq_tiles) {
+      const int q0 = my_qt * 128;
       const int i = q0 + row;
       const float sl2 = p.scale_log2;
       float m_run = -INFINITY, l_run = 0.f;
       int cnt = 0;
       bool ok = true;
-      for (int t = lo[s]; t <= hi[s]; ++t, ++cnt) {
+      for (int t = my_lo; t <= my_hi; ++t, ++cnt) {
         ok = __all_sync(0xffffffffu, mbar_wait(&s_full[s], cnt & 1, abort_flag));
         if (!ok) break;
         tc_fence_after();
         uint32_t r[128];
-        tmem_ld32(tS[s] + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_ld32(tS[s] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-        tmem_ld32(tS[s] + lane_off + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
-        tmem_ld32(tS[s] + lane_off + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
+        tmem_ld32(tSs + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(tSs + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_ld32(tSs + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
+        tmem_ld32(tSs + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
         tmem_ld_wait();
         const int k0 = t * 128;
         const bool full = (k0 + 127 <= q0) && (W < 0 || q0 + 127 - k0 <= W);
-        // 8 independent max chains instead of one 128-long dependent chain
-        float mx8[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
-        if (full) {
-#pragma unroll
-          for (int c = 0; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(r[c]));
-        } else {
+        // 4 independent 3-input max chains instead of one 128-long dependent chain
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (!full) {
           // visible columns of this row: [c_lo, c_hi] (empty when c_lo > c_hi)
           const int c_hi = i - k0;
           const int c_lo = (W < 0) ? -1 : i - W - k0;
@@ -238,11 +235,16 @@ __global__ void __launch_bounds__(384, 1)
           for (int c = 0; c < 128; ++c) {
             const bool vis = (c <= c_hi) & (c >= c_lo);
             r[c] = vis ? r[c] : __float_as_uint(-INFINITY);
-            mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(r[c]));
           }
         }
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+#pragma unroll
+        for (int c = 0; c < 128; c += 8) {
+          mx4[(c >> 3) & 3] = fmax3(mx4[(c >> 3) & 3], __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+          mx4[(c >> 3) & 3] = fmax3(mx4[(c >> 3) & 3], __uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
+          mx4[(c >> 3) & 3] = fmax3(mx4[(c >> 3) & 3], __uint_as_float(r[c + 4]), __uint_as_float(r[c + 5]));
+          mx4[(c >> 3) & 3] = fmax3(mx4[(c >> 3) & 3], __uint_as_float(r[c + 6]), __uint_as_float(r[c + 7]));
+        }
+        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
         const float m_tile = mx * sl2;
         bool rescale = false;
         float factor = 1.f;
@@ -255,30 +257,30 @@ __global__ void __launch_bounds__(384, 1)
           rescale = true;
         }
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-        float ls8[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) ls8[u] = 0.f;
+        // p = exp2(s * scale * log2e - m), two columns per packed FMA; row sum in packed adds
+        const float2 sl2v = make_float2(sl2, sl2), nm = make_float2(-m_use, -m_use);
+        float2 ls4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * c]), sl2, -m_use));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * c + 1]), sl2, -m_use));
-          ls8[c & 7] += p0 + p1;
-          r[c] = pack_bf16x2(p0, p1);
+          const float2 x = __ffma2_rn(make_float2(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), sl2v, nm);
+          const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          ls4[c & 3] = __fadd2_rn(ls4[c & 3], pp);
+          r[c] = pack_bf16x2(pp.x, pp.y);
         }
-        l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
-        tmem_st32(tS[s] + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_st32(tS[s] + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        l_run += ((ls4[0].x + ls4[0].y) + (ls4[1].x + ls4[1].y)) + ((ls4[2].x + ls4[2].y) + (ls4[3].x + ls4[3].y));
+        tmem_st32(tSs + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_st32(tSs + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
         // rescale only when some row of the warp needs it (O is stable: the MMA
         // warp waited for the previous PV before issuing this tile's S)
         if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
-            tmem_ld32(tO[s] + lane_off + c * 32, o);
+            tmem_ld32(tOs + c * 32, o);
             tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-            tmem_st32(tO[s] + lane_off + c * 32, o);
+            tmem_st32(tOs + c * 32, o);
           }
         }
         tmem_st_wait();
@@ -297,7 +299,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(tO[s] + lane_off + c * 32, o);
+          tmem_ld32(tOs + c * 32, o);
           tmem_ld_wait();
           uint4 v[4];
           uint32_t* pv = reinterpret_cast<uint32_t*>(v);
