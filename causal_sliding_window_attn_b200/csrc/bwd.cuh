@@ -560,26 +560,27 @@ __global__ void __launch_bounds__(256, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t id = idesc_bf16(128, D, true, true);  // A = dS (queries contiguous), B = K (d contiguous)
-      bool ok = true;
-      for (int i = 0; ok && i < steps; ++i) {
-        const int st = i % L::kStages;
-        if (!(ok = mbar_wait(&full[st], (i / L::kStages) & 1, abort_flag))) break;
-        tc_fence_after();
-        const uint32_t sds = sbase + st * L::kStage, sk = sds + L::kDS;
-        // A = dS (M = queries, K = keys) in the stored unit order: 128 bytes between
-        // core matrices along K, 512 along M; 16 keys per MMA = (kk / 2) * 8 KB + (kk & 1) * 256
-        const uint64_t da = sdesc_noswz(sds, 128, 512), db = sdesc_sw128(sk, 16384, 1024);
+    // whole warp runs the loop, one elected lane issues
+    const uint32_t leader = elect_one();
+    constexpr uint32_t id = idesc_bf16(128, D, true, true);  // A = dS (queries contiguous), B = K (d contiguous)
+    bool ok = true;
+    for (int i = 0; ok && i < steps; ++i) {
+      const int st = i % L::kStages;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&full[st], (i / L::kStages) & 1, abort_flag)))) break;
+      tc_fence_after();
+      const uint32_t sds = sbase + st * L::kStage, sk = sds + L::kDS;
+      // A = dS (M = queries, K = keys) in the stored unit order: 128 bytes between
+      // core matrices along K, 512 along M; 16 keys per MMA = (kk / 2) * 8 KB + (kk & 1) * 256
+      const uint64_t da = sdesc_noswz(sds, 128, 512), db = sdesc_sw128(sk, 16384, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem, da + ((ds_unit_offset(16 * kk, 0)) >> 4), db + ((kk * 2048) >> 4), id, (i > 0 || kk > 0));
-        mma_commit(&empty[st]);
-      }
-      mma_commit(done);
-      volatile int dummy = 0;
-      mbar_wait(done, 0, &dummy);
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ss(tmem, da + ((ds_unit_offset(16 * kk, 0)) >> 4), db + ((kk * 2048) >> 4), id, (i > 0 || kk > 0),
+               leader);
+      mma_commit(&empty[st], leader);
     }
+    mma_commit(done, leader);
+    volatile int dummy = 0;
+    mbar_wait(done, 0, &dummy);
   } else if (warp >= 4) {
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;

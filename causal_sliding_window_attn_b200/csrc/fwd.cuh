@@ -11,7 +11,8 @@
 // 2p+1. It walks the union of their key-tile ranges inside the causal/window
 // band; key tiles outside the band are never loaded.
 //   warp 0      TMA producer: Q once, then K/V tiles into a 2-stage ring
-//   warp 1      MMA issuer (one thread): S_s = Q_s K^T (SS), O_s += P_s V (TS)
+//   warp 1      MMA issuer (whole warp, one elected lane issues): S_s = Q_s K^T (SS),
+//               O_s += P_s V (TS)
 //   warp 2      TMEM allocator
 //   warps 4-7   softmax + epilogue for slot 0 (thread = query row)
 //   warps 8-11  softmax + epilogue for slot 1
@@ -148,54 +149,58 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
-      constexpr uint32_t idO = idesc_bf16(128, D, false, true);
-      // descriptors built once; each MMA adds (byte offset >> 4) to the start field
-      const uint64_t dQ0 = sdesc_sw128(sbase + L::kQ0, 16, 1024), dQ1 = sdesc_sw128(sbase + L::kQ1, 16, 1024);
-      const uint64_t dK0 = sdesc_sw128(sbase + L::kK0, 16, 1024);
-      const uint64_t dV0 = sdesc_sw128(sbase + L::kV0, 16384, 1024);
-      int cnt[2] = {0, 0};
-      bool ok = mbar_wait(q_full, 0, abort_flag);
+    // The whole warp runs the loop (descriptors stay warp-uniform); one elected lane
+    // issues. MMAs run in issue order, so S_s of the next key tile, issued after PV_s
+    // of this one, never overwrites P_s before PV_s has read it, and the softmax warps,
+    // which see S_s only through a commit issued after PV_s, find O_s stable.
+    const uint32_t leader = elect_one();
+    constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
+    constexpr uint32_t idO = idesc_bf16(128, D, false, true);
+    // descriptors built once; each MMA adds (byte offset >> 4) to the start field
+    const uint64_t dQ0 = sdesc_sw128(sbase + L::kQ0, 16, 1024), dQ1 = sdesc_sw128(sbase + L::kQ1, 16, 1024);
+    const uint64_t dK0 = sdesc_sw128(sbase + L::kK0, 16, 1024);
+    const uint64_t dV0 = sdesc_sw128(sbase + L::kV0, 16384, 1024);
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+    };
+    int cnt[2] = {0, 0};
+    bool ok = wait_all(q_full, 0);
+    tc_fence_after();
+    int n = 0;
+    for (int t = t_lo; ok && t <= t_hi; ++t, ++n) {
+      const int st = n & 1;
+      const uint32_t ph = (n >> 1) & 1;
+      if (!(ok = wait_all(&k_full[st], ph))) break;
       tc_fence_after();
-      int n = 0;
-      for (int t = t_lo; ok && t <= t_hi; ++t, ++n) {
-        const int st = n & 1;
-        const uint32_t ph = (n >> 1) & 1;
-        if (!(ok = mbar_wait(&k_full[st], ph, abort_flag))) break;
-        tc_fence_after();
-        for (int s = 0; s < 2; ++s) {
-          if (!(has[s] && lo[s] <= t && t <= hi[s])) continue;
-          // P_s of the previous tile lives where S_s goes: wait until PV has read it
-          if (cnt[s] > 0 && !(ok = mbar_wait(&pv_done[s], (cnt[s] - 1) & 1, abort_flag))) break;
-          tc_fence_after();
+      for (int s = 0; s < 2; ++s) {
+        if (!(has[s] && lo[s] <= t && t <= hi[s])) continue;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_ss(tS(s), (s ? dQ1 : dQ0) + (off >> 4), dK0 + ((st * L::kTile + off) >> 4), idS, kk > 0);
-          }
-          mma_commit(&s_full[s]);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(tS(s), (s ? dQ1 : dQ0) + (off >> 4), dK0 + ((st * L::kTile + off) >> 4), idS, kk > 0, leader);
         }
-        if (!ok) break;
-        if (!(ok = mbar_wait(&v_full[st], ph, abort_flag))) break;
-        tc_fence_after();
-        for (int s = 0; s < 2; ++s) {
-          if (!(has[s] && lo[s] <= t && t <= hi[s])) continue;
-          if (!(ok = mbar_wait(&p_full[s], cnt[s] & 1, abort_flag))) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tO(s), tS(s) + kk * 8, dV0 + ((st * L::kTile + kk * 2048) >> 4), idO, (cnt[s] > 0 || kk > 0));
-          mma_commit(&pv_done[s]);
-          ++cnt[s];
-        }
-        mma_commit(&kv_empty[st]);
+        mma_commit(&s_full[s], leader);
       }
-      // every MMA issued above has finished before TMEM is released
-      mma_commit(final_bar);
-      volatile int dummy = 0;
-      mbar_wait(final_bar, 0, &dummy);
+      if (!(ok = wait_all(&v_full[st], ph))) break;
+      tc_fence_after();
+      for (int s = 0; s < 2; ++s) {
+        if (!(has[s] && lo[s] <= t && t <= hi[s])) continue;
+        if (!(ok = wait_all(&p_full[s], cnt[s] & 1))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tO(s), tS(s) + kk * 8, dV0 + ((st * L::kTile + kk * 2048) >> 4), idO, (cnt[s] > 0 || kk > 0),
+                 leader);
+        mma_commit(&pv_done[s], leader);
+        ++cnt[s];
+      }
+      if (!ok) break;
+      mma_commit(&kv_empty[st], leader);
     }
+    // every MMA issued above has finished before TMEM is released
+    mma_commit(final_bar, leader);
+    volatile int dummy = 0;
+    mbar_wait(final_bar, 0, &dummy);
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
     const int s = (warp - 4) >> 2;
@@ -270,8 +275,8 @@ __global__ void __launch_bounds__(384, 1)
         l_run += ((ls4[0].x + ls4[0].y) + (ls4[1].x + ls4[1].y)) + ((ls4[2].x + ls4[2].y) + (ls4[3].x + ls4[3].y));
         tmem_st32(tSs + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
         tmem_st32(tSs + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-        // rescale only when some row of the warp needs it (O is stable: the MMA
-        // warp waited for the previous PV before issuing this tile's S)
+        // rescale only when some row of the warp needs it (O is stable: this tile's
+        // S was committed after the previous PV, so that PV has completed)
         if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
