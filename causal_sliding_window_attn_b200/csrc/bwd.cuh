@@ -103,7 +103,11 @@ struct BwdLayout {
   static constexpr int kExt = kDO + kDOStages * kTile;
   static constexpr int kExtOnes = kExt + (kQStages + kDOStages) * 512;
   static constexpr int kBar = kExtOnes + 256;
+#ifdef CSWA_TRACE
+  static constexpr int kUsed = kBar + 256;  // profiling builds keep 4 more barriers
+#else
   static constexpr int kUsed = kBar + 192;
+#endif
   static constexpr int kBytes = (kUsed + 1024 <= 232448) ? kUsed + 1024 : 232448;
   static_assert(kUsed <= 232448, "shared memory budget");
   static constexpr uint32_t kTmemCols = 512;
@@ -130,8 +134,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* do_full = q_empty + QS;            // [DS]
   uint64_t* do_empty = do_full + DS;           // [DS]  dV has read the dO tile
   uint64_t* s_full = do_empty + DS;            // S^T in TMEM
-  uint64_t* p_full = s_full + 1;               // P^T written over S^T
-  uint64_t* dp_full = p_full + 1;              // dP^T in TMEM
+  uint64_t* p_chunk = s_full + 1;              // [4] P^T of queries 16c..16c+15 of each half written
+  uint64_t* dp_full = p_chunk + 4;             // dP^T in TMEM
   uint64_t* ds_full = dp_full + 1;             // dS^T written over dP^T
   uint64_t* final_bar = ds_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
@@ -160,7 +164,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&do_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 256);
+    for (int c = 0; c < 4; ++c) mbar_init(&p_chunk[c], 256);
     mbar_init(dp_full, 1);
     mbar_init(ds_full, 256);
     mbar_init(final_bar, 1);
@@ -301,10 +305,20 @@ __global__ void __launch_bounds__(384, 1)
       const bool more = it + 1 < n_iters;
       if (tracer) CSWA_MARK(0, it, 0);
       if (more && !(ok = wait_all(&q_full[q1], ((it + 1) / QS) & 1))) break;
-      if (!(ok = wait_all(p_full, it & 1))) break;
-      if (tracer) CSWA_MARK(0, it, 1);
-      tc_fence_after();
-      issue_acc(tdV, tR0, dDO_mn, ds * L::kTile, it == 0);
+      // dV(it) chunk by chunk as the P/dS warps publish P^T: chunk c holds queries
+      // 16c..16c+15 of each half, i.e. the K steps c and 4 + c
+      for (int c = 0; c < 4; ++c) {
+        if (!(ok = wait_all(&p_chunk[c], it & 1))) break;
+        if (tracer && c == 0) CSWA_MARK(0, it, 1);
+        tc_fence_after();
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int kk = c + 4 * u;
+          mma_ts(tdV, tR0 + u * 64 + c * 8, dDO_mn + ((ds * L::kTile + kk * 2048) >> 4), idKV, (it > 0 || kk > 0),
+                 leader);
+        }
+      }
+      if (!ok) break;
       mma_commit(&do_empty[ds], leader);
 #ifdef CSWA_TRACE
       mma_commit(&trace_bar[0], leader);
@@ -365,6 +379,18 @@ __global__ void __launch_bounds__(384, 1)
     const int trole = 1 + half;
     (void)tracer;
     (void)trole;
+    // dS^T of the previous step (this warp's 32 keys x 64 queries) and where it goes in
+    // the workspace tile the dQ kernel reads; it is stored during this step's P phase,
+    // whose exp2 work leaves the load/store unit idle. The tile is written as 16-byte
+    // units (8 queries of one key) ordered so that every warp store covers 512
+    // contiguous bytes (see ds_unit_offset).
+    uint32_t dsk[32];
+    uint8_t* ds_dst = nullptr;
+    auto store_ds_units = [&](int g0, int g1) {
+#pragma unroll
+      for (int g = g0; g < g1; ++g)
+        *reinterpret_cast<uint4*>(ds_dst + g * 512) = make_uint4(dsk[4 * g], dsk[4 * g + 1], dsk[4 * g + 2], dsk[4 * g + 3]);
+    };
     bool ok = true;
     for (int it = 0; it < n_iters; ++it) {
       const int q0 = iter_q0(it) + 64 * half;  // first query of this thread's columns
@@ -383,33 +409,37 @@ __global__ void __launch_bounds__(384, 1)
       const int c_hi = (W < 0) ? 63 : j + W - q0;   //   and c <= c_hi
       // P = exp2(scale log2e (S - lse/scale)): the MMA has already added -lse/scale, so
       // one packed multiply per two columns; masked entries are set to 0 after the exp2,
-      // tiles inside the band skip the mask (a warp-uniform branch).
+      // tiles inside the band skip the mask (a warp-uniform branch). P^T goes back to
+      // TMEM in four chunks of 16 queries, each published on its own barrier so that
+      // dV starts on the first while the rest is computed. Chunk c's bf16 pairs land in
+      // columns 8c..8c+7, whose fp32 S^T (queries <= 16c+15) is already in registers.
       const float2 sl2v = make_float2(sl2, sl2);
 #pragma unroll
-      for (int c2 = 0; c2 < 32; ++c2) {
-        const float2 e = __fmul2_rn(make_float2(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1])), sl2v);
-        float y[2] = {ex2_approx(e.x), ex2_approx(e.y)};
-        if (!full) {
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[8];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int c = 2 * c2 + u;
-            y[u] = ((c >= c_lo) & (c <= c_hi)) ? y[u] : 0.f;
+        for (int c2 = 8 * c; c2 < 8 * c + 8; ++c2) {
+          const float2 e = __fmul2_rn(make_float2(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1])), sl2v);
+          float y[2] = {ex2_approx(e.x), ex2_approx(e.y)};
+          if (!full) {
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int col = 2 * c2 + u;
+              y[u] = ((col >= c_lo) & (col <= c_hi)) ? y[u] : 0.f;
+            }
           }
+          sr[2 * c2] = __float_as_uint(y[0]);
+          sr[2 * c2 + 1] = __float_as_uint(y[1]);
+          pk[c2 - 8 * c] = pack_bf16x2(y[0], y[1]);
         }
-        sr[2 * c2] = __float_as_uint(y[0]);
-        sr[2 * c2 + 1] = __float_as_uint(y[1]);
+        tmem_st8(tR0 + cols + 8 * c, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_chunk[c]);
+        if (tracer && c == 0) CSWA_MARK(trole, it, 3);
+        if (ds_dst) store_ds_units(2 * c, 2 * c + 2);
       }
       const float* pf = reinterpret_cast<const float*>(sr);
-      if (tracer) CSWA_MARK(trole, it, 3);
-      {
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pf[2 * c], pf[2 * c + 1]);
-        tmem_st32(tR0 + cols, pk);  // over this thread's own (already read) S^T columns
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(p_full);
       if (tracer) CSWA_MARK(trole, it, 4);
 
       ok = __all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, abort_flag));
@@ -418,7 +448,6 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       // dS = P * (dP - Delta): the MMA has already subtracted Delta; one packed multiply
       // per two columns, 32 columns at a time
-      uint32_t dsk[32];
 #pragma unroll
       for (int hc = 0; hc < 2; ++hc) {
         uint32_t dp[32];
@@ -438,18 +467,10 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before();
       mbar_arrive(ds_full);
       if (tracer) CSWA_MARK(trole, it, 7);
-      // dS^T of this warp's 32 keys x 64 queries into the workspace tile the dQ kernel
-      // reads (after the arrive: dK need not wait for these stores), as 16-byte units
-      // (8 queries of one key) ordered so that every warp store covers 512 contiguous
-      // bytes (see ds_unit_offset)
-      {
-        const long long tile = tile0 + (long long)iter_head(it) * p.tiles_per_bh + it % m_cnt;
-        uint8_t* dst = reinterpret_cast<uint8_t*>(p.ds) + (size_t)tile * 32768 + ds_unit_offset(r, 8 * half);
-#pragma unroll
-        for (int g = 0; g < 8; ++g)
-          *reinterpret_cast<uint4*>(dst + g * 512) = make_uint4(dsk[4 * g], dsk[4 * g + 1], dsk[4 * g + 2], dsk[4 * g + 3]);
-      }
+      const long long tile = tile0 + (long long)iter_head(it) * p.tiles_per_bh + it % m_cnt;
+      ds_dst = reinterpret_cast<uint8_t*>(p.ds) + (size_t)tile * 32768 + ds_unit_offset(r, 8 * half);
     }
+    if (ok && ds_dst) store_ds_units(0, 8);
     // ---------------------------------------------------------- dK (warps 4-7) / dV (8-11) epilogue
     ok = __all_sync(0xffffffffu, ok && mbar_wait(final_bar, 0, abort_flag));
     tc_fence_after();

@@ -111,7 +111,11 @@ attn_status_t rope_common(const void* x0, const void* x1, const void* dy0, const
   p.H[0] = Hq;
   p.H[1] = Hkv;
   p.eps = eps;
-  p.log2_base = std::log2((double)base);
+  for (int j = 0; j < D / 2; ++j) {
+    const double u = std::exp2(-2.0 * (double)j / (double)D * std::log2((double)base)) *
+                     0.15915494309189533576888376337251;  // turns per unit position
+    p.turns[j] = (unsigned long long)(u * 18446744073709551616.0);
+  }
   cudaStream_t st = as_stream(stream);
   const long long n_pos = (long long)B * T;
   if (D == 64) return bwd ? launch_rope<64, true>(p, n_pos, st) : launch_rope<64, false>(p, n_pos, st);

@@ -52,12 +52,51 @@ __device__ __forceinline__ uint4 ld_stream(const __nv_bfloat16* p) {
   return v;
 }
 
+// d += a.lo * b.lo + a.hi * b.hi for packed bf16 pairs, accumulated in fp32 (the
+// products of two bf16 values are exact in fp32): no conversion instructions.
+__device__ __forceinline__ float fma_bf16x2_f32(uint32_t a, uint32_t b, float d) {
+  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, al, bl, %0;\n\tfma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
+      : "+f"(d)
+      : "r"(a), "r"(b));
+  return d;
+}
+// d_lo += p * b.lo, d_hi += p * b.hi with p a bf16 value (in the low half of pp)
+__device__ __forceinline__ void fma_bf16_pair_f32(uint32_t pp, uint32_t b, float& lo, float& hi) {
+  asm("{\n\t.reg .b16 p, x, bl, bh;\n\tmov.b32 {p, x}, %2;\n\tmov.b32 {bl, bh}, %3;\n\t"
+      "fma.rn.f32.bf16 %0, p, bl, %0;\n\tfma.rn.f32.bf16 %1, p, bh, %1;\n\t}"
+      : "+f"(lo), "+f"(hi)
+      : "r"(pp), "r"(b));
+}
+
+// Sum of v[0..7] (one partial dot product per key) over the 16 lanes of a key-row
+// group, as a transposing butterfly: 8 shuffles for 8 keys. Lane lr ends with the
+// full sum of key (lr >> 1) & 7.
+__device__ __forceinline__ float reduce8x16(float (&v)[8], int lr) {
+  const bool b3 = lr & 8, b2 = lr & 4, b1 = lr & 2;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float send = b3 ? v[i] : v[i + 4], keep = b3 ? v[i + 4] : v[i];
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float send = b2 ? v[i] : v[i + 2], keep = b2 ? v[i + 2] : v[i];
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+  }
+  const float send = b1 ? v[0] : v[1], keep = b1 ? v[1] : v[0];
+  float r = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+  return r + __shfl_xor_sync(0xffffffffu, r, 1);
+}
+
 template <int D, int GMAX>
 __global__ void __launch_bounds__(128) decode_chunk_kernel(const DecodeParams p) {
   constexpr int LK = D / 8;          // lanes per key row
   constexpr int KPP = 128 / LK;      // key rows per pass
   constexpr int PASSES = kDecodeChunk / KPP;
-  constexpr int UNROLL = PASSES < 8 ? PASSES : 8;
+  constexpr int UNROLL = 8;          // key rows per thread in flight (the butterfly takes 8)
+  static_assert(PASSES % UNROLL == 0, "passes per chunk");
+  static_assert(LK == 16 || LK == 8, "lanes per key row");
   __shared__ float s_sc[GMAX][kDecodeChunk];
   __shared__ float s_red[GMAX][4];
   __shared__ float s_stat[GMAX][2];
@@ -73,51 +112,71 @@ __global__ void __launch_bounds__(128) decode_chunk_kernel(const DecodeParams p)
   const int k_begin = lo + chunk * kDecodeChunk;
   if (k_begin > P) return;
   const int nk = min(P, k_begin + kDecodeChunk - 1) - k_begin + 1;
+  // chunks before the last hold 128 cache rows and not the new token: no bounds
+  // checks, no row substitution
+  const bool full = (k_begin + kDecodeChunk - 1 < P);
   const int tid = threadIdx.x, lr = tid % LK, sub = tid / LK, warp = tid >> 5, lane = tid & 31;
   const int G = p.G;
   const bool append = p.kn != nullptr;
+  const size_t row_stride = (size_t)p.Hkv * D;          // elements between consecutive keys
+  const size_t pass_stride = row_stride * KPP;          // between a thread's consecutive rows
+  const size_t cache_off = (((size_t)b * p.Tmax + k_begin + sub) * p.Hkv + hk) * D + lr * 8;
+  const size_t fresh_off = ((size_t)b * p.Hkv + hk) * D + lr * 8;
 
-  float qf[GMAX][8];
+  uint32_t qv[GMAX][4];
 #pragma unroll
   for (int g = 0; g < GMAX; ++g) {
-    if (g < G) {
-      bf16x8_to_float(*reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.Hq + hk * G + g) * D + lr * 8),
-                      qf[g]);
-    }
+    const uint4 t = (g < G) ? *reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.Hq + hk * G + g) * D + lr * 8)
+                            : make_uint4(0, 0, 0, 0);
+    qv[g][0] = t.x, qv[g][1] = t.y, qv[g][2] = t.z, qv[g][3] = t.w;
   }
-  auto row_ptr = [&](const __nv_bfloat16* cache, const __nv_bfloat16* fresh, int j) {
-    return (append && j == P) ? fresh + ((size_t)b * p.Hkv + hk) * D + lr * 8
-                              : cache + (((size_t)b * p.Tmax + j) * p.Hkv + hk) * D + lr * 8;
+  // row kc of the chunk for this thread's pass u: cache row, or the new token at P
+  auto load_row = [&](const __nv_bfloat16* cache, const __nv_bfloat16* fresh, int u) {
+    const int kc = u * KPP + sub;
+    if (full) return ld_stream(cache + cache_off + u * pass_stride);
+    if (kc >= nk) return make_uint4(0, 0, 0, 0);
+    if (append && k_begin + kc == P) return ld_stream(fresh + fresh_off);
+    return ld_stream(cache + cache_off + u * pass_stride);
   };
 
-  // pass 1: scores
+  // pass 1: scores s = <q, k> * scale * log2(e)
   for (int ps = 0; ps < PASSES; ps += UNROLL) {
     uint4 kv[UNROLL];
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      const int kc = (ps + u) * KPP + sub;
-      kv[u] = kc < nk ? ld_stream(row_ptr(p.kc, p.kn, k_begin + kc)) : make_uint4(0, 0, 0, 0);
-    }
+    for (int u = 0; u < UNROLL; ++u) kv[u] = load_row(p.kc, p.kn, ps + u);
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      float kf[8];
-      bf16x8_to_float(kv[u], kf);
-      const int kc = (ps + u) * KPP + sub;
+    for (int g = 0; g < GMAX; ++g) {
+      if (g < G) {
+        float d[8];
 #pragma unroll
-      for (int g = 0; g < GMAX; ++g) {
-        if (g < G) {
-          float d = 0.f;
+        for (int u = 0; u < UNROLL; ++u) {
+          float t = 0.f;
+          t = fma_bf16x2_f32(qv[g][0], kv[u].x, t);
+          t = fma_bf16x2_f32(qv[g][1], kv[u].y, t);
+          t = fma_bf16x2_f32(qv[g][2], kv[u].z, t);
+          t = fma_bf16x2_f32(qv[g][3], kv[u].w, t);
+          d[u] = t;
+        }
+        float sum;
+        if (LK == 16) {
+          sum = reduce8x16(d, lr);
+          const int kc = (ps + ((lr >> 1) & 7)) * KPP + sub;
+          if ((lr & 1) == 0 && kc < nk) s_sc[g][kc] = sum * p.scale_log2;
+        } else {
+          // 8 lanes per row: reduce each key separately
 #pragma unroll
-          for (int e = 0; e < 8; ++e) d = fmaf(qf[g][e], kf[e], d);
+          for (int u = 0; u < UNROLL; ++u) {
+            float t = d[u];
 #pragma unroll
-          for (int o = LK / 2; o >= 1; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-          if (lr == 0 && kc < nk) s_sc[g][kc] = d * p.scale_log2;
+            for (int o = LK / 2; o >= 1; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+            const int kc = (ps + u) * KPP + sub;
+            if (lr == 0 && kc < nk) s_sc[g][kc] = t * p.scale_log2;
+          }
         }
       }
     }
   }
   __syncthreads();
-
   // pass 2: chunk max and exponentials (thread tid owns key tid)
 #pragma unroll
   for (int g = 0; g < GMAX; ++g) {
@@ -147,7 +206,7 @@ __global__ void __launch_bounds__(128) decode_chunk_kernel(const DecodeParams p)
   if (tid < G) s_stat[tid][1] = s_acc[0][tid][0] + s_acc[0][tid][1] + s_acc[0][tid][2] + s_acc[0][tid][3];
   __syncthreads();
 
-  // pass 3: acc = sum_j p_j v_j
+  // pass 3: acc = sum_j p_j v_j, p_j rounded to bf16 (as the PV product of attn_fwd)
   float acc[GMAX][8];
 #pragma unroll
   for (int g = 0; g < GMAX; ++g)
@@ -156,21 +215,19 @@ __global__ void __launch_bounds__(128) decode_chunk_kernel(const DecodeParams p)
   for (int ps = 0; ps < PASSES; ps += UNROLL) {
     uint4 vv[UNROLL];
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      const int kc = (ps + u) * KPP + sub;
-      vv[u] = kc < nk ? ld_stream(row_ptr(p.vc, p.vn, k_begin + kc)) : make_uint4(0, 0, 0, 0);
-    }
+    for (int u = 0; u < UNROLL; ++u) vv[u] = load_row(p.vc, p.vn, ps + u);
 #pragma unroll
     for (int u = 0; u < UNROLL; ++u) {
-      float vf[8];
-      bf16x8_to_float(vv[u], vf);
       const int kc = (ps + u) * KPP + sub;
 #pragma unroll
       for (int g = 0; g < GMAX; ++g) {
         if (g < G) {
-          const float pj = kc < nk ? s_sc[g][kc] : 0.f;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(pj, vf[e], acc[g][e]);
+          const float pj = (full || kc < nk) ? s_sc[g][kc] : 0.f;
+          const uint32_t pb = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(pj));
+          fma_bf16_pair_f32(pb, vv[u].x, acc[g][0], acc[g][1]);
+          fma_bf16_pair_f32(pb, vv[u].y, acc[g][2], acc[g][3]);
+          fma_bf16_pair_f32(pb, vv[u].z, acc[g][4], acc[g][5]);
+          fma_bf16_pair_f32(pb, vv[u].w, acc[g][6], acc[g][7]);
         }
       }
     }

@@ -164,35 +164,42 @@ __global__ void __launch_bounds__(384, 1)
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
     };
     int cnt[2] = {0, 0};
-    bool ok = wait_all(q_full, 0);
+    auto active = [&](int s, int t) { return has[s] && lo[s] <= t && t <= hi[s]; };
+    auto issue_S = [&](int s, int st) {
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+        mma_ss(tS(s), (s ? dQ1 : dQ0) + (off >> 4), dK0 + ((st * L::kTile + off) >> 4), idS, kk > 0, leader);
+      }
+      mma_commit(&s_full[s], leader);
+    };
+    // Ping-pong: S_s of key tile t+1 follows PV_s of tile t at once, so each slot's
+    // chain S -> softmax -> PV runs without waiting for the other slot's PV.
+    bool ok = wait_all(q_full, 0) && wait_all(&k_full[0], 0);
     tc_fence_after();
+    if (ok)
+      for (int s = 0; s < 2; ++s)
+        if (active(s, t_lo)) issue_S(s, 0);
     int n = 0;
     for (int t = t_lo; ok && t <= t_hi; ++t, ++n) {
       const int st = n & 1;
       const uint32_t ph = (n >> 1) & 1;
-      if (!(ok = wait_all(&k_full[st], ph))) break;
-      tc_fence_after();
-      for (int s = 0; s < 2; ++s) {
-        if (!(has[s] && lo[s] <= t && t <= hi[s])) continue;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tS(s), (s ? dQ1 : dQ0) + (off >> 4), dK0 + ((st * L::kTile + off) >> 4), idS, kk > 0, leader);
-        }
-        mma_commit(&s_full[s], leader);
-      }
+      const bool next = t + 1 <= t_hi;
       if (!(ok = wait_all(&v_full[st], ph))) break;
-      tc_fence_after();
+      if (next && !(ok = wait_all(&k_full[st ^ 1], ((n + 1) >> 1) & 1))) break;
       for (int s = 0; s < 2; ++s) {
-        if (!(has[s] && lo[s] <= t && t <= hi[s])) continue;
-        if (!(ok = wait_all(&p_full[s], cnt[s] & 1))) break;
-        tc_fence_after();
+        if (active(s, t)) {
+          if (!(ok = wait_all(&p_full[s], cnt[s] & 1))) break;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tO(s), tS(s) + kk * 8, dV0 + ((st * L::kTile + kk * 2048) >> 4), idO, (cnt[s] > 0 || kk > 0),
-                 leader);
-        mma_commit(&pv_done[s], leader);
-        ++cnt[s];
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tO(s), tS(s) + kk * 8, dV0 + ((st * L::kTile + kk * 2048) >> 4), idO, (cnt[s] > 0 || kk > 0),
+                   leader);
+          mma_commit(&pv_done[s], leader);
+          ++cnt[s];
+        }
+        tc_fence_after();
+        if (next && active(s, t + 1)) issue_S(s, st ^ 1);
       }
       if (!ok) break;
       mma_commit(&kv_empty[st], leader);

@@ -9,9 +9,9 @@
 // with p = t + pos[b] (pos may be null). Backward, with g = rotation of dy by -phi:
 //   dx = (g - xh (g . xh) / D) / r.
 //
-// HBM-bound elementwise work: D/8 lanes own one row, 16 bytes each (one
-// vector load per operand), the pair partner j + D/2 is a shuffle away. The
-// angles are computed once per position and shared by all its head rows.
+// HBM-bound elementwise work: D/8 lanes own one row, each holding both members
+// of its rotation pairs (two 8-byte loads per operand). The angles are computed
+// once per position and shared by all its head rows.
 #pragma once
 #include "ptx.cuh"
 
@@ -25,137 +25,155 @@ struct RopeParams {
   long long rows[2];  // B*T*Hq, B*T*Hkv (0 when the operand is absent)
   int T, H[2];
   float eps;
-  double log2_base;
+  // turns of pair j per unit position, as a 64-bit fixed-point fraction:
+  // U_j = (base^(-2j/D) / (2 pi)) * 2^64, computed on the host in double precision
+  unsigned long long turns[64];
 };
 
 // Each block owns kPosPerBlock consecutive (b, t) positions and every q and k
-// head row at them. It first builds one cos/sin table per position in shared
-// memory -- the angle of pair j at position p, in turns, is p * u_j with
-// u_j = omega_j / (2 pi), held as a 64-bit fixed-point fraction U_j = u_j 2^64,
-// so p * U_j mod 2^64 is the exact fractional turn for any 32-bit position and
-// its top 32 bits, read as signed, give the reduced angle in [-pi, pi) -- and
-// then streams the rows: D/8 lanes per row, one 16-byte load per operand.
+// head row at them (the block's q rows, and its k rows, are each one contiguous
+// range). The angle of pair j at position p, in turns, is p * U_j mod 2^64 (exact
+// for any 32-bit position); its top 32 bits, read as signed, give the reduced angle
+// in [-pi, pi). A block first issues the loads of its first rows, then builds one
+// cos/sin table per position in shared memory while they are in flight, and streams
+// the rows: D/8 lanes per row, lane l owning elements 4l..4l+3 of each half (so a
+// rotation pair never leaves its lane), kBatch rows per thread in flight.
 constexpr int kPosPerBlock = 8;
 
 template <int D, bool kBwd>
-__global__ void __launch_bounds__(256) rope_qknorm_kernel(const RopeParams p) {
+__global__ void __launch_bounds__(256, kBwd ? 3 : 4) rope_qknorm_kernel(const __grid_constant__ RopeParams p) {
   constexpr int kLanesPerRow = D / 8;
   constexpr int kHalf = D / 2;
-  __shared__ unsigned long long turns[kHalf];
-  __shared__ float2 cs[kPosPerBlock][kHalf];  // (cos, sin)
+  constexpr int kRowsPerRound = 256 / kLanesPerRow;
+  constexpr int kBatch = 4;  // rows per thread in flight (8 loads in the backward)
+  __shared__ float4 cs4[kPosPerBlock][kHalf / 2];  // (cos_j, sin_j, cos_j+1, sin_j+1)
 
   const long long n_pos = p.rows[0] > 0 ? p.rows[0] / p.H[0] : p.rows[1] / p.H[1];  // B * T
   const long long pos0 = (long long)blockIdx.x * kPosPerBlock;
   const int Hq = p.rows[0] > 0 ? p.H[0] : 0;
   const int Hk = p.rows[1] > 0 ? p.H[1] : 0;
-
-  for (int j = threadIdx.x; j < kHalf; j += blockDim.x) {
-    const double u = exp2(-2.0 * (double)j / (double)D * p.log2_base) * 0.15915494309189533576888376337251;
-    turns[j] = (unsigned long long)(u * 18446744073709551616.0);
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < kPosPerBlock * kHalf; e += blockDim.x) {
-    const int pi = e / kHalf, j = e % kHalf;
-    const long long bt = pos0 + pi;
-    float c = 1.f, sn = 0.f;
-    if (bt < n_pos) {
-      const int t = (int)(bt % p.T), b = (int)(bt / p.T);
-      const unsigned long long pos = (unsigned long long)(unsigned)(t + (p.pos ? p.pos[b] : 0));
-      const unsigned long long frac = pos * turns[j];
-      const float ang = (float)(int)(unsigned)(frac >> 32) * 1.4629180792671596e-09f;  // 2 pi / 2^32
-      __sincosf(ang, &sn, &c);
-    }
-    cs[pi][j] = make_float2(c, sn);
-  }
-  __syncthreads();
-
   const int n_pos_here = (int)min((long long)kPosPerBlock, n_pos - pos0);
   const int rows_q = n_pos_here * Hq, rows_k = n_pos_here * Hk;
-  const int tasks = (rows_q + rows_k) * kLanesPerRow;
+  const int rows_all = rows_q + rows_k;
   const int lr = threadIdx.x % kLanesPerRow;
-  const bool second_half = lr >= kLanesPerRow / 2;
-  const int j0 = (lr % (kLanesPerRow / 2)) * 8;
-  // every thread runs the same trip count so the row shuffles stay warp-uniform
-  const int trips = (kPosPerBlock * (Hq + Hk) * kLanesPerRow + blockDim.x - 1) / blockDim.x;
-  for (int tr = 0; tr < trips; ++tr) {
-    const int task = tr * blockDim.x + threadIdx.x;
-    const bool active = task < tasks;
-    const int row = task / kLanesPerRow;
-    const int seg = (row >= rows_q) ? 1 : 0;
-    const int rr = seg ? row - rows_q : row;                 // row within the segment, block-local
+  const int row0 = threadIdx.x / kLanesPerRow;
+  const int j0 = lr * 4;  // elements j0..j0+3 and kHalf + j0..kHalf + j0+3
+  const float inv_hq = Hq ? 1.f / (float)Hq : 0.f, inv_hk = Hk ? 1.f / (float)Hk : 0.f;
+  // every thread runs the same number of rounds so the row shuffles stay warp-uniform
+  const int rounds = (kPosPerBlock * (Hq + Hk) + kRowsPerRound - 1) / kRowsPerRound;
+
+  // block-local row -> (operand, element offset, position in block)
+  auto locate = [&](int row, int& seg, size_t& off, int& pi) {
+    seg = row >= rows_q;
+    const int rr = seg ? row - rows_q : row;
     const int H = seg ? Hk : Hq;
-    const int pi = active ? rr / H : 0;
-    const long long grow = (pos0 * H) + rr;                  // global row of the segment
-    float x[8], g[8];
-    if (active) {
-      const uint4 xv = *reinterpret_cast<const uint4*>(p.x[seg] + grow * D + lr * 8);
-      const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xv);
+    // rr < 2^20, so the float quotient truncates to the exact integer one
+    pi = __float2int_rz(((float)rr + 0.5f) * (seg ? inv_hk : inv_hq));
+    off = ((size_t)pos0 * H + rr) * D + j0;
+  };
+
+  for (int rd0 = 0; rd0 < rounds; rd0 += kBatch) {
+    uint2 xa[kBatch], xb[kBatch], ga[kBatch], gb[kBatch];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float2 f = __bfloat1622float2(x2[u]);
-        x[2 * u] = f.x;
-        x[2 * u + 1] = f.y;
-      }
+    for (int u = 0; u < kBatch; ++u) {
+      const int row = (rd0 + u) * kRowsPerRound + row0;
+      int seg, pi;
+      size_t off;
+      locate(row, seg, off, pi);
+      const bool active = row < rows_all;
+      xa[u] = active ? *reinterpret_cast<const uint2*>(p.x[seg] + off) : make_uint2(0, 0);
+      xb[u] = active ? *reinterpret_cast<const uint2*>(p.x[seg] + off + kHalf) : make_uint2(0, 0);
       if (kBwd) {
-        const uint4 gv = *reinterpret_cast<const uint4*>(p.dy[seg] + grow * D + lr * 8);
-        const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+        ga[u] = active ? *reinterpret_cast<const uint2*>(p.dy[seg] + off) : make_uint2(0, 0);
+        gb[u] = active ? *reinterpret_cast<const uint2*>(p.dy[seg] + off + kHalf) : make_uint2(0, 0);
+      }
+    }
+    if (rd0 == 0) {
+      // the cos/sin table, built while the first loads are in flight
+      for (int e = threadIdx.x; e < kPosPerBlock * kHalf; e += blockDim.x) {
+        const int pi = e / kHalf, j = e % kHalf;
+        const long long bt = pos0 + pi;
+        float c = 1.f, sn = 0.f;
+        if (bt < n_pos) {
+          const int t = (int)(bt % p.T), b = (int)(bt / p.T);
+          const unsigned long long pos = (unsigned long long)(unsigned)(t + (p.pos ? p.pos[b] : 0));
+          const unsigned long long frac = pos * p.turns[j];
+          const float ang = (float)(int)(unsigned)(frac >> 32) * 1.4629180792671596e-09f;  // 2 pi / 2^32
+          __sincosf(ang, &sn, &c);
+        }
+        reinterpret_cast<float2*>(&cs4[pi][0])[j] = make_float2(c, sn);
+      }
+      __syncthreads();
+    }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float2 f = __bfloat1622float2(g2[u]);
-          g[2 * u] = f.x;
-          g[2 * u + 1] = f.y;
+    for (int u = 0; u < kBatch; ++u) {
+      if (rd0 + u >= rounds) break;  // uniform across the block
+      const int row = (rd0 + u) * kRowsPerRound + row0;
+      int seg, pi;
+      size_t off;
+      locate(row, seg, off, pi);
+      const bool active = row < rows_all;
+      if (!active) pi = 0;
+      // a[i] = element j0 + i, b[i] = element kHalf + j0 + i
+      float a[4], bq[4];
+      {
+        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&xa[u]);
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&xb[u]);
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          const float2 fa = __bfloat1622float2(a2[v]), fb = __bfloat1622float2(b2[v]);
+          a[2 * v] = fa.x, a[2 * v + 1] = fa.y, bq[2 * v] = fb.x, bq[2 * v + 1] = fb.y;
         }
       }
-    } else {
+      float ss = 0.f;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) x[u] = g[u] = 0.f;
-    }
-    float ss = 0.f;
+      for (int v = 0; v < 4; ++v) ss = fmaf(a[v], a[v], fmaf(bq[v], bq[v], ss));
 #pragma unroll
-    for (int u = 0; u < 8; ++u) ss = fmaf(x[u], x[u], ss);
+      for (int o = kLanesPerRow / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float inv_r = rsqrtf(ss * (1.f / D) + p.eps);
+      const float4 t01 = cs4[pi][j0 / 2], t23 = cs4[pi][j0 / 2 + 1];
+      const float c[4] = {t01.x, t01.z, t23.x, t23.z}, s[4] = {t01.y, t01.w, t23.y, t23.w};
+      float oa[4], ob[4];
+      if (!kBwd) {
 #pragma unroll
-    for (int o = kLanesPerRow / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float inv_r = rsqrtf(ss * (1.f / D) + p.eps);
-    float c[8], s[8];
+        for (int v = 0; v < 4; ++v) {
+          const float xa_ = a[v] * inv_r, xb_ = bq[v] * inv_r;
+          oa[v] = fmaf(-xb_, s[v], xa_ * c[v]);
+          ob[v] = fmaf(xa_, s[v], xb_ * c[v]);
+        }
+      } else {
+        // g = rotation of dy by -phi
+        float ga_[4], gb_[4];
+        {
+          const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&ga[u]);
+          const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&gb[u]);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const float2 t = cs[pi][j0 + u];
-      c[u] = t.x;
-      s[u] = t.y;
-    }
-    float out[8];
-    if (!kBwd) {
-      float xh[8], partner[8];
+          for (int v = 0; v < 2; ++v) {
+            const float2 fa = __bfloat1622float2(a2[v]), fb = __bfloat1622float2(b2[v]);
+            ga_[2 * v] = fa.x, ga_[2 * v + 1] = fa.y, gb_[2 * v] = fb.x, gb_[2 * v + 1] = fb.y;
+          }
+        }
+        float gra[4], grb[4], dot = 0.f;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) xh[u] = x[u] * inv_r;
+        for (int v = 0; v < 4; ++v) {
+          gra[v] = fmaf(gb_[v], s[v], ga_[v] * c[v]);
+          grb[v] = fmaf(-ga_[v], s[v], gb_[v] * c[v]);
+          dot = fmaf(gra[v], a[v] * inv_r, fmaf(grb[v], bq[v] * inv_r, dot));
+        }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) partner[u] = __shfl_xor_sync(0xffffffffu, xh[u], kLanesPerRow / 2);
+        for (int o = kLanesPerRow / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        const float proj = dot * (1.f / D);
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        out[u] = second_half ? fmaf(partner[u], s[u], xh[u] * c[u]) : fmaf(-partner[u], s[u], xh[u] * c[u]);
-    } else {
-      // g = rotation of dy by -phi
-      float partner[8], gr[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) partner[u] = __shfl_xor_sync(0xffffffffu, g[u], kLanesPerRow / 2);
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        gr[u] = second_half ? fmaf(-partner[u], s[u], g[u] * c[u]) : fmaf(partner[u], s[u], g[u] * c[u]);
-      float dot = 0.f;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) dot = fmaf(gr[u], x[u] * inv_r, dot);
-#pragma unroll
-      for (int o = kLanesPerRow / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-      const float proj = dot * (1.f / D);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) out[u] = (gr[u] - x[u] * inv_r * proj) * inv_r;
-    }
-    if (active) {
-      uint4 ov;
-      uint32_t* o32 = reinterpret_cast<uint32_t*>(&ov);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) o32[u] = pack_bf16x2(out[2 * u], out[2 * u + 1]);
-      *reinterpret_cast<uint4*>(p.y[seg] + grow * D + lr * 8) = ov;
+        for (int v = 0; v < 4; ++v) {
+          oa[v] = (gra[v] - a[v] * inv_r * proj) * inv_r;
+          ob[v] = (grb[v] - bq[v] * inv_r * proj) * inv_r;
+        }
+      }
+      if (active) {
+        *reinterpret_cast<uint2*>(p.y[seg] + off) = make_uint2(pack_bf16x2(oa[0], oa[1]), pack_bf16x2(oa[2], oa[3]));
+        *reinterpret_cast<uint2*>(p.y[seg] + off + kHalf) =
+            make_uint2(pack_bf16x2(ob[0], ob[1]), pack_bf16x2(ob[2], ob[3]));
+      }
     }
   }
 }
