@@ -246,7 +246,9 @@ def run_gpu(args, rank, world, local):
     bwd_avg_ms = per_op["bwd"] / (2 * args.steps)
     bwd_tflops = flops_b / 2 / (bwd_avg_ms * 1e-3) / 1e12
     fwd_avg_ms = per_op["fwd"] / (2 * args.steps)
-    traffic = ncu_traffic("attn_bwd_kernel")
+    # DRAM bytes of one attn_bwd call = its three launches (ncu, window-1024 layer)
+    parts = [ncu_traffic(kn) for kn in ("attn_bwd_prep_kernel", "attn_bwd_kernel", "attn_bwd_dq_kernel")]
+    traffic = sum(parts) if all(x is not None for x in parts) else None
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
@@ -259,11 +261,13 @@ def run_gpu(args, rank, world, local):
         "fwd_tflops": round(flops_f / 2 / (fwd_avg_ms * 1e-3) / 1e12, 1),
         "bwd_tflops": round(bwd_tflops, 1),
         "bwd_tflops_fa_convention": round(bwd_tflops * 10 / 8, 1),
-        "roofline": {"kernel": "attn_bwd call (prep + main + dq cast launches), both layers", "bound": "tensor",
+        "roofline": {"kernel": "attn_bwd call (prep + main + dQ launches), both layers", "bound": "tensor",
                      "achieved": round(bwd_tflops, 1), "peak": peak_sus, "unit": "TFLOP/s",
                      "frac": round(bwd_tflops / peak_sus, 4),
                      "peak_kind": f"bf16 sustained ({pk_src}); burst {peak_burst}",
                      "traffic": traffic,
+                     "traffic_note": "ncu dram read+write bytes of one attn_bwd call (prep + main + dQ), "
+                                     "window-1024 layer; null when the kernel sources changed since the capture",
                      "algorithmic_flops_per_launch": flops_b / 2},
         "gpu_launches": 12 * args.steps,  # per layer: prologue, fwd, bwd prep/main/dq, prologue bwd
         "clocks": clocks.summary(),
@@ -426,7 +430,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=800)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="cswa", choices=["cswa", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the cpu_baseline oracle sample")

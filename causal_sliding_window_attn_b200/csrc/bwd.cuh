@@ -655,10 +655,18 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16*
   const long long row = gtid / LK;
   const int lr = (int)(gtid % LK);
   const bool active = row < rows;
-  // row enumerates (b, t, h) with t over the padded length
-  const int h = active ? (int)(row % Hq) : 0;
-  const long long bt = active ? row / Hq : 0;
-  const int t = (int)(bt % Tpad), b = (int)(bt / Tpad);
+  // row enumerates (b, t, h) with t over the padded length (32-bit math when it fits)
+  int h, t, b;
+  if (rows < (1ll << 31)) {
+    const unsigned r32 = active ? (unsigned)row : 0u;
+    h = (int)(r32 % (unsigned)Hq);
+    const unsigned bt = r32 / (unsigned)Hq;
+    t = (int)(bt % (unsigned)Tpad), b = (int)(bt / (unsigned)Tpad);
+  } else {
+    h = active ? (int)(row % Hq) : 0;
+    const long long bt = active ? row / Hq : 0;
+    t = (int)(bt % Tpad), b = (int)(bt / Tpad);
+  }
   const bool real = active && t < T;
   float dsum = 0.f;
   if (real) {

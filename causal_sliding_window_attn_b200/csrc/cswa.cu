@@ -50,8 +50,6 @@ bool encode_bthd(CUtensorMap* m, const void* base, int B, int T, int H, int D, i
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The stored dS^T tiles: a (rows, 128) bf16 matrix, box = 64 columns x 128 rows,
-// 128-byte swizzle (the shared-memory layout of one 64-query panel).
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool dims_ok(int B, int T, int Hq, int Hkv) {
   return B >= 1 && T >= 1 && Hq >= 1 && Hkv >= 1 && Hq % Hkv == 0 && (long long)B * T * Hq < (1ll << 40);

@@ -41,11 +41,13 @@ struct RopeParams {
 constexpr int kPosPerBlock = 8;
 
 template <int D, bool kBwd>
-__global__ void __launch_bounds__(256, kBwd ? 3 : 4) rope_qknorm_kernel(const __grid_constant__ RopeParams p) {
+__global__ void __launch_bounds__(256, 4) rope_qknorm_kernel(const __grid_constant__ RopeParams p) {
   constexpr int kLanesPerRow = D / 8;
   constexpr int kHalf = D / 2;
   constexpr int kRowsPerRound = 256 / kLanesPerRow;
-  constexpr int kBatch = 4;  // rows per thread in flight (8 loads in the backward)
+  // rows per thread in flight: 4 (8 loads of 8 bytes); the backward, with twice the
+  // loads per row and more live values, keeps 2 so that 4 blocks fit per SM
+  constexpr int kBatch = kBwd ? 2 : 4;
   __shared__ float4 cs4[kPosPerBlock][kHalf / 2];  // (cos_j, sin_j, cos_j+1, sin_j+1)
 
   const long long n_pos = p.rows[0] > 0 ? p.rows[0] / p.H[0] : p.rows[1] / p.H[1];  // B * T
