@@ -10,7 +10,7 @@
 // One CTA owns two 128-row query tiles ("slots") of one (b, h): tiles 2p and
 // 2p+1. It walks the union of their key-tile ranges inside the causal/window
 // band; key tiles outside the band are never loaded.
-//   warp 0      TMA producer: Q once, then K/V tiles into a 2-stage ring
+//   warp 0      TMA producer: Q once, then K and V tiles into 2-stage rings
 //   warp 1      MMA issuer (whole warp, one elected lane issues): S_s = Q_s K^T (SS),
 //               O_s += P_s V (TS)
 //   warp 2      TMEM allocator
@@ -57,13 +57,14 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;    // [2]
   uint64_t* v_full = bars + 3;    // [2]
-  uint64_t* kv_empty = bars + 5;  // [2]
+  uint64_t* k_empty = bars + 5;   // [2] S of the tile has read K
   uint64_t* s_full = bars + 7;    // [2]
   uint64_t* p_full = bars + 9;    // [2]
   uint64_t* pv_done = bars + 11;  // [2]
   uint64_t* final_bar = bars + 13;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 15);
+  uint64_t* v_empty = bars + 16;  // [2] PV of the tile has read V
 
   const int warp = warp_id(), lane = lane_id();
   const int h = blockIdx.x, b = blockIdx.y;
@@ -88,7 +89,8 @@ __global__ void __launch_bounds__(384, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 128);
       mbar_init(&pv_done[s], 1);
@@ -122,27 +124,30 @@ __global__ void __launch_bounds__(384, 1)
         if (has[s])
           for (int pn = 0; pn < L::kPanels; ++pn)
             tma_load_4d(smem + (s ? L::kQ1 : L::kQ0) + pn * 16384, &tm_q, q_full, pn * 64, h, qt[s] * 128, b);
-      int n = 0, last_issue[2] = {-1, -1};
+      // K and V stages are released separately (K once the S products have read it, V
+      // once the PV products have), so K of the next tile loads a whole tile ahead
+      int n = 0, last_k[2] = {-1, -1}, last_v[2] = {-1, -1};
       for (int t = t_lo; t <= t_hi; ++t, ++n) {
         const int st = n & 1;
         const uint32_t ph = (n >> 1) & 1;
-        if (!mbar_wait(&kv_empty[st], ph ^ 1, abort_flag)) break;
+        if (!mbar_wait(&k_empty[st], ph ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(&k_full[st], L::kTile);
         for (int pn = 0; pn < L::kPanels; ++pn)
           tma_load_4d(smem + L::kK0 + st * L::kTile + pn * 16384, &tm_k, &k_full[st], pn * 64, hk, t * 128, b);
+        last_k[st] = n;
+        if (!mbar_wait(&v_empty[st], ph ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(&v_full[st], L::kTile);
         for (int pn = 0; pn < L::kPanels; ++pn)
           tma_load_4d(smem + L::kV0 + st * L::kTile + pn * 16384, &tm_v, &v_full[st], pn * 64, hk, t * 128, b);
-        last_issue[st] = n;
+        last_v[st] = n;
       }
       if (*abort_flag) {
         // never leave with copies in flight: wait (bounded) for the last load of each stage
-        for (int st = 0; st < 2; ++st)
-          if (last_issue[st] >= 0) {
-            volatile int dummy = 0;
-            mbar_wait(&k_full[st], (last_issue[st] >> 1) & 1, &dummy);
-            mbar_wait(&v_full[st], (last_issue[st] >> 1) & 1, &dummy);
-          }
+        for (int st = 0; st < 2; ++st) {
+          volatile int dummy = 0;
+          if (last_k[st] >= 0) mbar_wait(&k_full[st], (last_k[st] >> 1) & 1, &dummy);
+          if (last_v[st] >= 0) mbar_wait(&v_full[st], (last_v[st] >> 1) & 1, &dummy);
+        }
         volatile int dummy = 0;
         mbar_wait(q_full, 0, &dummy);
       }
@@ -177,19 +182,26 @@ __global__ void __launch_bounds__(384, 1)
     // chain S -> softmax -> PV runs without waiting for the other slot's PV.
     bool ok = wait_all(q_full, 0) && wait_all(&k_full[0], 0);
     tc_fence_after();
-    if (ok)
+    if (ok) {
       for (int s = 0; s < 2; ++s)
         if (active(s, t_lo)) issue_S(s, 0);
+      mma_commit(&k_empty[0], leader);
+    }
     int n = 0;
+    const bool tracer = (lane == 0);
+    (void)tracer;
     for (int t = t_lo; ok && t <= t_hi; ++t, ++n) {
       const int st = n & 1;
       const uint32_t ph = (n >> 1) & 1;
       const bool next = t + 1 <= t_hi;
+      if (tracer) CSWA_MARK(0, n, 0);
       if (!(ok = wait_all(&v_full[st], ph))) break;
       if (next && !(ok = wait_all(&k_full[st ^ 1], ((n + 1) >> 1) & 1))) break;
+      if (tracer) CSWA_MARK(0, n, 1);
       for (int s = 0; s < 2; ++s) {
         if (active(s, t)) {
           if (!(ok = wait_all(&p_full[s], cnt[s] & 1))) break;
+          if (tracer) CSWA_MARK(0, n, 2 + 3 * s);
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
@@ -197,12 +209,15 @@ __global__ void __launch_bounds__(384, 1)
                    leader);
           mma_commit(&pv_done[s], leader);
           ++cnt[s];
+          if (tracer) CSWA_MARK(0, n, 3 + 3 * s);
         }
         tc_fence_after();
         if (next && active(s, t + 1)) issue_S(s, st ^ 1);
+        if (tracer) CSWA_MARK(0, n, 4 + 3 * s);
       }
       if (!ok) break;
-      mma_commit(&kv_empty[st], leader);
+      mma_commit(&v_empty[st], leader);                 // V(t) read by both PVs
+      if (next) mma_commit(&k_empty[st ^ 1], leader);  // K(t+1) read by both S
     }
     // every MMA issued above has finished before TMEM is released
     mma_commit(final_bar, leader);
@@ -225,8 +240,12 @@ __global__ void __launch_bounds__(384, 1)
       float m_run = -INFINITY, l_run = 0.f;
       int cnt = 0;
       bool ok = true;
+      const bool tracer = (quarter == 0 && lane == 0);
+      (void)tracer;
       for (int t = my_lo; t <= my_hi; ++t, ++cnt) {
+        if (tracer) CSWA_MARK(1 + s, cnt, 0);
         ok = __all_sync(0xffffffffu, mbar_wait(&s_full[s], cnt & 1, abort_flag));
+        if (tracer) CSWA_MARK(1 + s, cnt, 1);
         if (!ok) break;
         tc_fence_after();
         uint32_t r[128];
@@ -257,6 +276,7 @@ __global__ void __launch_bounds__(384, 1)
           mx4[(c >> 3) & 3] = fmax3(mx4[(c >> 3) & 3], __uint_as_float(r[c + 6]), __uint_as_float(r[c + 7]));
         }
         const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        if (tracer) CSWA_MARK(1 + s, cnt, 2);
         const float m_tile = mx * sl2;
         bool rescale = false;
         float factor = 1.f;
@@ -280,6 +300,7 @@ __global__ void __launch_bounds__(384, 1)
           r[c] = pack_bf16x2(pp.x, pp.y);
         }
         l_run += ((ls4[0].x + ls4[0].y) + (ls4[1].x + ls4[1].y)) + ((ls4[2].x + ls4[2].y) + (ls4[3].x + ls4[3].y));
+        if (tracer) CSWA_MARK(1 + s, cnt, 3);
         tmem_st32(tSs + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
         tmem_st32(tSs + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
         // rescale only when some row of the warp needs it (O is stable: this tile's
@@ -298,6 +319,7 @@ __global__ void __launch_bounds__(384, 1)
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&p_full[s]);
+        if (tracer) CSWA_MARK(1 + s, cnt, 4);
       }
       // ---------------------------------------------------------- epilogue
       if (ok && cnt > 0) ok = mbar_wait(&pv_done[s], (cnt - 1) & 1, abort_flag);
