@@ -503,8 +503,11 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-// dQ = scale * sum_n dS(m, n) K_n for one 128-row query tile m of one query head,
-// from the dS^T tiles bwd_main stored; accumulated in TMEM, written once as bf16.
+// dQ = scale * sum_n dS(m, n) K_n for every 128-row query tile m of every query
+// head, from the dS^T tiles bwd_main stored; accumulated in TMEM, written once as bf16.
+// Persistent: one CTA per SM walks the (m, h, b) items (m fastest) round-robin. A
+// 3-stage ring of (dS^T tile, K tile) runs on across items, and two TMEM accumulators
+// let the epilogue of one item overlap the MMAs of the next.
 template <int D>
 struct DqLayout {
   static constexpr int kStages = 3;
@@ -513,36 +516,46 @@ struct DqLayout {
   static constexpr int kStage = kDS + kK;
   static constexpr int kBar = kStages * kStage;
   static constexpr int kBytes = kBar + 256 + 1024;
-  static constexpr uint32_t kTmemCols = D < 32 ? 32 : D;
+  static constexpr uint32_t kTmemCols = 2 * D;  // two accumulators
 };
 
 template <int D>
 __global__ void __launch_bounds__(256, 1)
-    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const BwdParams p) {
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const BwdParams p, int n_items) {
   using L = DqLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  uint64_t* full = bars;                  // [kStages]
-  uint64_t* empty = bars + L::kStages;    // [kStages]
-  uint64_t* done = bars + 2 * L::kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * L::kStages + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * L::kStages + 2);
+  uint64_t* full = bars;                   // [kStages]
+  uint64_t* empty = bars + L::kStages;     // [kStages]
+  uint64_t* acc_full = bars + 2 * L::kStages;       // [2] an item's dQ is in TMEM
+  uint64_t* acc_empty = acc_full + 2;               // [2] the epilogue has read it
+  uint64_t* final_bar = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(final_bar + 2);
 
   const int warp = warp_id(), lane = lane_id();
-  // query tiles of one (b, h) are adjacent in launch order (they share K tiles in L2)
-  const int m = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int hk = h / p.G;
-  // key tiles n whose query range [n, n + span - 1] holds m
-  const int n_lo = max(0, m - p.span + 1);
-  const int steps = m - n_lo + 1;
+  // item -> (query tile m, head h, batch b), m fastest (neighbouring items share K in L2),
+  // and the key tiles n whose query range [n, n + span - 1] holds m
+  auto item_of = [&](int item, int& m, int& h, int& b, int& n_lo, int& steps) {
+    m = item % p.n_tiles;
+    const int hb = item / p.n_tiles;
+    h = hb % p.Hq;
+    b = hb / p.Hq;
+    n_lo = max(0, m - p.span + 1);
+    steps = m - n_lo + 1;
+  };
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(done, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&acc_full[s], 1);
+      mbar_init(&acc_empty[s], 128);
+    }
+    mbar_init(final_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -555,24 +568,30 @@ __global__ void __launch_bounds__(256, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = smem_u32(smem);
-  const long long bh_base = ((long long)b * p.Hq + h) * p.tiles_per_bh;
 
   if (warp == 0) {
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       int last_issue[L::kStages];
       for (int s = 0; s < L::kStages; ++s) last_issue[s] = -1;
-      for (int i = 0; i < steps; ++i) {
-        const int st = i % L::kStages;
-        const int n = n_lo + i;
-        if (!mbar_wait(&empty[st], ((i / L::kStages) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&full[st], L::kDS + L::kK);
-        const long long tile = bh_base + ds_tiles_before(n, p.n_tiles, p.span) + (m - n);
-        uint8_t* dst = smem + st * L::kStage;
-        bulk_load(dst, reinterpret_cast<const uint8_t*>(p.ds) + (size_t)tile * L::kDS, L::kDS, &full[st]);
-        for (int pn = 0; pn < D / 64; ++pn)
-          tma_load_4d(dst + L::kDS + pn * 16384, &tm_k, &full[st], pn * 64, hk, n * 128, b);
-        last_issue[st] = i;
+      int g = 0;  // ring step counter across items
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+        int m, h, b, n_lo, steps;
+        item_of(item, m, h, b, n_lo, steps);
+        const long long bh_base = ((long long)b * p.Hq + h) * p.tiles_per_bh;
+        for (int i = 0; i < steps; ++i, ++g) {
+          const int st = g % L::kStages;
+          const int n = n_lo + i;
+          if (!(ok = mbar_wait(&empty[st], ((g / L::kStages) & 1) ^ 1, abort_flag))) break;
+          mbar_arrive_expect_tx(&full[st], L::kDS + L::kK);
+          const long long tile = bh_base + ds_tiles_before(n, p.n_tiles, p.span) + (m - n);
+          uint8_t* dst = smem + st * L::kStage;
+          bulk_load(dst, reinterpret_cast<const uint8_t*>(p.ds) + (size_t)tile * L::kDS, L::kDS, &full[st]);
+          for (int pn = 0; pn < D / 64; ++pn)
+            tma_load_4d(dst + L::kDS + pn * 16384, &tm_k, &full[st], pn * 64, h / p.G, n * 128, b);
+          last_issue[st] = g;
+        }
       }
       if (*abort_flag) {
         volatile int dummy = 0;
@@ -584,37 +603,54 @@ __global__ void __launch_bounds__(256, 1)
     // whole warp runs the loop, one elected lane issues
     const uint32_t leader = elect_one();
     constexpr uint32_t id = idesc_bf16(128, D, true, true);  // A = dS (queries contiguous), B = K (d contiguous)
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+    };
+    int g = 0, k = 0;
     bool ok = true;
-    for (int i = 0; ok && i < steps; ++i) {
-      const int st = i % L::kStages;
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&full[st], (i / L::kStages) & 1, abort_flag)))) break;
-      tc_fence_after();
-      const uint32_t sds = sbase + st * L::kStage, sk = sds + L::kDS;
-      // A = dS (M = queries, K = keys) in the stored unit order: 128 bytes between
-      // core matrices along K, 512 along M; 16 keys per MMA = (kk / 2) * 8 KB + (kk & 1) * 256
-      const uint64_t da = sdesc_noswz(sds, 128, 512), db = sdesc_sw128(sk, 16384, 1024);
+    for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++k) {
+      int m, h, b, n_lo, steps;
+      item_of(item, m, h, b, n_lo, steps);
+      const int buf = k & 1;
+      // the epilogue has drained this accumulator (item k - 2)
+      if (!(ok = wait_all(&acc_empty[buf], ((k >> 1) & 1) ^ 1))) break;
+      for (int i = 0; i < steps; ++i, ++g) {
+        const int st = g % L::kStages;
+        if (!(ok = wait_all(&full[st], (g / L::kStages) & 1))) break;
+        tc_fence_after();
+        const uint32_t sds = sbase + st * L::kStage, sk = sds + L::kDS;
+        // A = dS (M = queries, K = keys) in the stored unit order: 128 bytes between
+        // core matrices along K, 512 along M; 16 keys per MMA = (kk / 2) * 8 KB + (kk & 1) * 256
+        const uint64_t da = sdesc_noswz(sds, 128, 512), db = sdesc_sw128(sk, 16384, 1024);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_ss(tmem, da + ((ds_unit_offset(16 * kk, 0)) >> 4), db + ((kk * 2048) >> 4), id, (i > 0 || kk > 0),
-               leader);
-      mma_commit(&empty[st], leader);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + buf * D, da + ((ds_unit_offset(16 * kk, 0)) >> 4), db + ((kk * 2048) >> 4), id,
+                 (i > 0 || kk > 0), leader);
+        mma_commit(&empty[st], leader);
+      }
+      if (!ok) break;
+      mma_commit(&acc_full[buf], leader);
     }
-    mma_commit(done, leader);
+    mma_commit(final_bar, leader);
     volatile int dummy = 0;
-    mbar_wait(done, 0, &dummy);
+    mbar_wait(final_bar, 0, &dummy);
   } else if (warp >= 4) {
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    const int i = m * 128 + row;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag));
-    tc_fence_after();
-    if (ok) {
+    int k = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++k) {
+      int m, h, b, n_lo, steps;
+      item_of(item, m, h, b, n_lo, steps);
+      const int buf = k & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (k >> 1) & 1, abort_flag))) break;
+      tc_fence_after();
+      const int i = m * 128 + row;
       __nv_bfloat16* dst = p.dq + ((size_t)((size_t)b * p.T + i) * p.Hq + h) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_off + c * 32, o);
+        tmem_ld32(tmem + buf * D + lane_off + c * 32, o);
         tmem_ld_wait();
         uint32_t w[16];
 #pragma unroll
@@ -626,6 +662,8 @@ __global__ void __launch_bounds__(256, 1)
           for (int u = 0; u < 4; ++u) d4[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
         }
       }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);
     }
   }
   __syncthreads();

@@ -50,6 +50,18 @@ bool encode_bthd(CUtensorMap* m, const void* base, int B, int T, int H, int D, i
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// SMs of the current device (looked up once per device)
+int sm_count() {
+  static int counts[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (counts[dev] == 0) {
+    int n = 0;
+    counts[dev] = (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) ? n : 148;
+  }
+  return counts[dev];
+}
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool dims_ok(int B, int T, int Hq, int Hkv) {
   return B >= 1 && T >= 1 && Hq >= 1 && Hkv >= 1 && Hq % Hkv == 0 && (long long)B * T * Hq < (1ll << 40);
@@ -216,7 +228,9 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
   p.scale_log2 = scale * kLog2e;
   attn_bwd_kernel<D><<<dim3(nt, Hkv, B), 384, BwdLayout<D>::kBytes, st>>>(tq, tk, tv, tdo, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
-  attn_bwd_dq_kernel<D><<<dim3(nt, Hq, B), 256, DqLayout<D>::kBytes, st>>>(tk, p);
+  const long long items = (long long)nt * Hq * B;
+  const int grid = (int)std::min<long long>(items, sm_count());
+  attn_bwd_dq_kernel<D><<<grid, 256, DqLayout<D>::kBytes, st>>>(tk, p, (int)items);
   return launched();
 }
 
@@ -308,7 +322,7 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
   if (Hq > 65535 || B > 65535 || tiles128(T) > 65535) return ATTN_ERR_INVALID_ARG;
   if ((long long)B * Hq * ds_tiles_before(tiles128(T), tiles128(T), bwd_span(tiles128(T), eff_window(window, T))) *
           128 >= (1ll << 31))
-    return ATTN_ERR_UNSUPPORTED;  // stored dS^T rows are addressed with 32-bit TMA coordinates
+    return ATTN_ERR_UNSUPPORTED;  // stored dS^T tile rows and dQ work items are counted in 32 bits
   cudaStream_t st = as_stream(stream);
   return D == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, workspace, B, T, Hq, Hkv, window, scale, st)
                  : launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, workspace, B, T, Hq, Hkv, window, scale, st);
