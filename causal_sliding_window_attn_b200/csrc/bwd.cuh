@@ -12,10 +12,13 @@
 //   bwd_prep     per query row, -lse_i/scale and -Delta_i as bf16 hi + lo pairs,
 //                laid out as one extra K = 16 step of an MMA (padded rows: a
 //                large negative lse term, so P = 0 there).
-//   bwd_main     one CTA per (128-key tile, KV head, batch). K and V stay in
-//                shared memory; the CTA walks every (query head of the group,
-//                128-row query tile) that sees the key tile, with Q and dO in
-//                rings of 3 and 2 stages. Per step, all MMAs M = 128, N = 128 (the
+//   bwd_main     persistent, one CTA per SM, walking (128-key tile, KV head,
+//                batch) items round-robin. For an item, K and V stay in shared
+//                memory and the CTA walks every (query head of the group, 128-row
+//                query tile) that sees the key tile, with Q and dO in rings of 3
+//                and 2 stages that run on across items; the next item's K and V
+//                load during the current item's last step, and its first S^T and
+//                dP^T are computed during the current item's dK/dV epilogue. Per step, all MMAs M = 128, N = 128 (the
 //                shape the tensor pipe runs at full rate), TMEM regions R0, R1 of
 //                128 columns each:
 //                  S^T' = K Q^T - lse/scale     (SS, + extension step) -> R0
@@ -55,7 +58,8 @@ struct BwdParams {
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   __nv_bfloat16* dq;
-  __nv_bfloat16* ds;   // stored dS^T tiles: 128 key rows x 128 query columns each, row-major
+  __nv_bfloat16* ds;   // stored dS^T tiles (see ds_unit_offset)
+  int* item_counter;   // [2] next work item of the main and dQ kernels (zeroed by the prep kernel)
   int T, Tpad, Hq, G, window, n_tiles, span;  // tiles of 128 rows; span = query tiles per key tile
   long long tiles_per_bh;                     // stored dS^T tiles per (batch, query head)
   float scale, scale_log2;
@@ -89,6 +93,22 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+// Work-item order of the persistent backward kernels. Items are (tile t, block blk)
+// pairs, blk = (head, batch) block of n_blocks, t of n_tiles; a tile's weight falls
+// as t grows. Blocks are taken 8 at a time (a super-block) and, inside one, the tile
+// index is the slow one: the heaviest tiles of 8 blocks first, then the next ones.
+// Handed out first come first served, this ends every super-block (and the whole
+// run) with the lightest items, while the CTAs running at the same time share the
+// tiles of those 8 blocks in L2.
+__host__ __device__ inline void sb_order(int item, int n_tiles, int n_blocks, int& t, int& blk) {
+  constexpr int kSB = 8;
+  const int s = item / (kSB * n_tiles);
+  const int w = min(kSB, n_blocks - kSB * s);
+  const int r = item - kSB * n_tiles * s;
+  t = r / w;
+  blk = kSB * s + r % w;
+}
+
 template <int D>
 struct BwdLayout {
   static constexpr int kQStages = 3, kDOStages = 2;
@@ -106,7 +126,7 @@ struct BwdLayout {
 #ifdef CSWA_TRACE
   static constexpr int kUsed = kBar + 256;  // profiling builds keep 4 more barriers
 #else
-  static constexpr int kUsed = kBar + 192;
+  static constexpr int kUsed = kBar + 224;
 #endif
   static constexpr int kBytes = (kUsed + 1024 <= 232448) ? kUsed + 1024 : 232448;
   static_assert(kUsed <= 232448, "shared memory budget");
@@ -117,7 +137,7 @@ template <int D>
 __global__ void __launch_bounds__(384, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const BwdParams p) {
+                    const BwdParams p, int n_items) {
   using L = BwdLayout<D>;
   constexpr int QS = L::kQStages, DS = L::kDOStages;
   extern __shared__ uint8_t smem_raw[];
@@ -129,7 +149,8 @@ __global__ void __launch_bounds__(384, 1)
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* kv_full = bars + 0;
-  uint64_t* q_full = bars + 1;                 // [QS]
+  uint64_t* kv_empty = bars + 1;               // the item's last S^T and dP^T have read K and V
+  uint64_t* q_full = bars + 2;                 // [QS]
   uint64_t* q_empty = q_full + QS;             // [QS]  dK has read the Q tile
   uint64_t* do_full = q_empty + QS;            // [DS]
   uint64_t* do_empty = do_full + DS;           // [DS]  dV has read the dO tile
@@ -137,24 +158,45 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* p_chunk = s_full + 1;              // [4] P^T of queries 16c..16c+15 of each half written
   uint64_t* dp_full = p_chunk + 4;             // dP^T in TMEM
   uint64_t* ds_full = dp_full + 1;             // dS^T written over dP^T
-  uint64_t* final_bar = ds_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(final_bar + 2);
+  uint64_t* final_bar = ds_full + 1;           // the item's dK and dV are complete in TMEM
+  uint64_t* acc_free = final_bar + 1;          // the epilogue has read them
+  uint64_t* done_bar = acc_free + 1;           // every MMA of the CTA has completed
+  uint64_t* item_full = done_bar + 1;          // the next work item's index is in item_slot
+  uint64_t* item_empty = item_full + 1;        // every role has read it
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(item_empty + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(item_empty + 2);
+  volatile int* item_slot = reinterpret_cast<volatile int*>(item_empty + 3);
 #ifdef CSWA_TRACE
-  uint64_t* trace_bar = final_bar + 3;  // [4] completion of dV, S, dK, dP groups (profiling builds)
+  uint64_t* trace_bar = item_empty + 4;  // [4] completion of dV, S, dK, dP groups (profiling builds)
 #endif
 
   const int warp = warp_id(), lane = lane_id();
-  // key tiles of one (b, KV head) are adjacent in launch order, so the CTAs that read
-  // the same Q/dO tiles run together and share them through L2
-  const int n = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int W = p.window, G = p.G;
-  const int k0 = n * 128;
-  const int m_cnt = min(p.n_tiles - n, p.span);
-  const int n_iters = G * m_cnt;
+  // Persistent: the CTAs share the (key tile n, KV head, batch) items through a
+  // global counter (first come, first served: CTAs that finish early take more), in
+  // super-block order (see sb_order): CTAs working at the same time read the same
+  // few blocks' Q/dO tiles through L2, and the last items handed out are light. Warp 2
+  // claims them and passes each index to the other roles through a one-deep slot.
+  // Every step of every item consumes one stage of the Q ring and one of the dO
+  // ring, so a step counter g running across the CTA's items gives all ring stages
+  // and per-step barrier phases.
+  struct Item {
+    int n, hk, b, m_cnt, n_iters;
+  };
+  auto item_of = [&](int item) {
+    Item it;
+    int blk;
+    sb_order(item, p.n_tiles, n_items / p.n_tiles, it.n, blk);
+    it.hk = blk % (p.Hq / G);
+    it.b = blk / (p.Hq / G);
+    it.m_cnt = min(p.n_tiles - it.n, p.span);
+    it.n_iters = G * it.m_cnt;
+    return it;
+  };
 
   if (warp == 0 && lane == 0) {
     mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
     for (int s = 0; s < QS; ++s) {
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
@@ -168,6 +210,10 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(dp_full, 1);
     mbar_init(ds_full, 256);
     mbar_init(final_bar, 1);
+    mbar_init(acc_free, 256);
+    mbar_init(done_bar, 1);
+    mbar_init(item_full, 1);
+    mbar_init(item_empty, 11);  // warps 0, 1, 3 and the eight P/dS warps
 #ifdef CSWA_TRACE
     for (int i = 0; i < 4; ++i) mbar_init(&trace_bar[i], 1);
 #endif
@@ -197,55 +243,82 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t tR0 = tmem, tR1 = tmem + 128, tdV = tmem + 256, tdK = tmem + 256 + D;
 
   const uint32_t sbase = smem_u32(smem);
-  auto iter_head = [&](int it) { return hk * G + it / m_cnt; };
-  auto iter_q0 = [&](int it) { return (n + it % m_cnt) * 128; };
+  // the k-th work item of this CTA (-1: none left, or the CTA gave up), read by a whole
+  // warp; one lane releases the slot for the role
+  auto take_item = [&](int k) {
+    int v = mbar_wait(item_full, k & 1, abort_flag) ? *item_slot : -1;
+    v = __shfl_sync(0xffffffffu, v, 0);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(item_empty);
+    return v;
+  };
 
   if (warp == 0 || warp == 3) {
     // ------------------------------------------------------------ producers
-    // warp 0: K, V and the Q ring; warp 3: the dO ring (its stages free up at a
-    // different point of the step, so it waits on its own). Each stage also takes
-    // the 512-byte row extension of its tile: -lse/scale with Q, -Delta with dO.
+    // warp 0: K and V of each item and the Q ring; warp 3: the dO ring (its stages
+    // free up at a different point of the step, so it waits on its own). Each stage
+    // also takes the 512-byte row extension of its tile: -lse/scale with Q, -Delta
+    // with dO. K and V of the next item load as soon as the current item's last S^T
+    // and dP^T have read the previous ones.
+    // The whole warp takes the items (the slot is read warp-wide); lane 0 issues.
+    const bool qside = (warp == 0);
+    const int nst = qside ? QS : DS;
+    int last_issue[3] = {-1, -1, -1};
+    int last_kv = -1;
     if (lane == 0) {
-      const bool qside = (warp == 0);
-      const int nst = qside ? QS : DS;
-      int last_issue[3] = {-1, -1, -1};
       if (qside) {
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
-        mbar_arrive_expect_tx(kv_full, 2 * L::kTile);
-        for (int pn = 0; pn < D / 64; ++pn) {
-          tma_load_4d(smem + L::kK + pn * L::kPanel, &tm_k, kv_full, pn * 64, hk, k0, b);
-          tma_load_4d(smem + L::kV + pn * L::kPanel, &tm_v, kv_full, pn * 64, hk, k0, b);
-        }
       } else {
         tma_prefetch_desc(&tm_do);
       }
-      uint64_t* full = qside ? q_full : do_full;
-      uint64_t* empty = qside ? q_empty : do_empty;
-      const CUtensorMap* tm = qside ? &tm_q : &tm_do;
-      const int base = qside ? L::kQ : L::kDO;
-      const uint8_t* ext = qside ? p.ext_lse : p.ext_delta;
-      uint8_t* ext_slot = smem + L::kExt + (qside ? 0 : QS * 512);
-      for (int it = 0; it < n_iters; ++it) {
-        const int st = it % nst;
-        const int h = iter_head(it), q0 = iter_q0(it);
-        if (qside) CSWA_MARK(3, it, 0);
-        if (!mbar_wait(&empty[st], ((it / nst) & 1) ^ 1, abort_flag)) break;
-        if (qside) CSWA_MARK(3, it, 1);
-        mbar_arrive_expect_tx(&full[st], L::kTile + 512);
-        for (int pn = 0; pn < D / 64; ++pn)
-          tma_load_4d(smem + base + st * L::kTile + pn * L::kPanel, tm, &full[st], pn * 64, h, q0, b);
-        bulk_load(ext_slot + st * 512, ext + (((size_t)b * p.Hq + h) * p.n_tiles + q0 / 128) * 512, 512, &full[st]);
-        last_issue[st] = it;
+    }
+    uint64_t* full = qside ? q_full : do_full;
+    uint64_t* empty = qside ? q_empty : do_empty;
+    const CUtensorMap* tm = qside ? &tm_q : &tm_do;
+    const int base = qside ? L::kQ : L::kDO;
+    const uint8_t* ext = qside ? p.ext_lse : p.ext_delta;
+    uint8_t* ext_slot = smem + L::kExt + (qside ? 0 : QS * 512);
+    int g = 0;
+    bool ok = true;
+    for (int k = 0;; ++k) {
+      const int item = take_item(k);
+      if (item < 0) break;
+      if (lane == 0) {
+        const Item I = item_of(item);
+        if (qside) {
+          if ((ok = mbar_wait(kv_empty, (k & 1) ^ 1, abort_flag))) {
+            mbar_arrive_expect_tx(kv_full, 2 * L::kTile);
+            for (int pn = 0; pn < D / 64; ++pn) {
+              tma_load_4d(smem + L::kK + pn * L::kPanel, &tm_k, kv_full, pn * 64, I.hk, I.n * 128, I.b);
+              tma_load_4d(smem + L::kV + pn * L::kPanel, &tm_v, kv_full, pn * 64, I.hk, I.n * 128, I.b);
+            }
+            last_kv = k;
+          }
+        }
+        for (int it = 0; ok && it < I.n_iters; ++it, ++g) {
+          const int st = g % nst;
+          const int h = I.hk * G + it / I.m_cnt, q0 = (I.n + it % I.m_cnt) * 128;
+          if (qside) CSWA_MARK(3, g, 0);
+          if (!(ok = mbar_wait(&empty[st], ((g / nst) & 1) ^ 1, abort_flag))) break;
+          if (qside) CSWA_MARK(3, g, 1);
+          mbar_arrive_expect_tx(&full[st], L::kTile + 512);
+          for (int pn = 0; pn < D / 64; ++pn)
+            tma_load_4d(smem + base + st * L::kTile + pn * L::kPanel, tm, &full[st], pn * 64, h, q0, I.b);
+          bulk_load(ext_slot + st * 512, ext + (((size_t)I.b * p.Hq + h) * p.n_tiles + q0 / 128) * 512, 512,
+                    &full[st]);
+          last_issue[st] = g;
+        }
       }
-      if (*abort_flag) {
-        // let every copy in flight land before the CTA's shared memory is released
-        volatile int dummy = 0;
-        for (int s = 0; s < nst; ++s)
-          if (last_issue[s] >= 0) mbar_wait(&full[s], (last_issue[s] / nst) & 1, &dummy);
-        if (qside) mbar_wait(kv_full, 0, &dummy);
-      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+    }
+    if (lane == 0 && *abort_flag) {
+      // let every copy in flight land before the CTA's shared memory is released
+      volatile int dummy = 0;
+      for (int s = 0; s < nst; ++s)
+        if (last_issue[s] >= 0) mbar_wait(&full[s], (last_issue[s] / nst) & 1, &dummy);
+      if (qside && last_kv >= 0) mbar_wait(kv_full, last_kv & 1, &dummy);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -277,8 +350,8 @@ __global__ void __launch_bounds__(384, 1)
       mma_ss(dst, dOnes, dX + ((xslot * 512) >> 4), idX, 1, leader);
       mma_commit(done, leader);
     };
-    // dV += P^T dO and dK += dS^T Q: A = the bf16 pairs packed over S^T / dP^T (queries
-    // 0-63 in columns 0-31, 64-127 in columns 64-95), B = dO or Q, MN-major
+    // dK += dS^T Q: A = the bf16 pairs packed over dP^T (queries 0-63 in columns 0-31,
+    // 64-127 in columns 64-95), B = Q, MN-major
     auto issue_acc = [&](uint32_t dst, uint32_t a_tmem, uint64_t dB, uint32_t boff, bool first) {
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
@@ -288,196 +361,225 @@ __global__ void __launch_bounds__(384, 1)
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
     };
-    bool ok = wait_all(kv_full, 0) && wait_all(&q_full[0], 0);
-    tc_fence_after();
-    if (ok) issue_R(tR0, dK_k, dQ_k, 0, 0, s_full);
-    ok = ok && wait_all(&do_full[0], 0);
-    tc_fence_after();
-    if (ok) issue_R(tR1, dV_k, dDO_k, 0, QS, dp_full);
     const bool tracer = (lane == 0);
     (void)tracer;
-    // Each step issues two bursts, each preceded by all of its waits (a barrier wait
-    // between two groups would let the tensor pipe run dry): dV(it) + S^T(it+1) once
-    // P^T(it) is written, dK(it) + dP^T(it+1) once dS^T(it) is written.
-    for (int it = 0; ok && it < n_iters; ++it) {
-      const int qs = it % QS, ds = it % DS;
-      const int q1 = (it + 1) % QS, d1 = (it + 1) % DS;
-      const bool more = it + 1 < n_iters;
-      if (tracer) CSWA_MARK(0, it, 0);
-      if (more && !(ok = wait_all(&q_full[q1], ((it + 1) / QS) & 1))) break;
-      // dV(it) chunk by chunk as the P/dS warps publish P^T: chunk c holds queries
-      // 16c..16c+15 of each half, i.e. the K steps c and 4 + c
-      for (int c = 0; c < 4; ++c) {
-        if (!(ok = wait_all(&p_chunk[c], it & 1))) break;
-        if (tracer && c == 0) CSWA_MARK(0, it, 1);
-        tc_fence_after();
+    int g0 = 0, k = 0;  // step counter at the item's first step; items done
+    bool ok = true;
+    for (;; ++k) {
+      const int item = take_item(k);
+      if (item < 0) break;
+      const Item I = item_of(item);
+      // S^T and dP^T of the item's first step, once its K, V, Q and dO are in
+      if (!(ok = wait_all(kv_full, k & 1) && wait_all(&q_full[g0 % QS], (g0 / QS) & 1))) break;
+      tc_fence_after();
+      issue_R(tR0, dK_k, dQ_k, (g0 % QS) * L::kTile, g0 % QS, s_full);
+      if (!(ok = wait_all(&do_full[g0 % DS], (g0 / DS) & 1))) break;
+      tc_fence_after();
+      issue_R(tR1, dV_k, dDO_k, (g0 % DS) * L::kTile, QS + g0 % DS, dp_full);
+      if (I.n_iters == 1) mma_commit(kv_empty, leader);  // K and V are no longer read
+      // Each step issues two bursts, each preceded by all of its waits (a barrier wait
+      // between two groups would let the tensor pipe run dry): dV(it) + S^T(it+1) once
+      // P^T(it) is written, dK(it) + dP^T(it+1) once dS^T(it) is written.
+      for (int it = 0; ok && it < I.n_iters; ++it) {
+        const int g = g0 + it;
+        const int qs = g % QS, ds = g % DS;
+        const int q1 = (g + 1) % QS, d1 = (g + 1) % DS;
+        const bool more = it + 1 < I.n_iters;
+        if (tracer) CSWA_MARK(0, g, 0);
+        if (more && !(ok = wait_all(&q_full[q1], ((g + 1) / QS) & 1))) break;
+        // the accumulators are free once the epilogue has read the previous item's
+        if (it == 0 && !(ok = wait_all(acc_free, (k & 1) ^ 1))) break;
+        // dV(it) chunk by chunk as the P/dS warps publish P^T: chunk c holds queries
+        // 16c..16c+15 of each half, i.e. the K steps c and 4 + c
+        for (int c = 0; c < 4; ++c) {
+          if (!(ok = wait_all(&p_chunk[c], g & 1))) break;
+          if (tracer && c == 0) CSWA_MARK(0, g, 1);
+          tc_fence_after();
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int kk = c + 4 * u;
-          mma_ts(tdV, tR0 + u * 64 + c * 8, dDO_mn + ((ds * L::kTile + kk * 2048) >> 4), idKV, (it > 0 || kk > 0),
-                 leader);
+          for (int u = 0; u < 2; ++u) {
+            const int kk = c + 4 * u;
+            mma_ts(tdV, tR0 + u * 64 + c * 8, dDO_mn + ((ds * L::kTile + kk * 2048) >> 4), idKV,
+                   (it > 0 || kk > 0), leader);
+          }
         }
+        if (!ok) break;
+        mma_commit(&do_empty[ds], leader);
+#ifdef CSWA_TRACE
+        mma_commit(&trace_bar[0], leader);
+#endif
+        if (tracer) CSWA_MARK(0, g, 2);
+        // S^T(it+1) overwrites P^T(it) only after dV(it) has read it: MMAs run in issue order
+        if (more) issue_R(tR0, dK_k, dQ_k, q1 * L::kTile, q1, s_full);
+#ifdef CSWA_TRACE
+        if (more) mma_commit(&trace_bar[1], leader);
+#endif
+        if (tracer) CSWA_MARK(0, g, 4);
+        if (more && !(ok = wait_all(&do_full[d1], ((g + 1) / DS) & 1))) break;
+        if (!(ok = wait_all(ds_full, g & 1))) break;
+        if (tracer) CSWA_MARK(0, g, 5);
+        tc_fence_after();
+        issue_acc(tdK, tR1, dQ_mn, qs * L::kTile, it == 0);
+        mma_commit(&q_empty[qs], leader);
+#ifdef CSWA_TRACE
+        mma_commit(&trace_bar[2], leader);
+#endif
+        if (tracer) CSWA_MARK(0, g, 6);
+        if (more) {
+          issue_R(tR1, dV_k, dDO_k, d1 * L::kTile, QS + d1, dp_full);
+          if (it + 2 == I.n_iters) mma_commit(kv_empty, leader);  // the item's last S^T and dP^T
+        }
+#ifdef CSWA_TRACE
+        if (more) mma_commit(&trace_bar[3], leader);
+#endif
+        if (tracer) CSWA_MARK(0, g, 7);
       }
       if (!ok) break;
-      mma_commit(&do_empty[ds], leader);
-#ifdef CSWA_TRACE
-      mma_commit(&trace_bar[0], leader);
-#endif
-      if (tracer) CSWA_MARK(0, it, 2);
-      // S^T(it+1) overwrites P^T(it) only after dV(it) has read it: MMAs run in issue order
-      if (more) issue_R(tR0, dK_k, dQ_k, q1 * L::kTile, q1, s_full);
-#ifdef CSWA_TRACE
-      if (more) mma_commit(&trace_bar[1], leader);
-#endif
-      if (tracer) CSWA_MARK(0, it, 4);
-      if (more && !(ok = wait_all(&do_full[d1], ((it + 1) / DS) & 1))) break;
-      if (!(ok = wait_all(ds_full, it & 1))) break;
-      if (tracer) CSWA_MARK(0, it, 5);
-      tc_fence_after();
-      issue_acc(tdK, tR1, dQ_mn, qs * L::kTile, it == 0);
-      mma_commit(&q_empty[qs], leader);
-#ifdef CSWA_TRACE
-      mma_commit(&trace_bar[2], leader);
-#endif
-      if (tracer) CSWA_MARK(0, it, 6);
-      if (more) issue_R(tR1, dV_k, dDO_k, d1 * L::kTile, QS + d1, dp_full);
-#ifdef CSWA_TRACE
-      if (more) mma_commit(&trace_bar[3], leader);
-#endif
-      if (tracer) CSWA_MARK(0, it, 7);
+      mma_commit(final_bar, leader);  // dK and dV of the item are complete
+      g0 += I.n_iters;
     }
-    mma_commit(final_bar, leader);
+    // every MMA issued above has finished before TMEM is released
+    mma_commit(done_bar, leader);
     volatile int dummy = 0;
-    mbar_wait(final_bar, 0, &dummy);
+    mbar_wait(done_bar, 0, &dummy);
   } else if (warp == 2) {
-#ifdef CSWA_TRACE
-    // profiling builds: the TMEM allocator warp records when each MMA group completes
+    // ------------------------------------------------------------ work scheduler
+    // claims the CTA's next item from the global counter once every role has read
+    // the previous one; -1 when none is left
     if (lane == 0) {
-      volatile int own_abort = 0;
-      for (int it = 0; it < n_iters && !own_abort; ++it) {
-        for (int g = 0; g < 4 && !own_abort; ++g) {
-          if ((g == 1 || g == 3) && it + 1 >= n_iters) continue;
-          if (!mbar_wait(&trace_bar[g], it & 1, &own_abort)) break;
-          CSWA_MARK(3, it, 4 + g);
-        }
+      for (int k = 0;; ++k) {
+        if (!mbar_wait(item_empty, (k & 1) ^ 1, abort_flag)) break;
+        const int idx = atomicAdd(p.item_counter, 1);
+        const int v = idx < n_items ? idx : -1;
+        *item_slot = v;
+        mbar_arrive(item_full);
+        if (v < 0) break;
       }
     }
-#endif
   } else if (warp >= 4) {
     // ------------------------------------------------------------ P and dS (thread = key row)
     // warps 4-7 take query columns 0-63, warps 8-11 columns 64-127 (warp 2 only allocates TMEM)
     const int half = (warp >= 8) ? 1 : 0;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const int j = k0 + r;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t cols = lane_off + 64 * half;  // this thread's S^T / dP^T columns
     const float sl2 = p.scale_log2;
-    // row r of the stored dS^T tile, this warpgroup's 64 queries
-    const long long tile0 = ((long long)b * p.Hq) * p.tiles_per_bh + ds_tiles_before(n, p.n_tiles, p.span);
     const bool tracer = ((warp == 4 || warp == 8) && lane == 0);
     const int trole = 1 + half;
     (void)tracer;
     (void)trole;
     // dS^T of the previous step (this warp's 32 keys x 64 queries) and where it goes in
-    // the workspace tile the dQ kernel reads; it is stored during this step's P phase,
-    // whose exp2 work leaves the load/store unit idle. The tile is written as 16-byte
-    // units (8 queries of one key) ordered so that every warp store covers 512
-    // contiguous bytes (see ds_unit_offset).
+    // the workspace tile the dQ kernel reads; it is stored during the next step's P
+    // phase, whose exp2 work leaves the load/store unit idle (an item's last one before
+    // its epilogue). The tile is written as 16-byte units (8 queries of one key) ordered
+    // so that every warp store covers 512 contiguous bytes (see ds_unit_offset).
     uint32_t dsk[32];
     uint8_t* ds_dst = nullptr;
-    auto store_ds_units = [&](int g0, int g1) {
+    auto store_ds_units = [&](int u0, int u1) {
 #pragma unroll
-      for (int g = g0; g < g1; ++g)
-        *reinterpret_cast<uint4*>(ds_dst + g * 512) = make_uint4(dsk[4 * g], dsk[4 * g + 1], dsk[4 * g + 2], dsk[4 * g + 3]);
+      for (int u = u0; u < u1; ++u)
+        *reinterpret_cast<uint4*>(ds_dst + u * 512) = make_uint4(dsk[4 * u], dsk[4 * u + 1], dsk[4 * u + 2], dsk[4 * u + 3]);
     };
     bool ok = true;
-    for (int it = 0; it < n_iters; ++it) {
-      const int q0 = iter_q0(it) + 64 * half;  // first query of this thread's columns
-      if (tracer) CSWA_MARK(trole, it, 0);
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full, it & 1, abort_flag));
-      if (tracer) CSWA_MARK(trole, it, 1);
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld32(tR0 + cols + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tR0 + cols + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld_wait();
-      if (tracer) CSWA_MARK(trole, it, 2);
-      const bool full = (k0 + 127 <= q0) && (W < 0 || q0 + 63 - k0 <= W);
-      const int c_lo = j - q0;                      // query q0 + c sees key j iff c >= c_lo
-      const int c_hi = (W < 0) ? 63 : j + W - q0;   //   and c <= c_hi
-      // P = exp2(scale log2e (S - lse/scale)): the MMA has already added -lse/scale, so
-      // one packed multiply per two columns; masked entries are set to 0 after the exp2,
-      // tiles inside the band skip the mask (a warp-uniform branch). P^T goes back to
-      // TMEM in four chunks of 16 queries, each published on its own barrier so that
-      // dV starts on the first while the rest is computed. Chunk c's bf16 pairs land in
-      // columns 8c..8c+7, whose fp32 S^T (queries <= 16c+15) is already in registers.
-      const float2 sl2v = make_float2(sl2, sl2);
+    int g0 = 0, k = 0;
+    for (;; ++k) {
+      const int item = take_item(k);
+      if (item < 0) break;
+      const Item I = item_of(item);
+      const int k0 = I.n * 128;
+      const int j = k0 + r;
+      // the item's first stored dS^T tile (key tile n of batch b, query head 0)
+      const long long tile0 = ((long long)I.b * p.Hq) * p.tiles_per_bh + ds_tiles_before(I.n, p.n_tiles, p.span);
+      for (int it = 0; it < I.n_iters; ++it) {
+        const int g = g0 + it;
+        const int q0 = (I.n + it % I.m_cnt) * 128 + 64 * half;  // first query of this thread's columns
+        if (tracer) CSWA_MARK(trole, g, 0);
+        ok = __all_sync(0xffffffffu, mbar_wait(s_full, g & 1, abort_flag));
+        if (tracer) CSWA_MARK(trole, g, 1);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t sr[64];
+        tmem_ld32(tR0 + cols + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(tR0 + cols + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld_wait();
+        if (tracer) CSWA_MARK(trole, g, 2);
+        const bool full = (k0 + 127 <= q0) && (W < 0 || q0 + 63 - k0 <= W);
+        const int c_lo = j - q0;                      // query q0 + c sees key j iff c >= c_lo
+        const int c_hi = (W < 0) ? 63 : j + W - q0;   //   and c <= c_hi
+        // P = exp2(scale log2e (S - lse/scale)): the MMA has already added -lse/scale, so
+        // one packed multiply per two columns; masked entries are set to 0 after the exp2,
+        // tiles inside the band skip the mask (a warp-uniform branch). P^T goes back to
+        // TMEM in four chunks of 16 queries, each published on its own barrier so that
+        // dV starts on the first while the rest is computed. Chunk c's bf16 pairs land in
+        // columns 8c..8c+7, whose fp32 S^T (queries <= 16c+15) is already in registers.
+        const float2 sl2v = make_float2(sl2, sl2);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[8];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[8];
 #pragma unroll
-        for (int c2 = 8 * c; c2 < 8 * c + 8; ++c2) {
-          const float2 e = __fmul2_rn(make_float2(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1])), sl2v);
-          float y[2] = {ex2_approx(e.x), ex2_approx(e.y)};
-          if (!full) {
+          for (int c2 = 8 * c; c2 < 8 * c + 8; ++c2) {
+            const float2 e = __fmul2_rn(make_float2(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1])), sl2v);
+            float y[2] = {ex2_approx(e.x), ex2_approx(e.y)};
+            if (!full) {
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int col = 2 * c2 + u;
-              y[u] = ((col >= c_lo) & (col <= c_hi)) ? y[u] : 0.f;
+              for (int u = 0; u < 2; ++u) {
+                const int col = 2 * c2 + u;
+                y[u] = ((col >= c_lo) & (col <= c_hi)) ? y[u] : 0.f;
+              }
             }
+            sr[2 * c2] = __float_as_uint(y[0]);
+            sr[2 * c2 + 1] = __float_as_uint(y[1]);
+            pk[c2 - 8 * c] = pack_bf16x2(y[0], y[1]);
           }
-          sr[2 * c2] = __float_as_uint(y[0]);
-          sr[2 * c2 + 1] = __float_as_uint(y[1]);
-          pk[c2 - 8 * c] = pack_bf16x2(y[0], y[1]);
+          tmem_st8(tR0 + cols + 8 * c, pk);
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&p_chunk[c]);
+          if (tracer && c == 0) CSWA_MARK(trole, g, 3);
+          if (ds_dst) store_ds_units(2 * c, 2 * c + 2);
         }
-        tmem_st8(tR0 + cols + 8 * c, pk);
+        const float* pf = reinterpret_cast<const float*>(sr);
+        if (tracer) CSWA_MARK(trole, g, 4);
+
+        ok = __all_sync(0xffffffffu, mbar_wait(dp_full, g & 1, abort_flag));
+        if (!ok) break;
+        if (tracer) CSWA_MARK(trole, g, 5);
+        tc_fence_after();
+        // dS = P * (dP - Delta): the MMA has already subtracted Delta; one packed multiply
+        // per two columns, 32 columns at a time
+#pragma unroll
+        for (int hc = 0; hc < 2; ++hc) {
+          uint32_t dp[32];
+          tmem_ld32(tR1 + cols + 32 * hc, dp);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c2 = 0; c2 < 16; ++c2) {
+            const int c = 32 * hc + 2 * c2;
+            const float2 d = __fmul2_rn(make_float2(pf[c], pf[c + 1]),
+                                        make_float2(__uint_as_float(dp[2 * c2]), __uint_as_float(dp[2 * c2 + 1])));
+            dsk[c / 2] = pack_bf16x2(d.x, d.y);
+          }
+        }
+        if (tracer) CSWA_MARK(trole, g, 6);
+        tmem_st32(tR1 + cols, dsk);  // over this thread's own (already read) dP^T columns
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&p_chunk[c]);
-        if (tracer && c == 0) CSWA_MARK(trole, it, 3);
-        if (ds_dst) store_ds_units(2 * c, 2 * c + 2);
+        mbar_arrive(ds_full);
+        if (tracer) CSWA_MARK(trole, g, 7);
+        const long long tile = tile0 + (long long)(I.hk * G + it / I.m_cnt) * p.tiles_per_bh + it % I.m_cnt;
+        ds_dst = reinterpret_cast<uint8_t*>(p.ds) + (size_t)tile * 32768 + ds_unit_offset(r, 8 * half);
       }
-      const float* pf = reinterpret_cast<const float*>(sr);
-      if (tracer) CSWA_MARK(trole, it, 4);
-
-      ok = __all_sync(0xffffffffu, mbar_wait(dp_full, it & 1, abort_flag));
       if (!ok) break;
-      if (tracer) CSWA_MARK(trole, it, 5);
+      // the item's last dS^T now: the epilogue needs the registers
+      store_ds_units(0, 8);
+      ds_dst = nullptr;
+      // ------------------------------------------------------ dK (warps 4-7) / dV (8-11) epilogue
+      ok = __all_sync(0xffffffffu, mbar_wait(final_bar, k & 1, abort_flag));
+      if (!ok) break;
       tc_fence_after();
-      // dS = P * (dP - Delta): the MMA has already subtracted Delta; one packed multiply
-      // per two columns, 32 columns at a time
-#pragma unroll
-      for (int hc = 0; hc < 2; ++hc) {
-        uint32_t dp[32];
-        tmem_ld32(tR1 + cols + 32 * hc, dp);
-        tmem_ld_wait();
-#pragma unroll
-        for (int c2 = 0; c2 < 16; ++c2) {
-          const int c = 32 * hc + 2 * c2;
-          const float2 d = __fmul2_rn(make_float2(pf[c], pf[c + 1]),
-                                      make_float2(__uint_as_float(dp[2 * c2]), __uint_as_float(dp[2 * c2 + 1])));
-          dsk[c / 2] = pack_bf16x2(d.x, d.y);
-        }
-      }
-      if (tracer) CSWA_MARK(trole, it, 6);
-      tmem_st32(tR1 + cols, dsk);  // over this thread's own (already read) dP^T columns
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(ds_full);
-      if (tracer) CSWA_MARK(trole, it, 7);
-      const long long tile = tile0 + (long long)iter_head(it) * p.tiles_per_bh + it % m_cnt;
-      ds_dst = reinterpret_cast<uint8_t*>(p.ds) + (size_t)tile * 32768 + ds_unit_offset(r, 8 * half);
-    }
-    if (ok && ds_dst) store_ds_units(0, 8);
-    // ---------------------------------------------------------- dK (warps 4-7) / dV (8-11) epilogue
-    ok = __all_sync(0xffffffffu, ok && mbar_wait(final_bar, 0, abort_flag));
-    tc_fence_after();
-    if (ok) {
       const uint32_t src = half ? tdV : tdK;
       const float mul = half ? 1.f : p.scale;
-      __nv_bfloat16* dst = (half ? p.dv : p.dk) + ((size_t)((size_t)b * p.T + j) * (p.Hq / G) + hk) * D;
+      __nv_bfloat16* dst = (half ? p.dv : p.dk) + ((size_t)((size_t)I.b * p.T + j) * (p.Hq / G) + I.hk) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -493,6 +595,10 @@ __global__ void __launch_bounds__(384, 1)
           for (int u = 0; u < 4; ++u) d4[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
         }
       }
+      // the accumulators may take the next item's first products
+      tc_fence_before();
+      mbar_arrive(acc_free);
+      g0 += I.n_iters;
     }
   }
 
@@ -505,9 +611,9 @@ __global__ void __launch_bounds__(384, 1)
 
 // dQ = scale * sum_n dS(m, n) K_n for every 128-row query tile m of every query
 // head, from the dS^T tiles bwd_main stored; accumulated in TMEM, written once as bf16.
-// Persistent: one CTA per SM walks the (m, h, b) items (m fastest) round-robin. A
-// 3-stage ring of (dS^T tile, K tile) runs on across items, and two TMEM accumulators
-// let the epilogue of one item overlap the MMAs of the next.
+// Persistent: one CTA per SM takes (m, h, b) items from a global counter (warp 3
+// claims them). A 3-stage ring of (dS^T tile, K tile) runs on across items, and two
+// TMEM accumulators let the epilogue of one item overlap the MMAs of the next.
 template <int D>
 struct DqLayout {
   static constexpr int kStages = 3;
@@ -531,17 +637,22 @@ __global__ void __launch_bounds__(256, 1)
   uint64_t* acc_full = bars + 2 * L::kStages;       // [2] an item's dQ is in TMEM
   uint64_t* acc_empty = acc_full + 2;               // [2] the epilogue has read it
   uint64_t* final_bar = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(final_bar + 2);
+  uint64_t* item_full = final_bar + 1;     // the next work item's index is in item_slot
+  uint64_t* item_empty = item_full + 1;    // every role has read it
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(item_empty + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(item_empty + 2);
+  volatile int* item_slot = reinterpret_cast<volatile int*>(item_empty + 3);
 
   const int warp = warp_id(), lane = lane_id();
-  // item -> (query tile m, head h, batch b), m fastest (neighbouring items share K in L2),
-  // and the key tiles n whose query range [n, n + span - 1] holds m
+  // item -> (query tile m, head h, batch b) in super-block order with the heaviest
+  // query tiles (the most key tiles) first, and the key tiles n whose query range
+  // [n, n + span - 1] holds m; items are handed out first come first served
   auto item_of = [&](int item, int& m, int& h, int& b, int& n_lo, int& steps) {
-    m = item % p.n_tiles;
-    const int hb = item / p.n_tiles;
-    h = hb % p.Hq;
-    b = hb / p.Hq;
+    int t, blk;
+    sb_order(item, p.n_tiles, n_items / p.n_tiles, t, blk);
+    m = p.n_tiles - 1 - t;
+    h = blk % p.Hq;
+    b = blk / p.Hq;
     n_lo = max(0, m - p.span + 1);
     steps = m - n_lo + 1;
   };
@@ -556,6 +667,8 @@ __global__ void __launch_bounds__(256, 1)
       mbar_init(&acc_empty[s], 128);
     }
     mbar_init(final_bar, 1);
+    mbar_init(item_full, 1);
+    mbar_init(item_empty, 6);  // warps 0, 1 and the four epilogue warps
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -568,15 +681,27 @@ __global__ void __launch_bounds__(256, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = smem_u32(smem);
+  // the k-th work item of this CTA (-1: none left, or the CTA gave up), read by a whole
+  // warp; one lane releases the slot for the role
+  auto take_item = [&](int k) {
+    int v = mbar_wait(item_full, k & 1, abort_flag) ? *item_slot : -1;
+    v = __shfl_sync(0xffffffffu, v, 0);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(item_empty);
+    return v;
+  };
 
   if (warp == 0) {
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_k);
-      int last_issue[L::kStages];
-      for (int s = 0; s < L::kStages; ++s) last_issue[s] = -1;
-      int g = 0;  // ring step counter across items
-      bool ok = true;
-      for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+    // producer: the whole warp takes the items, lane 0 issues
+    int last_issue[L::kStages];
+    for (int s = 0; s < L::kStages; ++s) last_issue[s] = -1;
+    if (lane == 0) tma_prefetch_desc(&tm_k);
+    int g = 0;  // ring step counter across items
+    bool ok = true;
+    for (int k = 0;; ++k) {
+      const int item = take_item(k);
+      if (item < 0) break;
+      if (lane == 0) {
         int m, h, b, n_lo, steps;
         item_of(item, m, h, b, n_lo, steps);
         const long long bh_base = ((long long)b * p.Hq + h) * p.tiles_per_bh;
@@ -593,11 +718,12 @@ __global__ void __launch_bounds__(256, 1)
           last_issue[st] = g;
         }
       }
-      if (*abort_flag) {
-        volatile int dummy = 0;
-        for (int s = 0; s < L::kStages; ++s)
-          if (last_issue[s] >= 0) mbar_wait(&full[s], (last_issue[s] / L::kStages) & 1, &dummy);
-      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+    }
+    if (lane == 0 && *abort_flag) {
+      volatile int dummy = 0;
+      for (int s = 0; s < L::kStages; ++s)
+        if (last_issue[s] >= 0) mbar_wait(&full[s], (last_issue[s] / L::kStages) & 1, &dummy);
     }
   } else if (warp == 1) {
     // whole warp runs the loop, one elected lane issues
@@ -606,9 +732,11 @@ __global__ void __launch_bounds__(256, 1)
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
     };
-    int g = 0, k = 0;
+    int g = 0;
     bool ok = true;
-    for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++k) {
+    for (int k = 0;; ++k) {
+      const int item = take_item(k);
+      if (item < 0) break;
       int m, h, b, n_lo, steps;
       item_of(item, m, h, b, n_lo, steps);
       const int buf = k & 1;
@@ -634,12 +762,26 @@ __global__ void __launch_bounds__(256, 1)
     mma_commit(final_bar, leader);
     volatile int dummy = 0;
     mbar_wait(final_bar, 0, &dummy);
+  } else if (warp == 3) {
+    // work scheduler: claims the CTA's next item from the global counter once every
+    // role has read the previous one; -1 when none is left
+    if (lane == 0) {
+      for (int k = 0;; ++k) {
+        if (!mbar_wait(item_empty, (k & 1) ^ 1, abort_flag)) break;
+        const int idx = atomicAdd(p.item_counter + 1, 1);
+        const int v = idx < n_items ? idx : -1;
+        *item_slot = v;
+        mbar_arrive(item_full);
+        if (v < 0) break;
+      }
+    }
   } else if (warp >= 4) {
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    int k = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++k) {
+    for (int k = 0;; ++k) {
+      const int item = take_item(k);
+      if (item < 0) break;
       int m, h, b, n_lo, steps;
       item_of(item, m, h, b, n_lo, steps);
       const int buf = k & 1;
@@ -685,9 +827,12 @@ __global__ void __launch_bounds__(256, 1)
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __nv_bfloat16* o, const __nv_bfloat16* dout,
                                                              const float* lse, uint8_t* ext_lse,
-                                                             uint8_t* ext_delta, int B, int T, int Tpad, int Hq,
-                                                             float inv_scale) {
+                                                             uint8_t* ext_delta, int* item_counter, int B, int T,
+                                                             int Tpad, int Hq, float inv_scale) {
   constexpr int LK = D / 8;
+  // the main and dQ kernels that follow on the stream hand out their work items from
+  // these two counters
+  if (blockIdx.x == 0 && threadIdx.x < 2) item_counter[threadIdx.x] = 0;
   const long long rows = (long long)B * Tpad * Hq;
   const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long row = gtid / LK;

@@ -158,6 +158,7 @@ struct BwdWorkspace {
   uint8_t* ext_lse;       // (B, Hq, Tpad / 128) x 512 bytes
   uint8_t* ext_delta;     // (B, Hq, Tpad / 128) x 512 bytes
   __nv_bfloat16* ds;      // stored dS^T tiles, 128 x 128 each
+  int* counter;           // [2] work-item counters of the main and dQ kernels (zeroed by the prep kernel)
   long long tiles_per_bh;
   int span;
 };
@@ -174,13 +175,15 @@ BwdWorkspace carve_bwd(void* ws, int B, int T, int Hq, int window) {
   w.ext_delta = p;
   p += align256((size_t)B * Hq * Tpad * 4);
   w.ds = reinterpret_cast<__nv_bfloat16*>(p);
+  p += align256((size_t)B * Hq * w.tiles_per_bh * 32768);
+  w.counter = reinterpret_cast<int*>(p);
   return w;
 }
 size_t bwd_ws_bytes(int B, int T, int Hq, int window) {
   const int nt = tiles128(T);
   const size_t Tpad = (size_t)nt * 128;
   const long long tiles = ds_tiles_before(nt, nt, bwd_span(nt, eff_window(window, T)));
-  return 2 * align256((size_t)B * Hq * Tpad * 4) + (size_t)B * Hq * tiles * 32768;
+  return 2 * align256((size_t)B * Hq * Tpad * 4) + align256((size_t)B * Hq * tiles * 32768) + 256;
 }
 
 template <int D>
@@ -205,8 +208,8 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
   {
     const long long threads = (long long)B * Tpad * Hq * (D / 8);
     attn_bwd_prep_kernel<D><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, w.ext_lse, w.ext_delta, B, T,
-        Tpad, Hq, 1.f / scale);
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, w.ext_lse, w.ext_delta, w.counter, B,
+        T, Tpad, Hq, 1.f / scale);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
   }
   BwdParams p{};
@@ -216,6 +219,7 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.ds = w.ds;
+  p.item_counter = w.counter;
   p.T = T;
   p.Tpad = Tpad;
   p.Hq = Hq;
@@ -226,7 +230,12 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
   p.tiles_per_bh = w.tiles_per_bh;
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
-  attn_bwd_kernel<D><<<dim3(nt, Hkv, B), 384, BwdLayout<D>::kBytes, st>>>(tq, tk, tv, tdo, p);
+  {
+    // persistent: one CTA per SM walks the (key tile, KV head, batch) items
+    const long long kv_items = (long long)nt * Hkv * B;
+    const int kv_grid = (int)std::min<long long>(kv_items, sm_count());
+    attn_bwd_kernel<D><<<kv_grid, 384, BwdLayout<D>::kBytes, st>>>(tq, tk, tv, tdo, p, (int)kv_items);
+  }
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
   const long long items = (long long)nt * Hq * B;
   const int grid = (int)std::min<long long>(items, sm_count());

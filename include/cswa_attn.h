@@ -82,11 +82,13 @@ attn_status_t attn_rope_qknorm_bwd(const void* q, const void* k, const void* dq_
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T,
                        int Hq, int Hkv, int D, int window, float scale, void* stream);
 
-/* Bytes of workspace attn_bwd needs for this window: the per-row lse*log2(e) and
- * Delta_i = dO_i . o_i (fp32, (B,Hq,Tpad), Tpad = T rounded up to a multiple of 128)
- * and the bf16 dS^T tiles (128 x 128) of every (query tile, key tile) pair inside
- * the causal window, kept between the main backward kernel and the dQ kernel:
- * about B*Hq*T*min(T, W+128)*2 bytes for window W (B*Hq*T^2 without a window). */
+/* Bytes of workspace attn_bwd needs for this window: per query row, -lse/scale and
+ * -Delta_i = -(dO_i . o_i) as bf16 hi/lo pairs (2 x B*Hq*Tpad*4 bytes, Tpad = T
+ * rounded up to a multiple of 128); the bf16 dS^T tiles (128 x 128) of every (query
+ * tile, key tile) pair inside the causal window, kept between the main backward
+ * kernel and the dQ kernel: about B*Hq*T*min(T, W+128)*2 bytes for window W
+ * (B*Hq*T^2 without a window); and 256 bytes for the main kernel's work counter.
+ * Nothing in it needs to be initialised. */
 size_t attn_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int window);
 
 /*

@@ -46,13 +46,13 @@ def test_bwd_workspace_size(L):
     B, T, Hq, Hkv, D = 8, 2048, 10, 10, 128
     rows = B * Hq * 2048 * 4
     # window 1024: key tile n sees min(16 - n, 9) query tiles -> 7*9 + (9+8+...+1) = 108
-    assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, 1024) == 2 * rows + B * Hq * 108 * 32768
+    assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, 1024) == 2 * rows + B * Hq * 108 * 32768 + 256
     # no window: the 16*17/2 = 136 tiles of the lower triangle; window >= T - 1 is the same
-    full = 2 * rows + B * Hq * 136 * 32768
+    full = 2 * rows + B * Hq * 136 * 32768 + 256
     assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, -1) == full
     assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, 2048) == full
     # ragged T pads the per-row arrays to whole 128-row tiles; window 0 keeps the diagonal only
-    assert L.attn_bwd_workspace_bytes(1, 130, 2, 1, 64, 0) == 2 * 2048 + 2 * 2 * 32768
+    assert L.attn_bwd_workspace_bytes(1, 130, 2, 1, 64, 0) == 2 * 2048 + 2 * 2 * 32768 + 256
     assert L.attn_bwd_workspace_bytes(1, 16, 3, 2, 128, -1) == 0     # Hq % Hkv != 0
     assert L.attn_bwd_workspace_bytes(1, 16, 2, 2, 96, -1) == 0      # head dim
 
