@@ -375,6 +375,7 @@ attn_status_t attn_decode(const void* q, void* kcache, void* vcache, const void*
   p.G = G;
   p.window = window;
   p.n_chunks = decode_chunks(Tmax, window);
+  if (p.n_chunks > kDecodeMaxChunks) return ATTN_ERR_UNSUPPORTED;  // more than 512k keys in view
   p.scale_log2 = scale * kLog2e;
   cudaStream_t st = as_stream(stream);
   const int gm = G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : 8;

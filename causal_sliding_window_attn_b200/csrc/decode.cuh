@@ -261,9 +261,19 @@ __global__ void __launch_bounds__(128) decode_chunk_kernel(const DecodeParams p)
   }
 }
 
+// Merge of the chunk partials of one (b, h): weights 2^(m_c - max m), o = sum of the
+// weighted acc / sum of the weighted l, lse. The chunk statistics are spread over the
+// block and reduced with shuffles; the weighted sum over chunks issues 8 loads at a
+// time (all L2 hits), so the merge costs a few load latencies, not two per chunk.
+constexpr int kDecodeMaxChunks = 4096;
 template <int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeParams p) {
-  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  static_assert(D % 32 == 0 && D >= 64, "block of D threads");
+  constexpr int NW = D / 32;
+  __shared__ float s_f[kDecodeMaxChunks];
+  __shared__ float s_red[NW];
+  __shared__ float s_bc;
+  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x, lane = d & 31, wp = d >> 5;
   const int P = p.pos[b];
   __nv_bfloat16* out = p.o + ((size_t)b * p.Hq + h) * D;
   if (P < 0 || P >= p.Tmax) {
@@ -274,13 +284,45 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeParams p)
   const int lo = p.window < 0 ? 0 : max(0, P - p.window);
   const int nc = (P - lo + kDecodeChunk) / kDecodeChunk;
   const float* w = p.ws + ((size_t)b * p.Hq + h) * p.n_chunks * (D + 2);
-  float M = -INFINITY;
-  for (int c = 0; c < nc; ++c) M = fmaxf(M, w[c * (D + 2) + D]);
-  float Lsum = 0.f, O = 0.f;
-  for (int c = 0; c < nc; ++c) {
+  // max of the chunk maxima
+  float mx = -INFINITY;
+  for (int c = d; c < nc; c += D) mx = fmaxf(mx, w[c * (D + 2) + D]);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) s_red[wp] = mx;
+  __syncthreads();
+  if (d == 0) {
+    float m = s_red[0];
+#pragma unroll
+    for (int i = 1; i < NW; ++i) m = fmaxf(m, s_red[i]);
+    s_bc = m;
+  }
+  __syncthreads();
+  const float M = s_bc;
+  // chunk weights and the weighted sum of l
+  float ls = 0.f;
+  for (int c = d; c < nc; c += D) {
     const float f = ex2_approx(w[c * (D + 2) + D] - M);
-    Lsum = fmaf(f, w[c * (D + 2) + D + 1], Lsum);
-    O = fmaf(f, w[c * (D + 2) + d], O);
+    s_f[c] = f;
+    ls = fmaf(f, w[c * (D + 2) + D + 1], ls);
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+  __syncthreads();  // s_red is reused; s_f is complete
+  if (lane == 0) s_red[wp] = ls;
+  __syncthreads();
+  float Lsum = 0.f;
+#pragma unroll
+  for (int i = 0; i < NW; ++i) Lsum += s_red[i];
+  // o[d] = sum_c f_c acc_c[d] / Lsum, 8 chunks per round
+  float O = 0.f;
+  for (int c0 = 0; c0 < nc; c0 += 8) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = (c0 + u < nc) ? w[(c0 + u) * (D + 2) + d] : 0.f;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (c0 + u < nc) O = fmaf(s_f[c0 + u], v[u], O);
   }
   out[d] = __float2bfloat16(O / Lsum);
   if (d == 0 && p.lse) p.lse[(size_t)b * p.Hq + h] = (M + __log2f(Lsum)) * 0.69314718055994531f;
