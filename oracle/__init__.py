@@ -23,5 +23,6 @@ from .attention import (  # noqa: F401
     attention_bwd_rows,
     attention_bwd_keys,
     decode,
+    prefill,
     useful_pairs,
 )

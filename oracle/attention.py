@@ -290,3 +290,52 @@ def decode(q, kcache, vcache, pos, window, scale, k_new=None, v_new=None):
             o[b, 0, h, :] = (e @ V) / l
             lse[b, h] = m + np.log(l)
     return o, lse, kc, vc
+
+
+# --------------------------------------------------------------------------
+# Chunked prefill against a KV cache  [AG6, AG7]
+# --------------------------------------------------------------------------
+def prefill(q, kcache, vcache, pos, window, scale, k_new=None, v_new=None, rows=None):
+    """A chunk of Tc new query tokens per sequence against its cache.
+
+    q (B, Tc, Hq, D); caches (B, Tmax, Hkv, D); pos (B,) = the number of
+    entries already in each cache, so chunk row t of sequence b sits at
+    position pos[b] + t. When k_new / v_new (B, Tc, Hkv, D) are given they are
+    first written into the caches at rows pos[b] .. pos[b] + Tc - 1 [AG7].
+    Row t then attends to the keys [max(0, p - window), p] of its own cache,
+    p = pos[b] + t: the training mask of ``visible`` in absolute positions
+    [AG3, AG6]. Cache rows past p are never read.
+    Returns o (B, R, Hq, D), lse (B, Hq, R) for the R requested chunk rows
+    (all Tc by default) and the updated caches.
+    """
+    q = _f64(q)
+    kc = _f64(kcache).copy()
+    vc = _f64(vcache).copy()
+    B, Tc, Hq, D = q.shape
+    G = _group(q, kc)
+    pos = np.asarray(pos, dtype=np.int64)
+    if k_new is not None:
+        kn, vn = _f64(k_new), _f64(v_new)
+        for b in range(B):
+            kc[b, pos[b]:pos[b] + Tc] = kn[b]
+            vc[b, pos[b]:pos[b] + Tc] = vn[b]
+    rows = np.arange(Tc) if rows is None else np.asarray(rows, dtype=np.int64)
+    o = np.empty((B, len(rows), Hq, D))
+    lse = np.empty((B, Hq, len(rows)))
+    for b in range(B):
+        p_rows = pos[b] + rows              # absolute positions of the requested rows
+        n_keys = int(p_rows.max()) + 1      # keys 0 .. the last row's position
+        j = np.arange(n_keys)
+        mask = visible(p_rows[:, None], j[None, :], window)
+        for h in range(Hq):
+            K = kc[b, :n_keys, h // G, :]
+            V = vc[b, :n_keys, h // G, :]
+            S = scale * (q[b, rows, h, :] @ K.T)
+            # masked entries are set, not added: NaN in an unused cache row stays out
+            S = np.where(mask, S, -np.inf)
+            m = S.max(axis=1, keepdims=True)
+            E = np.where(mask, np.exp(S - m), 0.0)
+            l = E.sum(axis=1, keepdims=True)
+            o[b, :, h, :] = (E / l) @ np.where(mask.any(axis=0)[:, None], V, 0.0)
+            lse[b, h, :] = (m + np.log(l))[:, 0]
+    return o, lse, kc, vc

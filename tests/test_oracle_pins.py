@@ -9,6 +9,8 @@
     prefix mean of v with lse = ln(n), sum_j dK_j = 0, sum_j dV_j = sum_i dO_i
   * torch's scaled_dot_product_attention and its autograd, in float64 on the CPU
   * decode at position p equals row p of the forward pass
+  * chunked prefill against a cache equals the same rows of one forward pass,
+    and a one-token chunk equals a decode step
 The last test plants plausible mistakes in the oracle and shows a pin fails.
 """
 import json
@@ -236,6 +238,62 @@ def check_decode_row(seed=10):
             allclose(l[b], l_full[b, :, pos[b]], 1e-13)
 
 
+def check_prefill_chunks(seed=12):
+    """Chunked prefill against a cache equals the rows of one forward pass.
+
+    (a) one sequence per batch entry fed in chunks of 5, 1, 7 and 11 tokens,
+    each chunk appending to caches that start out NaN; (b) ragged cache
+    lengths: sequence b holds its first pos[b] keys and NaN after them.
+    """
+    B, Tmax, Hq, Hkv, D = 3, 24, 4, 2, 8
+    qall, kall = rnd((B, Tmax, Hq, D), seed), rnd((B, Tmax, Hkv, D), seed + 1)
+    vall = rnd((B, Tmax, Hkv, D), seed + 2)
+    for W in (-1, 0, 3, 9):
+        o_full, l_full = oracle.attention_fwd(qall, kall, vall, W, 0.5)
+        kc = np.full((B, Tmax, Hkv, D), np.nan)
+        vc = np.full((B, Tmax, Hkv, D), np.nan)
+        bounds = [0, 5, 6, 13, 24]
+        for c0, c1 in zip(bounds[:-1], bounds[1:]):
+            pos = np.full(B, c0)
+            o, l, kc, vc = oracle.prefill(qall[:, c0:c1], kc, vc, pos, W, 0.5,
+                                          k_new=kall[:, c0:c1], v_new=vall[:, c0:c1])
+            allclose(o, o_full[:, c0:c1], 1e-13)
+            allclose(l, l_full[:, :, c0:c1], 1e-13)
+        allclose(kc, kall, 0.0)
+        allclose(vc, vall, 0.0)
+        pos = np.array([0, 3, 13])
+        Tc = 6
+        kc = np.full((B, Tmax, Hkv, D), np.nan)
+        vc = np.full((B, Tmax, Hkv, D), np.nan)
+        for b in range(B):
+            kc[b, :pos[b]] = kall[b, :pos[b]]
+            vc[b, :pos[b]] = vall[b, :pos[b]]
+        qc = np.stack([qall[b, pos[b]:pos[b] + Tc] for b in range(B)])
+        kn = np.stack([kall[b, pos[b]:pos[b] + Tc] for b in range(B)])
+        vn = np.stack([vall[b, pos[b]:pos[b] + Tc] for b in range(B)])
+        o, l, _, _ = oracle.prefill(qc, kc, vc, pos, W, 0.5, k_new=kn, v_new=vn)
+        o2, l2, _, _ = oracle.prefill(qc, kc, vc, pos, W, 0.5, k_new=kn, v_new=vn, rows=[5, 0, 2])
+        for b in range(B):
+            allclose(o[b], o_full[b, pos[b]:pos[b] + Tc], 1e-13)
+            allclose(l[b], l_full[b, :, pos[b]:pos[b] + Tc], 1e-13)
+            allclose(o2[b], o_full[b, pos[b] + np.array([5, 0, 2])], 1e-13)
+
+
+def check_prefill_one_token_is_decode(seed=13):
+    """A one-token chunk is a decode step (a separately written routine)."""
+    B, Tmax, Hq, Hkv, D = 3, 20, 6, 3, 8
+    kc, vc = rnd((B, Tmax, Hkv, D), seed), rnd((B, Tmax, Hkv, D), seed + 1)
+    q, kn, vn = rnd((B, 1, Hq, D), seed + 2), rnd((B, 1, Hkv, D), seed + 3), rnd((B, 1, Hkv, D), seed + 4)
+    pos = np.array([0, 11, 19])
+    for W in (-1, 4):
+        o, l, kc1, vc1 = oracle.prefill(q, kc, vc, pos, W, 0.7, k_new=kn, v_new=vn)
+        od, ld, kc2, vc2 = oracle.decode(q, kc, vc, pos, W, 0.7, k_new=kn, v_new=vn)
+        allclose(o, od, 1e-13)
+        allclose(l[:, :, 0], ld, 1e-13)
+        allclose(kc1, kc2, 0.0)
+        allclose(vc1, vc2, 0.0)
+
+
 # ---------------------------------------------------------------- tests
 def test_golden_two_token():
     check_golden()
@@ -302,6 +360,14 @@ def test_matches_torch_sdpa_fp64():
 
 def test_decode_equals_forward_row():
     check_decode_row()
+
+
+def test_prefill_chunks_equal_forward_rows():
+    check_prefill_chunks()
+
+
+def test_prefill_one_token_is_decode():
+    check_prefill_one_token_is_decode()
 
 
 def test_sampled_backward_matches_full():
@@ -380,6 +446,27 @@ def test_pins_catch_planted_mistakes(monkeypatch, name, attr, bad, check):
     monkeypatch.setattr(oracle, attr, bad, raising=False)
     with pytest.raises(AssertionError):
         check()
+
+
+def test_pins_catch_prefill_ignoring_the_cache(monkeypatch):
+    """A chunk that attends only to its own keys (the cache left out) must fail."""
+    def prefill_chunk_only(q, kcache, vcache, pos, window, scale, k_new=None, v_new=None, rows=None):
+        o, lse = oa.attention_fwd(q, k_new, v_new, window, scale, rows)
+        return o, lse, kcache, vcache
+    monkeypatch.setattr(oracle, "prefill", prefill_chunk_only)
+    with pytest.raises(AssertionError):
+        check_prefill_chunks()
+
+
+def test_pins_catch_prefill_positions_off_by_one(monkeypatch):
+    """Chunk row t must sit at pos + t; pos + t - 1 breaks the one-token == decode pin."""
+    real = oa.prefill
+    def shifted(q, kcache, vcache, pos, window, scale, k_new=None, v_new=None, rows=None):
+        o, lse, kc, vc = real(q, kcache, vcache, np.maximum(np.asarray(pos) - 1, 0), window, scale, k_new, v_new, rows)
+        return o, lse, kc, vc
+    monkeypatch.setattr(oracle, "prefill", shifted)
+    with pytest.raises(AssertionError):
+        check_prefill_one_token_is_decode()
 
 
 def test_pins_catch_wrong_gqa_mapping(monkeypatch):

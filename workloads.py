@@ -7,9 +7,10 @@ and rounds them to bf16.
 
 The shapes follow the nanochat d20 model (head_dim 128, 2048-token context,
 "SSSL" short/long layers; nanochat User Guide, 4 "The One Dial You Control" and
-13 "base_train full flag list"), a GQA variant, a long-context variant and a
-KV-cache decode batch. The pages train on text corpora; these synthetic
-tensors stand in for the activations that reach the attention block.
+13 "base_train full flag list"), a GQA variant, a long-context variant, a
+KV-cache decode batch and a chunked-prefill batch over ragged cache lengths.
+The pages train on text corpora; these synthetic tensors stand in for the
+activations that reach the attention block.
 """
 import math
 
@@ -28,6 +29,10 @@ CONFIGS = {
 
 DECODE = dict(B=32, Hq=10, Hkv=10, D=128, Tmax=2176, window=1024,
               len_lo=512, len_hi=2048, seed=4)
+
+# chunked prefill: a 512-token chunk per sequence on top of cache lengths U[0, 1536]
+PREFILL = dict(B=8, Hq=10, Hkv=10, D=128, T=512, Tmax=2048, window=1024,
+               len_lo=0, len_hi=1536, seed=5)
 
 
 def default_scale(D):
@@ -67,6 +72,35 @@ def decode_inputs(B, Hq, Hkv, D, Tmax, len_lo, len_hi, seed, **_):
     vn = torch.randn((B, 1, Hkv, D), generator=g, dtype=torch.float32)
     bf = torch.bfloat16
     return (lengths.to(torch.int32), kc.to(bf), vc.to(bf), q.to(bf), kn.to(bf), vn.to(bf))
+
+
+def prefill_inputs(B, Hq, Hkv, D, T, Tmax, len_lo, len_hi, seed, **_):
+    """Cache lengths and raw (pre-prologue) tensors for one chunked-prefill step.
+
+    Returns lengths int32 (B,), raw k cache (B, Tmax, Hkv, D), v cache, raw q
+    (B, T, Hq, D), raw k_new and v_new (B, T, Hkv, D); all bf16. The k cache goes
+    through the prologue at positions 0..Tmax-1; q and k_new at lengths[b] + t.
+    """
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    lengths = torch.randint(len_lo, len_hi + 1, (B,), generator=g, dtype=torch.int64)
+    kc = torch.randn((B, Tmax, Hkv, D), generator=g, dtype=torch.float32)
+    vc = torch.randn((B, Tmax, Hkv, D), generator=g, dtype=torch.float32)
+    q = torch.randn((B, T, Hq, D), generator=g, dtype=torch.float32)
+    kn = torch.randn((B, T, Hkv, D), generator=g, dtype=torch.float32)
+    vn = torch.randn((B, T, Hkv, D), generator=g, dtype=torch.float32)
+    bf = torch.bfloat16
+    return (lengths.to(torch.int32), kc.to(bf), vc.to(bf), q.to(bf), kn.to(bf), vn.to(bf))
+
+
+def prefill_pairs(lengths, T, window):
+    """Visible (query, key) pairs of one head over a prefill chunk: row t of
+    sequence b sits at position lengths[b] + t and sees min(position, W) + 1 keys."""
+    n = 0
+    for L in lengths:
+        for t in range(T):
+            p = L + t
+            n += (p if window < 0 else min(p, window)) + 1
+    return n
 
 
 def visible_pairs(T, window):
