@@ -9,7 +9,9 @@ prologue, attention forward, attention backward and the prologue backward.
 `value` is useful fwd+bwd TFLOP/s: 12*D per visible (query, key) pair (the
 pages' 3 x forward convention), masked work and recompute not counted. The
 KV-cache decode workload (32 sequences, lengths U[512, 2048], window 1024) is
-timed in the same run and reported under "decode" as HBM GB/s.
+timed in the same run and reported under "decode" as HBM GB/s, and the
+chunked-prefill workload (8 sequences, a 512-token chunk each on cache lengths
+U[0, 1536], window 1024) under "prefill" as useful TFLOP/s.
 
 Under torchrun each rank runs its own batch (weak scaling, no collective on
 the data path); times are the max over ranks. `--impl reference` times the
@@ -274,6 +276,7 @@ def run_gpu(args, rank, world, local):
     }
     if rank == 0 and not args.no_decode:
         result["decode"] = run_decode(cswa, dev, args, pk, pk_src)
+        result["prefill"] = run_prefill(cswa, dev, args, pk, pk_src)
     if not args.no_e2e:
         result["e2e"] = run_e2e(cswa, dev, args, q, k, v, do, L, scale, world, flops_f + flops_b)
     return result
@@ -316,6 +319,48 @@ def run_decode(cswa, dev, args, pk, pk_src):
                          "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
                          "traffic": ncu_traffic("decode_chunk_kernel"), "algorithmic_bytes": nbytes,
                          "peak_kind": pk_src}}
+
+
+def run_prefill(cswa, dev, args, pk, pk_src):
+    """Chunked prefill: a 512-token chunk per sequence against its KV cache (append +
+    tensor-core forward over the cache), useful FLOPs = 4 D per visible pair."""
+    c = workloads.PREFILL
+    B, Hq, Hkv, D, T, Tmax, W = c["B"], c["Hq"], c["Hkv"], c["D"], c["T"], c["Tmax"], c["window"]
+    lengths, kraw, vc, qraw, knraw, vn = workloads.prefill_inputs(**c)
+    kraw, vc, qraw, knraw, vn = (t.to(dev) for t in (kraw, vc, qraw, knraw, vn))
+    pos = lengths.to(dev)
+    _, kc = cswa.attn_rope_qknorm(None, kraw)
+    q, kn = cswa.attn_rope_qknorm(qraw, knraw, pos=pos)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, T), device=dev, dtype=torch.float32)
+    flush = torch.empty(256 * 1024 * 1024 // 4, device=dev, dtype=torch.float32)
+    reps = max(20, args.steps)
+    times = []
+    for i in range(5 + reps):
+        flush_l2(flush)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        # the same chunk is appended every call: the caches end up identical each time
+        cswa.attn_prefill(q, kc, vc, pos, W, k_new=kn, v_new=vn, o=o, lse=lse)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 5:
+            times.append(e0.elapsed_time(e1))
+    assert cswa.attn_get_status() == 0
+    ms = statistics.median(times)
+    flops = 4 * D * Hq * workloads.prefill_pairs(lengths.tolist(), T, W)
+    tf = flops / (ms * 1e-3) / 1e12
+    peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    return {"workload": "chunked prefill: 8 sequences, a 512-token chunk each on cache lengths U[0,1536] "
+                        "(seed 5), Hq=Hkv=10, D=128, Tmax=2048, window 1024, append of the chunk's k/v",
+            "us_per_step": round(ms * 1e3, 2), "us_p10": round(np.percentile(times, 10) * 1e3, 2),
+            "us_p90": round(np.percentile(times, 90) * 1e3, 2), "value": round(tf, 1), "unit": "TFLOP/s",
+            "l2": "flushed (256 MB write) before every call", "gpu_launches_per_step": 2,
+            "roofline": {"kernel": "attn_prefill (append + forward over the cache)", "bound": "tensor",
+                         "achieved": round(tf, 1), "peak": peak, "unit": "TFLOP/s", "frac": round(tf / peak, 4),
+                         "traffic": ncu_traffic("attn_fwd_kernel_prefill"),
+                         "traffic_note": "ncu dram read+write bytes of the forward-over-cache launch alone",
+                         "algorithmic_flops": flops, "peak_kind": f"bf16 burst ({pk_src})"}}
 
 
 def run_e2e(cswa, dev, args, q, k, v, do, L, scale, world, flops):

@@ -9,6 +9,7 @@ current CUDA stream. The functions carry the C ABI's names (include/cswa_attn.h)
     attn_fwd              attention forward -> (o, lse)
     attn_bwd              attention backward -> (dq, dk, dv)
     attn_decode           single-token decode against a KV cache -> (o, lse)
+    attn_prefill          a chunk of new tokens against a KV cache -> (o, lse)
 
 Tensors are bf16 CUDA tensors in BTHD layout (B, T, H, D), contiguous. There is
 no fallback: without the built library (or off an sm_100 GPU) every call raises.
@@ -21,7 +22,7 @@ import torch
 
 __all__ = [
     "AttnError", "lib", "attn_rope_qknorm", "attn_rope_qknorm_bwd", "attn_fwd", "attn_bwd",
-    "attn_bwd_workspace_bytes", "attn_decode", "attn_decode_workspace_bytes", "attn_get_status",
+    "attn_bwd_workspace_bytes", "attn_decode", "attn_decode_workspace_bytes", "attn_prefill", "attn_get_status",
     "attn_status_string", "LIB_PATH",
 ]
 
@@ -41,6 +42,7 @@ _SIGS = {
     "attn_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "attn_decode": (_i, [_vp] * 8 + [_i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "attn_decode_noalloc": (_i, [_vp] * 8 + [_i, _i, _i, _i, _i, _i, _f, _vp]),
+    "attn_prefill": (_i, [_vp] * 8 + [_i, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "attn_get_status": (_i, [_vp]),
     "attn_status_string": (ctypes.c_char_p, [_i]),
     "attn_device_supported": (_i, []),
@@ -194,6 +196,33 @@ def attn_decode(q, kcache, vcache, pos, window=-1, scale=None, k_new=None, v_new
         B, Tmax, Hq, Hkv, D, int(window), _default_scale(D, scale), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
     return o, lse
+
+
+def attn_prefill(q, kcache, vcache, pos, window=-1, scale=None, k_new=None, v_new=None, o=None, lse=None,
+                 stream=None):
+    """o (B,T,Hq,D), lse (B,Hq,T) for a chunk of T tokens per sequence at positions pos[b] + t.
+
+    Appends k_new / v_new (B,T,Hkv,D) into the caches at pos[b] first, in place.
+    Pass lse=False to skip the lse output.
+    """
+    B, T, Hq, D = _bf16("q", q).shape
+    _, Tmax, Hkv, _ = _bf16("kcache", kcache).shape
+    _bf16("vcache", vcache)
+    if (k_new is None) != (v_new is None):
+        raise ValueError("k_new and v_new go together")
+    if k_new is not None:
+        _bf16("k_new", k_new)
+        _bf16("v_new", v_new)
+    if not (pos.is_cuda and pos.dtype == torch.int32 and pos.numel() == B):
+        raise ValueError("pos must be an int32 CUDA tensor of B entries")
+    o = torch.empty_like(q) if o is None else _bf16("o", o)
+    if lse is None:
+        lse = torch.empty((B, Hq, T), device=q.device, dtype=torch.float32)
+    lse_t = None if lse is False else lse
+    _check("attn_prefill", lib().attn_prefill(
+        _ptr(q), _ptr(kcache), _ptr(vcache), _ptr(k_new), _ptr(v_new), _ptr(pos), _ptr(o), _ptr(lse_t),
+        B, T, Tmax, Hq, Hkv, D, int(window), _default_scale(D, scale), _stream(stream)))
+    return o, lse_t
 
 
 def attn_get_status(stream=None):

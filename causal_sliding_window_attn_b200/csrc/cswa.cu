@@ -82,6 +82,8 @@ bool set_smem_attrs() {
                                   FwdLayout<D>::kBytes) == cudaSuccess;
     r = r && cudaFuncSetAttribute(attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   BwdLayout<D>::kBytes) == cudaSuccess;
+    r = r && cudaFuncSetAttribute(attn_fwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  FwdLayout<D>::kBytes) == cudaSuccess;
     return r;
   }();
   return ok;
@@ -151,6 +153,34 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, f
   p.n_pairs = (p.nq_tiles + 1) / 2;
   dim3 grid(Hq, B, p.n_pairs);
   attn_fwd_kernel<D><<<grid, 384, FwdLayout<D>::kBytes, st>>>(tq, tk, tv, p);
+  return launched();
+}
+
+// Chunked prefill: the forward kernel in cache mode. q (B,T,Hq,D) is the chunk, the
+// caches (B,Tmax,Hkv,D) already hold its keys and values at rows pos[b] .. pos[b]+T-1.
+template <int D>
+attn_status_t launch_prefill(const void* q, const void* kc, const void* vc, const int32_t* pos, void* o, float* lse,
+                             int B, int T, int Tmax, int Hq, int Hkv, int window, float scale, cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  if (!encode_bthd(&tq, q, B, T, Hq, D) || !encode_bthd(&tk, kc, B, Tmax, Hkv, D) ||
+      !encode_bthd(&tv, vc, B, Tmax, Hkv, D))
+    return ATTN_ERR_LAUNCH;
+  if (!set_smem_attrs<D>()) return ATTN_ERR_LAUNCH;
+  FwdParams p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.T = T;
+  p.Hq = Hq;
+  p.G = Hq / Hkv;
+  p.window = (window >= Tmax) ? -1 : window;  // no position reaches Tmax
+  p.scale_log2 = scale * kLog2e;
+  p.nq_tiles = tiles128(T);
+  p.n_pairs = (p.nq_tiles + 1) / 2;
+  p.pos = pos;
+  p.Tmax = Tmax;
+  p.shift = 128 * p.nq_tiles - T;
+  dim3 grid(Hq, B, p.n_pairs);
+  attn_fwd_kernel<D, true><<<grid, 384, FwdLayout<D>::kBytes, st>>>(tq, tk, tv, p);
   return launched();
 }
 
@@ -411,6 +441,34 @@ attn_status_t attn_decode_noalloc(const void* q, void* kcache, void* vcache, con
                      stream);
 }
 
+attn_status_t attn_prefill(const void* q, void* kcache, void* vcache, const void* k_new, const void* v_new,
+                           const int32_t* pos, void* o, float* lse, int B, int T, int Tmax, int Hq, int Hkv, int D,
+                           int window, float scale, void* stream) {
+  if (!dims_ok(B, T, Hq, Hkv) || !dims_ok(B, Tmax, Hq, Hkv) || T > Tmax || !scale_ok(scale))
+    return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!q || !kcache || !vcache || !pos || !o || (k_new == nullptr) != (v_new == nullptr)) return ATTN_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, kcache, vcache, o};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return ATTN_ERR_INVALID_ARG;
+  if ((k_new && !aligned16(k_new)) || (v_new && !aligned16(v_new)) || (reinterpret_cast<uintptr_t>(pos) & 3u) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return ATTN_ERR_INVALID_ARG;
+  if (B > 65535 || Hq > 65535) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  if (k_new) {
+    const int row_vecs = Hkv * D / 8;  // 16-byte vectors per (b, t) row
+    const long long n = (long long)B * T * row_vecs;
+    const int grid = (int)std::min<long long>((n + 255) / 256, 8ll * sm_count());
+    kv_append_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
+                                           static_cast<uint4*>(kcache), static_cast<uint4*>(vcache), pos, T, Tmax,
+                                           row_vecs, n);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  }
+  return D == 64 ? launch_prefill<64>(q, kcache, vcache, pos, o, lse, B, T, Tmax, Hq, Hkv, window, scale, st)
+                 : launch_prefill<128>(q, kcache, vcache, pos, o, lse, B, T, Tmax, Hq, Hkv, window, scale, st);
+}
+
 attn_status_t attn_get_status(void* stream) {
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return ATTN_ERR_LAUNCH;
   unsigned v = 0, zero = 0;
@@ -428,7 +486,7 @@ const char* attn_status_string(attn_status_t s) {
     case ATTN_ERR_UNSUPPORTED: return "unsupported head dim or device";
     case ATTN_ERR_LAUNCH: return "CUDA launch or tensor-map encode failed";
     case ATTN_ERR_TIMEOUT: return "a device-side wait timed out";
-    case ATTN_ERR_DEVICE: return "a device-side range check failed (decode position out of range)";
+    case ATTN_ERR_DEVICE: return "a device-side range check failed (decode or prefill position out of range)";
   }
   return "unknown status";
 }

@@ -20,6 +20,17 @@
 // of S_s in place and feeds the PV product straight from tensor memory.
 // Softmax runs in the log2 domain; the running max is only moved (and O
 // rescaled) when it grows by more than 2^8, which leaves the result exact.
+//
+// Chunked prefill (kCache): the queries are a chunk of T new tokens of each
+// sequence, chunk row t at position pos[b] + t, and the keys and values are the
+// sequence's KV cache, which already holds the chunk's own entries (nanochat Admin
+// & Developer Guide, 6 "Attention: FA3 with SDPA Fallback": chunked / sliding-window
+// inference over a cache; 7 "KV cache"). The tile grid is anchored at the chunk's
+// END: query tile qt covers chunk rows 128 qt - shift .. 128 qt - shift + 127 with
+// shift = 128 ceil(T / 128) - T, and key tile t covers cache rows e0 + 128 t .. with
+// e0 = pos[b] - shift, so the last key row ever loaded is the chunk's last token and
+// no cache row past it (unwritten, possibly NaN) reaches a product. Rows before the
+// chunk or before position 0 come from the TMA's zero fill and are masked.
 #pragma once
 #include "ptx.cuh"
 
@@ -32,6 +43,10 @@ struct FwdParams {
   float scale_log2;  // scale * log2(e)
   int nq_tiles;
   int n_pairs;
+  // chunked prefill only
+  const int32_t* pos;  // (B) entries already in each cache = position of chunk row 0
+  int Tmax;            // cache rows
+  int shift;           // 128 * nq_tiles - T
 };
 
 template <int D>
@@ -46,7 +61,7 @@ struct FwdLayout {
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-template <int D>
+template <int D, bool kCache = false>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -71,6 +86,21 @@ __global__ void __launch_bounds__(384, 1)
   const int pair = p.n_pairs - 1 - blockIdx.z;  // heaviest tiles first
   const int hk = h / p.G;
   const int W = p.window;
+  // e0: position of tile row 0 (0 in training); shift: chunk row of a tile's first row
+  // is 128 qt - shift (0 in training)
+  int e0 = 0, shift = 0;
+  if constexpr (kCache) {
+    const int P = p.pos[b];
+    if (P < 0 || P > p.Tmax - p.T) {  // uniform over the CTA: nothing allocated yet
+      if (threadIdx.x == 0) atomicOr(&g_status, kStatusBadPosition);
+      return;
+    }
+    shift = p.shift;
+    e0 = P - shift;
+  }
+  // first key tile of query tile q: the one holding its first row's oldest visible
+  // key (an arithmetic shift: the floor also for the negative tiles of kCache)
+  auto lo_of = [&](int q) { return (((W < 0) ? 0 : max(0, e0 + q * 128 - W)) - e0) >> 7; };
 
   int qt[2], lo[2], hi[2];
   bool has[2];
@@ -79,7 +109,7 @@ __global__ void __launch_bounds__(384, 1)
     qt[s] = 2 * pair + s;
     has[s] = qt[s] < p.nq_tiles;
     hi[s] = qt[s];
-    lo[s] = (W < 0) ? 0 : max(0, qt[s] * 128 - W) / 128;
+    lo[s] = lo_of(qt[s]);
   }
   const int t_lo = lo[0];
   const int t_hi = has[1] ? hi[1] : hi[0];
@@ -123,7 +153,8 @@ __global__ void __launch_bounds__(384, 1)
       for (int s = 0; s < 2; ++s)
         if (has[s])
           for (int pn = 0; pn < L::kPanels; ++pn)
-            tma_load_4d(smem + (s ? L::kQ1 : L::kQ0) + pn * 16384, &tm_q, q_full, pn * 64, h, qt[s] * 128, b);
+            tma_load_4d(smem + (s ? L::kQ1 : L::kQ0) + pn * 16384, &tm_q, q_full, pn * 64, h, qt[s] * 128 - shift,
+                        b);
       // K and V stages are released separately (K once the S products have read it, V
       // once the PV products have), so K of the next tile loads a whole tile ahead
       int n = 0, last_k[2] = {-1, -1}, last_v[2] = {-1, -1};
@@ -133,12 +164,12 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait(&k_empty[st], ph ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(&k_full[st], L::kTile);
         for (int pn = 0; pn < L::kPanels; ++pn)
-          tma_load_4d(smem + L::kK0 + st * L::kTile + pn * 16384, &tm_k, &k_full[st], pn * 64, hk, t * 128, b);
+          tma_load_4d(smem + L::kK0 + st * L::kTile + pn * 16384, &tm_k, &k_full[st], pn * 64, hk, e0 + t * 128, b);
         last_k[st] = n;
         if (!mbar_wait(&v_empty[st], ph ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(&v_full[st], L::kTile);
         for (int pn = 0; pn < L::kPanels; ++pn)
-          tma_load_4d(smem + L::kV0 + st * L::kTile + pn * 16384, &tm_v, &v_full[st], pn * 64, hk, t * 128, b);
+          tma_load_4d(smem + L::kV0 + st * L::kTile + pn * 16384, &tm_v, &v_full[st], pn * 64, hk, e0 + t * 128, b);
         last_v[st] = n;
       }
       if (*abort_flag) {
@@ -231,10 +262,10 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const int my_qt = 2 * pair + s;
     const int my_hi = my_qt;
-    const int my_lo = (W < 0) ? 0 : max(0, my_qt * 128 - W) / 128;
+    const int my_lo = lo_of(my_qt);
     const uint32_t tSs = tS(s) + lane_off, tOs = tO(s) + lane_off;
     if (my_qt < p.nq_tiles) {
-      const int q0 = my_qt * 128;
+      const int q0 = e0 + my_qt * 128;  // position of the tile's first row
       const int i = q0 + row;
       const float sl2 = p.scale_log2;
       float m_run = -INFINITY, l_run = 0.f;
@@ -254,14 +285,15 @@ __global__ void __launch_bounds__(384, 1)
         tmem_ld32(tSs + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
         tmem_ld32(tSs + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
         tmem_ld_wait();
-        const int k0 = t * 128;
-        const bool full = (k0 + 127 <= q0) && (W < 0 || q0 + 127 - k0 <= W);
+        const int k0 = e0 + t * 128;
+        const bool full = (k0 + 127 <= q0) && (W < 0 || q0 + 127 - k0 <= W) && (!kCache || k0 >= 0);
         // 4 independent 3-input max chains instead of one 128-long dependent chain
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         if (!full) {
           // visible columns of this row: [c_lo, c_hi] (empty when c_lo > c_hi)
           const int c_hi = i - k0;
-          const int c_lo = (W < 0) ? -1 : i - W - k0;
+          int c_lo = (W < 0) ? -1 : i - W - k0;
+          if constexpr (kCache) c_lo = max(c_lo, -k0);  // no key before position 0
 #pragma unroll
           for (int c = 0; c < 128; ++c) {
             const bool vis = (c <= c_hi) & (c >= c_lo);
@@ -326,10 +358,11 @@ __global__ void __launch_bounds__(384, 1)
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
       if (ok) {
-        // tcgen05.ld is warp-collective: every lane loads, only rows < T store
-        const bool store = i < p.T;
+        // tcgen05.ld is warp-collective: every lane loads, only rows of [0, T) store
+        const int cr = my_qt * 128 - shift + row;  // output row (chunk row in kCache)
+        const bool store = (cr < p.T) && (!kCache || cr >= 0);
         const float inv_l = 1.f / l_run;
-        __nv_bfloat16* dst = p.o + ((size_t)((size_t)b * p.T + i) * p.Hq + h) * D;
+        __nv_bfloat16* dst = p.o + ((size_t)((size_t)b * p.T + cr) * p.Hq + h) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -346,7 +379,8 @@ __global__ void __launch_bounds__(384, 1)
             for (int e = 0; e < 4; ++e) d4[e] = v[e];
           }
         }
-        if (store) p.lse[((size_t)b * p.Hq + h) * p.T + i] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+        if (store && (!kCache || p.lse))
+          p.lse[((size_t)b * p.Hq + h) * p.T + cr] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
       }
     }
   }
@@ -355,6 +389,26 @@ __global__ void __launch_bounds__(384, 1)
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// Chunked prefill's cache append: rows t of k_new / v_new (B, T, Hkv, D) go to cache
+// rows pos[b] + t (B, Tmax, Hkv, D), 16 bytes per thread and step. A position that
+// leaves the cache is skipped here and reported by the attention kernel.
+__global__ void __launch_bounds__(256) kv_append_kernel(const uint4* __restrict__ kn, const uint4* __restrict__ vn,
+                                                        uint4* __restrict__ kc, uint4* __restrict__ vc,
+                                                        const int32_t* __restrict__ pos, int T, int Tmax,
+                                                        int row_vecs, long long n) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += stride) {
+    const long long row = e / row_vecs;  // (b, t)
+    const int c = (int)(e - row * row_vecs);
+    const int b = (int)(row / T), t = (int)(row - (long long)b * T);
+    const int P = pos[b];
+    if (P < 0 || P > Tmax - T) continue;
+    const long long d = ((long long)b * Tmax + P + t) * row_vecs + c;
+    kc[d] = kn[e];
+    vc[d] = vn[e];
   }
 }
 

@@ -129,6 +129,33 @@ attn_status_t attn_decode(const void* q, void* kcache, void* vcache, const void*
                           int window, float scale, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * attn_prefill -- a chunk of T new tokens per sequence against its KV cache
+ * (nanochat Admin & Developer Guide, 6 "Attention: FA3 with SDPA Fallback":
+ * chunked / sliding-window inference; 7 "KV cache": (B,T,H,D) caches with int32
+ * per-row positions, appended in place).
+ *   q (B,T,Hq,D) bf16, already through the prologue at positions pos[b] + t
+ *   (attn_rope_qknorm with the same pos does that).
+ *   kcache, vcache (B,Tmax,Hkv,D) bf16; pos int32 (B) device: entries already in
+ *   each cache, so chunk row t sits at position pos[b] + t; 0 <= pos[b] and
+ *   pos[b] + T <= Tmax.
+ *   k_new, v_new (B,T,Hkv,D) or both null: when given they are first written into
+ *   the caches at rows pos[b] .. pos[b] + T - 1 (in place); when null the caches
+ *   must already hold them there.
+ *   Chunk row t attends to keys [max(0, p - window), p] of its cache, p = pos[b] + t
+ *   (window < 0: [0, p]). Cache rows past pos[b] + T - 1 are never read, so they
+ *   may hold anything, NaN included.
+ *   o (B,T,Hq,D) bf16, lse (B,Hq,T) fp32 (natural log) or null.
+ * All device pointers are caller-owned, 16-byte aligned (pos and lse 4-byte).
+ * T <= Tmax, else ATTN_ERR_INVALID_ARG. A sequence whose pos[b] is out of range is
+ * neither appended nor computed (its rows of o and lse are left as they were)
+ * and raises ATTN_ERR_DEVICE in the status word. Two launches: the append copy,
+ * then the tensor-core forward over the cache.
+ */
+attn_status_t attn_prefill(const void* q, void* kcache, void* vcache, const void* k_new, const void* v_new,
+                           const int32_t* pos, void* o, float* lse, int B, int T, int Tmax, int Hq, int Hkv, int D,
+                           int window, float scale, void* stream);
+
+/*
  * attn_decode_noalloc -- attn_decode for callers that cannot allocate device memory.
  * (This entry point has no counterpart on the pages: it is a packaging variant.)
  *

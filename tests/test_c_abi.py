@@ -120,3 +120,20 @@ def test_decode_rejects_bad_args(L):
     a[10], a[11] = 18, 2                              # G = 9 > 8
     a[16] = L.attn_decode_workspace_bytes(2, 18, 128, 64, -1)
     assert L.attn_decode(*a) == UNSUPPORTED
+
+
+def test_prefill_rejects_bad_args(L):
+    # q, kcache, vcache, k_new, v_new, pos, o, lse, B, T, Tmax, Hq, Hkv, D, window, scale, stream
+    base = [P, P, P, P, P, P, P, P, 2, 100, 300, 4, 2, 128, -1, ctypes.c_float(0.1), None]
+    def call(i, v):
+        a = list(base)
+        a[i] = v
+        return L.attn_prefill(*a)
+    assert call(9, 301) == INVALID                    # chunk longer than the cache
+    assert call(3, None) == INVALID                   # v_new without k_new
+    assert call(5, None) == INVALID                   # null pos
+    assert call(5, ctypes.c_void_p(0x10002)) == INVALID  # pos not 4-byte aligned
+    assert call(1, MIS) == INVALID                    # misaligned k cache
+    assert call(12, 3) == INVALID                     # Hq % Hkv
+    assert call(15, ctypes.c_float(-1.0)) == INVALID  # scale
+    assert call(13, 96) == UNSUPPORTED                # head dim

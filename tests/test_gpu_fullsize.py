@@ -4,7 +4,8 @@ The oracle cannot expand every row at these sizes, so it checks sampled
 outputs it can compute one by one: whole query rows of o / lse / dq (rows at
 tile edges, window edges and the ends, plus random ones) for every batch and
 head, and dk / dv at clusters of keys (every query row that sees them is
-expanded). The prologue and its backward are checked on a batch slice.
+expanded). The prologue and its backward are checked on a batch slice. The
+decode and chunked-prefill workloads are checked on every (or sampled) row.
 """
 import numpy as np
 import pytest
@@ -95,3 +96,25 @@ def test_fullsize_decode(cswa):
     o_e2e, _, _, _ = oracle.decode(q_e2e, kc_e2e, f64(vc0), L, W, workloads.default_scale(D), k_new=kn_e2e,
                                    v_new=f64(vn))
     check_out("decode o (end-to-end)", f64(o), o_e2e, max_abs_tol=2e-2)
+
+
+def test_fullsize_prefill(cswa):
+    """The chunked-prefill workload: 8 sequences, a 512-token chunk each on top of
+    cache lengths U[0, 1536], window 1024; sampled chunk rows of every head."""
+    c = workloads.PREFILL
+    B, Hq, Hkv, D, T, Tmax, W = c["B"], c["Hq"], c["Hkv"], c["D"], c["T"], c["Tmax"], c["window"]
+    lengths, kraw, vc, qraw, knraw, vn = workloads.prefill_inputs(**c)
+    kraw, vc, qraw, knraw, vn = (t.cuda() for t in (kraw, vc, qraw, knraw, vn))
+    pos = lengths.cuda()
+    _, kc = cswa.attn_rope_qknorm(None, kraw)
+    q, kn = cswa.attn_rope_qknorm(qraw, knraw, pos=pos)
+    kc0, vc0 = kc.clone(), vc.clone()
+    o, lse = cswa.attn_prefill(q, kc, vc, pos, W, k_new=kn, v_new=vn)
+    torch.cuda.synchronize()
+    assert cswa.attn_get_status() == 0
+    rows = np.array(sorted({0, 1, 127, 128, 255, 256, 383, 384, 510, 511} |
+                           set(np.random.default_rng(7).integers(0, T, 12).tolist())))
+    o_ref, lse_ref, _, _ = oracle.prefill(f64(q), f64(kc0), f64(vc0), lengths.numpy(), W,
+                                          workloads.default_scale(D), k_new=f64(kn), v_new=f64(vn), rows=rows)
+    check_out("prefill o rows", f64(o)[:, rows], o_ref)
+    assert max_abs(f64(lse)[:, :, rows], lse_ref) <= LSE_MAX_ABS
