@@ -152,19 +152,29 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, f
   p.nq_tiles = tiles128(T);
   p.n_pairs = (p.nq_tiles + 1) / 2;
   dim3 grid(Hq, B, p.n_pairs);
-  attn_fwd_kernel<D><<<grid, 384, FwdLayout<D>::kBytes, st>>>(tq, tk, tv, p);
+  // the two chunk maps are unused in training: q's map stands in for them
+  attn_fwd_kernel<D><<<grid, 384, FwdLayout<D>::kBytes, st>>>(tq, tk, tv, tq, tq, p);
   return launched();
 }
 
-// Chunked prefill: the forward kernel in cache mode. q (B,T,Hq,D) is the chunk, the
-// caches (B,Tmax,Hkv,D) already hold its keys and values at rows pos[b] .. pos[b]+T-1.
+// Chunked prefill: the forward kernel in cache mode. q (B,T,Hq,D) is the chunk. With
+// k_new / v_new (B,T,Hkv,D) the chunk's keys are read from them and copied into the
+// caches (B,Tmax,Hkv,D) by the same launch; without, the caches already hold them at
+// rows pos[b] .. pos[b]+T-1.
 template <int D>
-attn_status_t launch_prefill(const void* q, const void* kc, const void* vc, const int32_t* pos, void* o, float* lse,
-                             int B, int T, int Tmax, int Hq, int Hkv, int window, float scale, cudaStream_t st) {
-  CUtensorMap tq, tk, tv;
+attn_status_t launch_prefill(const void* q, void* kc, void* vc, const void* kn, const void* vn, const int32_t* pos,
+                             void* o, float* lse, int B, int T, int Tmax, int Hq, int Hkv, int window, float scale,
+                             cudaStream_t st) {
+  CUtensorMap tq, tk, tv, tkn, tvn;
   if (!encode_bthd(&tq, q, B, T, Hq, D) || !encode_bthd(&tk, kc, B, Tmax, Hkv, D) ||
       !encode_bthd(&tv, vc, B, Tmax, Hkv, D))
     return ATTN_ERR_LAUNCH;
+  if (kn) {
+    if (!encode_bthd(&tkn, kn, B, T, Hkv, D) || !encode_bthd(&tvn, vn, B, T, Hkv, D)) return ATTN_ERR_LAUNCH;
+  } else {
+    tkn = tq;  // unused
+    tvn = tq;
+  }
   if (!set_smem_attrs<D>()) return ATTN_ERR_LAUNCH;
   FwdParams p{};
   p.o = static_cast<__nv_bfloat16*>(o);
@@ -178,9 +188,15 @@ attn_status_t launch_prefill(const void* q, const void* kc, const void* vc, cons
   p.n_pairs = (p.nq_tiles + 1) / 2;
   p.pos = pos;
   p.Tmax = Tmax;
-  p.shift = 128 * p.nq_tiles - T;
+  p.shift = kn ? 0 : 128 * p.nq_tiles - T;
+  p.B = B;
+  p.Hkv = Hkv;
+  p.kn = static_cast<const uint4*>(kn);
+  p.vn = static_cast<const uint4*>(vn);
+  p.kc = static_cast<uint4*>(kc);
+  p.vc = static_cast<uint4*>(vc);
   dim3 grid(Hq, B, p.n_pairs);
-  attn_fwd_kernel<D, true><<<grid, 384, FwdLayout<D>::kBytes, st>>>(tq, tk, tv, p);
+  attn_fwd_kernel<D, true><<<grid, 384, FwdLayout<D>::kBytes, st>>>(tq, tk, tv, tkn, tvn, p);
   return launched();
 }
 
@@ -456,17 +472,10 @@ attn_status_t attn_prefill(const void* q, void* kcache, void* vcache, const void
     return ATTN_ERR_INVALID_ARG;
   if (B > 65535 || Hq > 65535) return ATTN_ERR_INVALID_ARG;
   cudaStream_t st = as_stream(stream);
-  if (k_new) {
-    const int row_vecs = Hkv * D / 8;  // 16-byte vectors per (b, t) row
-    const long long n = (long long)B * T * row_vecs;
-    const int grid = (int)std::min<long long>((n + 255) / 256, 8ll * sm_count());
-    kv_append_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
-                                           static_cast<uint4*>(kcache), static_cast<uint4*>(vcache), pos, T, Tmax,
-                                           row_vecs, n);
-    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
-  }
-  return D == 64 ? launch_prefill<64>(q, kcache, vcache, pos, o, lse, B, T, Tmax, Hq, Hkv, window, scale, st)
-                 : launch_prefill<128>(q, kcache, vcache, pos, o, lse, B, T, Tmax, Hq, Hkv, window, scale, st);
+  return D == 64
+             ? launch_prefill<64>(q, kcache, vcache, k_new, v_new, pos, o, lse, B, T, Tmax, Hq, Hkv, window, scale, st)
+             : launch_prefill<128>(q, kcache, vcache, k_new, v_new, pos, o, lse, B, T, Tmax, Hq, Hkv, window, scale,
+                                   st);
 }
 
 attn_status_t attn_get_status(void* stream) {

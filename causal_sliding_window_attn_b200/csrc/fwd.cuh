@@ -25,12 +25,23 @@
 // sequence, chunk row t at position pos[b] + t, and the keys and values are the
 // sequence's KV cache, which already holds the chunk's own entries (nanochat Admin
 // & Developer Guide, 6 "Attention: FA3 with SDPA Fallback": chunked / sliding-window
-// inference over a cache; 7 "KV cache"). The tile grid is anchored at the chunk's
-// END: query tile qt covers chunk rows 128 qt - shift .. 128 qt - shift + 127 with
-// shift = 128 ceil(T / 128) - T, and key tile t covers cache rows e0 + 128 t .. with
-// e0 = pos[b] - shift, so the last key row ever loaded is the chunk's last token and
-// no cache row past it (unwritten, possibly NaN) reaches a product. Rows before the
-// chunk or before position 0 come from the TMA's zero fill and are masked.
+// inference over a cache; 7 "KV cache"). No cache row past the chunk's last token
+// (unwritten, possibly NaN) may reach a product, since 0 * NaN would poison the
+// rows that mask it. Two tile grids ensure that:
+//  * chunk given (k_new / v_new): the grid is anchored at the chunk's START. Key
+//    tile t >= 0 is read from k_new / v_new (rows past T are the TMA's zero fill),
+//    t < 0 from the cache (the last such tile ends at pos[b] - 1). The kernel never
+//    reads the cache at or past pos[b], so warp 3 copies the chunk into the cache
+//    while the tiles are computed (the CTA of the group's first query head copies
+//    its own query tiles' rows).
+//  * chunk already in the cache: the grid is anchored at the chunk's END. Query
+//    tile qt covers chunk rows 128 qt - shift .. with shift = 128 ceil(T/128) - T,
+//    key tile t covers cache rows pos[b] - shift + 128 t .., so the last key row
+//    loaded is the chunk's last token.
+// Rows before the chunk or before position 0 come from the TMA's zero fill and are
+// masked. The (sequence, pair) items are ranked by their key-tile count (read from
+// pos on the device) and handed to the CTAs heaviest first, so the last wave of
+// CTAs holds the lightest items.
 #pragma once
 #include "ptx.cuh"
 
@@ -46,8 +57,15 @@ struct FwdParams {
   // chunked prefill only
   const int32_t* pos;  // (B) entries already in each cache = position of chunk row 0
   int Tmax;            // cache rows
-  int shift;           // 128 * nq_tiles - T
+  int shift;           // 128 * nq_tiles - T, or 0 when the chunk comes from kn / vn
+  int B, Hkv;
+  const uint4* kn;     // the chunk's k / v (B, T, Hkv, D), or null
+  const uint4* vn;
+  uint4* kc;           // the caches (B, Tmax, Hkv, D)
+  uint4* vc;
 };
+
+constexpr int kMaxRankedItems = 256;  // prefill items ranked by weight (more: pair order)
 
 template <int D>
 struct FwdLayout {
@@ -64,7 +82,8 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 template <int D, bool kCache = false>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kn,
+                    const __grid_constant__ CUtensorMap tm_vn, const FwdParams p) {
   using L = FwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -82,25 +101,59 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* v_empty = bars + 16;  // [2] PV of the tile has read V
 
   const int warp = warp_id(), lane = lane_id();
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int pair = p.n_pairs - 1 - blockIdx.z;  // heaviest tiles first
+  const int h = blockIdx.x;
+  int b = blockIdx.y;
+  int pair = p.n_pairs - 1 - blockIdx.z;  // heaviest tiles first
   const int hk = h / p.G;
   const int W = p.window;
   // e0: position of tile row 0 (0 in training); shift: chunk row of a tile's first row
   // is 128 qt - shift (0 in training)
-  int e0 = 0, shift = 0;
+  int e0 = 0, shift = 0, P = 0;
+  // first key tile of query tile q: the one holding its first row's oldest visible
+  // key (an arithmetic shift: the floor also for the negative tiles of kCache)
+  auto lo_of_at = [&](int base, int q) { return (((W < 0) ? 0 : max(0, base + q * 128 - W)) - base) >> 7; };
   if constexpr (kCache) {
-    const int P = p.pos[b];
+    shift = p.shift;
+    const int n_items = p.B * p.n_pairs;
+    if (n_items <= kMaxRankedItems) {
+      // rank the (sequence, pair) items by key tiles, heaviest first (ties: lower index
+      // first); the CTA at launch rank blockIdx.z * B + blockIdx.y takes that rank's item
+      int* w = reinterpret_cast<int*>(smem + L::kV0 + L::kTile);  // free until the first V load
+      int* order = w + kMaxRankedItems;
+      for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
+        const int bi = i / p.n_pairs, pi = i - bi * p.n_pairs;
+        const int Pi = p.pos[bi];
+        int wt = -1;  // an item out of range only reports and leaves: last
+        if (Pi >= 0 && Pi <= p.Tmax - p.T) {
+          wt = 0;
+          for (int s2 = 0; s2 < 2; ++s2) {
+            const int q = 2 * pi + s2;
+            if (q < p.nq_tiles) wt += q - lo_of_at(Pi - shift, q) + 1;
+          }
+        }
+        w[i] = wt;
+      }
+      __syncthreads();
+      for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
+        const int wi = w[i];
+        int r = 0;
+        for (int j = 0; j < n_items; ++j) r += (w[j] > wi) | ((w[j] == wi) & (j < i));
+        order[r] = i;
+      }
+      __syncthreads();
+      const int item = order[blockIdx.z * p.B + blockIdx.y];
+      b = item / p.n_pairs;
+      pair = item - b * p.n_pairs;
+      __syncthreads();  // the scratch is V stage 1: read before anything else touches it
+    }
+    P = p.pos[b];
     if (P < 0 || P > p.Tmax - p.T) {  // uniform over the CTA: nothing allocated yet
       if (threadIdx.x == 0) atomicOr(&g_status, kStatusBadPosition);
       return;
     }
-    shift = p.shift;
     e0 = P - shift;
   }
-  // first key tile of query tile q: the one holding its first row's oldest visible
-  // key (an arithmetic shift: the floor also for the negative tiles of kCache)
-  auto lo_of = [&](int q) { return (((W < 0) ? 0 : max(0, e0 + q * 128 - W)) - e0) >> 7; };
+  auto lo_of = [&](int q) { return lo_of_at(e0, q); };
 
   int qt[2], lo[2], hi[2];
   bool has[2];
@@ -149,6 +202,10 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
+      if (kCache && p.kn) {
+        tma_prefetch_desc(&tm_kn);
+        tma_prefetch_desc(&tm_vn);
+      }
       mbar_arrive_expect_tx(q_full, (has[1] ? 2 : 1) * L::kTile);
       for (int s = 0; s < 2; ++s)
         if (has[s])
@@ -161,15 +218,20 @@ __global__ void __launch_bounds__(384, 1)
       for (int t = t_lo; t <= t_hi; ++t, ++n) {
         const int st = n & 1;
         const uint32_t ph = (n >> 1) & 1;
+        // key tiles at or past the chunk's start come from k_new / v_new when given
+        const bool fresh = kCache && p.kn && t >= 0;
+        const CUtensorMap* mk = fresh ? &tm_kn : &tm_k;
+        const CUtensorMap* mv = fresh ? &tm_vn : &tm_v;
+        const int row = fresh ? t * 128 : e0 + t * 128;
         if (!mbar_wait(&k_empty[st], ph ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(&k_full[st], L::kTile);
         for (int pn = 0; pn < L::kPanels; ++pn)
-          tma_load_4d(smem + L::kK0 + st * L::kTile + pn * 16384, &tm_k, &k_full[st], pn * 64, hk, e0 + t * 128, b);
+          tma_load_4d(smem + L::kK0 + st * L::kTile + pn * 16384, mk, &k_full[st], pn * 64, hk, row, b);
         last_k[st] = n;
         if (!mbar_wait(&v_empty[st], ph ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(&v_full[st], L::kTile);
         for (int pn = 0; pn < L::kPanels; ++pn)
-          tma_load_4d(smem + L::kV0 + st * L::kTile + pn * 16384, &tm_v, &v_full[st], pn * 64, hk, e0 + t * 128, b);
+          tma_load_4d(smem + L::kV0 + st * L::kTile + pn * 16384, mv, &v_full[st], pn * 64, hk, row, b);
         last_v[st] = n;
       }
       if (*abort_flag) {
@@ -254,6 +316,51 @@ __global__ void __launch_bounds__(384, 1)
     mma_commit(final_bar, leader);
     volatile int dummy = 0;
     mbar_wait(final_bar, 0, &dummy);
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------------ cache append (prefill)
+    // Warps 2 and 3 of the group's first query head copy the chunk rows of the CTA's
+    // own query tiles into the caches (each (b, KV head, row) exactly once), 8 vectors
+    // of k and 8 of v in flight per lane. Nothing in this launch reads those cache
+    // rows: the key tiles at or past pos[b] come from k_new / v_new.
+    if constexpr (kCache) {
+      if (p.kn && h % p.G == 0) {
+        constexpr int V = D / 8;  // 16-byte vectors per row
+        constexpr int kBatch = 8;
+        const int tid = (warp - 2) * 32 + lane;
+        const size_t rs = (size_t)p.Hkv * V;  // row stride in vectors
+#pragma unroll 1
+        for (int s2 = 0; s2 < 2; ++s2) {
+          if (!has[s2]) continue;
+          const int r0 = qt[s2] * 128, n = min(128, p.T - r0) * V;
+          const uint4* ks = p.kn + ((size_t)((size_t)b * p.T + r0) * p.Hkv + hk) * V;
+          const uint4* vs = p.vn + ((size_t)((size_t)b * p.T + r0) * p.Hkv + hk) * V;
+          uint4* kd = p.kc + ((size_t)((size_t)b * p.Tmax + P + r0) * p.Hkv + hk) * V;
+          uint4* vd = p.vc + ((size_t)((size_t)b * p.Tmax + P + r0) * p.Hkv + hk) * V;
+#pragma unroll 1
+          for (int e0b = 0; e0b < n; e0b += 64 * kBatch) {
+            uint4 kr[kBatch], vr[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+              const int e = e0b + u * 64 + tid;
+              if (e < n) {
+                const size_t off = (size_t)(e / V) * rs + (e % V);
+                kr[u] = ks[off];
+                vr[u] = vs[off];
+              }
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+              const int e = e0b + u * 64 + tid;
+              if (e < n) {
+                const size_t off = (size_t)(e / V) * rs + (e % V);
+                kd[off] = kr[u];
+                vd[off] = vr[u];
+              }
+            }
+          }
+        }
+      }
+    }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
     const int s = (warp - 4) >> 2;
@@ -389,26 +496,6 @@ __global__ void __launch_bounds__(384, 1)
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
-  }
-}
-
-// Chunked prefill's cache append: rows t of k_new / v_new (B, T, Hkv, D) go to cache
-// rows pos[b] + t (B, Tmax, Hkv, D), 16 bytes per thread and step. A position that
-// leaves the cache is skipped here and reported by the attention kernel.
-__global__ void __launch_bounds__(256) kv_append_kernel(const uint4* __restrict__ kn, const uint4* __restrict__ vn,
-                                                        uint4* __restrict__ kc, uint4* __restrict__ vc,
-                                                        const int32_t* __restrict__ pos, int T, int Tmax,
-                                                        int row_vecs, long long n) {
-  const long long stride = (long long)gridDim.x * blockDim.x;
-  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += stride) {
-    const long long row = e / row_vecs;  // (b, t)
-    const int c = (int)(e - row * row_vecs);
-    const int b = (int)(row / T), t = (int)(row - (long long)b * T);
-    const int P = pos[b];
-    if (P < 0 || P > Tmax - T) continue;
-    const long long d = ((long long)b * Tmax + P + t) * row_vecs + c;
-    kc[d] = kn[e];
-    vc[d] = vn[e];
   }
 }
 

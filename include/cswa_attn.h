@@ -148,8 +148,9 @@ attn_status_t attn_decode(const void* q, void* kcache, void* vcache, const void*
  * All device pointers are caller-owned, 16-byte aligned (pos and lse 4-byte).
  * T <= Tmax, else ATTN_ERR_INVALID_ARG. A sequence whose pos[b] is out of range is
  * neither appended nor computed (its rows of o and lse are left as they were)
- * and raises ATTN_ERR_DEVICE in the status word. Two launches: the append copy,
- * then the tensor-core forward over the cache.
+ * and raises ATTN_ERR_DEVICE in the status word. One launch: the tensor-core
+ * forward reads the chunk's keys from k_new / v_new and copies them into the
+ * caches on the way (no cache row at or past pos[b] is read when they are given).
  */
 attn_status_t attn_prefill(const void* q, void* kcache, void* vcache, const void* k_new, const void* v_new,
                            const int32_t* pos, void* o, float* lse, int B, int T, int Tmax, int Hq, int Hkv, int D,
