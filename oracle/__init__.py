@@ -24,5 +24,7 @@ from .attention import (  # noqa: F401
     attention_bwd_keys,
     decode,
     prefill,
+    layer_windows,
+    kv_replicate,
     useful_pairs,
 )

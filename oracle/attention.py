@@ -8,11 +8,14 @@ Sources (page title, section):
         rotary embeddings instead of learned positions; queries and keys are
         RMS-normalised with no learnable weight; grouped-query attention with
         n_kv_head <= n_head; a per-layer sliding window handed to flash
-        attention as a (left, right) pair ("Sliding-window attention").
+        attention as a (left, right) pair ("Sliding-window attention"): a
+        pattern of S (a quarter of the context, rounded up to a 128 tile) and
+        L (full context) tiled over the layers, the last layer always L.
   [AG6] nanochat Admin & Developer Guide, 6 "Attention: FA3 with SDPA Fallback":
         GQA through enable_gqa; single-token decode slices the KV window.
   [AG7] nanochat Admin & Developer Guide, 7 "KV cache": (B, T, H, D) caches,
-        int32 per-row positions, appended in place.
+        int32 per-row positions, appended in place; a batch-1 prefill cache
+        copied into a batch-N decode cache (one row per sample).
   [NG8] nanoGPT Administrator & Developer Guide, 8 "CausalSelfAttention":
         the manual path -- q k^T scaled by 1/sqrt(d), a triangular mask,
         softmax, then a product with v.
@@ -33,6 +36,9 @@ Readings where the pages are silent or disagree (all repeated in the design doc):
     is what repeating each KV head Hq/Hkv times means).
   * lse is the natural-log log-sum-exp of the scaled scores, shape (B, Hq, T).
   * The 1.2 QK gain of [AG3] is folded into ``scale``.
+  * The short window is a quarter of the context rounded up to a multiple of
+    128 (2048 -> 512); the example printed beside that rule (2048 -> 768) does
+    not follow from it and is not used.
 
 Everything is float64 numpy. Query rows are independent by definition, so the
 functions can be asked for a subset of rows; nothing else is blocked, fused or
@@ -339,3 +345,34 @@ def prefill(q, kcache, vcache, pos, window, scale, k_new=None, v_new=None, rows=
             o[b, :, h, :] = (E / l) @ np.where(mask.any(axis=0)[:, None], V, 0.0)
             lse[b, h, :] = (m + np.log(l))[:, 0]
     return o, lse, kc, vc
+
+
+# --------------------------------------------------------------------------
+# Layer stack: per-layer windows and batch-1 -> N cache replication  [AG3, AG7]
+# --------------------------------------------------------------------------
+def layer_windows(n_layer, seq_len, pattern="SSSL", short_window=None):
+    """Window of every layer: ``pattern`` tiled over the layers, 'L' = the full
+    context (returned as -1, unbounded), 'S' = a quarter of the context rounded
+    up to a whole 128-row tile (or ``short_window`` when given); the last layer
+    is always 'L' whatever the pattern says [AG3]."""
+    if not pattern or any(c not in "SL" for c in pattern) or n_layer < 1 or seq_len < 1:
+        raise ValueError("bad pattern or sizes")
+    if short_window is None or short_window <= 0:
+        quarter = -(-seq_len // 4)                  # ceil(seq_len / 4)
+        short_window = -(-quarter // 128) * 128     # up to a multiple of 128
+    out = []
+    for layer in range(n_layer):
+        c = "L" if layer == n_layer - 1 else pattern[layer % len(pattern)]
+        out.append(-1 if c == "L" else short_window)
+    return out
+
+
+def kv_replicate(k_src, v_src, k_dst, v_dst, rows):
+    """Copies rows [0, rows) of a batch-1 cache (n_layers, 1, Tsrc, H, D) into every
+    batch row of a batch-N cache (n_layers, N, Tmax, H, D) [AG7: a batch-1 prefill
+    is expanded across the samples]; the other rows of the destination are kept."""
+    k_out, v_out = np.array(k_dst, copy=True), np.array(v_dst, copy=True)
+    for n in range(k_out.shape[1]):
+        k_out[:, n, :rows] = np.asarray(k_src)[:, 0, :rows]
+        v_out[:, n, :rows] = np.asarray(v_src)[:, 0, :rows]
+    return k_out, v_out

@@ -11,6 +11,8 @@
   * decode at position p equals row p of the forward pass
   * chunked prefill against a cache equals the same rows of one forward pass,
     and a one-token chunk equals a decode step
+  * the per-layer window rule on hand-computed cases; a replicated batch-1 cache
+    decodes every sample exactly as the batch-1 cache does
 The last test plants plausible mistakes in the oracle and shows a pin fails.
 """
 import json
@@ -294,6 +296,49 @@ def check_prefill_one_token_is_decode(seed=13):
         allclose(vc1, vc2, 0.0)
 
 
+def check_layer_windows():
+    """The window rule as the nanochat guide states it, on hand-computed cases:
+    the pattern is tiled over the layers, L is the full context, S a quarter of it
+    rounded up to a 128 tile, and the last layer is L whatever the pattern says."""
+    w = oracle.layer_windows(20, 2048)                       # d20, default SSSL
+    assert w == [-1 if (l % 4 == 3 or l == 19) else 512 for l in range(20)]
+    assert oracle.layer_windows(6, 2048, "L") == [-1] * 6
+    assert oracle.layer_windows(5, 2048, "S") == [512, 512, 512, 512, -1]
+    assert oracle.layer_windows(1, 2048, "S") == [-1]
+    assert oracle.layer_windows(3, 2048, "SL") == [512, -1, -1]
+    assert oracle.layer_windows(4, 1000, "S")[0] == 256       # 250 -> 256
+    assert oracle.layer_windows(4, 4096, "S")[0] == 1024
+    assert oracle.layer_windows(4, 129, "S")[0] == 128        # 33 -> 128
+    assert oracle.layer_windows(4, 2048, "S", short_window=1024)[:3] == [1024] * 3
+    for T in (1, 127, 128, 511, 512, 513, 2048, 8191):
+        s = oracle.layer_windows(2, T, "S")[0]
+        assert s % 128 == 0 and s >= T / 4 and s < T / 4 + 128
+    for bad in ("", "SX", "s"):
+        with pytest.raises(ValueError):
+            oracle.layer_windows(4, 2048, bad)
+
+
+def check_kv_replicate(seed=14):
+    """A batch-1 prefill cache copied to N rows: every sample then decodes exactly as
+    it would against the batch-1 cache, and rows past the prompt keep their contents."""
+    L, Tsrc, Tmax, H, D, N, rows = 2, 12, 16, 2, 8, 3, 9
+    ks, vs = rnd((L, 1, Tsrc, H, D), seed), rnd((L, 1, Tsrc, H, D), seed + 1)
+    kd0, vd0 = rnd((L, N, Tmax, H, D), seed + 2), rnd((L, N, Tmax, H, D), seed + 3)
+    kd, vd = oracle.kv_replicate(ks, vs, kd0, vd0, rows)
+    allclose(kd[:, :, rows:], kd0[:, :, rows:], 0.0)
+    allclose(vd[:, :, rows:], vd0[:, :, rows:], 0.0)
+    q = rnd((N, 1, 4, D), seed + 4)
+    kn, vn = rnd((N, 1, H, D), seed + 5), rnd((N, 1, H, D), seed + 6)
+    pos = np.full(N, rows)
+    for l in range(L):
+        o, lse, _, _ = oracle.decode(q, kd[l], vd[l], pos, 5, 0.3, k_new=kn, v_new=vn)
+        for n in range(N):
+            o1, l1, _, _ = oracle.decode(q[n:n + 1], ks[l], vs[l], pos[:1], 5, 0.3, k_new=kn[n:n + 1],
+                                         v_new=vn[n:n + 1])
+            allclose(o[n], o1[0], 1e-13)
+            allclose(lse[n], l1[0], 1e-13)
+
+
 # ---------------------------------------------------------------- tests
 def test_golden_two_token():
     check_golden()
@@ -360,6 +405,14 @@ def test_matches_torch_sdpa_fp64():
 
 def test_decode_equals_forward_row():
     check_decode_row()
+
+
+def test_layer_windows():
+    check_layer_windows()
+
+
+def test_kv_replicate():
+    check_kv_replicate()
 
 
 def test_prefill_chunks_equal_forward_rows():
@@ -467,6 +520,16 @@ def test_pins_catch_prefill_positions_off_by_one(monkeypatch):
     monkeypatch.setattr(oracle, "prefill", shifted)
     with pytest.raises(AssertionError):
         check_prefill_one_token_is_decode()
+
+
+def test_pins_catch_layer_windows_without_a_final_full_layer(monkeypatch):
+    """The last layer must be L whatever the pattern says."""
+    def tiled_only(n_layer, seq_len, pattern="SSSL", short_window=None):
+        s = short_window or -(-(-(-seq_len // 4)) // 128) * 128
+        return [-1 if pattern[l % len(pattern)] == "L" else s for l in range(n_layer)]
+    monkeypatch.setattr(oracle, "layer_windows", tiled_only)
+    with pytest.raises(AssertionError):
+        check_layer_windows()
 
 
 def test_pins_catch_wrong_gqa_mapping(monkeypatch):
