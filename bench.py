@@ -11,7 +11,8 @@ pages' 3 x forward convention), masked work and recompute not counted. The
 KV-cache decode workload (32 sequences, lengths U[512, 2048], window 1024) is
 timed in the same run and reported under "decode" as HBM GB/s, and the
 chunked-prefill workload (8 sequences, a 512-token chunk each on cache lengths
-U[0, 1536], window 1024) under "prefill" as useful TFLOP/s.
+U[0, 1536], window 1024) under "prefill" as useful TFLOP/s, and the batch-1 -> 8
+KV-cache replication of a 20-layer stack under "kv_replicate" as GB/s.
 
 Under torchrun each rank runs its own batch (weak scaling, no collective on
 the data path); times are the max over ranks. `--impl reference` times the
@@ -277,6 +278,7 @@ def run_gpu(args, rank, world, local):
     if rank == 0 and not args.no_decode:
         result["decode"] = run_decode(cswa, dev, args, pk, pk_src)
         result["prefill"] = run_prefill(cswa, dev, args, pk, pk_src)
+        result["kv_replicate"] = run_replicate(cswa, dev, args, pk, pk_src)
     if not args.no_e2e:
         result["e2e"] = run_e2e(cswa, dev, args, q, k, v, do, L, scale, world, flops_f + flops_b)
     return result
@@ -362,6 +364,40 @@ def run_prefill(cswa, dev, args, pk, pk_src):
                          "traffic": ncu_traffic("attn_fwd_kernel_prefill"),
                          "traffic_note": "ncu dram read+write bytes of the prefill launch",
                          "algorithmic_flops": flops, "peak_kind": f"bf16 burst ({pk_src})"}}
+
+
+def run_replicate(cswa, dev, args, pk, pk_src):
+    """Batch-1 -> 8 cache replication over a 20-layer d20 stack: a 1024-token prompt
+    copied into 8 sample rows of (20, 8, 2048, 10, 128) k and v caches."""
+    n_layers, rows, Tmax, N, Hkv, D = 20, 1024, 2048, 8, 10, 128
+    ks = torch.randn((n_layers, 1, Tmax, Hkv, D), device=dev).to(torch.bfloat16)
+    vs = torch.randn((n_layers, 1, Tmax, Hkv, D), device=dev).to(torch.bfloat16)
+    kd = torch.empty((n_layers, N, Tmax, Hkv, D), device=dev, dtype=torch.bfloat16)
+    vd = torch.empty_like(kd)
+    times = []
+    for i in range(3 + 10):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        cswa.attn_kv_replicate(ks, vs, kd, vd, rows)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    row = Hkv * D * 2
+    nbytes = 2 * n_layers * rows * row * (1 + N)  # k and v: the prompt read once, written N times
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    hbm = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    return {"workload": "batch-1 -> 8 KV-cache replication: 20 layers, 1024-token prompt, Hkv=10, D=128, Tmax=2048",
+            "us_per_step": round(ms * 1e3, 1), "value": round(gbs, 1), "unit": "GB/s",
+            "l2": "inputs and outputs (1.9 GB) exceed L2", "gpu_launches_per_step": 0,
+            "copies_per_step": 2 * n_layers * (1 + math.ceil(math.log2(N))),
+            "roofline": {"kernel": "attn_kv_replicate (copy-engine copies, doubling rounds)", "bound": "hbm",
+                         "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                         "traffic": None, "algorithmic_bytes": nbytes,
+                         "note": "the doubling rounds read the copied rows again: the copy engines move "
+                                 "about 2x the algorithmic bytes",
+                         "peak_kind": pk_src}}
 
 
 def run_e2e(cswa, dev, args, q, k, v, do, L, scale, world, flops):

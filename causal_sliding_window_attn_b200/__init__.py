@@ -10,6 +10,8 @@ current CUDA stream. The functions carry the C ABI's names (include/cswa_attn.h)
     attn_bwd              attention backward -> (dq, dk, dv)
     attn_decode           single-token decode against a KV cache -> (o, lse)
     attn_prefill          a chunk of new tokens against a KV cache -> (o, lse)
+    attn_layer_window     the window of one layer of a stack (pattern such as "SSSL")
+    attn_kv_replicate     a batch-1 prefill cache copied to N sample rows
 
 Tensors are bf16 CUDA tensors in BTHD layout (B, T, H, D), contiguous. There is
 no fallback: without the built library (or off an sm_100 GPU) every call raises.
@@ -22,7 +24,8 @@ import torch
 
 __all__ = [
     "AttnError", "lib", "attn_rope_qknorm", "attn_rope_qknorm_bwd", "attn_fwd", "attn_bwd",
-    "attn_bwd_workspace_bytes", "attn_decode", "attn_decode_workspace_bytes", "attn_prefill", "attn_get_status",
+    "attn_bwd_workspace_bytes", "attn_decode", "attn_decode_workspace_bytes", "attn_prefill", "attn_layer_window",
+    "layer_windows", "attn_kv_replicate", "attn_get_status",
     "attn_status_string", "LIB_PATH",
 ]
 
@@ -43,6 +46,8 @@ _SIGS = {
     "attn_decode": (_i, [_vp] * 8 + [_i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "attn_decode_noalloc": (_i, [_vp] * 8 + [_i, _i, _i, _i, _i, _i, _f, _vp]),
     "attn_prefill": (_i, [_vp] * 8 + [_i, _i, _i, _i, _i, _i, _i, _f, _vp]),
+    "attn_layer_window": (_i, [ctypes.c_char_p, _i, _i, _i, _i]),
+    "attn_kv_replicate": (_i, [_vp] * 4 + [_i] * 7 + [_vp]),
     "attn_get_status": (_i, [_vp]),
     "attn_status_string": (ctypes.c_char_p, [_i]),
     "attn_device_supported": (_i, []),
@@ -223,6 +228,34 @@ def attn_prefill(q, kcache, vcache, pos, window=-1, scale=None, k_new=None, v_ne
         _ptr(q), _ptr(kcache), _ptr(vcache), _ptr(k_new), _ptr(v_new), _ptr(pos), _ptr(o), _ptr(lse_t),
         B, T, Tmax, Hq, Hkv, D, int(window), _default_scale(D, scale), _stream(stream)))
     return o, lse_t
+
+
+def attn_layer_window(pattern, layer, n_layer, seq_len, short_window=0):
+    """Window of one layer: -1 (full context) for L and for the last layer, else the
+    short window (a quarter of seq_len up to a 128 multiple unless short_window > 0)."""
+    w = int(lib().attn_layer_window(pattern.encode(), int(layer), int(n_layer), int(seq_len), int(short_window)))
+    if w < -1:
+        raise ValueError(f"bad window pattern {pattern!r} or sizes (layer {layer} of {n_layer}, seq_len {seq_len})")
+    return w
+
+
+def layer_windows(n_layer, seq_len, pattern="SSSL", short_window=0):
+    """The windows of every layer of an n_layer stack."""
+    return [attn_layer_window(pattern, l, n_layer, seq_len, short_window) for l in range(n_layer)]
+
+
+def attn_kv_replicate(k_src, v_src, k_dst, v_dst, rows, stream=None):
+    """Copies rows [0, rows) of the batch-1 caches (n_layers, 1, Tsrc, Hkv, D) into every
+    sample row of (n_layers, N, Tmax, Hkv, D), in place."""
+    L1, one, Tsrc, Hkv, D = _bf16("k_src", k_src, 5).shape
+    L2, N, Tmax, Hkv2, D2 = _bf16("k_dst", k_dst, 5).shape
+    if one != 1 or (L1, Hkv, D) != (L2, Hkv2, D2) or v_src.shape != k_src.shape or v_dst.shape != k_dst.shape:
+        raise ValueError("k_src/v_src must be (n_layers, 1, Tsrc, Hkv, D), k_dst/v_dst (n_layers, N, Tmax, Hkv, D)")
+    _bf16("v_src", v_src, 5)
+    _bf16("v_dst", v_dst, 5)
+    _check("attn_kv_replicate", lib().attn_kv_replicate(
+        _ptr(k_src), _ptr(v_src), _ptr(k_dst), _ptr(v_dst), L1, int(rows), Tsrc, N, Tmax, Hkv, D, _stream(stream)))
+    return k_dst, v_dst
 
 
 def attn_get_status(stream=None):

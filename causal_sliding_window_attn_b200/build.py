@@ -2,8 +2,9 @@
 
     python -m causal_sliding_window_attn_b200.build [--force] [-v]
 
-The library is one translation unit (csrc/cswa.cu) that includes every kernel;
-cudart is linked statically and the driver's tensor-map encoder is looked up
+The kernels and their launches are one translation unit (csrc/cswa.cu); the
+host-only helpers (host/*.cpp: per-layer windows, cache replication) are a
+second. cudart is linked statically and the driver's tensor-map encoder is looked up
 at run time, so the .so needs nothing but a CUDA 12.8+ driver.
 """
 import argparse
@@ -16,6 +17,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
+HOST = os.path.join(PKG, "host")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libcswa_attn.so")
 
@@ -33,7 +35,7 @@ def nvcc():
 
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh")) +
-                  glob.glob(os.path.join(INCLUDE, "*.h")))
+                  glob.glob(os.path.join(HOST, "*.cpp")) + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
 def stale():
@@ -48,7 +50,7 @@ def build(force=False, verbose=False):
     if not force and not stale():
         return LIB
     cmd = [nvcc(), *ARCH, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", LIB + ".tmp",
-           os.path.join(CSRC, "cswa.cu")]
+           os.path.join(CSRC, "cswa.cu"), *sorted(glob.glob(os.path.join(HOST, "*.cpp")))]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)

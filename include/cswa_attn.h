@@ -187,6 +187,35 @@ attn_status_t attn_decode_noalloc(const void* q, void* kcache, void* vcache, con
                                   const int32_t* pos, void* o, float* lse, int B, int Tmax, int Hq, int Hkv, int D,
                                   int window, float scale, void* stream);
 
+/*
+ * attn_layer_window -- the attention window of one layer of a stack
+ * (nanochat Admin & Developer Guide, 3 "Sliding-window attention").
+ *   pattern: a NUL-terminated string of 'S' and 'L' tiled over the layers
+ *   (nanochat's default is "SSSL"); layer in [0, n_layer).
+ * Returns -1 (unbounded: the full context) for an 'L' layer and for the last
+ * layer whatever the pattern says; for an 'S' layer short_window when it is > 0,
+ * else a quarter of seq_len rounded up to a multiple of 128 (2048 -> 512).
+ * Returns -2 for a null or empty pattern, any other character, or sizes out of
+ * range. Host only; needs no GPU.
+ */
+int attn_layer_window(const char* pattern, int layer, int n_layer, int seq_len, int short_window);
+
+/*
+ * attn_kv_replicate -- expand a batch-1 prefill cache across N samples
+ * (nanochat Admin & Developer Guide, 7 "KV cache" and "Generation flow": the
+ * prompt is prefilled once at batch 1, then its cache is copied to every row).
+ *   k_src, v_src: (n_layers, 1, Tmax_src, Hkv, D) bf16 device memory.
+ *   k_dst, v_dst: (n_layers, N, Tmax, Hkv, D) bf16 device memory.
+ * Copies rows [0, rows) of every layer into every sample row; the destination's
+ * other rows are left as they were. 0 <= rows <= min(Tmax_src, Tmax); the four
+ * buffers must not overlap (ATTN_ERR_INVALID_ARG). The caller sets each
+ * sample's position (cache_seqlens) to rows. Asynchronous device-to-device
+ * copies on `stream`, 1 + ceil(log2 N) rounds per layer and tensor, no kernel;
+ * a failed copy enqueue returns ATTN_ERR_LAUNCH.
+ */
+attn_status_t attn_kv_replicate(const void* k_src, const void* v_src, void* k_dst, void* v_dst, int n_layers,
+                                int rows, int Tmax_src, int N, int Tmax, int Hkv, int D, void* stream);
+
 /* Synchronises `stream`, then returns and clears the device status word of the
  * current device: ATTN_OK, ATTN_ERR_TIMEOUT or ATTN_ERR_DEVICE (or
  * ATTN_ERR_LAUNCH if a CUDA error is pending). */

@@ -137,3 +137,34 @@ def test_prefill_rejects_bad_args(L):
     assert call(12, 3) == INVALID                     # Hq % Hkv
     assert call(15, ctypes.c_float(-1.0)) == INVALID  # scale
     assert call(13, 96) == UNSUPPORTED                # head dim
+
+
+def test_layer_window_rule_on_cpu(L):
+    """attn_layer_window is host-only: checked here against the oracle's rule."""
+    import oracle
+    import causal_sliding_window_attn_b200 as m
+    for n_layer, T, pat, sw in ((20, 2048, "SSSL", 0), (12, 1000, "SL", 0), (5, 2048, "S", 1024), (1, 64, "S", 0),
+                                (7, 8192, "LSS", 0), (9, 129, "SSSSL", 0)):
+        assert m.layer_windows(n_layer, T, pat, sw) == oracle.layer_windows(n_layer, T, pat, sw or None)
+    assert L.attn_layer_window(b"SSSL", 0, 20, 2048, 0) == 512
+    assert L.attn_layer_window(b"SXSL", 0, 20, 2048, 0) == -2
+    assert L.attn_layer_window(b"", 0, 20, 2048, 0) == -2
+    assert L.attn_layer_window(None, 0, 20, 2048, 0) == -2
+    assert L.attn_layer_window(b"SSSL", 20, 20, 2048, 0) == -2
+    assert L.attn_layer_window(b"SSSL", -1, 20, 2048, 0) == -2
+
+
+def test_kv_replicate_rejects_bad_args(L):
+    A, B2, C, E = (ctypes.c_void_p(x) for x in (0x100000, 0x200000, 0x300000, 0x400000))
+    # k_src, v_src, k_dst, v_dst, n_layers, rows, Tmax_src, N, Tmax, Hkv, D, stream
+    base = [A, B2, C, E, 2, 8, 16, 3, 32, 2, 64, None]
+    def call(i, v):
+        a = list(base)
+        a[i] = v
+        return L.attn_kv_replicate(*a)
+    assert call(5, 17) == INVALID                      # more rows than the source holds
+    assert call(8, 4) == INVALID                       # more rows than the destination holds
+    assert call(0, None) == INVALID
+    assert call(7, 0) == INVALID                       # no samples
+    assert call(3, ctypes.c_void_p(0x300010)) == INVALID  # v_dst overlaps k_dst
+    assert call(5, 0) == 0                             # nothing to copy: ok, nothing enqueued
