@@ -168,3 +168,29 @@ def test_kv_replicate_rejects_bad_args(L):
     assert call(7, 0) == INVALID                       # no samples
     assert call(3, ctypes.c_void_p(0x300010)) == INVALID  # v_dst overlaps k_dst
     assert call(5, 0) == 0                             # nothing to copy: ok, nothing enqueued
+
+
+def test_size_limits_rejected_before_launch(L):
+    """Calls past the kernels' limits come back before anything is enqueued."""
+    f = ctypes.c_float(0.1)
+    # decode: more than 4096 chunks of 128 keys in view (an unbounded window over 600k rows)
+    Tmax = 600_000
+    ws = L.attn_decode_workspace_bytes(1, 1, 128, Tmax, -1)
+    assert ws > 0
+    assert L.attn_decode(P, P, P, None, None, P, P, P, 1, Tmax, 1, 1, 128, -1, f, P, ws, None) == UNSUPPORTED
+    # decode: a group of more than 8 query heads per KV head
+    ws = L.attn_decode_workspace_bytes(1, 9, 128, 64, -1)
+    assert L.attn_decode(P, P, P, None, None, P, P, P, 1, 64, 9, 1, 128, -1, f, P, ws, None) == UNSUPPORTED
+    # backward: stored dS^T tiles beyond 2^31 rows (B * Hq * tiles * 128)
+    B, T, H = 64, 65536, 64
+    ws = L.attn_bwd_workspace_bytes(B, T, H, H, 128, -1)
+    big = ctypes.c_void_p(0x100000000)
+    assert L.attn_bwd(*([P] * 9), big, ws, B, T, H, H, 128, -1, f, None) == UNSUPPORTED
+    # grid limits: 65535 sequences or query heads at most
+    assert L.attn_fwd(P, P, P, P, P, 65536, 16, 1, 1, 128, -1, f, None) == INVALID
+    assert L.attn_fwd(P, P, P, P, P, 1, 16, 65536, 1, 128, -1, f, None) == INVALID
+    assert L.attn_prefill(P, P, P, None, None, P, P, P, 65536, 16, 32, 1, 1, 128, -1, f, None) == INVALID
+    # empty inputs
+    assert L.attn_fwd(P, P, P, P, P, 1, 0, 1, 1, 128, -1, f, None) == INVALID
+    assert L.attn_prefill(P, P, P, None, None, P, P, P, 1, 0, 32, 1, 1, 128, -1, f, None) == INVALID
+    assert L.attn_decode(P, P, P, None, None, P, P, P, 0, 64, 1, 1, 128, -1, f, P, 1 << 20, None) == INVALID
