@@ -25,7 +25,7 @@ import torch
 __all__ = [
     "AttnError", "lib", "attn_rope_qknorm", "attn_rope_qknorm_bwd", "attn_fwd", "attn_bwd",
     "attn_bwd_workspace_bytes", "attn_decode", "attn_decode_workspace_bytes", "attn_prefill", "attn_layer_window",
-    "layer_windows", "attn_kv_replicate", "attn_get_status",
+    "layer_windows", "attn_kv_replicate", "attn_get_status", "attn_debug_set_wait_limit",
     "attn_status_string", "LIB_PATH",
 ]
 
@@ -49,6 +49,7 @@ _SIGS = {
     "attn_layer_window": (_i, [ctypes.c_char_p, _i, _i, _i, _i]),
     "attn_kv_replicate": (_i, [_vp] * 4 + [_i] * 7 + [_vp]),
     "attn_get_status": (_i, [_vp]),
+    "attn_debug_set_wait_limit": (_i, [ctypes.c_ulonglong, _vp]),
     "attn_status_string": (ctypes.c_char_p, [_i]),
     "attn_device_supported": (_i, []),
 }
@@ -256,6 +257,11 @@ def attn_kv_replicate(k_src, v_src, k_dst, v_dst, rows, stream=None):
     _check("attn_kv_replicate", lib().attn_kv_replicate(
         _ptr(k_src), _ptr(v_src), _ptr(k_dst), _ptr(v_dst), L1, int(rows), Tsrc, N, Tmax, Hkv, D, _stream(stream)))
     return k_dst, v_dst
+
+
+def attn_debug_set_wait_limit(ns, stream=None):
+    """Test hook: limit (ns) of the kernels' pipeline waits for later launches; 0 = default (2 s)."""
+    _check("attn_debug_set_wait_limit", lib().attn_debug_set_wait_limit(int(ns), _stream(stream)))
 
 
 def attn_get_status(stream=None):

@@ -313,12 +313,12 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
     }
-    if (lane == 0 && *abort_flag) {
-      // let every copy in flight land before the CTA's shared memory is released
-      volatile int dummy = 0;
+    if (lane == 0) {
+      // let every copy in flight land before the CTA's shared memory is released (at
+      // once after a normal run; an abort raised by another role may leave some pending)
       for (int s = 0; s < nst; ++s)
-        if (last_issue[s] >= 0) mbar_wait(&full[s], (last_issue[s] / nst) & 1, &dummy);
-      if (qside && last_kv >= 0) mbar_wait(kv_full, last_kv & 1, &dummy);
+        if (last_issue[s] >= 0) mbar_drain(&full[s], (last_issue[s] / nst) & 1);
+      if (qside && last_kv >= 0) mbar_drain(kv_full, last_kv & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -439,8 +439,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     // every MMA issued above has finished before TMEM is released
     mma_commit(done_bar, leader);
-    volatile int dummy = 0;
-    mbar_wait(done_bar, 0, &dummy);
+    mbar_drain(done_bar, 0);
   } else if (warp == 2) {
     // ------------------------------------------------------------ work scheduler
     // claims the CTA's next item from the global counter once every role has read
@@ -720,10 +719,10 @@ __global__ void __launch_bounds__(256, 1)
       }
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
     }
-    if (lane == 0 && *abort_flag) {
-      volatile int dummy = 0;
+    if (lane == 0) {
+      // every copy in flight lands before the CTA's shared memory is released
       for (int s = 0; s < L::kStages; ++s)
-        if (last_issue[s] >= 0) mbar_wait(&full[s], (last_issue[s] / L::kStages) & 1, &dummy);
+        if (last_issue[s] >= 0) mbar_drain(&full[s], (last_issue[s] / L::kStages) & 1);
     }
   } else if (warp == 1) {
     // whole warp runs the loop, one elected lane issues
@@ -760,8 +759,7 @@ __global__ void __launch_bounds__(256, 1)
       mma_commit(&acc_full[buf], leader);
     }
     mma_commit(final_bar, leader);
-    volatile int dummy = 0;
-    mbar_wait(final_bar, 0, &dummy);
+    mbar_drain(final_bar, 0);
   } else if (warp == 3) {
     // work scheduler: claims the CTA's next item from the global counter once every
     // role has read the previous one; -1 when none is left

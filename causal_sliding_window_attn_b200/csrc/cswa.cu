@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "cswa_attn.h"
@@ -74,19 +75,27 @@ constexpr float kLog2e = 1.4426950408889634f;
 inline int tiles128(int T) { return (T + 127) / 128; }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+constexpr int kMaxDevices = 64;
+
+// cudaFuncSetAttribute acts on the current device only, so the dynamic shared-memory
+// limits are raised once per (device, head dim): a process that drives several GPUs
+// sets them on each before its first launch there.
 template <int D>
 bool set_smem_attrs() {
-  // once per process and head dim; cudaFuncSetAttribute is per-function, device-independent here
-  static bool ok = [] {
-    bool r = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  FwdLayout<D>::kBytes) == cudaSuccess;
-    r = r && cudaFuncSetAttribute(attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  BwdLayout<D>::kBytes) == cudaSuccess;
-    r = r && cudaFuncSetAttribute(attn_fwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  FwdLayout<D>::kBytes) == cudaSuccess;
-    return r;
-  }();
-  return ok;
+  static std::atomic<bool> done[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  if (done[dev].load(std::memory_order_acquire)) return true;
+  bool r = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                FwdLayout<D>::kBytes) == cudaSuccess;
+  r = r && cudaFuncSetAttribute(attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                BwdLayout<D>::kBytes) == cudaSuccess;
+  r = r && cudaFuncSetAttribute(attn_fwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                FwdLayout<D>::kBytes) == cudaSuccess;
+  r = r && cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                DqLayout<D>::kBytes) == cudaSuccess;
+  if (r) done[dev].store(true, std::memory_order_release);
+  return r;
 }
 
 template <int D, bool kBwd>
@@ -100,8 +109,11 @@ attn_status_t launch_rope(const RopeParams& p, long long n_pos, cudaStream_t st)
 attn_status_t rope_common(const void* x0, const void* x1, const void* dy0, const void* dy1, void* y0, void* y1,
                           const int32_t* pos, int B, int T, int Hq, int Hkv, int D, float base, float eps,
                           void* stream, bool bwd) {
-  // the prologue treats q and k rows alike: no Hq/Hkv relation is needed here
-  if (B < 1 || T < 1 || (x0 && Hq < 1) || (x1 && Hkv < 1) || (long long)B * T * (Hq + Hkv) >= (1ll << 40) ||
+  // the prologue treats q and k rows alike: no Hq/Hkv relation is needed here. A block's
+  // row index reaches kPosPerBlock * H, which the kernel divides in float: H <= 65535
+  // keeps it exact
+  if (B < 1 || T < 1 || (x0 && (Hq < 1 || Hq > 65535)) || (x1 && (Hkv < 1 || Hkv > 65535)) ||
+      (long long)B * T * (Hq + Hkv) >= (1ll << 40) ||
       !(base > 1.f) || !std::isfinite(base) || !(eps >= 0.f) || !std::isfinite(eps))
     return ATTN_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
@@ -233,13 +245,6 @@ size_t bwd_ws_bytes(int B, int T, int Hq, int window) {
 }
 
 template <int D>
-bool set_dq_attr() {
-  static bool ok = cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        DqLayout<D>::kBytes) == cudaSuccess;
-  return ok;
-}
-
-template <int D>
 attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                          const float* lse, void* dq, void* dk, void* dv, void* ws, int B, int T, int Hq, int Hkv,
                          int window, float scale, cudaStream_t st) {
@@ -250,7 +255,7 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
   if (!encode_bthd(&tq, q, B, T, Hq, D) || !encode_bthd(&tk, k, B, T, Hkv, D) ||
       !encode_bthd(&tv, v, B, T, Hkv, D) || !encode_bthd(&tdo, dO, B, T, Hq, D))
     return ATTN_ERR_LAUNCH;
-  if (!set_smem_attrs<D>() || !set_dq_attr<D>()) return ATTN_ERR_LAUNCH;
+  if (!set_smem_attrs<D>()) return ATTN_ERR_LAUNCH;
   {
     const long long threads = (long long)B * Tpad * Hq * (D / 8);
     attn_bwd_prep_kernel<D><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
@@ -313,7 +318,6 @@ static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
 
 // The device address of g_noalloc_scratch, looked up once per device with that
 // device current (host code only sees a stand-in symbol, never the address).
-constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_addr[kMaxDevices] = {};
 
@@ -486,6 +490,15 @@ attn_status_t attn_get_status(void* stream) {
   if (v & (kStatusTimeout | kStatusLayout)) return ATTN_ERR_TIMEOUT;
   if (v & kStatusBadPosition) return ATTN_ERR_DEVICE;
   return ATTN_OK;
+}
+
+attn_status_t attn_debug_set_wait_limit(unsigned long long ns, void* stream) {
+  const unsigned long long v = ns ? ns : kWaitTimeoutNs;
+  if (v > kWaitTimeoutNs) return ATTN_ERR_INVALID_ARG;
+  // kernels already enqueued on `stream` keep the limit they started with
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return ATTN_ERR_LAUNCH;
+  if (cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)) != cudaSuccess) return ATTN_ERR_LAUNCH;
+  return cudaDeviceSynchronize() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
 const char* attn_status_string(attn_status_t s) {

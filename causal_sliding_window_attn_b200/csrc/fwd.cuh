@@ -234,16 +234,14 @@ __global__ void __launch_bounds__(384, 1)
           tma_load_4d(smem + L::kV0 + st * L::kTile + pn * 16384, mv, &v_full[st], pn * 64, hk, row, b);
         last_v[st] = n;
       }
-      if (*abort_flag) {
-        // never leave with copies in flight: wait (bounded) for the last load of each stage
-        for (int st = 0; st < 2; ++st) {
-          volatile int dummy = 0;
-          if (last_k[st] >= 0) mbar_wait(&k_full[st], (last_k[st] >> 1) & 1, &dummy);
-          if (last_v[st] >= 0) mbar_wait(&v_full[st], (last_v[st] >> 1) & 1, &dummy);
-        }
-        volatile int dummy = 0;
-        mbar_wait(q_full, 0, &dummy);
+      // never leave with copies in flight: wait (bounded) for the last load of each
+      // stage. After a normal run they were all consumed and these return at once; after
+      // an abort (raised by any role, before or after this loop ended) they may not be.
+      for (int st = 0; st < 2; ++st) {
+        if (last_k[st] >= 0) mbar_drain(&k_full[st], (last_k[st] >> 1) & 1);
+        if (last_v[st] >= 0) mbar_drain(&v_full[st], (last_v[st] >> 1) & 1);
       }
+      mbar_drain(q_full, 0);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -314,8 +312,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     // every MMA issued above has finished before TMEM is released
     mma_commit(final_bar, leader);
-    volatile int dummy = 0;
-    mbar_wait(final_bar, 0, &dummy);
+    mbar_drain(final_bar, 0);
   } else if (warp == 2 || warp == 3) {
     // ------------------------------------------------------------ cache append (prefill)
     // Warps 2 and 3 of the group's first query head copy the chunk rows of the CTA's

@@ -9,11 +9,15 @@ namespace cswa {
 
 // ---------------------------------------------------------------- status word
 // One word per device, OR-ed with error bits by kernels; read (and cleared) by
-// attn_get_status(). Waits never spin forever: after kWaitTimeoutNs they set
-// kStatusTimeout, raise the CTA's abort flag and fall through.
+// attn_get_status(). Waits never spin forever: a pipeline wait gives up after
+// g_wait_limit_ns (kWaitTimeoutNs unless a test shortened it through
+// attn_debug_set_wait_limit), sets kStatusTimeout, raises the CTA's abort flag
+// and falls through. Drain waits (a CTA letting its own copies and MMAs land
+// before it exits) always keep kWaitTimeoutNs and ignore the abort flag.
 enum : unsigned { kStatusTimeout = 1u, kStatusBadPosition = 2u, kStatusLayout = 4u };
 __device__ unsigned int g_status;
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
+__device__ unsigned long long g_wait_limit_ns = kWaitTimeoutNs;
 
 // Pipeline trace marks: compiled out unless CSWA_TRACE is defined (profiling
 // builds record clock64() per (CTA, role, step, tag) for the first CTAs).
@@ -90,17 +94,35 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 }
 
 // Wait for the phase of `bar` with parity `parity` to complete. Bounded: gives
-// up (and raises *abort) after kWaitTimeoutNs, or at once when *abort is set
+// up (and raises *abort) after g_wait_limit_ns, or at once when *abort is set
 // by another thread of the CTA. Returns false when it gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   const uint32_t b = smem_u32(bar);
   if (mbar_try_wait(b, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
+  const unsigned long long limit = *static_cast<volatile unsigned long long*>(&g_wait_limit_ns);
+  for (;;) {
     if (mbar_try_wait_sleep(b, parity)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+    if (globaltimer_ns() - t0 > limit) {
       *abort = 1;
+      atomicOr(&g_status, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
+// Drain wait before a CTA exits: the phase of `bar` is an operation this thread
+// issued itself (a TMA copy, or an MMA commit), which completes on its own. The
+// limit is always kWaitTimeoutNs, whatever a test set for the pipeline waits,
+// and the CTA's abort flag does not cut it short. Returns false on time-out.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint32_t b = smem_u32(bar);
+  if (mbar_try_wait(b, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (;;) {
+    if (mbar_try_wait_sleep(b, parity)) return true;
+    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
       atomicOr(&g_status, kStatusTimeout);
       return false;
     }

@@ -221,6 +221,24 @@ attn_status_t attn_kv_replicate(const void* k_src, const void* v_src, void* k_ds
  * ATTN_ERR_LAUNCH if a CUDA error is pending). */
 attn_status_t attn_get_status(void* stream);
 
+/*
+ * attn_debug_set_wait_limit -- test hook for the failure-detection path.
+ * Every wait inside the kernels is bounded: a wait on a pipeline stage (a tile
+ * copy, a tensor-core product, another warp's results) that has not completed
+ * after the limit gives up, records ATTN_ERR_TIMEOUT in the status word and
+ * makes its CTA wind down: every other wait of the CTA falls through, the CTA
+ * still waits for the copies and products it issued itself (those waits keep
+ * the default limit), frees its tensor memory and exits, leaving the outputs
+ * of that call undefined. This call sets the pipeline-wait limit, in
+ * nanoseconds, for launches made after it on the current device; 0 restores
+ * the default (2 s, also the maximum: a longer limit is ATTN_ERR_INVALID_ARG).
+ * A limit of a few nanoseconds makes ordinary waits run out, so a test can
+ * check that the status is reported and that the next call with the default
+ * limit is correct. It synchronises `stream` first and the device after, and
+ * is meant for tests only: the default is the right limit for real work.
+ */
+attn_status_t attn_debug_set_wait_limit(unsigned long long ns, void* stream);
+
 /* Static description of a status code. */
 const char* attn_status_string(attn_status_t status);
 

@@ -17,6 +17,7 @@ from .attention import (  # noqa: F401
     row_positions,
     prologue,
     prologue_bwd,
+    round_bf16,
     visible,
     attention_fwd,
     attention_bwd,

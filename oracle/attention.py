@@ -23,7 +23,7 @@ Sources (page title, section):
         12*H*Q*T FLOPs per token, i.e. forward 4*D per visible pair and
         backward twice that.
 
-Readings where the pages are silent or disagree (all repeated in the design doc):
+Readings where the pages are silent or disagree:
   * RoPE pairs dimension j with j + D/2 ("half split") and rotates by +phi,
     phi = p * base**(-2j/D). The base is an argument (10000 in every config;
     [AG3] prints 100000 for nanochat itself).
@@ -106,6 +106,20 @@ def rope_transpose(y, positions, base):
 def prologue(x, positions, base, eps):
     """RoPE(RMSNorm(x)): the fused prologue applied to q and to k [AG3]."""
     return rope(rms_norm(x, eps), positions, base)
+
+
+def round_bf16(x):
+    """Round to the nearest bfloat16 value, ties to even.
+
+    The pages keep the model's activations in bf16 ([AG6]: FA3 and its fallback
+    run in bf16), so the prologue's outputs reach the attention as bf16 values.
+    A bf16 number has 8 significant bits: with x = m * 2**e and 0.5 <= |m| < 1,
+    the rounded value is round_half_even(m * 2**8) * 2**(e - 8). Only the normal
+    range is handled (no value here is below 2**-126 in magnitude or overflows).
+    """
+    x = _f64(x)
+    m, e = np.frexp(x)
+    return np.ldexp(np.round(m * 256.0) / 256.0, e)
 
 
 def prologue_bwd(x, dy, positions, base, eps):

@@ -4,6 +4,9 @@ Tolerances (outputs: max-abs 1e-2 and relative L2 5e-3; gradients dQ/dK/dV:
 relative L2 1e-2) are the acceptance bar for the attention block; lse gets
 1e-3 absolute.
 """
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -11,17 +14,40 @@ OUT_MAX_ABS = 1e-2
 OUT_REL_L2 = 5e-3
 GRAD_REL_L2 = 1e-2
 LSE_MAX_ABS = 1e-3
-# End-to-end (raw inputs -> o) also carries the bf16 storage of q_hat and k_hat
-# between the prologue and the attention kernel: a relative perturbation of
-# up to 2^-9 per element moves each score by ~ scale * sqrt(D) * 2^-9, and o by
-# that times |v - o|, which reaches ~1e-2 on rows with few visible keys. Its
-# max-abs bar is therefore 2e-2; its relative L2 bar stays 5e-3.
+# Three parity levels for the attention output:
+#   kernel-only   oracle attention on the GPU's own bf16 q_hat, k_hat: the bar above.
+#   e2e-bf16      oracle prologue in fp64, its q_hat, k_hat rounded to bf16 (the pages keep
+#                 activations in bf16), oracle attention in fp64: the bar above.
+#   e2e-fp64      oracle prologue and attention in fp64 with no bf16 step. This also
+#                 measures the bf16 storage of q_hat, k_hat: a relative perturbation of up to
+#                 2^-9 per element moves each score by ~ scale * sqrt(D) * 2^-9, and o by that
+#                 times |v - o|, which reaches ~1e-2 on rows with few visible keys. Any bf16
+#                 tensor-core path carries it. Its max-abs bar is 2e-2, a departure from the
+#                 1e-2 output bar; its relative L2 bar stays 5e-3.
 E2E_MAX_ABS = 2e-2
 # bf16 outputs of elementwise kernels: round-to-nearest gives at most half an
 # ulp, i.e. 2^-9 relative; 2^-8 leaves room for the fp32 arithmetic before it.
 BF16_REL = 2.0 ** -8
 ROPE_BASE = 10000.0
 EPS = 1e-6
+
+
+# Measured errors, printed in pytest's terminal summary (and written as JSON to
+# $CSWA_PARITY_LOG when that is set) so that every run reports what it saw.
+RECORDS = []
+
+
+def record(test, level, **values):
+    RECORDS.append(dict(test=test, level=level, **{k: (round(float(v), 6) if isinstance(v, float) else v)
+                                                   for k, v in values.items()}))
+
+
+def dump_records():
+    path = os.environ.get("CSWA_PARITY_LOG")
+    if path and RECORDS:
+        os.makedirs(os.path.dirname(os.path.abspath(path)), exist_ok=True)
+        with open(path, "w") as f:
+            json.dump(RECORDS, f, indent=1)
 
 
 def f64(t):

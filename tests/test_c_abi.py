@@ -104,6 +104,11 @@ def test_rope_rejects_bad_args(L):
     assert L.attn_rope_qknorm(P, None, P, None, None, 1, 4, 2, 2, 128, f(1e4), f(-1.0), None) == INVALID
     assert L.attn_rope_qknorm(P, None, MIS, None, None, 1, 4, 2, 2, 128, f(1e4), f(1e-6), None) == INVALID
     assert L.attn_rope_qknorm(P, P, P, P, None, 1, 4, 2, 2, 32, f(1e4), f(1e-6), None) == UNSUPPORTED
+    # head counts above 65535 (the kernel's per-block row index must stay exact in float)
+    assert L.attn_rope_qknorm(P, None, P, None, None, 1, 4, 131072, 1, 128, f(1e4), f(1e-6), None) == INVALID
+    assert L.attn_rope_qknorm(None, P, None, P, None, 1, 4, 1, 65536, 128, f(1e4), f(1e-6), None) == INVALID
+    assert L.attn_rope_qknorm_bwd(P, None, P, None, P, None, None, 1, 4, 70000, 1, 128, f(1e4), f(1e-6),
+                                  None) == INVALID
 
 
 def test_decode_rejects_bad_args(L):
@@ -194,3 +199,8 @@ def test_size_limits_rejected_before_launch(L):
     assert L.attn_fwd(P, P, P, P, P, 1, 0, 1, 1, 128, -1, f, None) == INVALID
     assert L.attn_prefill(P, P, P, None, None, P, P, P, 1, 0, 32, 1, 1, 128, -1, f, None) == INVALID
     assert L.attn_decode(P, P, P, None, None, P, P, P, 0, 64, 1, 1, 128, -1, f, P, 1 << 20, None) == INVALID
+
+
+def test_wait_limit_hook_rejects_limits_above_the_default(L):
+    # checked before anything touches the device
+    assert L.attn_debug_set_wait_limit(3_000_000_000, None) == INVALID

@@ -13,8 +13,8 @@ import torch
 
 import oracle
 import workloads
-from tests.parity import (EPS, LSE_MAX_ABS, ROPE_BASE, check_bf16, check_grad, check_out, f64, max_abs,
-                          run_block)
+from tests.parity import (E2E_MAX_ABS, EPS, LSE_MAX_ABS, ROPE_BASE, check_bf16, check_grad, check_out, f64,
+                          max_abs, record, run_block)
 
 pytestmark = pytest.mark.gpu
 
@@ -47,9 +47,23 @@ def test_fullsize_sampled(cswa, name, W):
     vf, dof = f64(v), f64(do)
 
     rows = sample_rows(T, W, seed=T + W)
+    o_gpu = f64(g["o"])[:, rows]
     o_ref, lse_ref = oracle.attention_fwd(qh, kh, vf, W, scale, rows=rows)
-    check_out(f"{name} o rows", f64(g["o"])[:, rows], o_ref)
+    ma, rl = check_out(f"{name} o rows", o_gpu, o_ref)
+    tid = f"fullsize {name} W={W} ({len(rows)} rows x B x Hq)"
+    record(tid, "kernel-only", max_abs=ma, rel_l2=rl, max_abs_o=float(np.max(np.abs(o_ref))))
     assert max_abs(f64(g["lse"])[:, :, rows], lse_ref) <= LSE_MAX_ABS
+
+    # end to end on the same rows: the oracle's own prologue of the raw q, k
+    pos_all = oracle.row_positions(B, T)
+    qh_e, kh_e = oracle.prologue(f64(q), pos_all, ROPE_BASE, EPS), oracle.prologue(f64(k), pos_all, ROPE_BASE, EPS)
+    o_b16, _ = oracle.attention_fwd(oracle.round_bf16(qh_e), oracle.round_bf16(kh_e), vf, W, scale, rows=rows)
+    ma, rl = check_out(f"{name} o rows (end-to-end, bf16 q_hat/k_hat)", o_gpu, o_b16)
+    record(tid, "e2e-bf16", max_abs=ma, rel_l2=rl, max_abs_o=float(np.max(np.abs(o_b16))))
+    o_e2e, _ = oracle.attention_fwd(qh_e, kh_e, vf, W, scale, rows=rows)
+    ma, rl = check_out(f"{name} o rows (end-to-end)", o_gpu, o_e2e, max_abs_tol=E2E_MAX_ABS)
+    record(tid, "e2e-fp64", max_abs=ma, rel_l2=rl, max_abs_o=float(np.max(np.abs(o_e2e))))
+    del qh_e, kh_e
 
     bs = [0, B - 1] if B > 1 else [0]
     dq_ref = oracle.attention_bwd_rows(qh[bs], kh[bs], vf[bs], dof[bs], W, scale, rows)
@@ -86,7 +100,8 @@ def test_fullsize_decode(cswa):
     assert cswa.attn_get_status() == 0
     o_ref, lse_ref, _, _ = oracle.decode(f64(qd), f64(kc0), f64(vc0), lengths.numpy(), W,
                                          workloads.default_scale(D), k_new=f64(kn), v_new=f64(vn))
-    check_out("decode o", f64(o), o_ref)
+    ma, rl = check_out("decode o", f64(o), o_ref)
+    record("fullsize decode", "kernel-only", max_abs=ma, rel_l2=rl, max_abs_o=float(np.max(np.abs(o_ref))))
     assert max_abs(f64(lse), lse_ref) <= LSE_MAX_ABS
     # end-to-end: the oracle's own prologue of the raw cache and query
     L = lengths.numpy()
@@ -95,7 +110,13 @@ def test_fullsize_decode(cswa):
     kn_e2e = oracle.prologue(f64(knraw), oracle.row_positions(B, 1, L), ROPE_BASE, EPS)
     o_e2e, _, _, _ = oracle.decode(q_e2e, kc_e2e, f64(vc0), L, W, workloads.default_scale(D), k_new=kn_e2e,
                                    v_new=f64(vn))
-    check_out("decode o (end-to-end)", f64(o), o_e2e, max_abs_tol=2e-2)
+    ma, rl = check_out("decode o (end-to-end)", f64(o), o_e2e, max_abs_tol=E2E_MAX_ABS)
+    record("fullsize decode", "e2e-fp64", max_abs=ma, rel_l2=rl, max_abs_o=float(np.max(np.abs(o_e2e))))
+    r16 = oracle.round_bf16
+    o_b16, _, _, _ = oracle.decode(r16(q_e2e), r16(kc_e2e), f64(vc0), L, W, workloads.default_scale(D),
+                                   k_new=r16(kn_e2e), v_new=f64(vn))
+    ma, rl = check_out("decode o (end-to-end, bf16 q_hat/k_hat)", f64(o), o_b16)
+    record("fullsize decode", "e2e-bf16", max_abs=ma, rel_l2=rl, max_abs_o=float(np.max(np.abs(o_b16))))
 
 
 def test_fullsize_prefill(cswa):

@@ -13,6 +13,8 @@
     and a one-token chunk equals a decode step
   * the per-layer window rule on hand-computed cases; a replicated batch-1 cache
     decodes every sample exactly as the batch-1 cache does
+  * bf16 rounding: hand-computed ties and near-ties, and torch's own float32 ->
+    bfloat16 conversion on random float32 values
 The last test plants plausible mistakes in the oracle and shows a pin fails.
 """
 import json
@@ -445,6 +447,32 @@ def test_visible_pair_count():
         assert workloads.visible_pairs(T, W) == oracle.useful_pairs(T, W)
 
 
+def check_round_bf16_hand():
+    """Hand-computed bf16 roundings. Near 1 the bf16 spacing is 2**-7, so 1 + 2**-8 is a
+    tie (to the even neighbour 1), 1 + 3 * 2**-8 a tie (to 1 + 2**-6, whose last
+    mantissa bit is 0), and 1 + 2**-8 + 2**-20 just above a tie (up to 1 + 2**-7)."""
+    cases = [(1 + 2.0 ** -8, 1.0), (1 + 3 * 2.0 ** -8, 1 + 2.0 ** -6), (1 + 2.0 ** -8 + 2.0 ** -20, 1 + 2.0 ** -7),
+             (-(1 + 2.0 ** -8 + 2.0 ** -20), -(1 + 2.0 ** -7)), (3.0, 3.0), (0.1, 0.10009765625),
+             (255.5, 256.0), (2.0 ** -100 * 1.00390625, 2.0 ** -100), (0.0, 0.0)]
+    x = np.array([c[0] for c in cases])
+    allclose(oracle.round_bf16(x), [c[1] for c in cases], 0.0)
+
+
+def check_round_bf16_torch():
+    """On float32 inputs a single round-to-nearest-even to bf16 is what torch's
+    float32 -> bfloat16 conversion does: both must agree bit for bit."""
+    x = torch.from_numpy(rnd(100000, 31) * np.exp(rnd(100000, 32) * 4)).to(torch.float32)
+    ref = x.to(torch.bfloat16).to(torch.float64).numpy()
+    allclose(oracle.round_bf16(x.to(torch.float64).numpy()), ref, 0.0)
+
+
+def test_round_bf16():
+    check_round_bf16_hand()
+    check_round_bf16_torch()
+    y = oracle.round_bf16(rnd(1000, 33))
+    allclose(oracle.round_bf16(y), y, 0.0)  # idempotent
+
+
 # ---------------------------------------------------------------- planted mistakes
 def _rope_wrong_sign(x, positions, base):
     return oa.rope_transpose(x, positions, base)
@@ -499,6 +527,18 @@ def test_pins_catch_planted_mistakes(monkeypatch, name, attr, bad, check):
     monkeypatch.setattr(oracle, attr, bad, raising=False)
     with pytest.raises(AssertionError):
         check()
+
+
+def test_pins_catch_truncating_bf16_rounding(monkeypatch):
+    """Rounding toward zero instead of to nearest must fail the hand-computed cases."""
+    def truncate(x):
+        m, e = np.frexp(np.asarray(x, np.float64))
+        return np.ldexp(np.trunc(m * 256.0) / 256.0, e)
+    monkeypatch.setattr(oracle, "round_bf16", truncate)
+    with pytest.raises(AssertionError):
+        check_round_bf16_hand()
+    with pytest.raises(AssertionError):
+        check_round_bf16_torch()
 
 
 def test_pins_catch_prefill_ignoring_the_cache(monkeypatch):
