@@ -5,7 +5,8 @@
 One step is the whole hot path on one batch: for each layer of the nanochat-d20
 shaped pair (B=8, T=2048, Hq=Hkv=10, D=128; a short layer with window 1024 and
 a long layer with window 2048 = full causal) it runs the RoPE + QK-norm
-prologue, attention forward, attention backward and the prologue backward.
+prologue, attention forward, and the block backward (attention backward with the
+prologue backward fused into its kernels: gradients w.r.t. the raw q, k, v).
 `value` is useful fwd+bwd TFLOP/s: 12*D per visible (query, key) pair (the
 pages' 3 x forward convention), masked work and recompute not counted. The
 KV-cache decode workload (32 sequences, lengths U[512, 2048], window 1024) is
@@ -40,6 +41,7 @@ METRIC = "attention fwd+bwd TFLOP/s (useful FLOPs) & % bf16 peak; decode HBM GB/
 WORKLOAD = ("nanochat-d20 attention layer pair, fwd+bwd incl. RoPE+QK-norm prologue: B=8 T=2048 Hq=Hkv=10 "
             "D=128 bf16, windows 1024 (short layer) and 2048 (long layer)")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SUSTAINED_REGION_MS = 3000.0
 
 
 def peaks():
@@ -102,28 +104,62 @@ def decode_bytes(lengths, Hq, Hkv, D, W):
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons every 200 ms while running."""
+    """Samples the SM clock and the clock-event (throttle) reasons while running: through
+    NVML every 5 ms when the binding is present (short timed regions still get several
+    samples), else through nvidia-smi every 200 ms."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, index):
         self.index = index
-        self.rows = []
+        self.rows = []  # (sm_mhz, max_mhz, [reason names])
+        self.source = None
         self._stop = threading.Event()
         self._t = None
 
-    def _run(self):
+    def _nvml_handle(self, pynvml):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.index).uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.index)
+
+    def _run_nvml(self):
+        import pynvml
+        pynvml.nvmlInit()
+        h = self._nvml_handle(pynvml)
+        bits = [pynvml.nvmlClocksEventReasonHwSlowdown, pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                pynvml.nvmlClocksEventReasonSwThermalSlowdown, pynvml.nvmlClocksEventReasonSwPowerCap]
+        mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        self.source = "nvml, 5 ms"
+        while not self._stop.is_set():
+            sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+            r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+            self.rows.append((float(sm), float(mx), [n for n, b in zip(self.NAMES, bits) if r & b]))
+            self._stop.wait(0.005)
+
+    def _run_smi(self):
+        self.source = "nvidia-smi, 200 ms"
         while not self._stop.is_set():
             try:
                 out = subprocess.run(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
                                       "--format=csv,noheader,nounits"], capture_output=True, text=True,
                                      timeout=5).stdout.strip()
-                if out:
-                    self.rows.append([x.strip() for x in out.split(",")])
+                r = [x.strip() for x in out.split(",")]
+                if len(r) >= 9 and r[1].replace(".", "").isdigit():
+                    self.rows.append((float(r[1]), float(r[2]),
+                                      [n for i, n in enumerate(self.NAMES) if r[5 + i] == "Active"]))
             except Exception:
                 pass
             self._stop.wait(0.2)
+
+    def _run(self):
+        try:
+            self._run_nvml()
+        except Exception:
+            self._run_smi()
 
     def __enter__(self):
         self._t = threading.Thread(target=self._run, daemon=True)
@@ -136,13 +172,10 @@ class ClockSampler:
 
     def summary(self):
         if not self.rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
-        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in self.rows for i in range(4) if len(r) > 5 + i and r[5 + i] == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(self.rows)}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock samples"], "samples": 0}
+        return {"sm_mhz": statistics.median(r[0] for r in self.rows), "sm_max_mhz": max(r[1] for r in self.rows),
+                "reasons": sorted({n for r in self.rows for n in r[2]}), "samples": len(self.rows),
+                "source": self.source}
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -183,17 +216,18 @@ def run_gpu(args, rank, world, local):
     for W in windows:
         L.append(dict(W=W, qh=torch.empty_like(q), kh=torch.empty_like(k), o=torch.empty_like(q),
                       lse=torch.empty((B, Hq, T), device=dev, dtype=torch.float32),
-                      dqh=torch.empty_like(q), dkh=torch.empty_like(k), dv=torch.empty_like(v),
-                      dq=torch.empty_like(q), dk=torch.empty_like(k),
-                      ws=torch.empty(cswa.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, W), device=dev,
+                      dv=torch.empty_like(v), dq=torch.empty_like(q), dk=torch.empty_like(k),
+                      ws=torch.empty(cswa.attn_block_bwd_workspace_bytes(B, T, Hq, Hkv, D, W), device=dev,
                                      dtype=torch.uint8)))
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    per_op = {"prologue": 0.0, "fwd": 0.0, "bwd": 0.0, "prologue_bwd": 0.0}
+    per_op = {"prologue": 0.0, "fwd": 0.0, "bwd": 0.0}
     bwd_ms = [0.0, 0.0]
 
     def step(record):
+        # per layer: the prologue (q, k -> q_hat, k_hat), the forward, and the block backward
+        # (gradients w.r.t. the raw q, k: the prologue backward runs inside its kernels)
         for li, l in enumerate(L):
-            e = [ev() for _ in range(5)] if record else None
+            e = [ev() for _ in range(4)] if record else None
             if record:
                 e[0].record()
             cswa.attn_rope_qknorm(q, k, l["qh"], l["kh"])
@@ -202,13 +236,10 @@ def run_gpu(args, rank, world, local):
             cswa.attn_fwd(l["qh"], l["kh"], v, l["W"], scale, o=l["o"], lse=l["lse"])
             if record:
                 e[2].record()
-            cswa.attn_bwd(l["qh"], l["kh"], v, l["o"], do, l["lse"], l["W"], scale, dq=l["dqh"], dk=l["dkh"],
-                          dv=l["dv"], workspace=l["ws"])
+            cswa.attn_block_bwd(q, k, l["qh"], l["kh"], v, l["o"], do, l["lse"], l["W"], scale, dq=l["dq"],
+                                dk=l["dk"], dv=l["dv"], workspace=l["ws"])
             if record:
                 e[3].record()
-            cswa.attn_rope_qknorm_bwd(q, k, l["dqh"], l["dkh"], l["dq"], l["dk"])
-            if record:
-                e[4].record()
                 l["events"] = l.get("events", []) + [e]
 
     for _ in range(args.warmup):
@@ -233,7 +264,6 @@ def run_gpu(args, rank, world, local):
             per_op["prologue"] += e[0].elapsed_time(e[1])
             per_op["fwd"] += e[1].elapsed_time(e[2])
             bwd_ms[li] += e[2].elapsed_time(e[3])
-            per_op["prologue_bwd"] += e[3].elapsed_time(e[4])
     per_op["bwd"] = sum(bwd_ms)
     status = cswa.attn_get_status()
     assert status == 0, f"device status {status}"
@@ -246,10 +276,17 @@ def run_gpu(args, rank, world, local):
     pk, pk_src = peaks()
     peak_sus = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     peak_burst = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    # A timed region of a few seconds or more runs into the power cap: the sustained
+    # peak applies. A shorter one is a burst: the burst peak applies.
+    long_region = ms_total >= SUSTAINED_REGION_MS
+    peak_use = peak_sus if long_region else peak_burst
+    peak_kind = (f"bf16 {'sustained' if long_region else 'burst'} ({pk_src}): timed region "
+                 f"{ms_total / 1e3:.2f} s {'>=' if long_region else '<'} {SUSTAINED_REGION_MS / 1e3:.0f} s; "
+                 f"burst {peak_burst}, sustained {peak_sus}")
     bwd_avg_ms = per_op["bwd"] / (2 * args.steps)
     bwd_tflops = flops_b / 2 / (bwd_avg_ms * 1e-3) / 1e12
     fwd_avg_ms = per_op["fwd"] / (2 * args.steps)
-    # DRAM bytes of one attn_bwd call = its three launches (ncu, window-1024 layer)
+    # DRAM bytes of one attn_block_bwd call = its three launches (ncu, window-1024 layer)
     parts = [ncu_traffic(kn) for kn in ("attn_bwd_prep_kernel", "attn_bwd_kernel", "attn_bwd_dq_kernel")]
     traffic = sum(parts) if all(x is not None for x in parts) else None
     result = {
@@ -259,22 +296,34 @@ def run_gpu(args, rank, world, local):
         "config": {"workload": WORKLOAD, "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world}",
                    "l2": "no flush: each layer's inputs (q,k,v,dO: 168 MB) exceed the 126 MB L2"},
         "pct_bf16_peak": {"of_sustained": round(value / world / peak_sus, 4),
-                          "of_burst": round(value / world / peak_burst, 4), "peaks": pk_src},
+                          "of_burst": round(value / world / peak_burst, 4), "peaks": pk_src,
+                          "applies": "sustained" if long_region else "burst"},
         "breakdown_ms_per_step": {k2: round(v2 / args.steps, 4) for k2, v2 in per_op.items()},
         "fwd_tflops": round(flops_f / 2 / (fwd_avg_ms * 1e-3) / 1e12, 1),
         "bwd_tflops": round(bwd_tflops, 1),
         "bwd_tflops_fa_convention": round(bwd_tflops * 10 / 8, 1),
-        "roofline": {"kernel": "attn_bwd call (prep + main + dQ launches), both layers", "bound": "tensor",
-                     "achieved": round(bwd_tflops, 1), "peak": peak_sus, "unit": "TFLOP/s",
-                     "frac": round(bwd_tflops / peak_sus, 4),
-                     "peak_kind": f"bf16 sustained ({pk_src}); burst {peak_burst}",
+        "roofline": {"kernel": "attn_block_bwd call (prep + main + dq launches, prologue backward fused), "
+                               "both layers", "bound": "tensor",
+                     "achieved": round(bwd_tflops, 1), "peak": peak_use, "unit": "TFLOP/s",
+                     "frac": round(bwd_tflops / peak_use, 4),
+                     "peak_kind": peak_kind,
                      "traffic": traffic,
-                     "traffic_note": "ncu dram read+write bytes of one attn_bwd call (prep + main + dQ), "
+                     "traffic_note": "ncu dram read+write bytes of one attn_block_bwd call (prep + main + dq), "
                                      "window-1024 layer; null when the kernel sources changed since the capture",
                      "algorithmic_flops_per_launch": flops_b / 2},
-        "gpu_launches": 12 * args.steps,  # per layer: prologue, fwd, bwd prep/main/dq, prologue bwd
+        "gpu_launches": 10 * args.steps,  # per layer: prologue, fwd, bwd prep / main / dq
         "clocks": clocks.summary(),
     }
+    if not args.no_configs:
+        cfg_steps = max(3, args.steps // 4)
+        result["gqa"] = run_config(cswa, dev, "gqa", cfg_steps, world, rank, peak_use)
+        lc = run_config(cswa, dev, "long", cfg_steps, world, rank, peak_use)
+        pw, pf = (workloads.visible_pairs(8192, W) for W in (2048, -1))
+        lc["window_vs_full"] = {
+            "useful_flop_ratio": round(pw / pf, 4),
+            "time_ratio": round(lc["layers"]["2048"]["fwd_bwd_ms"] / lc["layers"]["-1"]["fwd_bwd_ms"], 4),
+            "note": "window 2048 over full causal on identical inputs: useful FLOPs and measured fwd+bwd time"}
+        result["long"] = lc
     if rank == 0 and not args.no_decode:
         result["decode"] = run_decode(cswa, dev, args, pk, pk_src)
         result["prefill"] = run_prefill(cswa, dev, args, pk, pk_src)
@@ -282,6 +331,48 @@ def run_gpu(args, rank, world, local):
     if not args.no_e2e:
         result["e2e"] = run_e2e(cswa, dev, args, q, k, v, do, L, scale, world, flops_f + flops_b)
     return result
+
+
+def run_config(cswa, dev, name, steps, world, rank, peak):
+    """fwd and bwd of each layer of a training config (the GQA layer, or the long-context
+    layers at window 2048 and full causal), timed with CUDA events over `steps` repetitions
+    after 3 warm-ups; useful TFLOP/s per layer. Inputs exceed L2."""
+    c = workloads.CONFIGS[name]
+    B, T, Hq, Hkv, D = c["B"], c["T"], c["Hq"], c["Hkv"], c["D"]
+    scale = workloads.default_scale(D)
+    q, k, v, do = (t.to(dev) for t in workloads.training_inputs(B, T, Hq, Hkv, D, shard_seed(c["seed"], rank)))
+    qh, kh = cswa.attn_rope_qknorm(q, k)
+    out = {"workload": f"{name}: B={B} T={T} Hq={Hq} Hkv={Hkv} D={D} bf16, fwd+bwd per layer (attention kernels; "
+                       f"prologue excluded)", "steps": steps, "layers": {}}
+    for W in c["windows"]:
+        o = torch.empty_like(qh)
+        lse = torch.empty((B, Hq, T), device=dev, dtype=torch.float32)
+        dq, dk, dv = torch.empty_like(qh), torch.empty_like(kh), torch.empty_like(v)
+        ws = torch.empty(cswa.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, W), device=dev, dtype=torch.uint8)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for i in range(3 + steps):
+            e = ev[i - 3] if i >= 3 else None
+            if e:
+                e[0].record()
+            cswa.attn_fwd(qh, kh, v, W, scale, o=o, lse=lse)
+            if e:
+                e[1].record()
+            cswa.attn_bwd(qh, kh, v, o, do, lse, W, scale, dq=dq, dk=dk, dv=dv, workspace=ws)
+            if e:
+                e[2].record()
+        torch.cuda.synchronize()
+        assert cswa.attn_get_status() == 0
+        f_ms = max_over_ranks(statistics.median(e[0].elapsed_time(e[1]) for e in ev), world)
+        b_ms = max_over_ranks(statistics.median(e[1].elapsed_time(e[2]) for e in ev), world)
+        ff, fb = layer_useful_flops(B, T, Hq, D, W)
+        out["layers"][str(W)] = {
+            "window": W, "fwd_ms": round(f_ms, 4), "bwd_ms": round(b_ms, 4), "fwd_bwd_ms": round(f_ms + b_ms, 4),
+            "fwd_tflops": round(world * ff / (f_ms * 1e-3) / 1e12, 1),
+            "bwd_tflops": round(world * fb / (b_ms * 1e-3) / 1e12, 1),
+            "fwd_bwd_tflops": round(world * (ff + fb) / ((f_ms + b_ms) * 1e-3) / 1e12, 1),
+            "frac_of_peak": round((ff + fb) / ((f_ms + b_ms) * 1e-3) / 1e12 / peak, 4)}
+        del o, lse, dq, dk, dv, ws
+    return out
 
 
 def run_decode(cswa, dev, args, pk, pk_src):
@@ -316,8 +407,9 @@ def run_decode(cswa, dev, args, pk, pk_src):
                         "Tmax=2176, window 1024, append of the new k/v",
             "us_per_step": round(ms * 1e3, 2), "us_p10": round(np.percentile(times, 10) * 1e3, 2),
             "us_p90": round(np.percentile(times, 90) * 1e3, 2), "value": round(gbs, 1), "unit": "GB/s",
-            "l2": "flushed (256 MB write) before every call", "gpu_launches_per_step": 2,
-            "roofline": {"kernel": "attn_decode (chunk + combine)", "bound": "hbm", "achieved": round(gbs, 1),
+            "l2": "flushed (256 MB write) before every call", "gpu_launches_per_step": 1,
+            "roofline": {"kernel": "attn_decode (one launch: chunks, merge by the last chunk CTA)", "bound": "hbm",
+                         "achieved": round(gbs, 1),
                          "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
                          "traffic": ncu_traffic("decode_chunk_kernel"), "algorithmic_bytes": nbytes,
                          "peak_kind": pk_src}}
@@ -420,9 +512,8 @@ def run_e2e(cswa, dev, args, q, k, v, do, L, scale, world, flops):
         for l in L:
             cswa.attn_rope_qknorm(q, k, l["qh"], l["kh"])
             cswa.attn_fwd(l["qh"], l["kh"], v, l["W"], scale, o=l["o"], lse=l["lse"])
-            cswa.attn_bwd(l["qh"], l["kh"], v, l["o"], do, l["lse"], l["W"], scale, dq=l["dqh"], dk=l["dkh"],
-                          dv=l["dv"], workspace=l["ws"])
-            cswa.attn_rope_qknorm_bwd(q, k, l["dqh"], l["dkh"], l["dq"], l["dk"])
+            cswa.attn_block_bwd(q, k, l["qh"], l["kh"], v, l["o"], do, l["lse"], l["W"], scale, dq=l["dq"],
+                                dk=l["dk"], dv=l["dv"], workspace=l["ws"])
         for lst in outs:
             for d, h in lst:
                 h.copy_(d, non_blocking=True)
@@ -447,65 +538,90 @@ def run_e2e(cswa, dev, args, q, k, v, do, L, scale, world, flops):
 
 
 # ------------------------------------------------------------------ CPU (oracle) arm
+REF_UNIT = ("one (sequence, head) unit of the d20 layer pair: the B=1, Hq=Hkv=1 slice (T=2048, D=128) of one "
+            "sequence and head, both windows (1024 and 2048), prologue + fwd + bwd + prologue bwd")
+
+
+class OracleUnits:
+    """The fp64 oracle on (sequence, head) units of the d20 layer pair: per unit, the
+    prologue, forward, backward and prologue backward of one head of one sequence, for
+    both layers. Units cycle through the heads of sequence 0."""
+
+    def __init__(self, seed_offset=0):
+        import oracle
+        self.oracle = oracle
+        c = workloads.CONFIGS["d20"]
+        self.c = c
+        self.scale = workloads.default_scale(c["D"])
+        self.q, self.k, self.v, self.do = workloads.training_inputs(1, c["T"], c["Hq"], c["Hkv"], c["D"],
+                                                                    c["seed"] + seed_offset)
+        self.pos = oracle.row_positions(1, c["T"])
+        self.n = 0
+
+    def run_one(self):
+        """Runs the next unit; returns its useful FLOPs (12 D per visible pair, both layers)."""
+        o, c = self.oracle, self.c
+        hs = slice(self.n % c["Hq"], self.n % c["Hq"] + 1)
+        self.n += 1
+        qf, kf, vf, dof = (t[:, :, hs].float().numpy().astype(np.float64) for t in (self.q, self.k, self.v, self.do))
+        flops = 0.0
+        for W in c["windows"]:
+            qh = o.prologue(qf, self.pos, workloads.ROPE_BASE, workloads.EPS)
+            kh = o.prologue(kf, self.pos, workloads.ROPE_BASE, workloads.EPS)
+            o.attention_fwd(qh, kh, vf, W, self.scale)
+            dqh, dkh, _ = o.attention_bwd(qh, kh, vf, dof, W, self.scale)
+            o.prologue_bwd(qf, dqh, self.pos, workloads.ROPE_BASE, workloads.EPS)
+            o.prologue_bwd(kf, dkh, self.pos, workloads.ROPE_BASE, workloads.EPS)
+            flops += 12.0 * c["D"] * workloads.visible_pairs(c["T"], W)
+        return flops
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count()
+
+
 def oracle_sample(seconds_budget, seed_offset=0):
-    """Times the fp64 oracle on (batch, head) units of the d20 pair until the budget
-    is spent: per unit, prologue + forward + backward + prologue backward of one
-    head of one sequence, for both layers. Returns (TFLOP/s, description, cores)."""
-    import oracle
-    c = workloads.CONFIGS["d20"]
-    B, T, Hq, Hkv, D = c["B"], c["T"], c["Hq"], c["Hkv"], c["D"]
-    scale = workloads.default_scale(D)
-    q, k, v, do = workloads.training_inputs(1, T, Hq, Hkv, D, c["seed"] + seed_offset)
-    pos = oracle.row_positions(1, T)
+    """Times the oracle on units until the budget is spent. Returns (TFLOP/s, description, cores)."""
+    u = OracleUnits(seed_offset)
     flops, units = 0.0, 0
     t0 = time.perf_counter()
-    h = 0
     while True:
-        hs = slice(h % Hq, h % Hq + 1)
-        qf, kf, vf, dof = (t[:, :, hs].float().numpy().astype(np.float64) for t in (q, k, v, do))
-        for W in c["windows"]:
-            qh = oracle.prologue(qf, pos, workloads.ROPE_BASE, workloads.EPS)
-            kh = oracle.prologue(kf, pos, workloads.ROPE_BASE, workloads.EPS)
-            oracle.attention_fwd(qh, kh, vf, W, scale)
-            dqh, dkh, _ = oracle.attention_bwd(qh, kh, vf, dof, W, scale)
-            oracle.prologue_bwd(qf, dqh, pos, workloads.ROPE_BASE, workloads.EPS)
-            oracle.prologue_bwd(kf, dkh, pos, workloads.ROPE_BASE, workloads.EPS)
-            flops += 12.0 * D * workloads.visible_pairs(T, W)
+        flops += u.run_one()
         units += 1
-        h += 1
         if time.perf_counter() - t0 >= seconds_budget:
             break
     dt = time.perf_counter() - t0
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        cores = os.cpu_count()
-    desc = (f"{units} (sequence, head) units of the d20 layer pair (both windows), fp64 numpy oracle, "
-            f"{dt:.1f} s")
-    return flops / dt / 1e12, desc, cores
+    desc = f"{units} units, each {REF_UNIT}; fp64 numpy oracle, {dt:.1f} s"
+    return flops / dt / 1e12, desc, cpu_cores()
 
 
 def run_reference(args, rank, world):
+    """The oracle as the reference arm. One step = one unit (a stated subset of the
+    workload, see REF_UNIT), timed on the host; ms_per_step is that measured time."""
     if rank != 0:
         return None
-    budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    u = OracleUnits()
     for _ in range(args.warmup):
-        oracle_sample(budget)
-    vals = []
-    t0 = time.perf_counter()
-    for s in range(args.steps):
-        v, desc, cores = oracle_sample(budget, seed_offset=0)
-        vals.append(v)
-    wall = time.perf_counter() - t0
-    value = statistics.median(vals)
-    ms = 12.0 * 128 * sum(workloads.visible_pairs(2048, W) for W in (1024, 2048)) * 80 / (value * 1e12) * 1e3
+        u.run_one()
+    flops, times = 0.0, []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        flops += u.run_one()
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = flops / total / 1e12
+    cores = cpu_cores()
+    sample = f"{args.steps} steps of one unit each ({REF_UNIT}), {total:.1f} s in total"
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "global_batch": 8, "seq_len": 2048, "parallelism": "cpu"},
-            "cpu_baseline": {"kind": "oracle", "value": value, "unit": "TFLOP/s", "cores": cores,
-                             "sample": desc + f" per step; {args.steps} steps in {wall:.1f} s"},
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "sample of the " + WORKLOAD + ": " + REF_UNIT + " per step",
+                       "global_batch": 1, "seq_len": 2048, "parallelism": "host cores"},
+            "cpu_baseline": {"kind": "oracle", "value": value, "unit": "TFLOP/s", "cores": cores, "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -519,6 +635,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the GQA and long-context sub-keys")
     args = ap.parse_args()
     rank, world, local = dist_setup(args.gpus)
     try:

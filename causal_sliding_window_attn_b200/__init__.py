@@ -8,6 +8,7 @@ current CUDA stream. The functions carry the C ABI's names (include/cswa_attn.h)
     attn_rope_qknorm_bwd  its backward
     attn_fwd              attention forward -> (o, lse)
     attn_bwd              attention backward -> (dq, dk, dv)
+    attn_block_bwd        the block's backward, prologue included -> (dq, dk, dv) w.r.t. raw q, k
     attn_decode           single-token decode against a KV cache -> (o, lse)
     attn_prefill          a chunk of new tokens against a KV cache -> (o, lse)
     attn_layer_window     the window of one layer of a stack (pattern such as "SSSL")
@@ -24,7 +25,7 @@ import torch
 
 __all__ = [
     "AttnError", "lib", "attn_rope_qknorm", "attn_rope_qknorm_bwd", "attn_fwd", "attn_bwd",
-    "attn_bwd_workspace_bytes", "attn_decode", "attn_decode_workspace_bytes", "attn_prefill", "attn_layer_window",
+    "attn_bwd_workspace_bytes", "attn_block_bwd", "attn_block_bwd_workspace_bytes", "attn_decode", "attn_decode_workspace_bytes", "attn_prefill", "attn_layer_window",
     "layer_windows", "attn_kv_replicate", "attn_get_status", "attn_debug_set_wait_limit",
     "attn_status_string", "LIB_PATH",
 ]
@@ -42,6 +43,8 @@ _SIGS = {
     "attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "attn_bwd_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "attn_bwd": (_i, [_vp] * 9 + [_vp, _sz, _i, _i, _i, _i, _i, _i, _f, _vp]),
+    "attn_block_bwd_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "attn_block_bwd": (_i, [_vp] * 12 + [_sz, _i, _i, _i, _i, _i, _i, _f, _f, _f, _vp]),
     "attn_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "attn_decode": (_i, [_vp] * 8 + [_i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "attn_decode_noalloc": (_i, [_vp] * 8 + [_i, _i, _i, _i, _i, _i, _f, _vp]),
@@ -177,6 +180,31 @@ def attn_bwd(q, k, v, o, dout, lse, window=-1, scale=None, dq=None, dk=None, dv=
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
         _ptr(workspace), workspace.numel() * workspace.element_size(), B, T, Hq, Hkv, D, int(window),
         _default_scale(D, scale), _stream(stream)))
+    return dq, dk, dv
+
+
+def attn_block_bwd_workspace_bytes(B, T, Hq, Hkv, D, window=-1):
+    return int(lib().attn_block_bwd_workspace_bytes(B, T, Hq, Hkv, D, int(window)))
+
+
+def attn_block_bwd(q, k, q_hat, k_hat, v, o, dout, lse, window=-1, scale=None, dq=None, dk=None, dv=None,
+                   workspace=None, rope_base=10000.0, eps=1e-6, stream=None):
+    """dq, dk (w.r.t. the raw q, k of the prologue) and dv of sum(dout * o) for
+    o = attn_fwd(*attn_rope_qknorm(q, k), v): attn_bwd with the prologue backward fused."""
+    B, T, Hq, D = _bf16("q", q).shape
+    Hkv = _bf16("k", k).shape[2]
+    for name, t in (("q_hat", q_hat), ("k_hat", k_hat), ("v", v), ("o", o), ("dout", dout)):
+        _bf16(name, t)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    nbytes = attn_block_bwd_workspace_bytes(B, T, Hq, Hkv, D, window)
+    if workspace is None:
+        workspace = torch.empty(nbytes, device=q.device, dtype=torch.uint8)
+    _check("attn_block_bwd", lib().attn_block_bwd(
+        _ptr(q), _ptr(k), _ptr(q_hat), _ptr(k_hat), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+        _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(), B, T, Hq, Hkv, D, int(window),
+        _default_scale(D, scale), float(rope_base), float(eps), _stream(stream)))
     return dq, dk, dv
 
 

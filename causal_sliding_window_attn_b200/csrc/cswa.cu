@@ -92,10 +92,19 @@ bool set_smem_attrs() {
                                 BwdLayout<D>::kBytes) == cudaSuccess;
   r = r && cudaFuncSetAttribute(attn_fwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 FwdLayout<D>::kBytes) == cudaSuccess;
-  r = r && cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                DqLayout<D>::kBytes) == cudaSuccess;
   if (r) done[dev].store(true, std::memory_order_release);
   return r;
+}
+
+// Rotary angle of pair j per unit position, omega_j / (2 pi) = base^(-2j/D) / (2 pi)
+// turns, as a 64-bit fixed-point fraction: position p's angle in turns is p * U_j
+// mod 2^64, exact for any 32-bit position.
+void rope_turns(int D, float base, unsigned long long* turns) {
+  for (int j = 0; j < D / 2; ++j) {
+    const double u = std::exp2(-2.0 * (double)j / (double)D * std::log2((double)base)) *
+                     0.15915494309189533576888376337251;  // turns per unit position
+    turns[j] = (unsigned long long)(u * 18446744073709551616.0);
+  }
 }
 
 template <int D, bool kBwd>
@@ -135,11 +144,7 @@ attn_status_t rope_common(const void* x0, const void* x1, const void* dy0, const
   p.H[0] = Hq;
   p.H[1] = Hkv;
   p.eps = eps;
-  for (int j = 0; j < D / 2; ++j) {
-    const double u = std::exp2(-2.0 * (double)j / (double)D * std::log2((double)base)) *
-                     0.15915494309189533576888376337251;  // turns per unit position
-    p.turns[j] = (unsigned long long)(u * 18446744073709551616.0);
-  }
+  rope_turns(D, base, p.turns);
   cudaStream_t st = as_stream(stream);
   const long long n_pos = (long long)B * T;
   if (D == 64) return bwd ? launch_rope<64, true>(p, n_pos, st) : launch_rope<64, false>(p, n_pos, st);
@@ -212,64 +217,94 @@ attn_status_t launch_prefill(const void* q, void* kc, void* vc, const void* kn, 
   return launched();
 }
 
+// attn_bwd's workspace: the row extensions of the S^T and dP^T MMAs (-lse/scale and
+// -Delta per query row, padded to 128-row tiles), the fp32 dQ accumulator, the work
+// counter, and for the fused block backward the rotary cos/sin table. O(B T Hq D).
 struct BwdWorkspace {
   uint8_t* ext_lse;       // (B, Hq, Tpad / 128) x 512 bytes
   uint8_t* ext_delta;     // (B, Hq, Tpad / 128) x 512 bytes
-  __nv_bfloat16* ds;      // stored dS^T tiles, 128 x 128 each
-  int* counter;           // [2] work-item counters of the main and dQ kernels (zeroed by the prep kernel)
-  long long tiles_per_bh;
-  int span;
+  float* dq_acc;          // (B, T, Hq, D) fp32
+  int* counter;           // the main kernel's work-item counter (zeroed by the prep kernel)
+  float2* rope_cs;        // (T, D/2) (cos, sin), block backward only
 };
 int eff_window(int window, int T) { return (window >= T) ? -1 : window; }
-BwdWorkspace carve_bwd(void* ws, int B, int T, int Hq, int window) {
-  const int nt = tiles128(T);
-  const size_t Tpad = (size_t)nt * 128;
-  BwdWorkspace w;
-  w.span = bwd_span(nt, eff_window(window, T));
-  w.tiles_per_bh = ds_tiles_before(nt, nt, w.span);
-  uint8_t* p = static_cast<uint8_t*>(ws);
-  w.ext_lse = p;
-  p += align256((size_t)B * Hq * Tpad * 4);
-  w.ext_delta = p;
-  p += align256((size_t)B * Hq * Tpad * 4);
-  w.ds = reinterpret_cast<__nv_bfloat16*>(p);
-  p += align256((size_t)B * Hq * w.tiles_per_bh * 32768);
-  w.counter = reinterpret_cast<int*>(p);
-  return w;
+size_t bwd_ws_parts(int B, int T, int Hq, int D, bool rope, BwdWorkspace* w, void* base) {
+  const size_t Tpad = (size_t)tiles128(T) * 128;
+  uint8_t* p = static_cast<uint8_t*>(base);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* at = p ? p + off : nullptr;
+    off += align256(bytes);
+    return at;
+  };
+  uint8_t* e1 = take((size_t)B * Hq * Tpad * 4);
+  uint8_t* e2 = take((size_t)B * Hq * Tpad * 4);
+  uint8_t* acc = take((size_t)B * T * Hq * D * 4);
+  uint8_t* cnt = take(256);
+  uint8_t* cs = rope ? take((size_t)T * (D / 2) * 8) : nullptr;
+  if (w) {
+    w->ext_lse = e1;
+    w->ext_delta = e2;
+    w->dq_acc = reinterpret_cast<float*>(acc);
+    w->counter = reinterpret_cast<int*>(cnt);
+    w->rope_cs = reinterpret_cast<float2*>(cs);
+  }
+  return off;
 }
-size_t bwd_ws_bytes(int B, int T, int Hq, int window) {
-  const int nt = tiles128(T);
-  const size_t Tpad = (size_t)nt * 128;
-  const long long tiles = ds_tiles_before(nt, nt, bwd_span(nt, eff_window(window, T)));
-  return 2 * align256((size_t)B * Hq * Tpad * 4) + align256((size_t)B * Hq * tiles * 32768) + 256;
-}
+
+// The fused prologue backward of the block variant: raw q and k, and the rotary
+// base and eps of the forward prologue (positions t). Null q_raw: plain attn_bwd.
+struct RopeBwd {
+  const void* q_raw;
+  const void* k_raw;
+  float base, eps;
+};
 
 template <int D>
 attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                          const float* lse, void* dq, void* dk, void* dv, void* ws, int B, int T, int Hq, int Hkv,
-                         int window, float scale, cudaStream_t st) {
+                         int window, float scale, const RopeBwd& rb, cudaStream_t st) {
   const int nt = tiles128(T);
   const int Tpad = nt * 128;
-  BwdWorkspace w = carve_bwd(ws, B, T, Hq, window);
+  const bool rope = rb.q_raw != nullptr;
+  BwdWorkspace w;
+  bwd_ws_parts(B, T, Hq, D, rope, &w, ws);
   CUtensorMap tq, tk, tv, tdo;
   if (!encode_bthd(&tq, q, B, T, Hq, D) || !encode_bthd(&tk, k, B, T, Hkv, D) ||
       !encode_bthd(&tv, v, B, T, Hkv, D) || !encode_bthd(&tdo, dO, B, T, Hq, D))
     return ATTN_ERR_LAUNCH;
   if (!set_smem_attrs<D>()) return ATTN_ERR_LAUNCH;
   {
+    PrepParams pp{};
+    pp.o = static_cast<const __nv_bfloat16*>(o);
+    pp.dout = static_cast<const __nv_bfloat16*>(dO);
+    pp.lse = lse;
+    pp.ext_lse = w.ext_lse;
+    pp.ext_delta = w.ext_delta;
+    pp.dq_acc = w.dq_acc;
+    pp.item_counter = w.counter;
+    pp.rope_cs = w.rope_cs;
+    pp.B = B;
+    pp.T = T;
+    pp.Tpad = Tpad;
+    pp.Hq = Hq;
+    pp.inv_scale = 1.f / scale;
     const long long threads = (long long)B * Tpad * Hq * (D / 8);
-    attn_bwd_prep_kernel<D><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, w.ext_lse, w.ext_delta, w.counter, B,
-        T, Tpad, Hq, 1.f / scale);
+    pp.row_blocks = (threads + 255) / 256;
+    long long blocks = pp.row_blocks;
+    if (rope) {
+      rope_turns(D, rb.base, pp.turns);
+      blocks += ((long long)T * (D / 2) + 255) / 256;
+    }
+    attn_bwd_prep_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(pp);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
   }
   BwdParams p{};
   p.ext_lse = w.ext_lse;
   p.ext_delta = w.ext_delta;
+  p.dq_acc = w.dq_acc;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
-  p.dq = static_cast<__nv_bfloat16*>(dq);
-  p.ds = w.ds;
   p.item_counter = w.counter;
   p.T = T;
   p.Tpad = Tpad;
@@ -277,10 +312,12 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
   p.G = Hq / Hkv;
   p.window = eff_window(window, T);
   p.n_tiles = nt;
-  p.span = w.span;
-  p.tiles_per_bh = w.tiles_per_bh;
+  p.span = bwd_span(nt, p.window);
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
+  p.k_raw = static_cast<const __nv_bfloat16*>(rb.k_raw);
+  p.rope_cs = w.rope_cs;
+  p.eps = rb.eps;
   {
     // persistent: one CTA per SM walks the (key tile, KV head, batch) items
     const long long kv_items = (long long)nt * Hkv * B;
@@ -288,9 +325,22 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
     attn_bwd_kernel<D><<<kv_grid, 384, BwdLayout<D>::kBytes, st>>>(tq, tk, tv, tdo, p, (int)kv_items);
   }
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
-  const long long items = (long long)nt * Hq * B;
-  const int grid = (int)std::min<long long>(items, sm_count());
-  attn_bwd_dq_kernel<D><<<grid, 256, DqLayout<D>::kBytes, st>>>(tk, p, (int)items);
+  DqParams dp{};
+  dp.dq_acc = w.dq_acc;
+  dp.dq = static_cast<__nv_bfloat16*>(dq);
+  dp.q_raw = static_cast<const __nv_bfloat16*>(rb.q_raw);
+  dp.rope_cs = w.rope_cs;
+  dp.rows = (long long)B * T * Hq;
+  dp.Hq = Hq;
+  dp.T = T;
+  dp.scale = scale;
+  dp.eps = rb.eps;
+  const long long per_block = 2 * (256 / (D / 8));
+  const unsigned grid = (unsigned)((dp.rows + per_block - 1) / per_block);
+  if (rope)
+    attn_bwd_dq_kernel<D, true><<<grid, 256, 0, st>>>(dp);
+  else
+    attn_bwd_dq_kernel<D, false><<<grid, 256, 0, st>>>(dp);
   return launched();
 }
 
@@ -298,15 +348,29 @@ template <int D, int GMAX>
 attn_status_t launch_decode(const DecodeParams& p, int B, cudaStream_t st) {
   dim3 g1(p.n_chunks, p.Hkv, B);
   decode_chunk_kernel<D, GMAX><<<g1, 128, 0, st>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
-  dim3 g2(p.Hq, B);
-  decode_combine_kernel<D><<<g2, D, 0, st>>>(p);
   return launched();
 }
 
 int decode_chunks(int Tmax, int window) {
   const int span = (window < 0 || window >= Tmax) ? Tmax : window + 1;
   return (span + kDecodeChunk - 1) / kDecodeChunk;
+}
+
+// attn_decode's workspace: the fp32 split-K partials (B, Hq, chunks, D + 2), rounded up
+// to 256 bytes, then one 8-byte arrival counter per (sequence, KV head) -- B * Hq of
+// them, enough for any Hkv <= Hq.
+size_t decode_ws_bytes(int B, int Hq, int D, int Tmax, int window) {
+  return align256((size_t)B * Hq * decode_chunks(Tmax, window) * (D + 2) * 4) + (size_t)B * Hq * 8;
+}
+
+// Tag of one decode call for its arrival counters: a fresh value per call in this
+// process (never 0, so zeroed memory never matches; a CUDA graph that captured a call
+// replays its tag, which the counters' reset to (tag, 0) allows).
+std::atomic<unsigned> g_decode_epoch{0};
+unsigned next_decode_epoch() {
+  unsigned e = g_decode_epoch.fetch_add(1, std::memory_order_relaxed) + 1;
+  if (e == 0) e = g_decode_epoch.fetch_add(1, std::memory_order_relaxed) + 1;
+  return e;
 }
 
 // ---------------------------------------------------------------- no-allocation decode
@@ -334,6 +398,30 @@ attn_status_t noalloc_scratch(void** out) {
   return ATTN_OK;
 }
 
+attn_status_t bwd_common(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                         const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B,
+                         int T, int Hq, int Hkv, int D, int window, float scale, const RopeBwd& rb, void* stream) {
+  if (!dims_ok(B, T, Hq, Hkv) || !scale_ok(scale)) return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q, k, v, o, dO, lse, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return ATTN_ERR_INVALID_ARG;
+  const bool rope = rb.q_raw != nullptr;
+  if (rope && (!rb.k_raw || !aligned16(rb.q_raw) || !aligned16(rb.k_raw) || !(rb.base > 1.f) ||
+               !std::isfinite(rb.base) || !(rb.eps >= 0.f) || !std::isfinite(rb.eps)))
+    return ATTN_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      ws_bytes < bwd_ws_parts(B, T, Hq, D, rope, nullptr, nullptr))
+    return ATTN_ERR_INVALID_ARG;
+  if (Hq > 65535 || B > 65535 || tiles128(T) > 65535) return ATTN_ERR_INVALID_ARG;
+  // work items and the prep kernel's blocks are counted in 32 bits
+  if ((long long)tiles128(T) * Hkv * B >= (1ll << 31) ||
+      (long long)B * tiles128(T) * 128 * Hq * (D / 8) / 256 + (long long)T * D / 512 >= (1ll << 31))
+    return ATTN_ERR_UNSUPPORTED;
+  cudaStream_t st = as_stream(stream);
+  return D == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, workspace, B, T, Hq, Hkv, window, scale, rb, st)
+                 : launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, workspace, B, T, Hq, Hkv, window, scale, rb, st);
+}
 }  // namespace
 
 extern "C" {
@@ -364,32 +452,38 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
 
 size_t attn_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int window) {
   if (!dims_ok(B, T, Hq, Hkv) || (D != 64 && D != 128)) return 0;
-  return bwd_ws_bytes(B, T, Hq, window);
+  (void)window;
+  return bwd_ws_parts(B, T, Hq, D, false, nullptr, nullptr);
 }
+
+size_t attn_block_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int window) {
+  if (!dims_ok(B, T, Hq, Hkv) || (D != 64 && D != 128)) return 0;
+  (void)window;
+  return bwd_ws_parts(B, T, Hq, D, true, nullptr, nullptr);
+}
+
 
 attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                        void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int T, int Hq, int Hkv,
                        int D, int window, float scale, void* stream) {
-  if (!dims_ok(B, T, Hq, Hkv) || !scale_ok(scale)) return ATTN_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
-  const void* ptrs[] = {q, k, v, o, dO, lse, dq, dk, dv};
-  for (const void* ptr : ptrs)
-    if (!ptr || !aligned16(ptr)) return ATTN_ERR_INVALID_ARG;
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
-      ws_bytes < attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, window))
-    return ATTN_ERR_INVALID_ARG;
-  if (Hq > 65535 || B > 65535 || tiles128(T) > 65535) return ATTN_ERR_INVALID_ARG;
-  if ((long long)B * Hq * ds_tiles_before(tiles128(T), tiles128(T), bwd_span(tiles128(T), eff_window(window, T))) *
-          128 >= (1ll << 31))
-    return ATTN_ERR_UNSUPPORTED;  // stored dS^T tile rows and dQ work items are counted in 32 bits
-  cudaStream_t st = as_stream(stream);
-  return D == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, workspace, B, T, Hq, Hkv, window, scale, st)
-                 : launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, workspace, B, T, Hq, Hkv, window, scale, st);
+  const RopeBwd none{nullptr, nullptr, 0.f, 0.f};
+  return bwd_common(q, k, v, o, dO, lse, dq, dk, dv, workspace, ws_bytes, B, T, Hq, Hkv, D, window, scale, none,
+                    stream);
+}
+
+attn_status_t attn_block_bwd(const void* q, const void* k, const void* q_hat, const void* k_hat, const void* v,
+                             const void* o, const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                             void* workspace, size_t ws_bytes, int B, int T, int Hq, int Hkv, int D, int window,
+                             float scale, float rope_base, float eps, void* stream) {
+  if (!q || !k) return ATTN_ERR_INVALID_ARG;
+  const RopeBwd rb{q, k, rope_base, eps};
+  return bwd_common(q_hat, k_hat, v, o, dO, lse, dq, dk, dv, workspace, ws_bytes, B, T, Hq, Hkv, D, window, scale, rb,
+                    stream);
 }
 
 size_t attn_decode_workspace_bytes(int B, int Hq, int D, int Tmax, int window) {
   if (B < 1 || Hq < 1 || Tmax < 1 || (D != 64 && D != 128)) return 0;
-  return (size_t)B * Hq * decode_chunks(Tmax, window) * (D + 2) * 4;
+  return decode_ws_bytes(B, Hq, D, Tmax, window);
 }
 
 attn_status_t attn_decode(const void* q, void* kcache, void* vcache, const void* k_new, const void* v_new,
@@ -398,7 +492,6 @@ attn_status_t attn_decode(const void* q, void* kcache, void* vcache, const void*
   if (!dims_ok(B, Tmax, Hq, Hkv) || !scale_ok(scale)) return ATTN_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
   const int G = Hq / Hkv;
-  if (G > 8) return ATTN_ERR_UNSUPPORTED;
   if (!q || !kcache || !vcache || !pos || !o || !workspace || (k_new == nullptr) != (v_new == nullptr))
     return ATTN_ERR_INVALID_ARG;
   const void* ptrs[] = {q, kcache, vcache, o, workspace};
@@ -409,6 +502,7 @@ attn_status_t attn_decode(const void* q, void* kcache, void* vcache, const void*
     return ATTN_ERR_INVALID_ARG;
   if (ws_bytes < attn_decode_workspace_bytes(B, Hq, D, Tmax, window) || Hkv > 65535 || B > 65535 || Hq > 65535)
     return ATTN_ERR_INVALID_ARG;
+  const size_t part_bytes = align256((size_t)B * Hq * decode_chunks(Tmax, window) * (D + 2) * 4);
   DecodeParams p{};
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.kc = static_cast<__nv_bfloat16*>(kcache);
@@ -419,6 +513,8 @@ attn_status_t attn_decode(const void* q, void* kcache, void* vcache, const void*
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.ws = static_cast<float*>(workspace);
+  p.counters = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) + part_bytes);
+  p.epoch = next_decode_epoch();
   p.Tmax = Tmax;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -456,7 +552,8 @@ attn_status_t attn_decode_noalloc(const void* q, void* kcache, void* vcache, con
   void* scratch = nullptr;
   const attn_status_t st = noalloc_scratch(&scratch);
   if (st != ATTN_OK) return st;
-  // every partial the combine step reads is written earlier in the same call: nothing to clear
+  // every partial the merge reads is written earlier in the same call, and the arrival
+  // counters are tagged per call (stale contents read as zero): nothing to clear
   return attn_decode(q, kcache, vcache, k_new, v_new, pos, o, lse, B, Tmax, Hq, Hkv, D, window, scale, scratch, need,
                      stream);
 }
@@ -500,6 +597,21 @@ attn_status_t attn_debug_set_wait_limit(unsigned long long ns, void* stream) {
   if (cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)) != cudaSuccess) return ATTN_ERR_LAUNCH;
   return cudaDeviceSynchronize() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
+
+#ifdef CSWA_TRACE
+// Profiling builds only: copies the pipeline trace marks (clock64 per CTA, role,
+// step and tag; see CSWA_MARK) to host memory.
+int attn_debug_trace_copy(void* dst, size_t bytes) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return 3;
+  return cudaMemcpyFromSymbol(dst, g_trace, bytes < sizeof(g_trace) ? bytes : sizeof(g_trace)) == cudaSuccess ? 0 : 3;
+}
+int attn_debug_trace_clear(void) {
+  static unsigned long long zeros[1024] = {};
+  for (size_t off = 0; off < sizeof(g_trace); off += sizeof(zeros))
+    if (cudaMemcpyToSymbol(g_trace, zeros, sizeof(zeros), off) != cudaSuccess) return 3;
+  return cudaDeviceSynchronize() == cudaSuccess ? 0 : 3;
+}
+#endif
 
 const char* attn_status_string(attn_status_t s) {
   switch (s) {

@@ -93,12 +93,12 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* v_full = bars + 3;    // [2]
   uint64_t* k_empty = bars + 5;   // [2] S of the tile has read K
   uint64_t* s_full = bars + 7;    // [2]
-  uint64_t* p_full = bars + 9;    // [2]
   uint64_t* pv_done = bars + 11;  // [2]
   uint64_t* final_bar = bars + 13;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 15);
   uint64_t* v_empty = bars + 16;  // [2] PV of the tile has read V
+  uint64_t* p_chunk = bars + 18;  // [2][4] P_s of keys 32c .. 32c+31 written over S_s
 
   const int warp = warp_id(), lane = lane_id();
   const int h = blockIdx.x;
@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&k_empty[s], 1);
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
+      for (int c = 0; c < 4; ++c) mbar_init(&p_chunk[4 * s + c], 128);
       mbar_init(&pv_done[s], 1);
     }
     mbar_init(final_bar, 1);
@@ -291,13 +291,20 @@ __global__ void __launch_bounds__(384, 1)
       if (tracer) CSWA_MARK(0, n, 1);
       for (int s = 0; s < 2; ++s) {
         if (active(s, t)) {
-          if (!(ok = wait_all(&p_full[s], cnt[s] & 1))) break;
-          if (tracer) CSWA_MARK(0, n, 2 + 3 * s);
-          tc_fence_after();
+          // PV_s chunk by chunk as the softmax warps publish P_s: chunk c holds keys
+          // 32c .. 32c+31 (K steps 2c, 2c+1) as bf16 pairs in columns 16c .. 16c+15
+          for (int c = 0; c < 4; ++c) {
+            if (!(ok = wait_all(&p_chunk[4 * s + c], cnt[s] & 1))) break;
+            if (tracer && c == 0) CSWA_MARK(0, n, 2 + 3 * s);
+            tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tO(s), tS(s) + kk * 8, dV0 + ((st * L::kTile + kk * 2048) >> 4), idO, (cnt[s] > 0 || kk > 0),
-                   leader);
+            for (int u = 0; u < 2; ++u) {
+              const int kk = 2 * c + u;
+              mma_ts(tO(s), tS(s) + kk * 8, dV0 + ((st * L::kTile + kk * 2048) >> 4), idO, (cnt[s] > 0 || kk > 0),
+                     leader);
+            }
+          }
+          if (!ok) break;
           mma_commit(&pv_done[s], leader);
           ++cnt[s];
           if (tracer) CSWA_MARK(0, n, 3 + 3 * s);
@@ -425,36 +432,43 @@ __global__ void __launch_bounds__(384, 1)
           rescale = true;
         }
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-        // p = exp2(s * scale * log2e - m), two columns per packed FMA; row sum in packed adds
+        // rescale O first, only when some row of the warp needs it (O is stable: this
+        // tile's S was committed after the previous PV, so that PV has completed), so that
+        // every P chunk published below may start its PV at once
+        if (__any_sync(0xffffffffu, rescale)) {
+          // 16 columns at a time: the row's 128 scores are still live in registers
+#pragma unroll 1
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t o[16];
+            tmem_ld16(tOs + c * 16, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+            tmem_st16(tOs + c * 16, o);
+          }
+          tmem_st_wait();
+        }
+        // p = exp2(s * scale * log2e - m), two columns per packed FMA; row sum in packed adds.
+        // Published in four chunks of 32 keys, each on its own barrier: chunk c's bf16 pairs
+        // land in columns 16c .. 16c+15, whose fp32 S (keys < 32c + 32) is already in registers
         const float2 sl2v = make_float2(sl2, sl2), nm = make_float2(-m_use, -m_use);
         float2 ls4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float2 x = __ffma2_rn(make_float2(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), sl2v, nm);
-          const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-          ls4[c & 3] = __fadd2_rn(ls4[c & 3], pp);
-          r[c] = pack_bf16x2(pp.x, pp.y);
+        for (int ch = 0; ch < 4; ++ch) {
+#pragma unroll
+          for (int c = 16 * ch; c < 16 * ch + 16; ++c) {
+            const float2 x =
+                __ffma2_rn(make_float2(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), sl2v, nm);
+            const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            ls4[c & 3] = __fadd2_rn(ls4[c & 3], pp);
+            r[c] = pack_bf16x2(pp.x, pp.y);
+          }
+          tmem_st16(tSs + 16 * ch, *reinterpret_cast<uint32_t(*)[16]>(&r[16 * ch]));
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&p_chunk[4 * s + ch]);
         }
         l_run += ((ls4[0].x + ls4[0].y) + (ls4[1].x + ls4[1].y)) + ((ls4[2].x + ls4[2].y) + (ls4[3].x + ls4[3].y));
-        if (tracer) CSWA_MARK(1 + s, cnt, 3);
-        tmem_st32(tSs + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_st32(tSs + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-        // rescale only when some row of the warp needs it (O is stable: this tile's
-        // S was committed after the previous PV, so that PV has completed)
-        if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tOs + c * 32, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-            tmem_st32(tOs + c * 32, o);
-          }
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&p_full[s]);
         if (tracer) CSWA_MARK(1 + s, cnt, 4);
       }
       // ---------------------------------------------------------- epilogue

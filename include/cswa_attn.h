@@ -82,13 +82,12 @@ attn_status_t attn_rope_qknorm_bwd(const void* q, const void* k, const void* dq_
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T,
                        int Hq, int Hkv, int D, int window, float scale, void* stream);
 
-/* Bytes of workspace attn_bwd needs for this window: per query row, -lse/scale and
- * -Delta_i = -(dO_i . o_i) as bf16 hi/lo pairs (2 x B*Hq*Tpad*4 bytes, Tpad = T
- * rounded up to a multiple of 128); the bf16 dS^T tiles (128 x 128) of every (query
- * tile, key tile) pair inside the causal window, kept between the main backward
- * kernel and the dQ kernel: about B*Hq*T*min(T, W+128)*2 bytes for window W
- * (B*Hq*T^2 without a window); and 256 bytes for the main kernel's work counter.
- * Nothing in it needs to be initialised. */
+/* Bytes of workspace attn_bwd needs: per query row, -lse/scale and -Delta_i =
+ * -(dO_i . o_i) as bf16 hi/lo pairs (2 x B*Hq*Tpad*4 bytes, Tpad = T rounded up to a
+ * multiple of 128); the fp32 dQ accumulator (B*T*Hq*D*4 bytes); and 256 bytes for
+ * the main kernel's work counter, each part rounded up to 256 bytes. O(B*T*Hq*D): it
+ * does not grow with the window. The window argument is accepted for symmetry and
+ * does not change the size. Nothing in it needs to be initialised. */
 size_t attn_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int window);
 
 /*
@@ -99,14 +98,44 @@ size_t attn_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int window
  * Inputs: q, k, v, o, dO (bf16) and lse (fp32) exactly as attn_fwd produced
  * them. Outputs dq (B,T,Hq,D), dk, dv (B,T,Hkv,D) bf16, fully overwritten.
  * workspace: device memory, 256-byte aligned, of ws_bytes >=
- * attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, window). Calls whose stored dS^T
- * tiles would exceed 2^31 rows return ATTN_ERR_UNSUPPORTED.
+ * attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, window). Three launches: a per-row
+ * preparation, the tensor-core main kernel (dK and dV complete per key tile; dQ
+ * partials added into the workspace's fp32 accumulator), and dq = scale x the
+ * accumulator as bf16. Sizes whose work items would not fit 32-bit counters return
+ * ATTN_ERR_UNSUPPORTED.
  */
 attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                        const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B,
                        int T, int Hq, int Hkv, int D, int window, float scale, void* stream);
 
-/* Bytes of workspace attn_decode needs (fp32 split-K partials). */
+/* Bytes of workspace attn_block_bwd needs: attn_bwd's, plus the rotary cos/sin table
+ * (T*D/2*8 bytes, rounded up to 256). */
+size_t attn_block_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int window);
+
+/*
+ * attn_block_bwd -- the backward of the whole attention block of training,
+ * prologue included (nanochat Admin & Developer Guide, 3: RMS-norm of q and k
+ * without weight, then RoPE at positions t; the softmax backward as in
+ * attn_bwd): gradients with respect to the RAW q, k and to v, of sum(dO * o) for
+ *   q_hat, k_hat = attn_rope_qknorm(q, k) (pos null),  o = attn_fwd(q_hat, k_hat, v).
+ * It computes what attn_bwd followed by attn_rope_qknorm_bwd computes, with the
+ * prologue backward done on the way out of the kernels (the dK epilogue of the
+ * main kernel and the dq pass): dq_hat and dk_hat never reach memory.
+ *   q (B,T,Hq,D), k (B,T,Hkv,D): the raw inputs of the prologue.
+ *   q_hat, k_hat: the prologue's outputs for them (rope_base, eps as given here).
+ *   v, o, dO, lse: as for attn_bwd. Outputs dq, dk (raw-input gradients) and dv.
+ *   workspace: 256-byte aligned, >= attn_block_bwd_workspace_bytes(...).
+ * Same checks, errors and launches as attn_bwd; rope_base > 1 and eps >= 0.
+ */
+attn_status_t attn_block_bwd(const void* q, const void* k, const void* q_hat, const void* k_hat, const void* v,
+                             const void* o, const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                             void* workspace, size_t ws_bytes, int B, int T, int Hq, int Hkv, int D, int window,
+                             float scale, float rope_base, float eps, void* stream);
+
+/* Bytes of workspace attn_decode needs: the fp32 split-K partials (B*Hq*chunks*(D+2)*4
+ * bytes, chunks = ceil(min(window+1, Tmax) / 128), rounded up to 256) and one 8-byte
+ * arrival counter per (sequence, head). Nothing in it needs to be initialised: the
+ * counters carry a per-call tag, so stale or garbage contents read as zero. */
 size_t attn_decode_workspace_bytes(int B, int Hq, int D, int Tmax, int window);
 
 /*
@@ -120,9 +149,12 @@ size_t attn_decode_workspace_bytes(int B, int Hq, int D, int Tmax, int window);
  *   already hold the new token's entry at pos[b].
  *   The token attends to keys [max(0, pos[b] - window), pos[b]].
  *   o (B,1,Hq,D) bf16; lse (B,Hq) fp32 or null.
- * Hq/Hkv <= 8 (ATTN_ERR_UNSUPPORTED above). A pos[b] out of range leaves NaN
- * in that row's outputs and raises ATTN_ERR_DEVICE in the status word.
- * Memory-bound split-K over key chunks.
+ * Any group size Hq/Hkv. A pos[b] out of range leaves NaN in that row's outputs and
+ * raises ATTN_ERR_DEVICE in the status word.
+ * Memory-bound split-K over 128-key chunks in one launch: every cache byte is read
+ * once, and the last chunk of each (sequence, KV head) to finish merges the chunks.
+ * Calls that share a workspace must be ordered (one stream): overlapping calls race
+ * on it.
  */
 attn_status_t attn_decode(const void* q, void* kcache, void* vcache, const void* k_new, const void* v_new,
                           const int32_t* pos, void* o, float* lse, int B, int Tmax, int Hq, int Hkv, int D,
@@ -167,9 +199,10 @@ attn_status_t attn_prefill(const void* q, void* kcache, void* vcache, const void
  * (same arguments minus the workspace) but keeps the split-K partials in a
  * fixed scratch array that the library itself holds in device memory.
  *
- *   - Limit: the partials of one call, attn_decode_workspace_bytes(B, Hq, D,
- *     Tmax, window), must fit in the fixed 4 MiB scratch (4194304 bytes; e.g.
- *     32 sequences x 16 query heads at window 1024 and D = 128 need 2.4 MB).
+ *   - Limit: what one call needs, attn_decode_workspace_bytes(B, Hq, D, Tmax,
+ *     window) (its partials and arrival counters), must fit in the fixed 4 MiB
+ *     scratch (4194304 bytes; e.g. 32 sequences x 16 query heads at window 1024
+ *     and D = 128 need 2.4 MB).
  *     Larger calls return ATTN_ERR_INVALID_ARG and enqueue nothing.
  *   - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
  *     The scratch is a file-scope __device__ array, so every GPU that loads the
@@ -181,7 +214,8 @@ attn_status_t attn_prefill(const void* q, void* kcache, void* vcache, const void
  *     contents. Calls whose kernels overlap on the GPU (different streams, no
  *     ordering between them) race on it and give undefined results; calls on
  *     one stream are safe. No part of it needs to start at zero: every partial
- *     a call reads is written earlier in that same call.
+ *     a call reads is written earlier in that same call, and the arrival
+ *     counters carry a per-call tag.
  */
 attn_status_t attn_decode_noalloc(const void* q, void* kcache, void* vcache, const void* k_new, const void* v_new,
                                   const int32_t* pos, void* o, float* lse, int B, int Tmax, int Hq, int Hkv, int D,

@@ -97,12 +97,14 @@ def check_grad(name, a, ref, rel_tol=GRAD_REL_L2):
 
 
 def run_block(cswa, q, k, v, do, window, scale):
-    """prologue -> fwd -> bwd -> prologue bwd on the GPU; returns a dict of CUDA tensors."""
+    """prologue -> fwd -> bwd -> prologue bwd on the GPU, and the same backward through
+    attn_block_bwd (prologue backward fused: dq_f, dk_f, dv_f); a dict of CUDA tensors."""
     q, k, v, do = (t.cuda() for t in (q, k, v, do))
     qh, kh = cswa.attn_rope_qknorm(q, k, rope_base=ROPE_BASE, eps=EPS)
     o, lse = cswa.attn_fwd(qh, kh, v, window, scale)
     dqh, dkh, dv = cswa.attn_bwd(qh, kh, v, o, do, lse, window, scale)
     dq, dk = cswa.attn_rope_qknorm_bwd(q, k, dqh, dkh, rope_base=ROPE_BASE, eps=EPS)
+    dq_f, dk_f, dv_f = cswa.attn_block_bwd(q, k, qh, kh, v, o, do, lse, window, scale, rope_base=ROPE_BASE, eps=EPS)
     torch.cuda.synchronize()
     assert cswa.attn_get_status() == 0
-    return dict(qh=qh, kh=kh, o=o, lse=lse, dqh=dqh, dkh=dkh, dv=dv, dq=dq, dk=dk)
+    return dict(qh=qh, kh=kh, o=o, lse=lse, dqh=dqh, dkh=dkh, dv=dv, dq=dq, dk=dk, dq_f=dq_f, dk_f=dk_f, dv_f=dv_f)

@@ -41,26 +41,30 @@ def test_status_strings(L):
 
 
 def test_bwd_workspace_size(L):
-    # lse*log2e and Delta (fp32, padded to 128-row tiles) + one 32 KB dS^T tile per
-    # (key tile, query tile) pair inside the window
+    # two arrays of per-row extension pairs (fp32-sized, padded to 128-row tiles), the
+    # fp32 dQ accumulator and the work counter; each part rounded up to 256 bytes. The
+    # window does not change it.
     B, T, Hq, Hkv, D = 8, 2048, 10, 10, 128
     rows = B * Hq * 2048 * 4
-    # window 1024: key tile n sees min(16 - n, 9) query tiles -> 7*9 + (9+8+...+1) = 108
-    assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, 1024) == 2 * rows + B * Hq * 108 * 32768 + 256
-    # no window: the 16*17/2 = 136 tiles of the lower triangle; window >= T - 1 is the same
-    full = 2 * rows + B * Hq * 136 * 32768 + 256
-    assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, -1) == full
-    assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, 2048) == full
-    # ragged T pads the per-row arrays to whole 128-row tiles; window 0 keeps the diagonal only
-    assert L.attn_bwd_workspace_bytes(1, 130, 2, 1, 64, 0) == 2 * 2048 + 2 * 2 * 32768 + 256
+    acc = B * T * Hq * D * 4
+    for W in (1024, -1, 2048, 0):
+        assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, W) == 2 * rows + acc + 256
+    # the block backward adds the (T, D/2) cos/sin table of float pairs
+    assert L.attn_block_bwd_workspace_bytes(B, T, Hq, Hkv, D, 1024) == 2 * rows + acc + 256 + T * 64 * 8
+    # ragged T pads the per-row arrays to whole 128-row tiles (130 -> 256); the accumulator
+    # holds the T real rows, rounded up to 256 bytes
+    assert L.attn_bwd_workspace_bytes(1, 130, 2, 1, 64, 0) == 2 * 2048 + 130 * 2 * 64 * 4 + 256
+    assert L.attn_block_bwd_workspace_bytes(1, 3, 1, 1, 64, -1) == 2 * 512 + 768 + 256 + 768
     assert L.attn_bwd_workspace_bytes(1, 16, 3, 2, 128, -1) == 0     # Hq % Hkv != 0
     assert L.attn_bwd_workspace_bytes(1, 16, 2, 2, 96, -1) == 0      # head dim
 
 
 def test_decode_workspace_size(L):
-    # 1025 visible keys at most -> 9 chunks of 128
-    assert L.attn_decode_workspace_bytes(32, 10, 128, 2176, 1024) == 32 * 10 * 9 * 130 * 4
-    assert L.attn_decode_workspace_bytes(2, 4, 64, 300, -1) == 2 * 4 * 3 * 66 * 4
+    # fp32 partials (B, Hq, chunks, D + 2) rounded up to 256 bytes, then an 8-byte
+    # arrival counter per (sequence, head); 1025 visible keys at most -> 9 chunks of 128
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert L.attn_decode_workspace_bytes(32, 10, 128, 2176, 1024) == up(32 * 10 * 9 * 130 * 4) + 32 * 10 * 8
+    assert L.attn_decode_workspace_bytes(2, 4, 64, 300, -1) == up(2 * 4 * 3 * 66 * 4) + 2 * 4 * 8
 
 
 P = ctypes.c_void_p(0x10000)      # a 16-byte aligned stand-in; never dereferenced
@@ -97,6 +101,22 @@ def test_bwd_rejects_bad_args(L):
     assert call(15, 96) == UNSUPPORTED                # head dim
 
 
+def test_block_bwd_rejects_bad_args(L):
+    ws = L.attn_block_bwd_workspace_bytes(1, 128, 4, 2, 128, 64)
+    f = ctypes.c_float
+    base = [P] * 11 + [P, ws, 1, 128, 4, 2, 128, 64, f(0.1), f(1e4), f(1e-6), None]
+    def call(i, v):
+        a = list(base)
+        a[i] = v
+        return L.attn_block_bwd(*a)
+    assert call(12, L.attn_bwd_workspace_bytes(1, 128, 4, 2, 128, 64)) == INVALID  # no room for the table
+    assert call(0, None) == INVALID                   # null raw q
+    assert call(1, MIS) == INVALID                    # misaligned raw k
+    assert call(20, f(1.0)) == INVALID                # rope base
+    assert call(21, f(-1.0)) == INVALID               # eps
+    assert call(17, 96) == UNSUPPORTED                # head dim
+
+
 def test_rope_rejects_bad_args(L):
     f = ctypes.c_float
     assert L.attn_rope_qknorm(None, None, None, None, None, 1, 4, 2, 2, 128, f(1e4), f(1e-6), None) == INVALID
@@ -121,10 +141,6 @@ def test_decode_rejects_bad_args(L):
     assert call(16, ws - 4) == INVALID
     assert call(3, P) == INVALID                      # k_new without v_new
     assert call(10, 5) == INVALID                     # Hq % Hkv
-    a = list(base)
-    a[10], a[11] = 18, 2                              # G = 9 > 8
-    a[16] = L.attn_decode_workspace_bytes(2, 18, 128, 64, -1)
-    assert L.attn_decode(*a) == UNSUPPORTED
 
 
 def test_prefill_rejects_bad_args(L):
@@ -183,13 +199,11 @@ def test_size_limits_rejected_before_launch(L):
     ws = L.attn_decode_workspace_bytes(1, 1, 128, Tmax, -1)
     assert ws > 0
     assert L.attn_decode(P, P, P, None, None, P, P, P, 1, Tmax, 1, 1, 128, -1, f, P, ws, None) == UNSUPPORTED
-    # decode: a group of more than 8 query heads per KV head
-    ws = L.attn_decode_workspace_bytes(1, 9, 128, 64, -1)
-    assert L.attn_decode(P, P, P, None, None, P, P, P, 1, 64, 9, 1, 128, -1, f, P, ws, None) == UNSUPPORTED
-    # backward: stored dS^T tiles beyond 2^31 rows (B * Hq * tiles * 128)
-    B, T, H = 64, 65536, 64
+    # backward: more than 2^31 work items (key tiles x KV heads x sequences)
+    B, T, H = 1023, 65535 * 128, 128
     ws = L.attn_bwd_workspace_bytes(B, T, H, H, 128, -1)
     big = ctypes.c_void_p(0x100000000)
+    assert ws > 0
     assert L.attn_bwd(*([P] * 9), big, ws, B, T, H, H, 128, -1, f, None) == UNSUPPORTED
     # grid limits: 65535 sequences or query heads at most
     assert L.attn_fwd(P, P, P, P, P, 65536, 16, 1, 1, 128, -1, f, None) == INVALID

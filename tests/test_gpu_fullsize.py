@@ -84,6 +84,13 @@ def test_fullsize_sampled(cswa, name, W):
                                                                            ROPE_BASE, EPS))
     check_grad("dk (prologue bwd)", f64(g["dk"][:1]), oracle.prologue_bwd(f64(k[:1]), f64(g["dkh"][:1]), pos,
                                                                            ROPE_BASE, EPS))
+    # attn_block_bwd (prologue backward fused) against the oracle's prologue backward of the
+    # GPU's own attention gradients on the same batch row; dv must equal attn_bwd's closely
+    check_grad("dq (attn_block_bwd)", f64(g["dq_f"][:1]), oracle.prologue_bwd(f64(q[:1]), f64(g["dqh"][:1]), pos,
+                                                                               ROPE_BASE, EPS))
+    check_grad("dk (attn_block_bwd)", f64(g["dk_f"][:1]), oracle.prologue_bwd(f64(k[:1]), f64(g["dkh"][:1]), pos,
+                                                                               ROPE_BASE, EPS))
+    check_grad("dv (attn_block_bwd)", f64(g["dv_f"]), f64(g["dv"]), 2e-3)
 
 
 def test_fullsize_decode(cswa):

@@ -86,9 +86,14 @@ def test_block_matches_oracle(cswa, case):
     check_grad("dv", f64(g["dv"]), dv_ref)
     # backward through the prologue, end-to-end from the raw inputs
     dqe, dke, dve = oracle.attention_bwd(qh_ref, kh_ref, vf, dof, W, scale)
-    check_grad("dq (end-to-end)", f64(g["dq"]), oracle.prologue_bwd(qf, dqe, pos, ROPE_BASE, EPS))
-    check_grad("dk (end-to-end)", f64(g["dk"]), oracle.prologue_bwd(kf, dke, pos, ROPE_BASE, EPS))
+    dq_e2e, dk_e2e = oracle.prologue_bwd(qf, dqe, pos, ROPE_BASE, EPS), oracle.prologue_bwd(kf, dke, pos, ROPE_BASE, EPS)
+    check_grad("dq (end-to-end)", f64(g["dq"]), dq_e2e)
+    check_grad("dk (end-to-end)", f64(g["dk"]), dk_e2e)
     check_grad("dv (end-to-end)", f64(g["dv"]), dve)
+    # the block backward: the prologue backward fused into the kernels' epilogues
+    record(tid, "block-bwd", dq_rel_l2=check_grad("dq (attn_block_bwd)", f64(g["dq_f"]), dq_e2e),
+           dk_rel_l2=check_grad("dk (attn_block_bwd)", f64(g["dk_f"]), dk_e2e),
+           dv_rel_l2=check_grad("dv (attn_block_bwd)", f64(g["dv_f"]), dve))
 
 
 def test_prologue_positions_and_inplace(cswa):
@@ -193,6 +198,30 @@ def test_decode_small(cswa, W, append):
 
 def test_decode_d64_gqa8(cswa):
     _decode_case(cswa, 2, 700, 8, 1, 64, 300, [650, 5], seed=22, append=True)
+
+
+@pytest.mark.parametrize("Hq,Hkv,D", [(16, 1, 128), (32, 2, 64), (12, 1, 128)])
+def test_decode_wide_groups(cswa, Hq, Hkv, D):
+    """Groups of more than 8 query heads per KV head (sub-groups of 8 in one CTA)."""
+    _decode_case(cswa, 3, 900, Hq, Hkv, D, 700, [899, 0, 431], seed=24, append=True)
+
+
+def test_decode_repeated_calls_share_a_workspace(cswa):
+    """The arrival counters in the workspace are tagged per call: a workspace reused
+    across calls (and one that starts out holding garbage) gives the same results."""
+    B, Tmax, Hq, Hkv, D, W = 4, 600, 4, 2, 128, 256
+    g = torch.Generator().manual_seed(25)
+    q = torch.randn((B, 1, Hq, D), generator=g).to(torch.bfloat16).cuda()
+    kc = torch.randn((B, Tmax, Hkv, D), generator=g).to(torch.bfloat16).cuda()
+    vc = torch.randn((B, Tmax, Hkv, D), generator=g).to(torch.bfloat16).cuda()
+    pos = torch.tensor([599, 10, 300, 128], dtype=torch.int32).cuda()
+    ws = torch.randint(0, 255, (cswa.attn_decode_workspace_bytes(B, Hq, D, Tmax, W),), dtype=torch.uint8).cuda()
+    ref, lref = cswa.attn_decode(q, kc, vc, pos, W)
+    for _ in range(3):
+        o, l = cswa.attn_decode(q, kc, vc, pos, W, workspace=ws)
+        torch.cuda.synchronize()
+        assert cswa.attn_get_status() == 0
+        assert torch.equal(o, ref) and torch.equal(l, lref)
 
 
 def test_decode_equals_forward_row(cswa):

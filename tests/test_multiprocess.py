@@ -56,9 +56,23 @@ def test_reference_arm_runs_on_rank0_only(monkeypatch):
     import bench
 
     class A:
-        steps, warmup = 1, 0
-    monkeypatch.setattr(bench, "oracle_sample", lambda budget, seed_offset=0: (1e-3, "stub sample", 4))
+        steps, warmup = 2, 1
+
+    class Units:  # stands in for the oracle: a fixed amount of work per unit
+        calls = 0
+
+        def __init__(self, seed_offset=0):
+            pass
+
+        def run_one(self):
+            Units.calls += 1
+            return 1e9
+    monkeypatch.setattr(bench, "OracleUnits", Units)
     assert bench.run_reference(A, 1, 2) is None
+    assert Units.calls == 0
     res = bench.run_reference(A, 0, 2)
+    assert Units.calls == 3  # warm-up + timed steps, one unit each
     assert res["impl"] == "reference" and res["cpu_baseline"]["kind"] == "oracle"
-    assert res["e2e"]["h2d_bytes_per_step"] == 0 and res["value"] == 1e-3
+    assert res["e2e"]["h2d_bytes_per_step"] == 0 and res["value"] > 0
+    assert res["e2e"]["value"] == res["value"] == res["cpu_baseline"]["value"]
+    assert "per step" in res["config"]["workload"]
