@@ -22,7 +22,6 @@ fp64 CPU oracle on a bounded sample of the same workload instead.
 import argparse
 import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -324,6 +323,7 @@ def run_gpu(args, rank, world, local):
             "time_ratio": round(lc["layers"]["2048"]["fwd_bwd_ms"] / lc["layers"]["-1"]["fwd_bwd_ms"], 4),
             "note": "window 2048 over full causal on identical inputs: useful FLOPs and measured fwd+bwd time"}
         result["long"] = lc
+        result["fp8"] = run_fp8(cswa, dev, cfg_steps, world, rank, peak_use)
     if rank == 0 and not args.no_decode:
         result["decode"] = run_decode(cswa, dev, args, pk, pk_src)
         result["prefill"] = run_prefill(cswa, dev, args, pk, pk_src)
@@ -372,6 +372,52 @@ def run_config(cswa, dev, name, steps, world, rank, peak):
             "fwd_bwd_tflops": round(world * (ff + fb) / ((f_ms + b_ms) * 1e-3) / 1e12, 1),
             "frac_of_peak": round((ff + fb) / ((f_ms + b_ms) * 1e-3) / 1e12 / peak, 4)}
         del o, lse, dq, dk, dv, ws
+    return out
+
+
+def run_fp8(cswa, dev, steps, world, rank, peak):
+    """The e4m3 forward on the d20 layers (tensorwise-quantized q_hat, k_hat, v), useful
+    TFLOP/s (4 D per visible pair) per window, and the three quantizations timed apart.
+    The peak is the bf16 one: FP8 tensor cores run at twice that, so "of_bf16_peak" above
+    0.5 would already mean more than the fp8 roofline allows for a bf16-shaped pipeline."""
+    c = workloads.CONFIGS["d20"]
+    B, T, Hq, Hkv, D = c["B"], c["T"], c["Hq"], c["Hkv"], c["D"]
+    scale = workloads.default_scale(D)
+    q, k, v, _ = (t.to(dev) for t in workloads.training_inputs(B, T, Hq, Hkv, D, shard_seed(c["seed"], rank)))
+    qh, kh = cswa.attn_rope_qknorm(q, k)
+    desc = torch.empty(3, device=dev, dtype=torch.float32)
+    q8 = torch.empty(qh.shape, device=dev, dtype=torch.uint8)
+    k8 = torch.empty(kh.shape, device=dev, dtype=torch.uint8)
+    v8 = torch.empty(v.shape, device=dev, dtype=torch.uint8)
+
+    def quantize():
+        cswa.attn_quantize_fp8(qh, q8, desc[0:1])
+        cswa.attn_quantize_fp8(kh, k8, desc[1:2])
+        cswa.attn_quantize_fp8(v, v8, desc[2:3])
+    out = {"workload": f"d20 layers: B={B} T={T} Hq=Hkv={Hq} D={D}, e4m3 q_hat/k_hat/v (tensorwise scales), "
+                       "attention forward on the e4m3 tensor cores", "steps": steps, "layers": {}}
+    o = torch.empty_like(qh)
+    lse = torch.empty((B, Hq, T), device=dev, dtype=torch.float32)
+    for W in c["windows"]:
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for i in range(3 + steps):
+            e = ev[i - 3] if i >= 3 else None
+            if e:
+                e[0].record()
+            quantize()
+            if e:
+                e[1].record()
+            cswa.attn_fwd_fp8(q8, k8, v8, desc, W, scale, o=o, lse=lse)
+            if e:
+                e[2].record()
+        torch.cuda.synchronize()
+        assert cswa.attn_get_status() == 0
+        qms = max_over_ranks(statistics.median(e[0].elapsed_time(e[1]) for e in ev), world)
+        fms = max_over_ranks(statistics.median(e[1].elapsed_time(e[2]) for e in ev), world)
+        ff, _ = layer_useful_flops(B, T, Hq, D, W)
+        tf = world * ff / (fms * 1e-3) / 1e12
+        out["layers"][str(W)] = {"window": W, "fwd_ms": round(fms, 4), "fwd_tflops": round(tf, 1),
+                                 "of_bf16_peak": round(tf / world / peak, 4), "quantize_ms": round(qms, 4)}
     return out
 
 
@@ -482,13 +528,11 @@ def run_replicate(cswa, dev, args, pk, pk_src):
     hbm = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     return {"workload": "batch-1 -> 8 KV-cache replication: 20 layers, 1024-token prompt, Hkv=10, D=128, Tmax=2048",
             "us_per_step": round(ms * 1e3, 1), "value": round(gbs, 1), "unit": "GB/s",
-            "l2": "inputs and outputs (1.9 GB) exceed L2", "gpu_launches_per_step": 0,
-            "copies_per_step": 2 * n_layers * (1 + math.ceil(math.log2(N))),
-            "roofline": {"kernel": "attn_kv_replicate (copy-engine copies, doubling rounds)", "bound": "hbm",
+            "l2": "inputs and outputs (1.9 GB) exceed L2", "gpu_launches_per_step": 1,
+            "roofline": {"kernel": "attn_kv_replicate (broadcast kernel: each prompt vector read once, "
+                                   "stored to the N samples)", "bound": "hbm",
                          "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
-                         "traffic": None, "algorithmic_bytes": nbytes,
-                         "note": "the doubling rounds read the copied rows again: the copy engines move "
-                                 "about 2x the algorithmic bytes",
+                         "traffic": ncu_traffic("kv_replicate_kernel"), "algorithmic_bytes": nbytes,
                          "peak_kind": pk_src}}
 
 

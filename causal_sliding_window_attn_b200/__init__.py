@@ -9,6 +9,8 @@ current CUDA stream. The functions carry the C ABI's names (include/cswa_attn.h)
     attn_fwd              attention forward -> (o, lse)
     attn_bwd              attention backward -> (dq, dk, dv)
     attn_block_bwd        the block's backward, prologue included -> (dq, dk, dv) w.r.t. raw q, k
+    attn_quantize_fp8     tensorwise e4m3 quantization -> (codes, dequantization factor)
+    attn_fwd_fp8          attention forward on e4m3 operands -> (o, lse)
     attn_decode           single-token decode against a KV cache -> (o, lse)
     attn_prefill          a chunk of new tokens against a KV cache -> (o, lse)
     attn_layer_window     the window of one layer of a stack (pattern such as "SSSL")
@@ -25,7 +27,8 @@ import torch
 
 __all__ = [
     "AttnError", "lib", "attn_rope_qknorm", "attn_rope_qknorm_bwd", "attn_fwd", "attn_bwd",
-    "attn_bwd_workspace_bytes", "attn_block_bwd", "attn_block_bwd_workspace_bytes", "attn_decode", "attn_decode_workspace_bytes", "attn_prefill", "attn_layer_window",
+    "attn_bwd_workspace_bytes", "attn_block_bwd", "attn_block_bwd_workspace_bytes", "attn_quantize_fp8",
+    "attn_fwd_fp8", "attn_decode", "attn_decode_workspace_bytes", "attn_prefill", "attn_layer_window",
     "layer_windows", "attn_kv_replicate", "attn_get_status", "attn_debug_set_wait_limit",
     "attn_status_string", "LIB_PATH",
 ]
@@ -45,6 +48,9 @@ _SIGS = {
     "attn_bwd": (_i, [_vp] * 9 + [_vp, _sz, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "attn_block_bwd_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "attn_block_bwd": (_i, [_vp] * 12 + [_sz, _i, _i, _i, _i, _i, _i, _f, _f, _f, _vp]),
+    "attn_quantize_fp8_workspace_bytes": (_sz, [ctypes.c_longlong]),
+    "attn_quantize_fp8": (_i, [_vp, ctypes.c_longlong, _vp, _vp, _vp, _sz, _vp]),
+    "attn_fwd_fp8": (_i, [_vp] * 6 + [_i] * 6 + [_f, _vp]),
     "attn_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "attn_decode": (_i, [_vp] * 8 + [_i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "attn_decode_noalloc": (_i, [_vp] * 8 + [_i, _i, _i, _i, _i, _i, _f, _vp]),
@@ -156,6 +162,41 @@ def attn_fwd(q, k, v, window=-1, scale=None, o=None, lse=None, stream=None):
     lse = torch.empty((B, Hq, T), device=q.device, dtype=torch.float32) if lse is None else lse
     _check("attn_fwd", lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, T, Hq, Hkv, D,
                                       int(window), _default_scale(D, scale), _stream(stream)))
+    return o, lse
+
+
+def attn_quantize_fp8(x, x8=None, descale=None, workspace=None, stream=None):
+    """x8 (uint8 e4m3 codes, x's shape), descale (1 float on the device): tensorwise e4m3
+    quantization of the bf16 CUDA tensor x; x ~ x8 * descale."""
+    if not (isinstance(x, torch.Tensor) and x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous()):
+        raise ValueError("x must be a contiguous bf16 CUDA tensor")
+    n = x.numel()
+    x8 = torch.empty(x.shape, device=x.device, dtype=torch.uint8) if x8 is None else x8
+    descale = torch.empty(1, device=x.device, dtype=torch.float32) if descale is None else descale
+    nbytes = int(lib().attn_quantize_fp8_workspace_bytes(n))
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 4), device=x.device, dtype=torch.uint8)
+    _check("attn_quantize_fp8", lib().attn_quantize_fp8(
+        _ptr(x), n, _ptr(x8), _ptr(descale), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+    return x8, descale
+
+
+def attn_fwd_fp8(q8, k8, v8, descale, window=-1, scale=None, o=None, lse=None, stream=None):
+    """o (bf16), lse of attention on e4m3 codes q8 (B,T,Hq,128), k8, v8 (B,T,Hkv,128); descale
+    holds the three dequantization factors (q, k, v) as a float32 CUDA tensor."""
+    for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == torch.uint8 and t.dim() == 4
+                and t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous 4-d uint8 CUDA tensor of e4m3 codes")
+    if not (descale.is_cuda and descale.dtype == torch.float32 and descale.numel() >= 3 and descale.is_contiguous()):
+        raise ValueError("descale must hold 3 float32 values on the device")
+    B, T, Hq, D = q8.shape
+    Hkv = k8.shape[2]
+    o = torch.empty((B, T, Hq, D), device=q8.device, dtype=torch.bfloat16) if o is None else _bf16("o", o)
+    lse = torch.empty((B, Hq, T), device=q8.device, dtype=torch.float32) if lse is None else lse
+    _check("attn_fwd_fp8", lib().attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(descale), _ptr(o), _ptr(lse), B, T,
+                                              Hq, Hkv, D, int(window), _default_scale(D, scale), _stream(stream)))
     return o, lse
 
 

@@ -15,6 +15,8 @@
 #include "decode.cuh"
 #include "fwd.cuh"
 #include "prologue.cuh"
+#include "quant.cuh"
+#include "replicate.cuh"
 
 using namespace cswa;
 
@@ -37,17 +39,19 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// BTHD bf16 tensor as a 4-D tensor map (D, H, T, B); box = 64 x 1 x rows x 1
-// (one rows-high, 128-byte-wide panel), 128-byte swizzle, zero fill past T.
-bool encode_bthd(CUtensorMap* m, const void* base, int B, int T, int H, int D, int rows = 128) {
+// BTHD tensor as a 4-D tensor map (D, H, T, B); box = one rows-high, 128-byte-wide
+// panel (64 bf16 or 128 one-byte elements) x 1 x rows x 1, 128-byte swizzle, zero fill
+// past T. elem = 2 (bf16) or 1 (e4m3 codes).
+bool encode_bthd(CUtensorMap* m, const void* base, int B, int T, int H, int D, int rows = 128, int elem = 2) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-  const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
-  const cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
+  const cuuint64_t strides[3] = {(cuuint64_t)D * elem, (cuuint64_t)H * D * elem, (cuuint64_t)T * H * D * elem};
+  const cuuint32_t box[4] = {(cuuint32_t)(128 / elem), 1, (cuuint32_t)rows, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return fn(m, elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 4,
+            const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -92,6 +96,11 @@ bool set_smem_attrs() {
                                 BwdLayout<D>::kBytes) == cudaSuccess;
   r = r && cudaFuncSetAttribute(attn_fwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 FwdLayout<D>::kBytes) == cudaSuccess;
+  r = r && cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                DqLayout<D>::kBytes) == cudaSuccess;
+  if constexpr (D == 128)
+    r = r && cudaFuncSetAttribute(attn_fwd_kernel<D, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  FwdLayout<D, true>::kBytes) == cudaSuccess;
   if (r) done[dev].store(true, std::memory_order_release);
   return r;
 }
@@ -174,6 +183,32 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, f
   return launched();
 }
 
+// The fp8 forward: e4m3 codes of q, k, v (one byte per element, BTHD) and their three
+// dequantization factors in device memory; D = 128.
+attn_status_t launch_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* descale, void* o, float* lse,
+                             int B, int T, int Hq, int Hkv, int window, float scale, cudaStream_t st) {
+  constexpr int D = 128;
+  CUtensorMap tq, tk, tv;
+  if (!encode_bthd(&tq, q8, B, T, Hq, D, 128, 1) || !encode_bthd(&tk, k8, B, T, Hkv, D, 128, 1) ||
+      !encode_bthd(&tv, v8, B, T, Hkv, D, 128, 1))
+    return ATTN_ERR_LAUNCH;
+  if (!set_smem_attrs<D>()) return ATTN_ERR_LAUNCH;
+  FwdParams p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.T = T;
+  p.Hq = Hq;
+  p.G = Hq / Hkv;
+  p.window = (window >= T) ? -1 : window;
+  p.scale_log2 = scale * kLog2e;
+  p.nq_tiles = tiles128(T);
+  p.n_pairs = (p.nq_tiles + 1) / 2;
+  p.descale = descale;
+  dim3 grid(Hq, B, p.n_pairs);
+  attn_fwd_kernel<D, false, true><<<grid, 384, FwdLayout<D, true>::kBytes, st>>>(tq, tk, tv, tq, tq, p);
+  return launched();
+}
+
 // Chunked prefill: the forward kernel in cache mode. q (B,T,Hq,D) is the chunk. With
 // k_new / v_new (B,T,Hkv,D) the chunk's keys are read from them and copied into the
 // caches (B,Tmax,Hkv,D) by the same launch; without, the caches already hold them at
@@ -218,18 +253,24 @@ attn_status_t launch_prefill(const void* q, void* kc, void* vc, const void* kn, 
 }
 
 // attn_bwd's workspace: the row extensions of the S^T and dP^T MMAs (-lse/scale and
-// -Delta per query row, padded to 128-row tiles), the fp32 dQ accumulator, the work
-// counter, and for the fused block backward the rotary cos/sin table. O(B T Hq D).
+// -Delta per query row, padded to 128-row tiles), the bf16 dS^T tiles of every (key
+// tile, query tile) pair inside the window, the two work counters, and for the block
+// backward the rotary cos/sin table.
 struct BwdWorkspace {
   uint8_t* ext_lse;       // (B, Hq, Tpad / 128) x 512 bytes
   uint8_t* ext_delta;     // (B, Hq, Tpad / 128) x 512 bytes
-  float* dq_acc;          // (B, T, Hq, D) fp32
-  int* counter;           // the main kernel's work-item counter (zeroed by the prep kernel)
+  __nv_bfloat16* ds;      // stored dS^T tiles, 128 x 128 each
+  int* counter;           // [2] work-item counters of the main and dQ kernels (zeroed by the prep kernel)
   float2* rope_cs;        // (T, D/2) (cos, sin), block backward only
+  long long tiles_per_bh;
+  int span;
 };
 int eff_window(int window, int T) { return (window >= T) ? -1 : window; }
-size_t bwd_ws_parts(int B, int T, int Hq, int D, bool rope, BwdWorkspace* w, void* base) {
-  const size_t Tpad = (size_t)tiles128(T) * 128;
+size_t bwd_ws_parts(int B, int T, int Hq, int D, int window, bool rope, BwdWorkspace* w, void* base) {
+  const int nt = tiles128(T);
+  const size_t Tpad = (size_t)nt * 128;
+  const int span = bwd_span(nt, eff_window(window, T));
+  const long long tiles = ds_tiles_before(nt, nt, span);
   uint8_t* p = static_cast<uint8_t*>(base);
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -239,15 +280,17 @@ size_t bwd_ws_parts(int B, int T, int Hq, int D, bool rope, BwdWorkspace* w, voi
   };
   uint8_t* e1 = take((size_t)B * Hq * Tpad * 4);
   uint8_t* e2 = take((size_t)B * Hq * Tpad * 4);
-  uint8_t* acc = take((size_t)B * T * Hq * D * 4);
+  uint8_t* ds = take((size_t)B * Hq * tiles * 32768);
   uint8_t* cnt = take(256);
   uint8_t* cs = rope ? take((size_t)T * (D / 2) * 8) : nullptr;
   if (w) {
     w->ext_lse = e1;
     w->ext_delta = e2;
-    w->dq_acc = reinterpret_cast<float*>(acc);
+    w->ds = reinterpret_cast<__nv_bfloat16*>(ds);
     w->counter = reinterpret_cast<int*>(cnt);
     w->rope_cs = reinterpret_cast<float2*>(cs);
+    w->tiles_per_bh = tiles;
+    w->span = span;
   }
   return off;
 }
@@ -268,7 +311,7 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
   const int Tpad = nt * 128;
   const bool rope = rb.q_raw != nullptr;
   BwdWorkspace w;
-  bwd_ws_parts(B, T, Hq, D, rope, &w, ws);
+  bwd_ws_parts(B, T, Hq, D, window, rope, &w, ws);
   CUtensorMap tq, tk, tv, tdo;
   if (!encode_bthd(&tq, q, B, T, Hq, D) || !encode_bthd(&tk, k, B, T, Hkv, D) ||
       !encode_bthd(&tv, v, B, T, Hkv, D) || !encode_bthd(&tdo, dO, B, T, Hq, D))
@@ -281,7 +324,6 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
     pp.lse = lse;
     pp.ext_lse = w.ext_lse;
     pp.ext_delta = w.ext_delta;
-    pp.dq_acc = w.dq_acc;
     pp.item_counter = w.counter;
     pp.rope_cs = w.rope_cs;
     pp.B = B;
@@ -302,9 +344,10 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
   BwdParams p{};
   p.ext_lse = w.ext_lse;
   p.ext_delta = w.ext_delta;
-  p.dq_acc = w.dq_acc;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.ds = w.ds;
   p.item_counter = w.counter;
   p.T = T;
   p.Tpad = Tpad;
@@ -312,10 +355,12 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
   p.G = Hq / Hkv;
   p.window = eff_window(window, T);
   p.n_tiles = nt;
-  p.span = bwd_span(nt, p.window);
+  p.span = w.span;
+  p.tiles_per_bh = w.tiles_per_bh;
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
   p.k_raw = static_cast<const __nv_bfloat16*>(rb.k_raw);
+  p.q_raw = static_cast<const __nv_bfloat16*>(rb.q_raw);
   p.rope_cs = w.rope_cs;
   p.eps = rb.eps;
   {
@@ -325,22 +370,9 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
     attn_bwd_kernel<D><<<kv_grid, 384, BwdLayout<D>::kBytes, st>>>(tq, tk, tv, tdo, p, (int)kv_items);
   }
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
-  DqParams dp{};
-  dp.dq_acc = w.dq_acc;
-  dp.dq = static_cast<__nv_bfloat16*>(dq);
-  dp.q_raw = static_cast<const __nv_bfloat16*>(rb.q_raw);
-  dp.rope_cs = w.rope_cs;
-  dp.rows = (long long)B * T * Hq;
-  dp.Hq = Hq;
-  dp.T = T;
-  dp.scale = scale;
-  dp.eps = rb.eps;
-  const long long per_block = 2 * (256 / (D / 8));
-  const unsigned grid = (unsigned)((dp.rows + per_block - 1) / per_block);
-  if (rope)
-    attn_bwd_dq_kernel<D, true><<<grid, 256, 0, st>>>(dp);
-  else
-    attn_bwd_dq_kernel<D, false><<<grid, 256, 0, st>>>(dp);
+  const long long items = (long long)nt * Hq * B;
+  const int grid = (int)std::min<long long>(items, sm_count());
+  attn_bwd_dq_kernel<D><<<grid, 256, DqLayout<D>::kBytes, st>>>(tk, p, (int)items);
   return launched();
 }
 
@@ -411,12 +443,14 @@ attn_status_t bwd_common(const void* q, const void* k, const void* v, const void
                !std::isfinite(rb.base) || !(rb.eps >= 0.f) || !std::isfinite(rb.eps)))
     return ATTN_ERR_INVALID_ARG;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
-      ws_bytes < bwd_ws_parts(B, T, Hq, D, rope, nullptr, nullptr))
+      ws_bytes < bwd_ws_parts(B, T, Hq, D, window, rope, nullptr, nullptr))
     return ATTN_ERR_INVALID_ARG;
   if (Hq > 65535 || B > 65535 || tiles128(T) > 65535) return ATTN_ERR_INVALID_ARG;
-  // work items and the prep kernel's blocks are counted in 32 bits
-  if ((long long)tiles128(T) * Hkv * B >= (1ll << 31) ||
-      (long long)B * tiles128(T) * 128 * Hq * (D / 8) / 256 + (long long)T * D / 512 >= (1ll << 31))
+  // stored dS^T tile rows, the dQ kernel's work items and the prep kernel's blocks are
+  // counted in 32 bits
+  const int nt = tiles128(T);
+  if ((long long)B * Hq * ds_tiles_before(nt, nt, bwd_span(nt, eff_window(window, T))) * 128 >= (1ll << 31) ||
+      (long long)B * nt * 128 * Hq * (D / 8) / 256 + (long long)T * D / 512 >= (1ll << 31))
     return ATTN_ERR_UNSUPPORTED;
   cudaStream_t st = as_stream(stream);
   return D == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, workspace, B, T, Hq, Hkv, window, scale, rb, st)
@@ -452,14 +486,12 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
 
 size_t attn_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int window) {
   if (!dims_ok(B, T, Hq, Hkv) || (D != 64 && D != 128)) return 0;
-  (void)window;
-  return bwd_ws_parts(B, T, Hq, D, false, nullptr, nullptr);
+  return bwd_ws_parts(B, T, Hq, D, window, false, nullptr, nullptr);
 }
 
 size_t attn_block_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int window) {
   if (!dims_ok(B, T, Hq, Hkv) || (D != 64 && D != 128)) return 0;
-  (void)window;
-  return bwd_ws_parts(B, T, Hq, D, true, nullptr, nullptr);
+  return bwd_ws_parts(B, T, Hq, D, window, true, nullptr, nullptr);
 }
 
 
@@ -577,6 +609,84 @@ attn_status_t attn_prefill(const void* q, void* kcache, void* vcache, const void
              ? launch_prefill<64>(q, kcache, vcache, k_new, v_new, pos, o, lse, B, T, Tmax, Hq, Hkv, window, scale, st)
              : launch_prefill<128>(q, kcache, vcache, k_new, v_new, pos, o, lse, B, T, Tmax, Hq, Hkv, window, scale,
                                    st);
+}
+
+size_t attn_quantize_fp8_workspace_bytes(long long n) {
+  if (n < 8 || n % 8) return 0;
+  return (size_t)kQuantMaxBlocks * 4;
+}
+
+attn_status_t attn_quantize_fp8(const void* x, long long n, void* x8, float* descale, void* workspace,
+                                size_t ws_bytes, void* stream) {
+  if (n < 8 || n % 8 || !x || !x8 || !descale || !workspace || !aligned16(x) ||
+      (reinterpret_cast<uintptr_t>(x8) & 7u) || (reinterpret_cast<uintptr_t>(descale) & 3u) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 3u) || ws_bytes < attn_quantize_fp8_workspace_bytes(n))
+    return ATTN_ERR_INVALID_ARG;
+  const long long n8 = n / 8;
+  const int blocks = (int)std::min<long long>((n8 + 255) / 256, kQuantMaxBlocks);
+  cudaStream_t st = as_stream(stream);
+  float* part = static_cast<float*>(workspace);
+  quant_amax_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint4*>(x), n8, part);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+  quant_e4m3_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint4*>(x), n8, part, blocks, static_cast<uint2*>(x8),
+                                            descale);
+  return launched();
+}
+
+attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* descale, void* o, float* lse,
+                           int B, int T, int Hq, int Hkv, int D, int window, float scale, void* stream) {
+  if (!dims_ok(B, T, Hq, Hkv) || !scale_ok(scale)) return ATTN_ERR_INVALID_ARG;
+  if (D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!q8 || !k8 || !v8 || !descale || !o || !lse || !aligned16(q8) || !aligned16(k8) || !aligned16(v8) ||
+      !aligned16(o) || !aligned16(lse) || (reinterpret_cast<uintptr_t>(descale) & 3u))
+    return ATTN_ERR_INVALID_ARG;
+  if (B > 65535 || Hq > 65535) return ATTN_ERR_INVALID_ARG;
+  return launch_fwd_fp8(q8, k8, v8, descale, o, lse, B, T, Hq, Hkv, window, scale, as_stream(stream));
+}
+
+attn_status_t attn_kv_replicate(const void* k_src, const void* v_src, void* k_dst, void* v_dst, int n_layers,
+                                int rows, int Tmax_src, int N, int Tmax, int Hkv, int D, void* stream) {
+  if (!k_src || !v_src || !k_dst || !v_dst || n_layers < 1 || rows < 0 || Tmax_src < 1 || N < 1 || Tmax < 1 ||
+      Hkv < 1 || D < 1 || rows > Tmax_src || rows > Tmax)
+    return ATTN_ERR_INVALID_ARG;
+  const size_t row_bytes = (size_t)Hkv * D * 2;
+  const size_t src_layer = (size_t)Tmax_src * row_bytes;  // batch-1 source: layer stride
+  const size_t dst_sample = (size_t)Tmax * row_bytes;     // destination: sample stride ...
+  const size_t dst_layer = (size_t)N * dst_sample;        // ... and layer stride
+  const size_t src_bytes = (size_t)n_layers * src_layer, dst_bytes = (size_t)n_layers * dst_layer;
+  auto disjoint = [](const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x + na <= y || y + nb <= x;
+  };
+  if (!disjoint(k_dst, dst_bytes, v_dst, dst_bytes) || !disjoint(k_dst, dst_bytes, k_src, src_bytes) ||
+      !disjoint(k_dst, dst_bytes, v_src, src_bytes) || !disjoint(v_dst, dst_bytes, k_src, src_bytes) ||
+      !disjoint(v_dst, dst_bytes, v_src, src_bytes))
+    return ATTN_ERR_INVALID_ARG;
+  if (rows == 0) return ATTN_OK;
+  // the widest vector every pointer and stride allows
+  const uintptr_t align = reinterpret_cast<uintptr_t>(k_src) | reinterpret_cast<uintptr_t>(v_src) |
+                          reinterpret_cast<uintptr_t>(k_dst) | reinterpret_cast<uintptr_t>(v_dst) | row_bytes;
+  const int vec = (align % 16 == 0) ? 16 : (align % 4 == 0) ? 4 : 2;
+  ReplicateParams p{};
+  p.src[0] = static_cast<const uint8_t*>(k_src);
+  p.src[1] = static_cast<const uint8_t*>(v_src);
+  p.dst[0] = static_cast<uint8_t*>(k_dst);
+  p.dst[1] = static_cast<uint8_t*>(v_dst);
+  p.vec_per_layer = (long long)((size_t)rows * row_bytes / vec);
+  p.src_layer = (long long)(src_layer / vec);
+  p.dst_layer = (long long)(dst_layer / vec);
+  p.dst_sample = (long long)(dst_sample / vec);
+  p.total = 2 * (long long)n_layers * p.vec_per_layer;
+  p.N = N;
+  const long long blocks = std::min<long long>((p.total + 255) / 256, (long long)sm_count() * 8);
+  cudaStream_t st = as_stream(stream);
+  if (vec == 16)
+    kv_replicate_kernel<uint4><<<(unsigned)blocks, 256, 0, st>>>(p);
+  else if (vec == 4)
+    kv_replicate_kernel<uint32_t><<<(unsigned)blocks, 256, 0, st>>>(p);
+  else
+    kv_replicate_kernel<uint16_t><<<(unsigned)blocks, 256, 0, st>>>(p);
+  return launched();
 }
 
 attn_status_t attn_get_status(void* stream) {

@@ -115,8 +115,11 @@ __device__ __forceinline__ unsigned decode_arrive(unsigned long long* cnt, unsig
   return 0u;
 }
 
+// resident CTAs per SM the register allocation must allow (65536 / (128 x registers))
+constexpr int decode_min_blocks(int gmax) { return gmax == 1 ? 9 : gmax == 2 ? 7 : gmax == 4 ? 5 : 3; }
+
 template <int D, int GMAX>
-__global__ void __launch_bounds__(128) decode_chunk_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(128, decode_min_blocks(GMAX)) decode_chunk_kernel(const DecodeParams p) {
   constexpr int LK = D / 8;          // lanes per key row
   constexpr int KPP = 128 / LK;      // key rows per pass
   constexpr int PASSES = kDecodeChunk / KPP;
@@ -168,10 +171,12 @@ __global__ void __launch_bounds__(128) decode_chunk_kernel(const DecodeParams p)
     return ld_stream(cache + cache_off + u * pass_stride);
   };
 
-  // the group's query heads in sub-groups of GMAX; a sub-group after the first reads
-  // the chunk's rows again, from L2
-  for (int g0 = 0; g0 < G; g0 += GMAX) {
-    const int gn = min(GMAX, G - g0);
+  // the group's query heads in sub-groups of GMAX (only the widest instantiation sees
+  // groups larger than GMAX); a sub-group after the first reads the chunk's rows
+  // again, from L2
+  constexpr bool kWide = (GMAX == 8);
+  for (int g0 = 0; g0 < (kWide ? G : 1); g0 += GMAX) {
+    const int gn = kWide ? min(GMAX, G - g0) : G;
     uint32_t qv[GMAX][4];
 #pragma unroll
     for (int g = 0; g < GMAX; ++g) {

@@ -63,14 +63,17 @@ struct FwdParams {
   const uint4* vn;
   uint4* kc;           // the caches (B, Tmax, Hkv, D)
   uint4* vc;
+  // fp8 forward only: the dequantization factors of q, k, v (device memory, 3 floats)
+  const float* descale;
 };
 
 constexpr int kMaxRankedItems = 256;  // prefill items ranked by weight (more: pair order)
 
-template <int D>
+template <int D, bool kFp8 = false>
 struct FwdLayout {
-  static constexpr int kTile = 128 * D * 2;  // bytes of one 128-row bf16 tile
-  static constexpr int kPanels = D / 64;     // 128-byte-wide panels per tile
+  static constexpr int kElem = kFp8 ? 1 : 2;  // bytes per element: e4m3 or bf16
+  static constexpr int kTile = 128 * D * kElem;  // bytes of one 128-row tile
+  static constexpr int kPanels = D * kElem / 128;  // 128-byte-wide panels per tile
   static constexpr int kQ0 = 0, kQ1 = kTile, kK0 = 2 * kTile, kV0 = 4 * kTile;
   static constexpr int kBar = 6 * kTile;
   static constexpr int kBytes = kBar + 256 + 1024;  // + barriers + alignment slack
@@ -79,12 +82,14 @@ struct FwdLayout {
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-template <int D, bool kCache = false>
+template <int D, bool kCache = false, bool kFp8 = false>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kn,
                     const __grid_constant__ CUtensorMap tm_vn, const FwdParams p) {
-  using L = FwdLayout<D>;
+  static_assert(!kFp8 || (D == 128 && !kCache), "the fp8 forward takes D = 128, training layout");
+  using L = FwdLayout<D, kFp8>;
+  constexpr int kPanelElems = 128 / L::kElem;  // elements across one 128-byte panel
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
@@ -210,8 +215,8 @@ __global__ void __launch_bounds__(384, 1)
       for (int s = 0; s < 2; ++s)
         if (has[s])
           for (int pn = 0; pn < L::kPanels; ++pn)
-            tma_load_4d(smem + (s ? L::kQ1 : L::kQ0) + pn * 16384, &tm_q, q_full, pn * 64, h, qt[s] * 128 - shift,
-                        b);
+            tma_load_4d(smem + (s ? L::kQ1 : L::kQ0) + pn * 16384, &tm_q, q_full, pn * kPanelElems, h,
+                        qt[s] * 128 - shift, b);
       // K and V stages are released separately (K once the S products have read it, V
       // once the PV products have), so K of the next tile loads a whole tile ahead
       int n = 0, last_k[2] = {-1, -1}, last_v[2] = {-1, -1};
@@ -226,12 +231,12 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait(&k_empty[st], ph ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(&k_full[st], L::kTile);
         for (int pn = 0; pn < L::kPanels; ++pn)
-          tma_load_4d(smem + L::kK0 + st * L::kTile + pn * 16384, mk, &k_full[st], pn * 64, hk, row, b);
+          tma_load_4d(smem + L::kK0 + st * L::kTile + pn * 16384, mk, &k_full[st], pn * kPanelElems, hk, row, b);
         last_k[st] = n;
         if (!mbar_wait(&v_empty[st], ph ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(&v_full[st], L::kTile);
         for (int pn = 0; pn < L::kPanels; ++pn)
-          tma_load_4d(smem + L::kV0 + st * L::kTile + pn * 16384, mv, &v_full[st], pn * 64, hk, row, b);
+          tma_load_4d(smem + L::kV0 + st * L::kTile + pn * 16384, mv, &v_full[st], pn * kPanelElems, hk, row, b);
         last_v[st] = n;
       }
       // never leave with copies in flight: wait (bounded) for the last load of each
@@ -250,8 +255,11 @@ __global__ void __launch_bounds__(384, 1)
     // of this one, never overwrites P_s before PV_s has read it, and the softmax warps,
     // which see S_s only through a commit issued after PV_s, find O_s stable.
     const uint32_t leader = elect_one();
-    constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
-    constexpr uint32_t idO = idesc_bf16(128, D, false, true);
+    constexpr uint32_t idS = kFp8 ? idesc_e4m3(128, 128, false, false) : idesc_bf16(128, 128, false, false);
+    constexpr uint32_t idO = kFp8 ? idesc_e4m3(128, D, false, true) : idesc_bf16(128, D, false, true);
+    // a K step is 32 bytes of a row: 16 bf16 or 32 e4m3 elements
+    constexpr int kKSteps = D * L::kElem / 32;       // steps of S = Q K^T
+    constexpr int kPVSteps = 128 * L::kElem / 32;    // steps of O += P V (128 keys)
     // descriptors built once; each MMA adds (byte offset >> 4) to the start field
     const uint64_t dQ0 = sdesc_sw128(sbase + L::kQ0, 16, 1024), dQ1 = sdesc_sw128(sbase + L::kQ1, 16, 1024);
     const uint64_t dK0 = sdesc_sw128(sbase + L::kK0, 16, 1024);
@@ -263,9 +271,12 @@ __global__ void __launch_bounds__(384, 1)
     auto active = [&](int s, int t) { return has[s] && lo[s] <= t && t <= hi[s]; };
     auto issue_S = [&](int s, int st) {
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
+      for (int kk = 0; kk < kKSteps; ++kk) {
         const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-        mma_ss(tS(s), (s ? dQ1 : dQ0) + (off >> 4), dK0 + ((st * L::kTile + off) >> 4), idS, kk > 0, leader);
+        if constexpr (kFp8)
+          mma_ss_f8(tS(s), (s ? dQ1 : dQ0) + (off >> 4), dK0 + ((st * L::kTile + off) >> 4), idS, kk > 0, leader);
+        else
+          mma_ss(tS(s), (s ? dQ1 : dQ0) + (off >> 4), dK0 + ((st * L::kTile + off) >> 4), idS, kk > 0, leader);
       }
       mma_commit(&s_full[s], leader);
     };
@@ -292,16 +303,22 @@ __global__ void __launch_bounds__(384, 1)
       for (int s = 0; s < 2; ++s) {
         if (active(s, t)) {
           // PV_s chunk by chunk as the softmax warps publish P_s: chunk c holds keys
-          // 32c .. 32c+31 (K steps 2c, 2c+1) as bf16 pairs in columns 16c .. 16c+15
+          // 32c .. 32c+31, as bf16 pairs in columns 16c .. 16c+15 (K steps 2c, 2c+1) or
+          // as e4m3 quadruples in columns 8c .. 8c+7 (K step c); a K step reads 8 columns
+          // of P and 32 bytes x its keys of V
+          constexpr int kPer = kPVSteps / 4;
           for (int c = 0; c < 4; ++c) {
             if (!(ok = wait_all(&p_chunk[4 * s + c], cnt[s] & 1))) break;
             if (tracer && c == 0) CSWA_MARK(0, n, 2 + 3 * s);
             tc_fence_after();
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int kk = 2 * c + u;
-              mma_ts(tO(s), tS(s) + kk * 8, dV0 + ((st * L::kTile + kk * 2048) >> 4), idO, (cnt[s] > 0 || kk > 0),
-                     leader);
+            for (int u = 0; u < kPer; ++u) {
+              const int kk = kPer * c + u;
+              const uint64_t bv = dV0 + ((st * L::kTile + kk * (32 / L::kElem) * 128) >> 4);
+              if constexpr (kFp8)
+                mma_ts_f8(tO(s), tS(s) + kk * 8, bv, idO, (cnt[s] > 0 || kk > 0), leader);
+              else
+                mma_ts(tO(s), tS(s) + kk * 8, bv, idO, (cnt[s] > 0 || kk > 0), leader);
             }
           }
           if (!ok) break;
@@ -378,7 +395,12 @@ __global__ void __launch_bounds__(384, 1)
     if (my_qt < p.nq_tiles) {
       const int q0 = e0 + my_qt * 128;  // position of the tile's first row
       const int i = q0 + row;
-      const float sl2 = p.scale_log2;
+      // fp8: the scores carry the quantization scales of q and k
+      const float sl2 = kFp8 ? p.scale_log2 * (p.descale[0] * p.descale[1]) : p.scale_log2;
+      // fp8: P is scaled by 2^8 before its e4m3 rounding (the exponent gets + 8) and must
+      // stay below 448, so the running max moves whenever it grows
+      constexpr float kThreshold = kFp8 ? 0.f : kRescaleThreshold;
+      constexpr float kPBias = kFp8 ? 8.f : 0.f;
       float m_run = -INFINITY, l_run = 0.f;
       int cnt = 0;
       bool ok = true;
@@ -425,7 +447,7 @@ __global__ void __launch_bounds__(384, 1)
         float factor = 1.f;
         if (cnt == 0) {
           m_run = m_tile;
-        } else if (m_tile > m_run + kRescaleThreshold) {
+        } else if (m_tile > m_run + kThreshold) {
           factor = ex2_approx(m_run - m_tile);
           m_run = m_tile;
           l_run *= factor;
@@ -451,19 +473,36 @@ __global__ void __launch_bounds__(384, 1)
         // p = exp2(s * scale * log2e - m), two columns per packed FMA; row sum in packed adds.
         // Published in four chunks of 32 keys, each on its own barrier: chunk c's bf16 pairs
         // land in columns 16c .. 16c+15, whose fp32 S (keys < 32c + 32) is already in registers
-        const float2 sl2v = make_float2(sl2, sl2), nm = make_float2(-m_use, -m_use);
+        const float2 sl2v = make_float2(sl2, sl2), nm = make_float2(kPBias - m_use, kPBias - m_use);
         float2 ls4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
+          if constexpr (kFp8) {
+            // e4m3 quadruples of keys 32ch .. 32ch+31 into columns 8ch .. 8ch+7, whose fp32
+            // S (keys < 8ch + 8) is already in registers
 #pragma unroll
-          for (int c = 16 * ch; c < 16 * ch + 16; ++c) {
-            const float2 x =
-                __ffma2_rn(make_float2(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), sl2v, nm);
-            const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            ls4[c & 3] = __fadd2_rn(ls4[c & 3], pp);
-            r[c] = pack_bf16x2(pp.x, pp.y);
+            for (int c = 8 * ch; c < 8 * ch + 8; ++c) {
+              const float2 x0 =
+                  __ffma2_rn(make_float2(__uint_as_float(r[4 * c]), __uint_as_float(r[4 * c + 1])), sl2v, nm);
+              const float2 x1 =
+                  __ffma2_rn(make_float2(__uint_as_float(r[4 * c + 2]), __uint_as_float(r[4 * c + 3])), sl2v, nm);
+              const float2 p0 = make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
+              const float2 p1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
+              ls4[c & 3] = __fadd2_rn(ls4[c & 3], __fadd2_rn(p0, p1));
+              r[c] = pack_e4m3x4(p0.x, p0.y, p1.x, p1.y);
+            }
+            tmem_st8(tSs + 8 * ch, *reinterpret_cast<uint32_t(*)[8]>(&r[8 * ch]));
+          } else {
+#pragma unroll
+            for (int c = 16 * ch; c < 16 * ch + 16; ++c) {
+              const float2 x =
+                  __ffma2_rn(make_float2(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), sl2v, nm);
+              const float2 pp = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+              ls4[c & 3] = __fadd2_rn(ls4[c & 3], pp);
+              r[c] = pack_bf16x2(pp.x, pp.y);
+            }
+            tmem_st16(tSs + 16 * ch, *reinterpret_cast<uint32_t(*)[16]>(&r[16 * ch]));
           }
-          tmem_st16(tSs + 16 * ch, *reinterpret_cast<uint32_t(*)[16]>(&r[16 * ch]));
           tmem_st_wait();
           tc_fence_before();
           mbar_arrive(&p_chunk[4 * s + ch]);
@@ -479,7 +518,8 @@ __global__ void __launch_bounds__(384, 1)
         // tcgen05.ld is warp-collective: every lane loads, only rows of [0, T) store
         const int cr = my_qt * 128 - shift + row;  // output row (chunk row in kCache)
         const bool store = (cr < p.T) && (!kCache || cr >= 0);
-        const float inv_l = 1.f / l_run;
+        // fp8: O and l both carry P's 2^8, and O the quantization scale of v
+        const float inv_l = (kFp8 ? p.descale[2] : 1.f) / l_run;
         __nv_bfloat16* dst = p.o + ((size_t)((size_t)b * p.T + cr) * p.Hq + h) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -498,7 +538,7 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         if (store && (!kCache || p.lse))
-          p.lse[((size_t)b * p.Hq + h) * p.T + cr] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+          p.lse[((size_t)b * p.Hq + h) * p.T + cr] = (m_run + __log2f(l_run) - kPBias) * 0.69314718055994531f;
       }
     }
   }

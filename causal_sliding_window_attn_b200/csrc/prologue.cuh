@@ -9,9 +9,9 @@
 // with p = t + pos[b] (pos may be null). Backward, with g = rotation of dy by -phi:
 //   dx = (g - xh (g . xh) / D) / r.
 //
-// HBM-bound elementwise work: D/8 lanes own one row, each holding both members
-// of its rotation pairs (two 8-byte loads per operand). The angles are computed
-// once per position and shared by all its head rows.
+// HBM-bound elementwise work: D / (2 kRopeVec) lanes own one row, each holding both
+// members of its rotation pairs (one load of kRopeVec values from each half per
+// operand). The angles are computed once per position and shared by all its head rows.
 #pragma once
 #include "ptx.cuh"
 
@@ -36,17 +36,48 @@ struct RopeParams {
 // for any 32-bit position); its top 32 bits, read as signed, give the reduced angle
 // in [-pi, pi). A block first issues the loads of its first rows, then builds one
 // cos/sin table per position in shared memory while they are in flight, and streams
-// the rows: D/8 lanes per row, lane l owning elements 4l..4l+3 of each half (so a
-// rotation pair never leaves its lane), kBatch rows per thread in flight.
+// the rows: D / (2 kRopeVec) lanes per row, lane l owning elements kRopeVec l ..
+// kRopeVec (l + 1) - 1 of each half (so a rotation pair never leaves its lane), kBatch
+// rows per thread in flight.
 constexpr int kPosPerBlock = 8;
+// elements of each half a lane owns: 4 (two 8-byte loads per row and operand)
+constexpr int kRopeVec = 4;
+
+// kE consecutive bf16 values (8 or 16 bytes) as floats
+template <int kE>
+__device__ __forceinline__ void load_bf16(const __nv_bfloat16* src, bool active, float (&f)[kE]) {
+  uint32_t w[kE / 2];
+  if constexpr (kE == 4) {
+    const uint2 v = active ? *reinterpret_cast<const uint2*>(src) : make_uint2(0, 0);
+    w[0] = v.x, w[1] = v.y;
+  } else {
+    const uint4 v = active ? *reinterpret_cast<const uint4*>(src) : make_uint4(0, 0, 0, 0);
+    w[0] = v.x, w[1] = v.y, w[2] = v.z, w[3] = v.w;
+  }
+#pragma unroll
+  for (int u = 0; u < kE / 2; ++u) {
+    f[2 * u] = __uint_as_float(w[u] << 16);
+    f[2 * u + 1] = __uint_as_float(w[u] & 0xffff0000u);
+  }
+}
+template <int kE>
+__device__ __forceinline__ void store_bf16(__nv_bfloat16* dst, const float (&f)[kE]) {
+  if constexpr (kE == 4) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
+  } else {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                                pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+  }
+}
 
 template <int D, bool kBwd>
 __global__ void __launch_bounds__(256, 4) rope_qknorm_kernel(const __grid_constant__ RopeParams p) {
-  constexpr int kLanesPerRow = D / 8;
+  constexpr int kE = kRopeVec;
+  constexpr int kLanesPerRow = D / (2 * kE);
   constexpr int kHalf = D / 2;
   constexpr int kRowsPerRound = 256 / kLanesPerRow;
-  // rows per thread in flight: 4 (8 loads of 8 bytes); the backward, with twice the
-  // loads per row and more live values, keeps 2 so that 4 blocks fit per SM
+  // rows per thread in flight: the forward keeps 4, the backward (twice the loads per
+  // row, more live values) 2, so that 4 blocks fit per SM
   constexpr int kBatch = kBwd ? 2 : 4;
   __shared__ float4 cs4[kPosPerBlock][kHalf / 2];  // (cos_j, sin_j, cos_j+1, sin_j+1)
 
@@ -59,7 +90,7 @@ __global__ void __launch_bounds__(256, 4) rope_qknorm_kernel(const __grid_consta
   const int rows_all = rows_q + rows_k;
   const int lr = threadIdx.x % kLanesPerRow;
   const int row0 = threadIdx.x / kLanesPerRow;
-  const int j0 = lr * 4;  // elements j0..j0+3 and kHalf + j0..kHalf + j0+3
+  const int j0 = lr * kE;  // elements j0..j0+kE-1 and kHalf + j0..
   const float inv_hq = Hq ? 1.f / (float)Hq : 0.f, inv_hk = Hk ? 1.f / (float)Hk : 0.f;
   // every thread runs the same number of rounds so the row shuffles stay warp-uniform
   const int rounds = (kPosPerBlock * (Hq + Hk) + kRowsPerRound - 1) / kRowsPerRound;
@@ -75,7 +106,7 @@ __global__ void __launch_bounds__(256, 4) rope_qknorm_kernel(const __grid_consta
   };
 
   for (int rd0 = 0; rd0 < rounds; rd0 += kBatch) {
-    uint2 xa[kBatch], xb[kBatch], ga[kBatch], gb[kBatch];
+    float xa[kBatch][kE], xb[kBatch][kE], ga[kBatch][kE], gb[kBatch][kE];
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int row = (rd0 + u) * kRowsPerRound + row0;
@@ -83,11 +114,11 @@ __global__ void __launch_bounds__(256, 4) rope_qknorm_kernel(const __grid_consta
       size_t off;
       locate(row, seg, off, pi);
       const bool active = row < rows_all;
-      xa[u] = active ? *reinterpret_cast<const uint2*>(p.x[seg] + off) : make_uint2(0, 0);
-      xb[u] = active ? *reinterpret_cast<const uint2*>(p.x[seg] + off + kHalf) : make_uint2(0, 0);
+      load_bf16<kE>(p.x[seg] + off, active, xa[u]);
+      load_bf16<kE>(p.x[seg] + off + kHalf, active, xb[u]);
       if (kBwd) {
-        ga[u] = active ? *reinterpret_cast<const uint2*>(p.dy[seg] + off) : make_uint2(0, 0);
-        gb[u] = active ? *reinterpret_cast<const uint2*>(p.dy[seg] + off + kHalf) : make_uint2(0, 0);
+        load_bf16<kE>(p.dy[seg] + off, active, ga[u]);
+        load_bf16<kE>(p.dy[seg] + off + kHalf, active, gb[u]);
       }
     }
     if (rd0 == 0) {
@@ -116,48 +147,36 @@ __global__ void __launch_bounds__(256, 4) rope_qknorm_kernel(const __grid_consta
       locate(row, seg, off, pi);
       const bool active = row < rows_all;
       if (!active) pi = 0;
-      // a[i] = element j0 + i, b[i] = element kHalf + j0 + i
-      float a[4], bq[4];
-      {
-        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&xa[u]);
-        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&xb[u]);
-#pragma unroll
-        for (int v = 0; v < 2; ++v) {
-          const float2 fa = __bfloat1622float2(a2[v]), fb = __bfloat1622float2(b2[v]);
-          a[2 * v] = fa.x, a[2 * v + 1] = fa.y, bq[2 * v] = fb.x, bq[2 * v + 1] = fb.y;
-        }
-      }
+      // a[i] = element j0 + i, bq[i] = element kHalf + j0 + i
+      const float* a = xa[u];
+      const float* bq = xb[u];
       float ss = 0.f;
 #pragma unroll
-      for (int v = 0; v < 4; ++v) ss = fmaf(a[v], a[v], fmaf(bq[v], bq[v], ss));
+      for (int v = 0; v < kE; ++v) ss = fmaf(a[v], a[v], fmaf(bq[v], bq[v], ss));
 #pragma unroll
       for (int o = kLanesPerRow / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
       const float inv_r = rsqrtf(ss * (1.f / D) + p.eps);
-      const float4 t01 = cs4[pi][j0 / 2], t23 = cs4[pi][j0 / 2 + 1];
-      const float c[4] = {t01.x, t01.z, t23.x, t23.z}, s[4] = {t01.y, t01.w, t23.y, t23.w};
-      float oa[4], ob[4];
+      float c[kE], s[kE];
+#pragma unroll
+      for (int v = 0; v < kE / 2; ++v) {
+        const float4 t = cs4[pi][j0 / 2 + v];
+        c[2 * v] = t.x, s[2 * v] = t.y, c[2 * v + 1] = t.z, s[2 * v + 1] = t.w;
+      }
+      float oa[kE], ob[kE];
       if (!kBwd) {
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
+        for (int v = 0; v < kE; ++v) {
           const float xa_ = a[v] * inv_r, xb_ = bq[v] * inv_r;
           oa[v] = fmaf(-xb_, s[v], xa_ * c[v]);
           ob[v] = fmaf(xa_, s[v], xb_ * c[v]);
         }
       } else {
         // g = rotation of dy by -phi
-        float ga_[4], gb_[4];
-        {
-          const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&ga[u]);
-          const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&gb[u]);
+        const float* ga_ = ga[u];
+        const float* gb_ = gb[u];
+        float gra[kE], grb[kE], dot = 0.f;
 #pragma unroll
-          for (int v = 0; v < 2; ++v) {
-            const float2 fa = __bfloat1622float2(a2[v]), fb = __bfloat1622float2(b2[v]);
-            ga_[2 * v] = fa.x, ga_[2 * v + 1] = fa.y, gb_[2 * v] = fb.x, gb_[2 * v + 1] = fb.y;
-          }
-        }
-        float gra[4], grb[4], dot = 0.f;
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
+        for (int v = 0; v < kE; ++v) {
           gra[v] = fmaf(gb_[v], s[v], ga_[v] * c[v]);
           grb[v] = fmaf(-ga_[v], s[v], gb_[v] * c[v]);
           dot = fmaf(gra[v], a[v] * inv_r, fmaf(grb[v], bq[v] * inv_r, dot));
@@ -166,15 +185,14 @@ __global__ void __launch_bounds__(256, 4) rope_qknorm_kernel(const __grid_consta
         for (int o = kLanesPerRow / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
         const float proj = dot * (1.f / D);
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
+        for (int v = 0; v < kE; ++v) {
           oa[v] = (gra[v] - a[v] * inv_r * proj) * inv_r;
           ob[v] = (grb[v] - bq[v] * inv_r * proj) * inv_r;
         }
       }
       if (active) {
-        *reinterpret_cast<uint2*>(p.y[seg] + off) = make_uint2(pack_bf16x2(oa[0], oa[1]), pack_bf16x2(oa[2], oa[3]));
-        *reinterpret_cast<uint2*>(p.y[seg] + off + kHalf) =
-            make_uint2(pack_bf16x2(ob[0], ob[1]), pack_bf16x2(ob[2], ob[3]));
+        store_bf16<kE>(p.y[seg] + off, oa);
+        store_bf16<kE>(p.y[seg] + off + kHalf, ob);
       }
     }
   }

@@ -82,12 +82,13 @@ attn_status_t attn_rope_qknorm_bwd(const void* q, const void* k, const void* dq_
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T,
                        int Hq, int Hkv, int D, int window, float scale, void* stream);
 
-/* Bytes of workspace attn_bwd needs: per query row, -lse/scale and -Delta_i =
- * -(dO_i . o_i) as bf16 hi/lo pairs (2 x B*Hq*Tpad*4 bytes, Tpad = T rounded up to a
- * multiple of 128); the fp32 dQ accumulator (B*T*Hq*D*4 bytes); and 256 bytes for
- * the main kernel's work counter, each part rounded up to 256 bytes. O(B*T*Hq*D): it
- * does not grow with the window. The window argument is accepted for symmetry and
- * does not change the size. Nothing in it needs to be initialised. */
+/* Bytes of workspace attn_bwd needs for this window: per query row, -lse/scale and
+ * -Delta_i = -(dO_i . o_i) as bf16 hi/lo pairs (2 x B*Hq*Tpad*4 bytes, Tpad = T
+ * rounded up to a multiple of 128); the bf16 dS^T tiles (128 x 128) of every (query
+ * tile, key tile) pair inside the causal window, kept between the main backward
+ * kernel and the dQ kernel: about B*Hq*T*min(T, W+128)*2 bytes for window W
+ * (B*Hq*T^2 without a window); and 256 bytes for the work counters; each part
+ * rounded up to 256 bytes. Nothing in it needs to be initialised. */
 size_t attn_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int window);
 
 /*
@@ -99,9 +100,9 @@ size_t attn_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int window
  * them. Outputs dq (B,T,Hq,D), dk, dv (B,T,Hkv,D) bf16, fully overwritten.
  * workspace: device memory, 256-byte aligned, of ws_bytes >=
  * attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, window). Three launches: a per-row
- * preparation, the tensor-core main kernel (dK and dV complete per key tile; dQ
- * partials added into the workspace's fp32 accumulator), and dq = scale x the
- * accumulator as bf16. Sizes whose work items would not fit 32-bit counters return
+ * preparation, the tensor-core main kernel (dK and dV complete per key tile, the
+ * dS^T tiles stored to the workspace) and the tensor-core dQ kernel (dQ = scale dS K
+ * from the stored tiles). Calls whose stored dS^T tiles would exceed 2^31 rows return
  * ATTN_ERR_UNSUPPORTED.
  */
 attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
@@ -131,6 +132,40 @@ attn_status_t attn_block_bwd(const void* q, const void* k, const void* q_hat, co
                              const void* o, const void* dO, const float* lse, void* dq, void* dk, void* dv,
                              void* workspace, size_t ws_bytes, int B, int T, int Hq, int Hkv, int D, int window,
                              float scale, float rope_base, float eps, void* stream);
+
+/* Bytes of workspace attn_quantize_fp8 needs for n elements (per-block maxima). */
+size_t attn_quantize_fp8_workspace_bytes(long long n);
+
+/*
+ * attn_quantize_fp8 -- tensorwise dynamic scaling of a bf16 tensor to float8 e4m3
+ * (nanochat Admin & Developer Guide, 5 "Precision: Explicit dtype & FP8": one
+ * scale per tensor from its absolute maximum, forward tensors in e4m3):
+ *   amax = max |x|,  s = 448 / amax (1 when amax = 0),  x8 = e4m3(x * s)
+ * with s and x * s computed in fp32 and the rounding to nearest even, saturating
+ * at +-448. Writes the n one-byte codes to x8 and the dequantization factor
+ * amax / 448 (x ~ x8 * descale) to *descale, both device memory.
+ *   x: n bf16 values, 16-byte aligned, n a multiple of 8; x8: n bytes, 8-byte
+ *   aligned; descale: one float, device memory, 4-byte aligned.
+ *   workspace: >= attn_quantize_fp8_workspace_bytes(n) bytes of device memory.
+ * Two launches (maxima, then codes); nothing else is read or written.
+ */
+attn_status_t attn_quantize_fp8(const void* x, long long n, void* x8, float* descale, void* workspace,
+                                size_t ws_bytes, void* stream);
+
+/*
+ * attn_fwd_fp8 -- attn_fwd on e4m3 operands (nanochat Admin & Developer Guide, 6
+ * "Attention: FA3 with SDPA Fallback": FA3 runs in bf16 or fp8; 5: the tensorwise
+ * e4m3 recipe). q8 (B,T,Hq,128), k8, v8 (B,T,Hkv,128): e4m3 codes, one byte per
+ * element, BTHD, as attn_quantize_fp8 writes them; descale: three floats in device
+ * memory, the dequantization factors of q, k and v in that order. Computes
+ *   S = scale * (q8 dq) (k8 dk)^T on the causal window, o = softmax(S) (v8 dv),
+ * with the products on the e4m3 tensor cores (fp32 accumulation) and P rounded to
+ * e4m3 (scaled by 2^8) for the P V product; the row sums use the unrounded P.
+ * o (B,T,Hq,128) bf16, lse (B,Hq,T) fp32 as for attn_fwd. D must be 128
+ * (ATTN_ERR_UNSUPPORTED otherwise); other checks as for attn_fwd.
+ */
+attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* descale, void* o, float* lse,
+                           int B, int T, int Hq, int Hkv, int D, int window, float scale, void* stream);
 
 /* Bytes of workspace attn_decode needs: the fp32 split-K partials (B*Hq*chunks*(D+2)*4
  * bytes, chunks = ceil(min(window+1, Tmax) / 128), rounded up to 256) and one 8-byte
@@ -243,9 +278,10 @@ int attn_layer_window(const char* pattern, int layer, int n_layer, int seq_len, 
  * Copies rows [0, rows) of every layer into every sample row; the destination's
  * other rows are left as they were. 0 <= rows <= min(Tmax_src, Tmax); the four
  * buffers must not overlap (ATTN_ERR_INVALID_ARG). The caller sets each
- * sample's position (cache_seqlens) to rows. Asynchronous device-to-device
- * copies on `stream`, 1 + ceil(log2 N) rounds per layer and tensor, no kernel;
- * a failed copy enqueue returns ATTN_ERR_LAUNCH.
+ * sample's position (cache_seqlens) to rows. One launch on `stream`: each vector
+ * of the prompt rows is read once and stored to every sample (16-byte vectors when
+ * the pointers and the row size allow, else 4 or 2 bytes); a failed launch returns
+ * ATTN_ERR_LAUNCH.
  */
 attn_status_t attn_kv_replicate(const void* k_src, const void* v_src, void* k_dst, void* v_dst, int n_layers,
                                 int rows, int Tmax_src, int N, int Tmax, int Hkv, int D, void* stream);

@@ -18,6 +18,9 @@ from .attention import (  # noqa: F401
     prologue,
     prologue_bwd,
     round_bf16,
+    round_e4m3,
+    quantize_e4m3_tensorwise,
+    E4M3_MAX,
     visible,
     attention_fwd,
     attention_bwd,

@@ -11,8 +11,12 @@ Sources (page title, section):
         attention as a (left, right) pair ("Sliding-window attention"): a
         pattern of S (a quarter of the context, rounded up to a 128 tile) and
         L (full context) tiled over the layers, the last layer always L.
+  [AG5] nanochat Admin & Developer Guide, 5 "Precision: Explicit dtype & FP8":
+        the FP8 path scales each tensor by one factor (tensorwise, dynamic) and
+        keeps forward tensors in float8 e4m3.
   [AG6] nanochat Admin & Developer Guide, 6 "Attention: FA3 with SDPA Fallback":
-        GQA through enable_gqa; single-token decode slices the KV window.
+        GQA through enable_gqa; single-token decode slices the KV window; FA3
+        runs in bf16 or fp8.
   [AG7] nanochat Admin & Developer Guide, 7 "KV cache": (B, T, H, D) caches,
         int32 per-row positions, appended in place; a batch-1 prefill cache
         copied into a batch-N decode cache (one row per sample).
@@ -359,6 +363,44 @@ def prefill(q, kcache, vcache, pos, window, scale, k_new=None, v_new=None, rows=
             o[b, :, h, :] = (E / l) @ np.where(mask.any(axis=0)[:, None], V, 0.0)
             lse[b, h, :] = (m + np.log(l))[:, 0]
     return o, lse, kc, vc
+
+
+# --------------------------------------------------------------------------
+# FP8 operands: e4m3 rounding and tensorwise scaling  [AG5, AG6]
+# --------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def round_e4m3(x):
+    """Round to the nearest float8 e4m3 ("fn": finite-only) value, ties to even,
+    saturating at +-448 [AG5: forward tensors in float8_e4m3fn].
+
+    e4m3: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits. A normal value
+    in [2**e, 2**(e+1)) (e >= -6) has 4 significant bits, so its spacing is
+    2**(e-3); below 2**-6 the values are the subnormals k * 2**-9 (k = 0..7). The
+    largest finite value is 448 = 1.75 * 2**8; rounding saturates there instead
+    of overflowing (there is no infinity).
+    """
+    x = _f64(x)
+    a = np.abs(x)
+    _, e = np.frexp(a)                 # a = m * 2**e with 0.5 <= m < 1: leading bit 2**(e-1)
+    q = np.maximum(e - 4, -9).astype(np.float64)   # spacing exponent: 3 bits below the leading one
+    r = np.minimum(np.round(a / np.exp2(q)) * np.exp2(q), E4M3_MAX)   # np.round: half to even
+    return np.copysign(r, x)
+
+
+def quantize_e4m3_tensorwise(x):
+    """Tensorwise dynamic scaling to e4m3 [AG5: the FP8 recipe scales each tensor by
+    one factor from its absolute maximum]: s = 448 / amax(|x|) and codes =
+    round_e4m3(x * s), the scale and the product taken in float32 as the device
+    computes them (a quantised code is decided in the kernel's precision). amax = 0
+    gives s = 1. Returns (codes as float64 values, s); the dequantized tensor is
+    codes / s."""
+    x32 = np.asarray(x, dtype=np.float32)
+    amax = np.float32(np.max(np.abs(x32))) if x32.size else np.float32(0)
+    s = np.float32(1) if amax == 0 else np.float32(E4M3_MAX) / amax
+    codes = round_e4m3((x32 * s).astype(np.float64))
+    return codes, float(s)
 
 
 # --------------------------------------------------------------------------

@@ -41,20 +41,21 @@ def test_status_strings(L):
 
 
 def test_bwd_workspace_size(L):
-    # two arrays of per-row extension pairs (fp32-sized, padded to 128-row tiles), the
-    # fp32 dQ accumulator and the work counter; each part rounded up to 256 bytes. The
-    # window does not change it.
+    # -lse/scale and -Delta row pairs (fp32-sized, padded to 128-row tiles) + one 32 KB
+    # dS^T tile per (key tile, query tile) pair inside the window + the work counters
     B, T, Hq, Hkv, D = 8, 2048, 10, 10, 128
     rows = B * Hq * 2048 * 4
-    acc = B * T * Hq * D * 4
-    for W in (1024, -1, 2048, 0):
-        assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, W) == 2 * rows + acc + 256
+    # window 1024: key tile n sees min(16 - n, 9) query tiles -> 7*9 + (9+8+...+1) = 108
+    assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, 1024) == 2 * rows + B * Hq * 108 * 32768 + 256
+    # no window: the 16*17/2 = 136 tiles of the lower triangle; window >= T - 1 is the same
+    full = 2 * rows + B * Hq * 136 * 32768 + 256
+    assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, -1) == full
+    assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, 2048) == full
     # the block backward adds the (T, D/2) cos/sin table of float pairs
-    assert L.attn_block_bwd_workspace_bytes(B, T, Hq, Hkv, D, 1024) == 2 * rows + acc + 256 + T * 64 * 8
-    # ragged T pads the per-row arrays to whole 128-row tiles (130 -> 256); the accumulator
-    # holds the T real rows, rounded up to 256 bytes
-    assert L.attn_bwd_workspace_bytes(1, 130, 2, 1, 64, 0) == 2 * 2048 + 130 * 2 * 64 * 4 + 256
-    assert L.attn_block_bwd_workspace_bytes(1, 3, 1, 1, 64, -1) == 2 * 512 + 768 + 256 + 768
+    assert L.attn_block_bwd_workspace_bytes(B, T, Hq, Hkv, D, -1) == full + T * 64 * 8
+    # ragged T pads the per-row arrays to whole 128-row tiles; window 0 keeps the diagonal only
+    assert L.attn_bwd_workspace_bytes(1, 130, 2, 1, 64, 0) == 2 * 2048 + 2 * 2 * 32768 + 256
+    assert L.attn_block_bwd_workspace_bytes(1, 3, 1, 1, 64, -1) == 2 * 512 + 32768 + 256 + 768
     assert L.attn_bwd_workspace_bytes(1, 16, 3, 2, 128, -1) == 0     # Hq % Hkv != 0
     assert L.attn_bwd_workspace_bytes(1, 16, 2, 2, 96, -1) == 0      # head dim
 
@@ -199,8 +200,8 @@ def test_size_limits_rejected_before_launch(L):
     ws = L.attn_decode_workspace_bytes(1, 1, 128, Tmax, -1)
     assert ws > 0
     assert L.attn_decode(P, P, P, None, None, P, P, P, 1, Tmax, 1, 1, 128, -1, f, P, ws, None) == UNSUPPORTED
-    # backward: more than 2^31 work items (key tiles x KV heads x sequences)
-    B, T, H = 1023, 65535 * 128, 128
+    # backward: stored dS^T tiles beyond 2^31 rows (B * Hq * tiles * 128)
+    B, T, H = 64, 65536, 64
     ws = L.attn_bwd_workspace_bytes(B, T, H, H, 128, -1)
     big = ctypes.c_void_p(0x100000000)
     assert ws > 0
@@ -218,3 +219,19 @@ def test_size_limits_rejected_before_launch(L):
 def test_wait_limit_hook_rejects_limits_above_the_default(L):
     # checked before anything touches the device
     assert L.attn_debug_set_wait_limit(3_000_000_000, None) == INVALID
+
+
+def test_fp8_entry_points_reject_bad_args(L):
+    f = ctypes.c_float(0.1)
+    assert L.attn_quantize_fp8_workspace_bytes(1024) == 4096
+    assert L.attn_quantize_fp8_workspace_bytes(12) == 0               # not a multiple of 8
+    ws = L.attn_quantize_fp8_workspace_bytes(64)
+    assert L.attn_quantize_fp8(P, 60, P, P, P, ws, None) == INVALID   # n % 8
+    assert L.attn_quantize_fp8(None, 64, P, P, P, ws, None) == INVALID
+    assert L.attn_quantize_fp8(MIS, 64, P, P, P, ws, None) == INVALID  # x misaligned
+    assert L.attn_quantize_fp8(P, 64, P, P, P, ws - 4, None) == INVALID
+    # q8, k8, v8, descale, o, lse, B, T, Hq, Hkv, D, window, scale, stream
+    assert L.attn_fwd_fp8(P, P, P, P, P, P, 1, 128, 2, 1, 64, -1, f, None) == UNSUPPORTED   # D = 64
+    assert L.attn_fwd_fp8(P, P, P, None, P, P, 1, 128, 2, 1, 128, -1, f, None) == INVALID  # no descale
+    assert L.attn_fwd_fp8(P, P, P, P, P, P, 1, 128, 3, 2, 128, -1, f, None) == INVALID     # Hq % Hkv
+    assert L.attn_fwd_fp8(MIS, P, P, P, P, P, 1, 128, 2, 1, 128, -1, f, None) == INVALID   # misaligned

@@ -15,6 +15,9 @@
     decodes every sample exactly as the batch-1 cache does
   * bf16 rounding: hand-computed ties and near-ties, and torch's own float32 ->
     bfloat16 conversion on random float32 values
+  * e4m3 rounding: hand-computed ties, subnormals and saturation, and torch's own
+    float32 -> float8_e4m3fn conversion on random in-range float32 values; the
+    tensorwise scale maps the absolute maximum to 448
 The last test plants plausible mistakes in the oracle and shows a pin fails.
 """
 import json
@@ -473,6 +476,52 @@ def test_round_bf16():
     allclose(oracle.round_bf16(y), y, 0.0)  # idempotent
 
 
+def check_round_e4m3_hand():
+    """Hand-computed e4m3 roundings. Near 1 the spacing is 2**-3: 1.0625 is a tie (to
+    1, even mantissa), 1.1875 a tie (to 1.25), 1.9375 a tie that carries into the next
+    binade (2). The top binade [256, 448] has spacing 32: 464 is a tie (to 448), and
+    values past 448 saturate. Subnormals are k * 2**-9: 2**-10 is a tie (to 0),
+    3 * 2**-10 a tie (to 2**-8), 2**-6 - 2**-10 = 7.5 * 2**-9 a tie up to the smallest
+    normal 2**-6."""
+    cases = [(1.0625, 1.0), (1.1875, 1.25), (1.9375, 2.0), (-1.0625, -1.0), (448.0, 448.0), (464.0, 448.0),
+             (480.0, 448.0), (1e6, 448.0), (-500.0, -448.0), (2.0 ** -10, 0.0), (3 * 2.0 ** -10, 2.0 ** -8),
+             (2.0 ** -9, 2.0 ** -9), (2.0 ** -6 - 2.0 ** -10, 2.0 ** -6), (0.1, 0.1015625), (5.0, 5.0),
+             (5.2, 5.0), (5.3, 5.5), (0.0, 0.0)]
+    x = np.array([c[0] for c in cases])
+    allclose(oracle.round_e4m3(x), [c[1] for c in cases], 0.0)
+
+
+def check_round_e4m3_torch():
+    """On in-range float32 inputs a single round-to-nearest-even to e4m3 is what torch's
+    float32 -> float8_e4m3fn conversion does: both must agree bit for bit."""
+    r = (rnd(100000, 41) * np.exp(rnd(100000, 42) * 3)).astype(np.float32)
+    r = r[np.abs(r) < 440]
+    ref = torch.from_numpy(r).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    allclose(oracle.round_e4m3(r.astype(np.float64)), ref, 0.0)
+
+
+def test_round_e4m3():
+    check_round_e4m3_hand()
+    check_round_e4m3_torch()
+    y = oracle.round_e4m3(rnd(5000, 43) * 30)
+    allclose(oracle.round_e4m3(y), y, 0.0)                       # idempotent
+    assert len(np.unique(np.abs(y))) <= 127                       # at most the 127 non-negative finite values
+
+
+def test_quantize_e4m3_tensorwise():
+    x = rnd((4, 33, 2, 16), 44)
+    codes, s = oracle.quantize_e4m3_tensorwise(x)
+    assert np.max(np.abs(codes)) == oracle.E4M3_MAX              # the absolute maximum maps to 448
+    assert s == float(np.float32(448) / np.float32(np.max(np.abs(np.float32(x)))))
+    deq = codes / s
+    normal = np.abs(x) * s >= 2.0 ** -6
+    # a normal e4m3 value is within half a spacing (2**-4 relative) of its input
+    assert np.all(np.abs(deq - x)[normal] <= 2.0 ** -4 * np.abs(x)[normal] * (1 + 1e-6))
+    assert np.all(np.abs(deq - x)[~normal] <= 2.0 ** -10 / s * (1 + 1e-6))
+    z_codes, z_s = oracle.quantize_e4m3_tensorwise(np.zeros(8))
+    assert z_s == 1.0 and not np.any(z_codes)
+
+
 # ---------------------------------------------------------------- planted mistakes
 def _rope_wrong_sign(x, positions, base):
     return oa.rope_transpose(x, positions, base)
@@ -539,6 +588,27 @@ def test_pins_catch_truncating_bf16_rounding(monkeypatch):
         check_round_bf16_hand()
     with pytest.raises(AssertionError):
         check_round_bf16_torch()
+
+
+@pytest.mark.parametrize("bad", ["truncate", "four_bits"])
+def test_pins_catch_wrong_e4m3_rounding(monkeypatch, bad):
+    """Rounding toward zero, or keeping one mantissa bit too many, must fail the pins."""
+    def wrong(x):
+        x = np.asarray(x, np.float64)
+        a = np.abs(x)
+        _, e = np.frexp(a)
+        if bad == "truncate":
+            q = np.maximum(e - 4, -9).astype(np.float64)
+            r = np.floor(a / np.exp2(q)) * np.exp2(q)
+        else:
+            q = np.maximum(e - 5, -10).astype(np.float64)
+            r = np.round(a / np.exp2(q)) * np.exp2(q)
+        return np.copysign(np.minimum(r, 448.0), x)
+    monkeypatch.setattr(oracle, "round_e4m3", wrong)
+    with pytest.raises(AssertionError):
+        check_round_e4m3_hand()
+    with pytest.raises(AssertionError):
+        check_round_e4m3_torch()
 
 
 def test_pins_catch_prefill_ignoring_the_cache(monkeypatch):
