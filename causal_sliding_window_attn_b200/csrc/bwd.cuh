@@ -34,11 +34,14 @@
 //                the elementwise warps work on this one. dS^T leaves as bf16
 //                tiles for bwd_dq (plain 512-byte coalesced stores). dK, dV are
 //                complete in the CTA (the whole group is walked here), so they
-//                are written once, as bf16, with no atomics.
+//                are written once, as bf16, with no atomics: each goes through
+//                the Q or dO ring stage of the item's last step (lent to the
+//                epilogue until its TMA stores have read it) and leaves as TMA
+//                stores of 32-row boxes.
 //   bwd_dq       one CTA per (128-row query tile, query head, batch):
 //                dQ = scale * sum over key tiles of dS K, accumulated in TMEM
 //                from the stored dS^T tiles (one bulk copy each) and K tiles,
-//                written once as bf16.
+//                written once as bf16 through a staging tile and TMA stores.
 // Splitting dQ out keeps fp32 dQ reductions out of the main kernel, whose
 // TMEM (512 columns) and shared memory are fully used. (A variant that reduced a
 // per-step dQ tile into an fp32 accumulator in L2 instead -- 64 KB of 16-byte
@@ -46,10 +49,13 @@
 // 14 bytes per clock per SM.)
 // For the block backward (attn_block_bwd) the dK epilogue and the dQ kernel's
 // epilogue also apply the prologue backward, so dk and dq come out with respect to
-// the raw k and q (rows read once, cos/sin from a table the prep kernel builds).
+// the raw k and q: the raw tile arrives by TMA in the staging buffer, the rotary
+// angles are computed from the row's position, and the result overwrites the raw
+// rows in place before the store.
 // Warp roles in bwd_main: 0 TMA (K, V, Q ring), 1 MMA issuer (whole warp, one
-// elected lane issues), 2 TMEM allocator, 3 TMA (dO ring), 4-7 and 8-11 P/dS
-// (thread = key row; query columns 0-63 and 64-127), then the dK and dV epilogues.
+// elected lane issues), 2 TMEM allocator and work scheduler, 3 TMA (dO ring),
+// 4-7 and 8-11 P/dS (thread = key row; query columns 0-63 and 64-127), then
+// the dK (4-7) and dV (8-11) epilogues.
 #pragma once
 #include "ptx.cuh"
 
@@ -61,20 +67,17 @@ struct BwdParams {
   // of the S^T and dP^T MMAs reads them (see attn_bwd_prep_kernel)
   const uint8_t* ext_lse;
   const uint8_t* ext_delta;
-  __nv_bfloat16* dk;
-  __nv_bfloat16* dv;
-  __nv_bfloat16* dq;
   __nv_bfloat16* ds;   // stored dS^T tiles (see ds_unit_offset)
   int* item_counter;   // [2] next work item of the main and dQ kernels (zeroed by the prep kernel)
   int T, Tpad, Hq, G, window, n_tiles, span;  // tiles of 128 rows; span = query tiles per key tile
   long long tiles_per_bh;                     // stored dS^T tiles per (batch, query head)
   float scale, scale_log2;
-  // fused prologue backward (attn_block_bwd): dk and dq with respect to the raw k and q,
-  // whose rows are read in the dK epilogue and the dQ kernel's epilogue; null otherwise
-  const __nv_bfloat16* k_raw;
-  const __nv_bfloat16* q_raw;
-  const float2* rope_cs;  // (T, D/2): (cos, sin) of t * omega_j
+  // fused prologue backward (attn_block_bwd): dk and dq with respect to the raw k and
+  // q (whose tensor maps the kernels take), the RMS-norm eps and the turns of rotary
+  // pair j per unit position as 64-bit fixed-point fractions (see rope_cos_sin)
+  int rope;
   float eps;
+  unsigned long long turns[64];
 };
 
 // Query tiles that see key tile n: [n, n + min(n_tiles - n, span) - 1], where
@@ -105,79 +108,23 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
-// Prologue backward of one row held whole by one thread (nanochat Admin & Developer
-// Guide, 3: RMS-norm without weight, then RoPE). dy_chunk(c0, v) fills v with elements
-// c0 .. c0+15 of the gradient with respect to the prologue output (fp32); x is the raw
-// row (bf16), cs[j] = (cos, sin) of the row's angle for pair (j, j + D/2). Writes
-//   dx = (g - xh (g . xh) / D) / r,  r = sqrt(mean(x^2) + eps),  xh = x / r,
-// g = dy rotated by -phi, as bf16 to dst when `store` is set. dy is asked for twice per
-// element (a dot product pass, then the output pass) so that no full row of it stays in
-// registers. Every lane of a warp runs the same steps (dy_chunk may be warp-collective);
-// a lane with nothing to store passes store = false and any valid x and cs rows.
-template <int D, typename DyChunk>
-__device__ __forceinline__ void prologue_bwd_row(DyChunk&& dy_chunk, const __nv_bfloat16* x,
-                                                 const float2* cs, float eps, __nv_bfloat16* dst, bool store) {
-  constexpr int H = D / 2;
-  // the raw row: the sum of squares first, then re-read (from L1) chunk by chunk
-  float ss = 0.f;
+// Prologue backward of 16 rotary pairs (j0 .. j0+15, and j0 + D/2 ..) of one row held
+// by one thread (nanochat Admin & Developer Guide, 3: RMS-norm without weight, then
+// RoPE). With dy the gradient with respect to the prologue output and x the raw row:
+//   g = dy rotated by -phi,  r = sqrt(mean(x^2) + eps),  xh = x / r,
+//   dx = (g - xh (g . xh) / D) / r.
+// rotate_back: g of the pairs from dy (both halves, fp32, in place).
+template <int D>
+__device__ __forceinline__ void rope_rotate_back(const unsigned long long* turns, unsigned pos, int j0,
+                                                 float (&a)[16], float (&b)[16]) {
 #pragma unroll
-  for (int v = 0; v < D / 8; ++v) {
-    const uint4 t = *reinterpret_cast<const uint4*>(x + 8 * v);
-    const uint32_t w[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float lo = __uint_as_float(w[u] << 16), hi = __uint_as_float(w[u] & 0xffff0000u);
-      ss = fmaf(lo, lo, fmaf(hi, hi, ss));
-    }
-  }
-  const float inv_r = rsqrtf(ss * (1.f / D) + eps);
-  auto x16 = [&](int c0, float (&v)[16]) {
-    const uint4 t0 = *reinterpret_cast<const uint4*>(x + c0), t1 = *reinterpret_cast<const uint4*>(x + c0 + 8);
-    const uint32_t w[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      v[2 * u] = __uint_as_float(w[u] << 16) * inv_r;
-      v[2 * u + 1] = __uint_as_float(w[u] & 0xffff0000u) * inv_r;
-    }
-  };
-  float dot = 0.f;
-#pragma unroll 1
-  for (int pass = 0; pass < 2; ++pass) {
-    const float proj = dot * (1.f / D);
-#pragma unroll 1
-    for (int c0 = 0; c0 < H; c0 += 16) {
-      float a[16], b[16], xa[16], xb[16];
-      dy_chunk(c0, a);      // elements c0 .. c0+15
-      dy_chunk(H + c0, b);  // elements H + c0 .. H + c0 + 15
-      x16(c0, xa);
-      x16(H + c0, xb);
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const float2 t = cs[c0 + u];
-        const float ga = fmaf(b[u], t.y, a[u] * t.x);
-        const float gb = fmaf(-a[u], t.y, b[u] * t.x);
-        if (pass == 0) {
-          dot = fmaf(ga, xa[u], fmaf(gb, xb[u], dot));
-        } else {
-          a[u] = (ga - xa[u] * proj) * inv_r;
-          b[u] = (gb - xb[u] * proj) * inv_r;
-        }
-      }
-      if (pass == 1 && store) {
-        uint32_t oa[8], ob[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          oa[u] = pack_bf16x2(a[2 * u], a[2 * u + 1]);
-          ob[u] = pack_bf16x2(b[2 * u], b[2 * u + 1]);
-        }
-        uint4* da = reinterpret_cast<uint4*>(dst + c0);
-        uint4* db = reinterpret_cast<uint4*>(dst + H + c0);
-        da[0] = make_uint4(oa[0], oa[1], oa[2], oa[3]);
-        da[1] = make_uint4(oa[4], oa[5], oa[6], oa[7]);
-        db[0] = make_uint4(ob[0], ob[1], ob[2], ob[3]);
-        db[1] = make_uint4(ob[4], ob[5], ob[6], ob[7]);
-      }
-    }
+  for (int u = 0; u < 16; ++u) {
+    float c, sn;
+    rope_cos_sin(pos, turns[j0 + u], c, sn);
+    const float ga = fmaf(b[u], sn, a[u] * c);
+    const float gb = fmaf(-a[u], sn, b[u] * c);
+    a[u] = ga;
+    b[u] = gb;
   }
 }
 
@@ -211,21 +158,21 @@ struct BwdLayout {
   static constexpr int kExt = kDO + kDOStages * kTile;
   static constexpr int kExtOnes = kExt + (kQStages + kDOStages) * 512;
   static constexpr int kBar = kExtOnes + 256;
-#ifdef CSWA_TRACE
-  static constexpr int kUsed = kBar + 256;  // profiling builds keep 4 more barriers
-#else
-  static constexpr int kUsed = kBar + 224;
-#endif
+  static constexpr int kNumBars = 29;
+  // the barriers, then three 4-byte slots (TMEM base, abort flag, work item)
+  static constexpr int kUsed = kBar + kNumBars * 8 + 16;
   static constexpr int kBytes = (kUsed + 1024 <= 232448) ? kUsed + 1024 : 232448;
   static_assert(kUsed <= 232448, "shared memory budget");
   static constexpr uint32_t kTmemCols = 512;
 };
 
+// tm_kr: the raw k (block backward only); tm_dk, tm_dv: the outputs, 32-row boxes.
 template <int D>
 __global__ void __launch_bounds__(384, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const BwdParams p, int n_items) {
+                    const __grid_constant__ CUtensorMap tm_kr, const __grid_constant__ CUtensorMap tm_dk,
+                    const __grid_constant__ CUtensorMap tm_dv, const __grid_constant__ BwdParams p, int n_items) {
   using L = BwdLayout<D>;
   constexpr int QS = L::kQStages, DS = L::kDOStages;
   extern __shared__ uint8_t smem_raw[];
@@ -240,23 +187,23 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* kv_empty = bars + 1;               // the item's last S^T and dP^T have read K and V
   uint64_t* q_full = bars + 2;                 // [QS]
   uint64_t* q_empty = q_full + QS;             // [QS]  dK has read the Q tile
-  uint64_t* do_full = q_empty + QS;            // [DS]
+  uint64_t* q_borrow = q_empty + QS;           // [QS]  the dK epilogue is done with a lent stage
+  uint64_t* do_full = q_borrow + QS;           // [DS]
   uint64_t* do_empty = do_full + DS;           // [DS]  dV has read the dO tile
-  uint64_t* s_full = do_empty + DS;            // S^T in TMEM
+  uint64_t* do_borrow = do_empty + DS;         // [DS]  the dV epilogue is done with a lent stage
+  uint64_t* s_full = do_borrow + DS;           // S^T in TMEM
   uint64_t* p_chunk = s_full + 1;              // [4] P^T of queries 16c..16c+15 of each half written
   uint64_t* dp_full = p_chunk + 4;             // dP^T in TMEM
   uint64_t* ds_full = dp_full + 1;             // dS^T written over dP^T
   uint64_t* final_bar = ds_full + 1;           // the item's dK and dV are complete in TMEM
   uint64_t* acc_free = final_bar + 1;          // the epilogue has read them
-  uint64_t* done_bar = acc_free + 1;           // every MMA of the CTA has completed
-  uint64_t* item_full = done_bar + 1;          // the next work item's index is in item_slot
+  uint64_t* item_full = acc_free + 1;          // the next work item's index is in item_slot
   uint64_t* item_empty = item_full + 1;        // every role has read it
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(item_empty + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(item_empty + 2);
-  volatile int* item_slot = reinterpret_cast<volatile int*>(item_empty + 3);
-#ifdef CSWA_TRACE
-  uint64_t* trace_bar = item_empty + 4;  // [4] completion of dV, S, dK, dP groups (profiling builds)
-#endif
+  uint64_t* kr_full = item_empty + 1;          // the raw k tile is in the lent Q stage
+  static_assert(L::kNumBars == 2 + 3 * QS + 3 * DS + 9 + 2 + 1, "barrier count");
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(kr_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(kr_full + 1) + 1;
+  volatile int* item_slot = reinterpret_cast<volatile int*>(kr_full + 1) + 2;
 
   const int warp = warp_id(), lane = lane_id();
   const int W = p.window, G = p.G;
@@ -288,10 +235,12 @@ __global__ void __launch_bounds__(384, 1)
     for (int s = 0; s < QS; ++s) {
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
+      mbar_init(&q_borrow[s], 4);  // the four dK epilogue warps
     }
     for (int s = 0; s < DS; ++s) {
       mbar_init(&do_full[s], 1);
       mbar_init(&do_empty[s], 1);
+      mbar_init(&do_borrow[s], 4);  // the four dV epilogue warps
     }
     mbar_init(s_full, 1);
     for (int c = 0; c < 4; ++c) mbar_init(&p_chunk[c], 256);
@@ -299,12 +248,9 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(ds_full, 256);
     mbar_init(final_bar, 1);
     mbar_init(acc_free, 256);
-    mbar_init(done_bar, 1);
     mbar_init(item_full, 1);
     mbar_init(item_empty, 11);  // warps 0, 1, 3 and the eight P/dS warps
-#ifdef CSWA_TRACE
-    for (int i = 0; i < 4; ++i) mbar_init(&trace_bar[i], 1);
-#endif
+    mbar_init(kr_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -347,7 +293,9 @@ __global__ void __launch_bounds__(384, 1)
     // free up at a different point of the step, so it waits on its own). Each stage
     // also takes the 512-byte row extension of its tile: -lse/scale with Q, -Delta
     // with dO. K and V of the next item load as soon as the current item's last S^T
-    // and dP^T have read the previous ones.
+    // and dP^T have read the previous ones. The stage of an item's last step is lent
+    // to that item's dK (Q ring) or dV (dO ring) epilogue as its staging buffer: it
+    // is loaded again only once the epilogue has released it (the borrow barrier).
     // The whole warp takes the items (the slot is read warp-wide); lane 0 issues.
     const bool qside = (warp == 0);
     const int nst = qside ? QS : DS;
@@ -364,6 +312,8 @@ __global__ void __launch_bounds__(384, 1)
     }
     uint64_t* full = qside ? q_full : do_full;
     uint64_t* empty = qside ? q_empty : do_empty;
+    uint64_t* borrow = qside ? q_borrow : do_borrow;
+    uint32_t lent = 0, lent_par = 0;  // per stage: lent to an epilogue; parity of its next release
     const CUtensorMap* tm = qside ? &tm_q : &tm_do;
     const int base = qside ? L::kQ : L::kDO;
     const uint8_t* ext = qside ? p.ext_lse : p.ext_delta;
@@ -382,6 +332,9 @@ __global__ void __launch_bounds__(384, 1)
               tma_load_4d(smem + L::kK + pn * L::kPanel, &tm_k, kv_full, pn * 64, I.hk, I.n * 128, I.b);
               tma_load_4d(smem + L::kV + pn * L::kPanel, &tm_v, kv_full, pn * 64, I.hk, I.n * 128, I.b);
             }
+            // the raw k rows the dK epilogue will load: on their way to L2 now
+            if (p.rope)
+              for (int pn = 0; pn < D / 64; ++pn) tma_prefetch_l2_4d(&tm_kr, pn * 64, I.hk, I.n * 128, I.b);
             last_kv = k;
           }
         }
@@ -389,6 +342,11 @@ __global__ void __launch_bounds__(384, 1)
           const int st = g % nst;
           const int h = I.hk * G + it / I.m_cnt, q0 = (I.n + it % I.m_cnt) * 128;
           if (qside) CSWA_MARK(3, g, 0);
+          if ((lent >> st) & 1u) {
+            if (!(ok = mbar_wait(&borrow[st], (lent_par >> st) & 1u, abort_flag))) break;
+            lent &= ~(1u << st);
+            lent_par ^= 1u << st;
+          }
           if (!(ok = mbar_wait(&empty[st], ((g / nst) & 1) ^ 1, abort_flag))) break;
           if (qside) CSWA_MARK(3, g, 1);
           mbar_arrive_expect_tx(&full[st], L::kTile + 512);
@@ -397,6 +355,7 @@ __global__ void __launch_bounds__(384, 1)
           bulk_load(ext_slot + st * 512, ext + (((size_t)I.b * p.Hq + h) * p.n_tiles + q0 / 128) * 512, 512,
                     &full[st]);
           last_issue[st] = g;
+          if (it + 1 == I.n_iters) lent |= 1u << st;
         }
       }
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
@@ -492,15 +451,9 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (!ok) break;
         mma_commit(&do_empty[ds], leader);
-#ifdef CSWA_TRACE
-        mma_commit(&trace_bar[0], leader);
-#endif
         if (tracer) CSWA_MARK(0, g, 2);
         // S^T(it+1) overwrites P^T(it) only after dV(it) has read it: MMAs run in issue order
         if (more) issue_R(tR0, dK_k, dQ_k, q1 * L::kTile, q1, s_full);
-#ifdef CSWA_TRACE
-        if (more) mma_commit(&trace_bar[1], leader);
-#endif
         if (tracer) CSWA_MARK(0, g, 4);
         if (more && !(ok = wait_all(&do_full[d1], ((g + 1) / DS) & 1))) break;
         if (!(ok = wait_all(ds_full, g & 1))) break;
@@ -508,26 +461,26 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_after();
         issue_acc(tdK, tR1, dQ_mn, qs * L::kTile, it == 0);
         mma_commit(&q_empty[qs], leader);
-#ifdef CSWA_TRACE
-        mma_commit(&trace_bar[2], leader);
-#endif
         if (tracer) CSWA_MARK(0, g, 6);
         if (more) {
           issue_R(tR1, dV_k, dDO_k, d1 * L::kTile, QS + d1, dp_full);
           if (it + 2 == I.n_iters) mma_commit(kv_empty, leader);  // the item's last S^T and dP^T
         }
-#ifdef CSWA_TRACE
-        if (more) mma_commit(&trace_bar[3], leader);
-#endif
         if (tracer) CSWA_MARK(0, g, 7);
       }
       if (!ok) break;
       mma_commit(final_bar, leader);  // dK and dV of the item are complete
       g0 += I.n_iters;
     }
-    // every MMA issued above has finished before TMEM is released
-    mma_commit(done_bar, leader);
-    mbar_drain(done_bar, 0);
+    // every MMA issued above has finished before TMEM is released. Items 0 .. k-1 each
+    // committed one phase of final_bar, the last of which covers every MMA of a normal
+    // run; after an abort, one more phase covers those issued since (final_bar gets no
+    // other commit, so neither wait can find its phase already overtaken).
+    if (k > 0) mbar_drain(final_bar, (k - 1) & 1);
+    if (!ok) {
+      mma_commit(final_bar, leader);
+      mbar_drain(final_bar, k & 1);
+    }
   } else if (warp == 2) {
     // ------------------------------------------------------------ work scheduler
     // claims the CTA's next item from the global counter once every role has read
@@ -569,6 +522,7 @@ __global__ void __launch_bounds__(384, 1)
     };
     bool ok = true;
     int g0 = 0, k = 0;
+    int kr_pending = -1;  // warp 4, lane 0: the item whose raw k load nobody has waited for yet
     for (;; ++k) {
       const int item = take_item(k);
       if (item < 0) break;
@@ -661,49 +615,132 @@ __global__ void __launch_bounds__(384, 1)
       store_ds_units(0, 8);
       ds_dst = nullptr;
       // ------------------------------------------------------ dK (warps 4-7) / dV (8-11) epilogue
-      ok = __all_sync(0xffffffffu, mbar_wait(final_bar, k & 1, abort_flag));
+      // Thread = key row j of the tile. The accumulator goes to bf16 in the ring stage
+      // of the item's last step (the Q stage for dK, the dO stage for dV: lent by the
+      // producers, whose last reader -- the last dK or dV MMA -- has completed), in the
+      // 128-byte-swizzled layout of a TMA tile; each warp then stores its 32 rows with
+      // one TMA store per 64-column panel (rows past T are not written) and returns the
+      // stage once the stores have read it. dV is complete as soon as the last dV MMA
+      // is (it released its dO stage), a step ahead of dK.
+      const int g_last = g0 + I.n_iters - 1;
+      const int st_last = half ? g_last % DS : g_last % QS;
+      uint8_t* stage = smem + (half ? L::kDO : L::kQ) + st_last * L::kTile;
+      // (profiling builds: epilogue marks of the CTA's first 8 items at steps 56-63)
+      const int emark = 56 + (k & 7);
+      if (tracer && k < 8) CSWA_MARK(trole, emark, 0);
+      ok = __all_sync(0xffffffffu, half ? mbar_wait(&do_empty[st_last], (g_last / DS) & 1, abort_flag)
+                                        : mbar_wait(final_bar, k & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      const uint32_t src = half ? tdV : tdK;
-      const float mul = half ? 1.f : p.scale;
-      const size_t krow = ((size_t)I.b * p.T + j) * (p.Hq / G) + I.hk;
-      __nv_bfloat16* dst = (half ? p.dv : p.dk) + krow * D;
-      if (!half && p.k_raw) {
-        // dk with respect to the raw k: the prologue backward on the way out. tcgen05.ld is
-        // warp-collective, so rows past T run the same steps on row T - 1's inputs and
-        // store nothing.
-        auto dy_chunk = [&](int c0, float (&v)[16]) {
-          uint32_t t[16];
-          tmem_ld16(src + lane_off + c0, t);
+      if (tracer && k < 8) CSWA_MARK(trole, emark, 1);
+      const uint32_t src = (half ? tdV : tdK) + lane_off;
+      if (!half && p.rope) {
+        // dk with respect to the raw k: the prologue backward on the way out. The raw
+        // tile goes into the stage now (it was on its way to L2 since the item began)
+        // while dy is rotated back in TMEM; then the row statistics, then dx in place.
+        if (warp == 4 && lane == 0) {
+          mbar_arrive_expect_tx(kr_full, L::kTile);
+          for (int pn = 0; pn < D / 64; ++pn)
+            tma_load_4d(stage + pn * L::kPanel, &tm_kr, kr_full, pn * 64, I.hk, k0, I.b);
+          kr_pending = k;
+        }
+        constexpr int H = D / 2;
+#pragma unroll 1
+        for (int j0 = 0; j0 < H; j0 += 16) {
+          uint32_t ta[16], tb[16];
+          tmem_ld16(src + j0, ta);
+          tmem_ld16(src + H + j0, tb);
+          tmem_ld_wait();
+          float a[16], b[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) a[u] = __uint_as_float(ta[u]) * p.scale, b[u] = __uint_as_float(tb[u]) * p.scale;
+          rope_rotate_back<D>(p.turns, (unsigned)j, j0, a, b);
+#pragma unroll
+          for (int u = 0; u < 16; ++u) ta[u] = __float_as_uint(a[u]), tb[u] = __float_as_uint(b[u]);
+          tmem_st16(src + j0, ta);
+          tmem_st16(src + H + j0, tb);
+        }
+        tmem_st_wait();
+        ok = __all_sync(0xffffffffu, mbar_wait(kr_full, k & 1, abort_flag));
+        if (!ok) break;
+        if (warp == 4 && lane == 0) kr_pending = -1;
+        float ss = 0.f, gx = 0.f;
+#pragma unroll 1
+        for (int j0 = 0; j0 < H; j0 += 16) {
+          uint32_t ta[16], tb[16];
+          tmem_ld16(src + j0, ta);
+          tmem_ld16(src + H + j0, tb);
+          float xa[16], xb[16];
+          tile_ld16(stage, r, j0, xa);
+          tile_ld16(stage, r, H + j0, xb);
           tmem_ld_wait();
 #pragma unroll
-          for (int u = 0; u < 16; ++u) v[u] = __uint_as_float(t[u]) * mul;
-        };
-        const int jj = min(j, p.T - 1);
-        const size_t krow_in = ((size_t)I.b * p.T + jj) * (p.Hq / G) + I.hk;
-        prologue_bwd_row<D>(dy_chunk, p.k_raw + krow_in * D, p.rope_cs + (size_t)jj * (D / 2), p.eps, dst, j < p.T);
+          for (int u = 0; u < 16; ++u) {
+            ss = fmaf(xa[u], xa[u], fmaf(xb[u], xb[u], ss));
+            gx = fmaf(__uint_as_float(ta[u]), xa[u], fmaf(__uint_as_float(tb[u]), xb[u], gx));
+          }
+        }
+        const float inv_r = rsqrtf(ss * (1.f / D) + p.eps);
+        const float c1 = gx * inv_r * inv_r * (1.f / D);  // (g . xh) / D, applied to x / r
+#pragma unroll 1
+        for (int j0 = 0; j0 < H; j0 += 16) {
+          uint32_t ta[16], tb[16];
+          tmem_ld16(src + j0, ta);
+          tmem_ld16(src + H + j0, tb);
+          float xa[16], xb[16];
+          tile_ld16(stage, r, j0, xa);
+          tile_ld16(stage, r, H + j0, xb);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            xa[u] = (__uint_as_float(ta[u]) - xa[u] * c1) * inv_r;
+            xb[u] = (__uint_as_float(tb[u]) - xb[u] * c1) * inv_r;
+          }
+          tile_st16(stage, r, j0, xa);
+          tile_st16(stage, r, H + j0, xb);
+        }
       } else {
+        // 64 columns per TMEM round trip (four loads, one wait)
+        const float mul = half ? 1.f : p.scale;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(src + lane_off + c * 32, o);
-        tmem_ld_wait();
-        uint32_t w[16];
+        for (int c0 = 0; c0 < D; c0 += 64) {
+          uint32_t t[4][16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * mul, __uint_as_float(o[2 * e + 1]) * mul);
-        if (j < p.T) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+          for (int e = 0; e < 4; ++e) tmem_ld16(src + c0 + 16 * e, t[e]);
+          tmem_ld_wait();
 #pragma unroll
-          for (int u = 0; u < 4; ++u) d4[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+          for (int e = 0; e < 4; ++e) {
+            float v[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) v[u] = __uint_as_float(t[e][u]) * mul;
+            tile_st16(stage, r, c0 + 16 * e, v);
+          }
         }
       }
-      }
+      if (tracer && k < 8) CSWA_MARK(trole, emark, 2);
       // the accumulators may take the next item's first products
       tc_fence_before();
       mbar_arrive(acc_free);
+      // the warp's 32 rows leave as TMA stores; the stage goes back to the producer
+      // once they have read it
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        for (int pn = 0; pn < D / 64; ++pn)
+          tma_store_4d(half ? &tm_dv : &tm_dk, stage + pn * L::kPanel + quarter * 4096, pn * 64, I.hk, k0 + 32 * quarter,
+                       I.b);
+        bulk_commit();
+        if (tracer && k < 8) CSWA_MARK(trole, emark, 3);
+        bulk_wait_read0();
+        if (tracer && k < 8) CSWA_MARK(trole, emark, 4);
+        mbar_arrive(half ? &do_borrow[st_last] : &q_borrow[st_last]);
+      }
       g0 += I.n_iters;
     }
+    // before the CTA's shared memory goes: the stores have completed, and a raw k load
+    // left behind by an abort has landed
+    if (lane == 0) bulk_wait0();
+    if (kr_pending >= 0) mbar_drain(kr_full, kr_pending & 1);
   }
 
   __syncthreads();
@@ -717,21 +754,28 @@ __global__ void __launch_bounds__(384, 1)
 // head, from the dS^T tiles bwd_main stored; accumulated in TMEM, written once as bf16.
 // Persistent: one CTA per SM takes (m, h, b) items from a global counter (warp 3
 // claims them). A 3-stage ring of (dS^T tile, K tile) runs on across items, and two
-// TMEM accumulators let the epilogue of one item overlap the MMAs of the next.
+// TMEM accumulators let the epilogue of one item overlap the MMAs of the next. The
+// epilogue (warps 4-7, thread = query row) turns the accumulator into bf16 rows of a
+// staging tile that each warp stores with TMA (its 32 rows); for the block backward
+// the warp first loads its 32 raw q rows there by TMA and writes dq in their place.
 template <int D>
 struct DqLayout {
   static constexpr int kStages = 3;
   static constexpr int kDS = 32768;            // one dS^T tile (128 keys x 128 queries bf16)
   static constexpr int kK = 128 * D * 2;       // one K tile
   static constexpr int kStage = kDS + kK;
-  static constexpr int kBar = kStages * kStage;
+  static constexpr int kX = kStages * kStage;  // the epilogue's staging tile (128 rows)
+  static constexpr int kBar = kX + 128 * D * 2;
   static constexpr int kBytes = kBar + 256 + 1024;
   static constexpr uint32_t kTmemCols = 2 * D;  // two accumulators
 };
 
+// tm_qr: the raw q (block backward only), tm_dq: the output; both 32-row boxes.
 template <int D>
 __global__ void __launch_bounds__(256, 1)
-    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const BwdParams p, int n_items) {
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_qr,
+                       const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ BwdParams p,
+                       int n_items) {
   using L = DqLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -743,9 +787,10 @@ __global__ void __launch_bounds__(256, 1)
   uint64_t* final_bar = acc_empty + 2;
   uint64_t* item_full = final_bar + 1;     // the next work item's index is in item_slot
   uint64_t* item_empty = item_full + 1;    // every role has read it
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(item_empty + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(item_empty + 2);
-  volatile int* item_slot = reinterpret_cast<volatile int*>(item_empty + 3);
+  uint64_t* x_full = item_empty + 1;       // [4] an epilogue warp's raw q rows have landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(x_full + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(x_full + 5);
+  volatile int* item_slot = reinterpret_cast<volatile int*>(x_full + 6);
 
   const int warp = warp_id(), lane = lane_id();
   // item -> (query tile m, head h, batch b) in super-block order with the heaviest
@@ -773,6 +818,7 @@ __global__ void __launch_bounds__(256, 1)
     mbar_init(final_bar, 1);
     mbar_init(item_full, 1);
     mbar_init(item_empty, 6);  // warps 0, 1 and the four epilogue warps
+    for (int q = 0; q < 4; ++q) mbar_init(&x_full[q], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -882,49 +928,117 @@ __global__ void __launch_bounds__(256, 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    uint8_t* xs = smem + L::kX;  // this warp's rows: 32 * quarter .. + 31 of each panel
+    int x_pending = -1;          // lane 0: the item whose raw q load nobody has waited for yet
     for (int k = 0;; ++k) {
       const int item = take_item(k);
       if (item < 0) break;
       int m, h, b, n_lo, steps;
       item_of(item, m, h, b, n_lo, steps);
       const int buf = k & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (k >> 1) & 1, abort_flag))) break;
-      tc_fence_after();
       const int i = m * 128 + row;
-      __nv_bfloat16* dst = p.dq + ((size_t)((size_t)b * p.T + i) * p.Hq + h) * D;
-      if (p.q_raw) {
-        // dq with respect to the raw q: the prologue backward on the way out (rows past T
-        // run the same warp-collective loads on row T - 1's inputs and store nothing)
-        const uint32_t src = tmem + buf * D + lane_off;
-        auto dy_chunk = [&](int c0, float (&v)[16]) {
-          uint32_t t[16];
-          tmem_ld16(src + c0, t);
-          tmem_ld_wait();
-#pragma unroll
-          for (int u = 0; u < 16; ++u) v[u] = __uint_as_float(t[u]) * p.scale;
-        };
-        const int ii = min(i, p.T - 1);
-        prologue_bwd_row<D>(dy_chunk, p.q_raw + ((size_t)((size_t)b * p.T + ii) * p.Hq + h) * D,
-                            p.rope_cs + (size_t)ii * (D / 2), p.eps, dst, i < p.T);
-      } else {
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tmem + buf * D + lane_off + c * 32, o);
-        tmem_ld_wait();
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * p.scale, __uint_as_float(o[2 * e + 1]) * p.scale);
-        if (i < p.T) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) d4[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+      if (lane == 0) {
+        // the previous item's stores must have read the rows before they are reused
+        bulk_wait_read0();
+        if (p.rope) {
+          mbar_arrive_expect_tx(&x_full[quarter], 32 * D * 2);
+          for (int pn = 0; pn < D / 64; ++pn)
+            tma_load_4d(xs + pn * 16384 + quarter * 4096, &tm_qr, &x_full[quarter], pn * 64, h, m * 128 + 32 * quarter,
+                        b);
+          x_pending = k;
         }
       }
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (k >> 1) & 1, abort_flag))) break;
+      tc_fence_after();
+      const uint32_t src = tmem + buf * D + lane_off;
+      if (p.rope) {
+        // dq with respect to the raw q: dy rotated back in TMEM, the row statistics, then
+        // dx written over the raw row
+        constexpr int H = D / 2;
+#pragma unroll 1
+        for (int j0 = 0; j0 < H; j0 += 16) {
+          uint32_t ta[16], tb[16];
+          tmem_ld16(src + j0, ta);
+          tmem_ld16(src + H + j0, tb);
+          tmem_ld_wait();
+          float a[16], bb[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) a[u] = __uint_as_float(ta[u]) * p.scale, bb[u] = __uint_as_float(tb[u]) * p.scale;
+          rope_rotate_back<D>(p.turns, (unsigned)i, j0, a, bb);
+#pragma unroll
+          for (int u = 0; u < 16; ++u) ta[u] = __float_as_uint(a[u]), tb[u] = __float_as_uint(bb[u]);
+          tmem_st16(src + j0, ta);
+          tmem_st16(src + H + j0, tb);
+        }
+        tmem_st_wait();
+        if (!__all_sync(0xffffffffu, mbar_wait(&x_full[quarter], k & 1, abort_flag))) break;
+        if (lane == 0) x_pending = -1;
+        float ss = 0.f, gx = 0.f;
+#pragma unroll 1
+        for (int j0 = 0; j0 < H; j0 += 16) {
+          uint32_t ta[16], tb[16];
+          tmem_ld16(src + j0, ta);
+          tmem_ld16(src + H + j0, tb);
+          float xa[16], xb[16];
+          tile_ld16(xs, row, j0, xa);
+          tile_ld16(xs, row, H + j0, xb);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            ss = fmaf(xa[u], xa[u], fmaf(xb[u], xb[u], ss));
+            gx = fmaf(__uint_as_float(ta[u]), xa[u], fmaf(__uint_as_float(tb[u]), xb[u], gx));
+          }
+        }
+        const float inv_r = rsqrtf(ss * (1.f / D) + p.eps);
+        const float c1 = gx * inv_r * inv_r * (1.f / D);
+#pragma unroll 1
+        for (int j0 = 0; j0 < H; j0 += 16) {
+          uint32_t ta[16], tb[16];
+          tmem_ld16(src + j0, ta);
+          tmem_ld16(src + H + j0, tb);
+          float xa[16], xb[16];
+          tile_ld16(xs, row, j0, xa);
+          tile_ld16(xs, row, H + j0, xb);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            xa[u] = (__uint_as_float(ta[u]) - xa[u] * c1) * inv_r;
+            xb[u] = (__uint_as_float(tb[u]) - xb[u] * c1) * inv_r;
+          }
+          tile_st16(xs, row, j0, xa);
+          tile_st16(xs, row, H + j0, xb);
+        }
+      } else {
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 64) {
+          uint32_t t[4][16];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) tmem_ld16(src + c0 + 16 * e, t[e]);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float v[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) v[u] = __uint_as_float(t[e][u]) * p.scale;
+            tile_st16(xs, row, c0 + 16 * e, v);
+          }
+        }
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        for (int pn = 0; pn < D / 64; ++pn)
+          tma_store_4d(&tm_dq, xs + pn * 16384 + quarter * 4096, pn * 64, h, m * 128 + 32 * quarter, b);
+        bulk_commit();
+      }
+      (void)i;
+    }
+    if (lane == 0) {
+      bulk_wait0();
+      if (x_pending >= 0) mbar_drain(&x_full[quarter], x_pending & 1);
     }
   }
   __syncthreads();
@@ -950,80 +1064,76 @@ struct PrepParams {
   uint8_t* ext_lse;
   uint8_t* ext_delta;
   int* item_counter;
-  float2* rope_cs;           // (T, D/2), or null
-  long long row_blocks;      // blocks of the row part; the blocks after them fill rope_cs
   int B, T, Tpad, Hq;
   float inv_scale;
-  // turns of rotary pair j per unit position as a 64-bit fixed-point fraction (as the
-  // prologue kernel computes its angles)
-  unsigned long long turns[64];
 };
 
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __grid_constant__ PrepParams p) {
   constexpr int LK = D / 8;
-  if (blockIdx.x >= p.row_blocks) {
-    // the cos/sin table of the rotary angles: entry (t, j) = angle t * omega_j
-    const long long e = (blockIdx.x - p.row_blocks) * (long long)blockDim.x + threadIdx.x;
-    if (e < (long long)p.T * (D / 2)) {
-      const int t = (int)(e / (D / 2)), jj = (int)(e % (D / 2));
-      const unsigned long long frac = (unsigned long long)(unsigned)t * p.turns[jj];
-      const float ang = (float)(int)(unsigned)(frac >> 32) * 1.4629180792671596e-09f;  // 2 pi / 2^32
-      float c, sn;
-      __sincosf(ang, &sn, &c);
-      p.rope_cs[e] = make_float2(c, sn);
-    }
-    return;
-  }
   // the main and dQ kernels that follow on the stream hand out their work items from
   // these two counters
   if (blockIdx.x == 0 && threadIdx.x < 2) p.item_counter[threadIdx.x] = 0;
   const int B = p.B, T = p.T, Tpad = p.Tpad, Hq = p.Hq;
   const long long rows = (long long)B * Tpad * Hq;
-  const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long long row = gtid / LK;
-  const int lr = (int)(gtid % LK);
-  const bool active = row < rows;
-  // row enumerates (b, t, h) with t over the padded length (32-bit math when it fits)
-  int h, t, b;
-  if (rows < (1ll << 31)) {
-    const unsigned r32 = active ? (unsigned)row : 0u;
-    h = (int)(r32 % (unsigned)Hq);
-    const unsigned bt = r32 / (unsigned)Hq;
-    t = (int)(bt % (unsigned)Tpad), b = (int)(bt / (unsigned)Tpad);
-  } else {
-    h = active ? (int)(row % Hq) : 0;
-    const long long bt = active ? row / Hq : 0;
-    t = (int)(bt % Tpad), b = (int)(bt / Tpad);
-  }
-  const bool real = active && t < T;
-  float dsum = 0.f;
-  if (real) {
-    const size_t off = ((size_t)((size_t)b * T + t) * Hq + h) * D + lr * 8;
-    const uint4 ov = *reinterpret_cast<const uint4*>(p.o + off);
-    const uint4 gv = *reinterpret_cast<const uint4*>(p.dout + off);
-    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
-    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+  // each thread takes kRows rows (row0 + u * kRowsPerPass), all their loads in flight
+  // before the sums
+  constexpr int kRows = 2, kRowsPerPass = 256 / LK;
+  const long long row0 = (long long)blockIdx.x * (kRows * kRowsPerPass) + threadIdx.x / LK;
+  const int lr = threadIdx.x % LK;
+  int hh[kRows], tt[kRows], bb[kRows];
+  bool real[kRows];
+  uint4 ov[kRows], gv[kRows];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float2 a = __bfloat1622float2(o2[u]), c = __bfloat1622float2(g2[u]);
-      dsum = fmaf(a.x, c.x, fmaf(a.y, c.y, dsum));
+  for (int u = 0; u < kRows; ++u) {
+    const long long row = row0 + u * kRowsPerPass;
+    const bool active = row < rows;
+    // row enumerates (b, t, h) with t over the padded length (32-bit math when it fits)
+    if (rows < (1ll << 31)) {
+      const unsigned r32 = active ? (unsigned)row : 0u;
+      hh[u] = (int)(r32 % (unsigned)Hq);
+      const unsigned bt = r32 / (unsigned)Hq;
+      tt[u] = (int)(bt % (unsigned)Tpad), bb[u] = (int)(bt / (unsigned)Tpad);
+    } else {
+      hh[u] = active ? (int)(row % Hq) : 0;
+      const long long bt = active ? row / Hq : 0;
+      tt[u] = (int)(bt % Tpad), bb[u] = (int)(bt / Tpad);
+    }
+    real[u] = active && tt[u] < T;
+    ov[u] = gv[u] = make_uint4(0, 0, 0, 0);
+    if (real[u]) {
+      const size_t off = ((size_t)((size_t)bb[u] * T + tt[u]) * Hq + hh[u]) * D + lr * 8;
+      ov[u] = *reinterpret_cast<const uint4*>(p.o + off);
+      gv[u] = *reinterpret_cast<const uint4*>(p.dout + off);
     }
   }
 #pragma unroll
-  for (int s = LK / 2; s >= 1; s >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, s);
-  if (active && lr == 0) {
-    // clamped to stay finite in bf16 (a huge 1/scale must not turn x into -inf)
-    const float x = real ? fminf(fmaxf(-p.lse[((size_t)b * Hq + h) * T + t] * p.inv_scale, -3.0e38f), 3.0e38f)
-                         : -1e30f;
-    const float y = real ? -dsum : 0.f;
-    const int i = t & 127;
-    const size_t at = (((size_t)b * Hq + h) * (Tpad / 128) + t / 128) * 512 + (i >> 3) * 32 + (i & 7) * 2;
-    const __nv_bfloat16 xh = __float2bfloat16_rn(x), yh = __float2bfloat16_rn(y);
-    *reinterpret_cast<__nv_bfloat16*>(p.ext_lse + at) = xh;
-    *reinterpret_cast<__nv_bfloat16*>(p.ext_lse + at + 16) = __float2bfloat16_rn(x - __bfloat162float(xh));
-    *reinterpret_cast<__nv_bfloat16*>(p.ext_delta + at) = yh;
-    *reinterpret_cast<__nv_bfloat16*>(p.ext_delta + at + 16) = __float2bfloat16_rn(y - __bfloat162float(yh));
+  for (int u = 0; u < kRows; ++u) {
+    const long long row = row0 + u * kRowsPerPass;
+    const int h = hh[u], t = tt[u], b = bb[u];
+    float dsum = 0.f;
+    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov[u]);
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv[u]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 a = __bfloat1622float2(o2[e]), c = __bfloat1622float2(g2[e]);
+      dsum = fmaf(a.x, c.x, fmaf(a.y, c.y, dsum));
+    }
+#pragma unroll
+    for (int sh = LK / 2; sh >= 1; sh >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, sh);
+    if (row < rows && lr == 0) {
+      // clamped to stay finite in bf16 (a huge 1/scale must not turn x into -inf)
+      const float x = real[u] ? fminf(fmaxf(-p.lse[((size_t)b * Hq + h) * T + t] * p.inv_scale, -3.0e38f), 3.0e38f)
+                              : -1e30f;
+      const float y = real[u] ? -dsum : 0.f;
+      const int i = t & 127;
+      const size_t at = (((size_t)b * Hq + h) * (Tpad / 128) + t / 128) * 512 + (i >> 3) * 32 + (i & 7) * 2;
+      const __nv_bfloat16 xh = __float2bfloat16_rn(x), yh = __float2bfloat16_rn(y);
+      *reinterpret_cast<__nv_bfloat16*>(p.ext_lse + at) = xh;
+      *reinterpret_cast<__nv_bfloat16*>(p.ext_lse + at + 16) = __float2bfloat16_rn(x - __bfloat162float(xh));
+      *reinterpret_cast<__nv_bfloat16*>(p.ext_delta + at) = yh;
+      *reinterpret_cast<__nv_bfloat16*>(p.ext_delta + at + 16) = __float2bfloat16_rn(y - __bfloat162float(yh));
+    }
   }
 }
 

@@ -163,8 +163,9 @@ attn_status_t rope_common(const void* x0, const void* x1, const void* dy0, const
 template <int D>
 attn_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int T, int Hq,
                          int Hkv, int window, float scale, cudaStream_t st) {
-  CUtensorMap tq, tk, tv;
-  if (!encode_bthd(&tq, q, B, T, Hq, D) || !encode_bthd(&tk, k, B, T, Hkv, D) || !encode_bthd(&tv, v, B, T, Hkv, D))
+  CUtensorMap tq, tk, tv, to;
+  if (!encode_bthd(&tq, q, B, T, Hq, D) || !encode_bthd(&tk, k, B, T, Hkv, D) || !encode_bthd(&tv, v, B, T, Hkv, D) ||
+      !encode_bthd(&to, o, B, T, Hq, D, 32))
     return ATTN_ERR_LAUNCH;
   if (!set_smem_attrs<D>()) return ATTN_ERR_LAUNCH;
   FwdParams p{};
@@ -179,7 +180,7 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, f
   p.n_pairs = (p.nq_tiles + 1) / 2;
   dim3 grid(Hq, B, p.n_pairs);
   // the two chunk maps are unused in training: q's map stands in for them
-  attn_fwd_kernel<D><<<grid, 384, FwdLayout<D>::kBytes, st>>>(tq, tk, tv, tq, tq, p);
+  attn_fwd_kernel<D><<<grid, 384, FwdLayout<D>::kBytes, st>>>(tq, tk, tv, tq, tq, to, p);
   return launched();
 }
 
@@ -205,7 +206,7 @@ attn_status_t launch_fwd_fp8(const void* q8, const void* k8, const void* v8, con
   p.n_pairs = (p.nq_tiles + 1) / 2;
   p.descale = descale;
   dim3 grid(Hq, B, p.n_pairs);
-  attn_fwd_kernel<D, false, true><<<grid, 384, FwdLayout<D, true>::kBytes, st>>>(tq, tk, tv, tq, tq, p);
+  attn_fwd_kernel<D, false, true><<<grid, 384, FwdLayout<D, true>::kBytes, st>>>(tq, tk, tv, tq, tq, tq, p);
   return launched();
 }
 
@@ -248,25 +249,23 @@ attn_status_t launch_prefill(const void* q, void* kc, void* vc, const void* kn, 
   p.kc = static_cast<uint4*>(kc);
   p.vc = static_cast<uint4*>(vc);
   dim3 grid(Hq, B, p.n_pairs);
-  attn_fwd_kernel<D, true><<<grid, 384, FwdLayout<D>::kBytes, st>>>(tq, tk, tv, tkn, tvn, p);
+  attn_fwd_kernel<D, true><<<grid, 384, FwdLayout<D>::kBytes, st>>>(tq, tk, tv, tkn, tvn, tq, p);
   return launched();
 }
 
-// attn_bwd's workspace: the row extensions of the S^T and dP^T MMAs (-lse/scale and
-// -Delta per query row, padded to 128-row tiles), the bf16 dS^T tiles of every (key
-// tile, query tile) pair inside the window, the two work counters, and for the block
-// backward the rotary cos/sin table.
+// attn_bwd's (and attn_block_bwd's) workspace: the row extensions of the S^T and dP^T
+// MMAs (-lse/scale and -Delta per query row, padded to 128-row tiles), the bf16 dS^T
+// tiles of every (key tile, query tile) pair inside the window, and the two work counters.
 struct BwdWorkspace {
   uint8_t* ext_lse;       // (B, Hq, Tpad / 128) x 512 bytes
   uint8_t* ext_delta;     // (B, Hq, Tpad / 128) x 512 bytes
   __nv_bfloat16* ds;      // stored dS^T tiles, 128 x 128 each
   int* counter;           // [2] work-item counters of the main and dQ kernels (zeroed by the prep kernel)
-  float2* rope_cs;        // (T, D/2) (cos, sin), block backward only
   long long tiles_per_bh;
   int span;
 };
 int eff_window(int window, int T) { return (window >= T) ? -1 : window; }
-size_t bwd_ws_parts(int B, int T, int Hq, int D, int window, bool rope, BwdWorkspace* w, void* base) {
+size_t bwd_ws_parts(int B, int T, int Hq, int window, BwdWorkspace* w, void* base) {
   const int nt = tiles128(T);
   const size_t Tpad = (size_t)nt * 128;
   const int span = bwd_span(nt, eff_window(window, T));
@@ -282,13 +281,11 @@ size_t bwd_ws_parts(int B, int T, int Hq, int D, int window, bool rope, BwdWorks
   uint8_t* e2 = take((size_t)B * Hq * Tpad * 4);
   uint8_t* ds = take((size_t)B * Hq * tiles * 32768);
   uint8_t* cnt = take(256);
-  uint8_t* cs = rope ? take((size_t)T * (D / 2) * 8) : nullptr;
   if (w) {
     w->ext_lse = e1;
     w->ext_delta = e2;
     w->ds = reinterpret_cast<__nv_bfloat16*>(ds);
     w->counter = reinterpret_cast<int*>(cnt);
-    w->rope_cs = reinterpret_cast<float2*>(cs);
     w->tiles_per_bh = tiles;
     w->span = span;
   }
@@ -311,11 +308,22 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
   const int Tpad = nt * 128;
   const bool rope = rb.q_raw != nullptr;
   BwdWorkspace w;
-  bwd_ws_parts(B, T, Hq, D, window, rope, &w, ws);
-  CUtensorMap tq, tk, tv, tdo;
+  bwd_ws_parts(B, T, Hq, window, &w, ws);
+  // operands (128-row boxes), the outputs (32-row boxes: one per epilogue warp), and
+  // for the block backward the raw k (128 rows, one load per tile) and q (32 rows)
+  CUtensorMap tq, tk, tv, tdo, tdk, tdv, tdq, tkr, tqr;
   if (!encode_bthd(&tq, q, B, T, Hq, D) || !encode_bthd(&tk, k, B, T, Hkv, D) ||
-      !encode_bthd(&tv, v, B, T, Hkv, D) || !encode_bthd(&tdo, dO, B, T, Hq, D))
+      !encode_bthd(&tv, v, B, T, Hkv, D) || !encode_bthd(&tdo, dO, B, T, Hq, D) ||
+      !encode_bthd(&tdk, dk, B, T, Hkv, D, 32) || !encode_bthd(&tdv, dv, B, T, Hkv, D, 32) ||
+      !encode_bthd(&tdq, dq, B, T, Hq, D, 32))
     return ATTN_ERR_LAUNCH;
+  if (rope) {
+    if (!encode_bthd(&tkr, rb.k_raw, B, T, Hkv, D) || !encode_bthd(&tqr, rb.q_raw, B, T, Hq, D, 32))
+      return ATTN_ERR_LAUNCH;
+  } else {
+    tkr = tk;  // not read
+    tqr = tdq;
+  }
   if (!set_smem_attrs<D>()) return ATTN_ERR_LAUNCH;
   {
     PrepParams pp{};
@@ -325,28 +333,19 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
     pp.ext_lse = w.ext_lse;
     pp.ext_delta = w.ext_delta;
     pp.item_counter = w.counter;
-    pp.rope_cs = w.rope_cs;
     pp.B = B;
     pp.T = T;
     pp.Tpad = Tpad;
     pp.Hq = Hq;
     pp.inv_scale = 1.f / scale;
-    const long long threads = (long long)B * Tpad * Hq * (D / 8);
-    pp.row_blocks = (threads + 255) / 256;
-    long long blocks = pp.row_blocks;
-    if (rope) {
-      rope_turns(D, rb.base, pp.turns);
-      blocks += ((long long)T * (D / 2) + 255) / 256;
-    }
-    attn_bwd_prep_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(pp);
+    // 256 threads take 2 * 256 / (D / 8) rows (D / 8 lanes per row, two rows per lane)
+    const long long rows = (long long)B * Tpad * Hq, per_block = 2 * 256 / (D / 8);
+    attn_bwd_prep_kernel<D><<<(unsigned)((rows + per_block - 1) / per_block), 256, 0, st>>>(pp);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
   }
   BwdParams p{};
   p.ext_lse = w.ext_lse;
   p.ext_delta = w.ext_delta;
-  p.dk = static_cast<__nv_bfloat16*>(dk);
-  p.dv = static_cast<__nv_bfloat16*>(dv);
-  p.dq = static_cast<__nv_bfloat16*>(dq);
   p.ds = w.ds;
   p.item_counter = w.counter;
   p.T = T;
@@ -359,20 +358,20 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
   p.tiles_per_bh = w.tiles_per_bh;
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
-  p.k_raw = static_cast<const __nv_bfloat16*>(rb.k_raw);
-  p.q_raw = static_cast<const __nv_bfloat16*>(rb.q_raw);
-  p.rope_cs = w.rope_cs;
+  p.rope = rope ? 1 : 0;
   p.eps = rb.eps;
+  if (rope) rope_turns(D, rb.base, p.turns);
   {
     // persistent: one CTA per SM walks the (key tile, KV head, batch) items
     const long long kv_items = (long long)nt * Hkv * B;
     const int kv_grid = (int)std::min<long long>(kv_items, sm_count());
-    attn_bwd_kernel<D><<<kv_grid, 384, BwdLayout<D>::kBytes, st>>>(tq, tk, tv, tdo, p, (int)kv_items);
+    attn_bwd_kernel<D><<<kv_grid, 384, BwdLayout<D>::kBytes, st>>>(tq, tk, tv, tdo, tkr, tdk, tdv, p,
+                                                                    (int)kv_items);
   }
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
   const long long items = (long long)nt * Hq * B;
   const int grid = (int)std::min<long long>(items, sm_count());
-  attn_bwd_dq_kernel<D><<<grid, 256, DqLayout<D>::kBytes, st>>>(tk, p, (int)items);
+  attn_bwd_dq_kernel<D><<<grid, 256, DqLayout<D>::kBytes, st>>>(tk, tqr, tdq, p, (int)items);
   return launched();
 }
 
@@ -443,14 +442,14 @@ attn_status_t bwd_common(const void* q, const void* k, const void* v, const void
                !std::isfinite(rb.base) || !(rb.eps >= 0.f) || !std::isfinite(rb.eps)))
     return ATTN_ERR_INVALID_ARG;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
-      ws_bytes < bwd_ws_parts(B, T, Hq, D, window, rope, nullptr, nullptr))
+      ws_bytes < bwd_ws_parts(B, T, Hq, window, nullptr, nullptr))
     return ATTN_ERR_INVALID_ARG;
   if (Hq > 65535 || B > 65535 || tiles128(T) > 65535) return ATTN_ERR_INVALID_ARG;
   // stored dS^T tile rows, the dQ kernel's work items and the prep kernel's blocks are
   // counted in 32 bits
   const int nt = tiles128(T);
   if ((long long)B * Hq * ds_tiles_before(nt, nt, bwd_span(nt, eff_window(window, T))) * 128 >= (1ll << 31) ||
-      (long long)B * nt * 128 * Hq * (D / 8) / 256 + (long long)T * D / 512 >= (1ll << 31))
+      (long long)B * nt * 128 * Hq * (D / 8) / 256 >= (1ll << 31))
     return ATTN_ERR_UNSUPPORTED;
   cudaStream_t st = as_stream(stream);
   return D == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, workspace, B, T, Hq, Hkv, window, scale, rb, st)
@@ -486,12 +485,12 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
 
 size_t attn_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int window) {
   if (!dims_ok(B, T, Hq, Hkv) || (D != 64 && D != 128)) return 0;
-  return bwd_ws_parts(B, T, Hq, D, window, false, nullptr, nullptr);
+  return bwd_ws_parts(B, T, Hq, window, nullptr, nullptr);
 }
 
 size_t attn_block_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int window) {
   if (!dims_ok(B, T, Hq, Hkv) || (D != 64 && D != 128)) return 0;
-  return bwd_ws_parts(B, T, Hq, D, window, true, nullptr, nullptr);
+  return bwd_ws_parts(B, T, Hq, window, nullptr, nullptr);
 }
 
 

@@ -86,10 +86,14 @@ template <int D, bool kCache = false, bool kFp8 = false>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kn,
-                    const __grid_constant__ CUtensorMap tm_vn, const FwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_vn, const __grid_constant__ CUtensorMap tm_o,
+                    const FwdParams p) {
   static_assert(!kFp8 || (D == 128 && !kCache), "the fp8 forward takes D = 128, training layout");
   using L = FwdLayout<D, kFp8>;
   constexpr int kPanelElems = 128 / L::kElem;  // elements across one 128-byte panel
+  // the bf16 training forward writes o with TMA stores from the slot's Q tile (tm_o:
+  // 32-row boxes); the prefill and the fp8 forward store rows directly
+  constexpr bool kTmaO = !kCache && !kFp8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
@@ -514,7 +518,33 @@ __global__ void __launch_bounds__(384, 1)
       if (ok && cnt > 0) ok = mbar_wait(&pv_done[s], (cnt - 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
-      if (ok) {
+      if (ok && kTmaO) {
+        // O / l as bf16 rows of the slot's Q tile (every S of the slot has read it), in
+        // the TMA layout; the warp stores its 32 rows (rows past T are not written)
+        const int cr = my_qt * 128 + row;
+        const float inv_l = 1.f / l_run;
+        uint8_t* stg = smem + (s ? L::kQ1 : L::kQ0);
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t t0[16], t1[16];
+          tmem_ld16(tOs + c0, t0);
+          tmem_ld16(tOs + c0 + 16, t1);
+          tmem_ld_wait();
+          float v0[16], v1[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) v0[u] = __uint_as_float(t0[u]) * inv_l, v1[u] = __uint_as_float(t1[u]) * inv_l;
+          tile_st16(stg, row, c0, v0);
+          tile_st16(stg, row, c0 + 16, v1);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          for (int pn = 0; pn < D / 64; ++pn)
+            tma_store_4d(&tm_o, stg + pn * 16384 + quarter * 4096, pn * 64, h, my_qt * 128 + 32 * quarter, b);
+          bulk_commit();
+        }
+        if (cr < p.T) p.lse[((size_t)b * p.Hq + h) * p.T + cr] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+      } else if (ok) {
         // tcgen05.ld is warp-collective: every lane loads, only rows of [0, T) store
         const int cr = my_qt * 128 - shift + row;  // output row (chunk row in kCache)
         const bool store = (cr < p.T) && (!kCache || cr >= 0);
@@ -543,6 +573,8 @@ __global__ void __launch_bounds__(384, 1)
     }
   }
 
+  // the o stores have completed before the CTA's shared memory goes
+  if (kTmaO && warp >= 4 && lane == 0) bulk_wait0();
   __syncthreads();
   if (warp == 2) {
     tc_fence_after();

@@ -129,10 +129,7 @@ __global__ void __launch_bounds__(256, 4) rope_qknorm_kernel(const __grid_consta
         float c = 1.f, sn = 0.f;
         if (bt < n_pos) {
           const int t = (int)(bt % p.T), b = (int)(bt / p.T);
-          const unsigned long long pos = (unsigned long long)(unsigned)(t + (p.pos ? p.pos[b] : 0));
-          const unsigned long long frac = pos * p.turns[j];
-          const float ang = (float)(int)(unsigned)(frac >> 32) * 1.4629180792671596e-09f;  // 2 pi / 2^32
-          __sincosf(ang, &sn, &c);
+          rope_cos_sin((unsigned)(t + (p.pos ? p.pos[b] : 0)), p.turns[j], c, sn);
         }
         reinterpret_cast<float2*>(&cs4[pi][0])[j] = make_float2(c, sn);
       }

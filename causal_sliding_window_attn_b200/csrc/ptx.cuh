@@ -149,6 +149,27 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* m, uin
       : "memory");
 }
 
+// 4-D tiled store shared -> global, tracked in the issuing thread's bulk async-group.
+// Rows past the tensor's extent are not written.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* m, const void* src, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+// 4-D tile of a tensor map into L2 (no shared memory, no completion to wait for)
+__device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap* m, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the thread's committed bulk stores have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// ... and have completed
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // ---------------------------------------------------------------- tcgen05
 // Instruction descriptor for kind::f16 with bf16 A/B and an f32 accumulator.
 // a_mn / b_mn select MN-major (transposed) operands in shared memory.
@@ -333,15 +354,15 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
                "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
                : "memory");
 }
+// 32 lanes x 2 consecutive 32-bit columns
+__device__ __forceinline__ void tmem_ld2(uint32_t taddr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st2(uint32_t taddr, uint32_t r0, uint32_t r1) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr), "r"(r0), "r"(r1) : "memory");
+}
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// ---------------------------------------------------------------- global reductions
-// *addr += (a, b, c, d) as one 16-byte fp32 reduction in L2 (no return value)
-__device__ __forceinline__ void red_add_f32x4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
 
 // ---------------------------------------------------------------- misc math
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -357,6 +378,39 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+// cos and sin of the rotary angle p * omega_j, given U_j = (omega_j / (2 pi)) * 2^64 (the
+// turns of pair j per unit position, 64-bit fixed point): p * U_j mod 2^64 is the angle
+// in turns, exact for any 32-bit position, and its top 32 bits read as signed give the
+// reduced angle in [-pi, pi).
+__device__ __forceinline__ void rope_cos_sin(unsigned pos, unsigned long long turn, float& c, float& s) {
+  const unsigned long long frac = (unsigned long long)pos * turn;
+  const float ang = (float)(int)(unsigned)(frac >> 32) * 1.4629180792671596e-09f;  // 2 pi / 2^32
+  __sincosf(ang, &s, &c);
+}
+// 16 consecutive bf16 columns c0 .. c0+15 (c0 a multiple of 16) of row r of a 128-row
+// tile in the 128-byte-swizzled panel layout TMA uses (64 columns per 16 KB panel, 128
+// bytes per row, 16-byte unit u of row r stored at unit u ^ (r & 7)). A warp of 32
+// consecutive rows touches every bank 4 times per access: no conflicts beyond that.
+__device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
+  return (uint32_t)((c >> 6) * 16384 + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4));
+}
+__device__ __forceinline__ void tile_ld16(const uint8_t* tile, int r, int c0, float (&v)[16]) {
+  const uint4 a = *reinterpret_cast<const uint4*>(tile + sw128_offset(r, c0));
+  const uint4 b = *reinterpret_cast<const uint4*>(tile + sw128_offset(r, c0 + 8));
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    v[2 * u] = __uint_as_float(w[u] << 16);
+    v[2 * u + 1] = __uint_as_float(w[u] & 0xffff0000u);
+  }
+}
+__device__ __forceinline__ void tile_st16(uint8_t* tile, int r, int c0, const float (&v)[16]) {
+  uint32_t w[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) w[u] = pack_bf16x2(v[2 * u], v[2 * u + 1]);
+  *reinterpret_cast<uint4*>(tile + sw128_offset(r, c0)) = make_uint4(w[0], w[1], w[2], w[3]);
+  *reinterpret_cast<uint4*>(tile + sw128_offset(r, c0 + 8)) = make_uint4(w[4], w[5], w[6], w[7]);
 }
 __device__ __forceinline__ uint32_t warp_id() { return threadIdx.x >> 5; }
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }

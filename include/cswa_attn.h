@@ -109,8 +109,8 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
                        const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B,
                        int T, int Hq, int Hkv, int D, int window, float scale, void* stream);
 
-/* Bytes of workspace attn_block_bwd needs: attn_bwd's, plus the rotary cos/sin table
- * (T*D/2*8 bytes, rounded up to 256). */
+/* Bytes of workspace attn_block_bwd needs: the same as attn_bwd's (the rotary angles
+ * are computed in the kernels, from each row's position). */
 size_t attn_block_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int window);
 
 /*
@@ -121,7 +121,8 @@ size_t attn_block_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int 
  *   q_hat, k_hat = attn_rope_qknorm(q, k) (pos null),  o = attn_fwd(q_hat, k_hat, v).
  * It computes what attn_bwd followed by attn_rope_qknorm_bwd computes, with the
  * prologue backward done on the way out of the kernels (the dK epilogue of the
- * main kernel and the dq pass): dq_hat and dk_hat never reach memory.
+ * main kernel and the dQ kernel's epilogue, each on a raw tile it loads by TMA):
+ * dq_hat and dk_hat never reach memory.
  *   q (B,T,Hq,D), k (B,T,Hkv,D): the raw inputs of the prologue.
  *   q_hat, k_hat: the prologue's outputs for them (rope_base, eps as given here).
  *   v, o, dO, lse: as for attn_bwd. Outputs dq, dk (raw-input gradients) and dv.

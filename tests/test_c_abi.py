@@ -51,11 +51,11 @@ def test_bwd_workspace_size(L):
     full = 2 * rows + B * Hq * 136 * 32768 + 256
     assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, -1) == full
     assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, 2048) == full
-    # the block backward adds the (T, D/2) cos/sin table of float pairs
-    assert L.attn_block_bwd_workspace_bytes(B, T, Hq, Hkv, D, -1) == full + T * 64 * 8
+    # the block backward needs no more (its rotary angles are computed in the kernels)
+    assert L.attn_block_bwd_workspace_bytes(B, T, Hq, Hkv, D, -1) == full
     # ragged T pads the per-row arrays to whole 128-row tiles; window 0 keeps the diagonal only
     assert L.attn_bwd_workspace_bytes(1, 130, 2, 1, 64, 0) == 2 * 2048 + 2 * 2 * 32768 + 256
-    assert L.attn_block_bwd_workspace_bytes(1, 3, 1, 1, 64, -1) == 2 * 512 + 32768 + 256 + 768
+    assert L.attn_block_bwd_workspace_bytes(1, 3, 1, 1, 64, -1) == 2 * 512 + 32768 + 256
     assert L.attn_bwd_workspace_bytes(1, 16, 3, 2, 128, -1) == 0     # Hq % Hkv != 0
     assert L.attn_bwd_workspace_bytes(1, 16, 2, 2, 96, -1) == 0      # head dim
 
@@ -110,7 +110,7 @@ def test_block_bwd_rejects_bad_args(L):
         a = list(base)
         a[i] = v
         return L.attn_block_bwd(*a)
-    assert call(12, L.attn_bwd_workspace_bytes(1, 128, 4, 2, 128, 64)) == INVALID  # no room for the table
+    assert call(12, ws - 1) == INVALID                # workspace too small
     assert call(0, None) == INVALID                   # null raw q
     assert call(1, MIS) == INVALID                    # misaligned raw k
     assert call(20, f(1.0)) == INVALID                # rope base
