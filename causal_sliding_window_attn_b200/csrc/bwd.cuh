@@ -523,6 +523,18 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
     int g0 = 0, k = 0;
     int kr_pending = -1;  // warp 4, lane 0: the item whose raw k load nobody has waited for yet
+    // the ring stage this warp lent its last epilogue, returned once the TMA stores have
+    // read it: during the next item's first P phase, so that the read overlaps the
+    // exponentials (the dO stage after the first chunk, as the producer reloads it a step
+    // ahead; the Q stage after the last)
+    int lent_stage = -1;
+    auto return_stage = [&]() {
+      if (lane == 0) {
+        bulk_wait_read0();
+        mbar_arrive(half ? &do_borrow[lent_stage] : &q_borrow[lent_stage]);
+      }
+      lent_stage = -1;
+    };
     for (;; ++k) {
       const int item = take_item(k);
       if (item < 0) break;
@@ -578,6 +590,7 @@ __global__ void __launch_bounds__(384, 1)
           mbar_arrive(&p_chunk[c]);
           if (tracer && c == 0) CSWA_MARK(trole, g, 3);
           if (ds_dst) store_ds_units(2 * c, 2 * c + 2);
+          if (lent_stage >= 0 && c == (half ? 0 : 3)) return_stage();
         }
         const float* pf = reinterpret_cast<const float*>(sr);
         if (tracer) CSWA_MARK(trole, g, 4);
@@ -627,6 +640,7 @@ __global__ void __launch_bounds__(384, 1)
       uint8_t* stage = smem + (half ? L::kDO : L::kQ) + st_last * L::kTile;
       // (profiling builds: epilogue marks of the CTA's first 8 items at steps 56-63)
       const int emark = 56 + (k & 7);
+      (void)emark;
       if (tracer && k < 8) CSWA_MARK(trole, emark, 0);
       ok = __all_sync(0xffffffffu, half ? mbar_wait(&do_empty[st_last], (g_last / DS) & 1, abort_flag)
                                         : mbar_wait(final_bar, k & 1, abort_flag));
@@ -731,12 +745,11 @@ __global__ void __launch_bounds__(384, 1)
                        I.b);
         bulk_commit();
         if (tracer && k < 8) CSWA_MARK(trole, emark, 3);
-        bulk_wait_read0();
-        if (tracer && k < 8) CSWA_MARK(trole, emark, 4);
-        mbar_arrive(half ? &do_borrow[st_last] : &q_borrow[st_last]);
       }
+      lent_stage = st_last;
       g0 += I.n_iters;
     }
+    if (lent_stage >= 0) return_stage();
     // before the CTA's shared memory goes: the stores have completed, and a raw k load
     // left behind by an abort has landed
     if (lane == 0) bulk_wait0();

@@ -50,10 +50,6 @@ __device__ __forceinline__ void bf16x8_to_float(const uint4& v, float (&f)[8]) {
   }
 }
 
-__device__ __forceinline__ void prefetch_l2(const __nv_bfloat16* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-
 __device__ __forceinline__ uint4 ld_stream(const __nv_bfloat16* p) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -174,18 +170,6 @@ __global__ void __launch_bounds__(128, decode_min_blocks(GMAX)) decode_chunk_ker
     if (append && k_begin + kc == P) return ld_stream(fresh + fresh_off);
     return ld_stream(cache + cache_off + u * pass_stride);
   };
-
-  // Every cache row of the chunk is requested into L2 at once (thread tid: row tid of
-  // K and of V, two 128-byte lines each), so the chunk's 64 KB are in flight while
-  // the scores are computed and pass 3 reads V from L2.
-  if (tid < nk && !(append && k_begin + tid == P)) {
-    const size_t roff = (((size_t)b * p.Tmax + k_begin + tid) * p.Hkv + hk) * D;
-#pragma unroll
-    for (int e = 0; e < D; e += 64) {
-      prefetch_l2(p.kc + roff + e);
-      prefetch_l2(p.vc + roff + e);
-    }
-  }
 
   // the group's query heads in sub-groups of GMAX (only the widest instantiation sees
   // groups larger than GMAX); a sub-group after the first reads the chunk's rows
