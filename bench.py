@@ -104,7 +104,8 @@ def decode_bytes(lengths, Hq, Hkv, D, W):
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     """Samples the SM clock and the clock-event (throttle) reasons while running: through
-    NVML every 5 ms when the binding is present (short timed regions still get several
+    NVML every millisecond when the binding is present (NVML is set up when the sampler is
+    made, before the timed region, so that a region of a few milliseconds still gets
     samples), else through nvidia-smi every 200 ms."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -117,6 +118,17 @@ class ClockSampler:
         self.source = None
         self._stop = threading.Event()
         self._t = None
+        self._nvml = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = self._nvml_handle(pynvml)
+            bits = [pynvml.nvmlClocksEventReasonHwSlowdown, pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                    pynvml.nvmlClocksEventReasonSwThermalSlowdown, pynvml.nvmlClocksEventReasonSwPowerCap]
+            mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self._nvml = (pynvml, h, bits, mx)
+        except Exception:
+            self._nvml = None
 
     def _nvml_handle(self, pynvml):
         try:
@@ -126,18 +138,13 @@ class ClockSampler:
             return pynvml.nvmlDeviceGetHandleByIndex(self.index)
 
     def _run_nvml(self):
-        import pynvml
-        pynvml.nvmlInit()
-        h = self._nvml_handle(pynvml)
-        bits = [pynvml.nvmlClocksEventReasonHwSlowdown, pynvml.nvmlClocksEventReasonHwThermalSlowdown,
-                pynvml.nvmlClocksEventReasonSwThermalSlowdown, pynvml.nvmlClocksEventReasonSwPowerCap]
-        mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
-        self.source = "nvml, 5 ms"
+        pynvml, h, bits, mx = self._nvml
+        self.source = "nvml, 1 ms"
         while not self._stop.is_set():
             sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
             r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
             self.rows.append((float(sm), float(mx), [n for n, b in zip(self.NAMES, bits) if r & b]))
-            self._stop.wait(0.005)
+            self._stop.wait(0.001)
 
     def _run_smi(self):
         self.source = "nvidia-smi, 200 ms"
@@ -155,10 +162,12 @@ class ClockSampler:
             self._stop.wait(0.2)
 
     def _run(self):
-        try:
-            self._run_nvml()
-        except Exception:
-            self._run_smi()
+        if self._nvml is not None:
+            try:
+                return self._run_nvml()
+            except Exception:
+                pass
+        self._run_smi()
 
     def __enter__(self):
         self._t = threading.Thread(target=self._run, daemon=True)
