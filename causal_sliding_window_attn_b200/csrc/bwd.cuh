@@ -1083,58 +1083,55 @@ struct PrepParams {
 
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __grid_constant__ PrepParams p) {
-  constexpr int LK = D / 8;
+  // blockIdx.y = batch b; the block's rows are (t, h) rows of that batch, t over the
+  // padded length. LK lanes per row, 16 elements each; every thread takes kRows rows
+  // (r0 + u * kRowsPerPass) with all their loads in flight before the sums, and forms
+  // o . dO with mixed bf16 x bf16 -> fp32 FMAs (no conversions).
+  constexpr int LK = D / 16;
+  constexpr int kRows = 2, kRowsPerPass = 256 / LK;
   // the main and dQ kernels that follow on the stream hand out their work items from
   // these two counters
-  if (blockIdx.x == 0 && threadIdx.x < 2) p.item_counter[threadIdx.x] = 0;
-  const int B = p.B, T = p.T, Tpad = p.Tpad, Hq = p.Hq;
-  const long long rows = (long long)B * Tpad * Hq;
-  // each thread takes kRows rows (row0 + u * kRowsPerPass), all their loads in flight
-  // before the sums
-  constexpr int kRows = 2, kRowsPerPass = 256 / LK;
-  const long long row0 = (long long)blockIdx.x * (kRows * kRowsPerPass) + threadIdx.x / LK;
-  const int lr = threadIdx.x % LK;
-  int hh[kRows], tt[kRows], bb[kRows];
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 2) p.item_counter[threadIdx.x] = 0;
+  const int b = blockIdx.y;
+  const int T = p.T, Tpad = p.Tpad, Hq = p.Hq;
+  const int rows = Tpad * Hq;  // < 2^31 (the host checks the stored tile rows, which bound it)
+  const int r0 = blockIdx.x * (kRows * kRowsPerPass) + (int)threadIdx.x / LK;
+  const int lr = (int)threadIdx.x % LK;
+  int hh[kRows], tt[kRows];
   bool real[kRows];
-  uint4 ov[kRows], gv[kRows];
+  uint4 ov[kRows][2], gv[kRows][2];
 #pragma unroll
   for (int u = 0; u < kRows; ++u) {
-    const long long row = row0 + u * kRowsPerPass;
-    const bool active = row < rows;
-    // row enumerates (b, t, h) with t over the padded length (32-bit math when it fits)
-    if (rows < (1ll << 31)) {
-      const unsigned r32 = active ? (unsigned)row : 0u;
-      hh[u] = (int)(r32 % (unsigned)Hq);
-      const unsigned bt = r32 / (unsigned)Hq;
-      tt[u] = (int)(bt % (unsigned)Tpad), bb[u] = (int)(bt / (unsigned)Tpad);
-    } else {
-      hh[u] = active ? (int)(row % Hq) : 0;
-      const long long bt = active ? row / Hq : 0;
-      tt[u] = (int)(bt % Tpad), bb[u] = (int)(bt / Tpad);
-    }
-    real[u] = active && tt[u] < T;
-    ov[u] = gv[u] = make_uint4(0, 0, 0, 0);
+    const int r = r0 + u * kRowsPerPass;
+    tt[u] = r / Hq;
+    hh[u] = r - tt[u] * Hq;
+    real[u] = r < rows && tt[u] < T;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) ov[u][e] = gv[u][e] = make_uint4(0, 0, 0, 0);
     if (real[u]) {
-      const size_t off = ((size_t)((size_t)bb[u] * T + tt[u]) * Hq + hh[u]) * D + lr * 8;
-      ov[u] = *reinterpret_cast<const uint4*>(p.o + off);
-      gv[u] = *reinterpret_cast<const uint4*>(p.dout + off);
+      const size_t off = ((size_t)((size_t)b * T + tt[u]) * Hq + hh[u]) * D + lr * 16;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        ov[u][e] = *reinterpret_cast<const uint4*>(p.o + off + 8 * e);
+        gv[u][e] = *reinterpret_cast<const uint4*>(p.dout + off + 8 * e);
+      }
     }
   }
 #pragma unroll
   for (int u = 0; u < kRows; ++u) {
-    const long long row = row0 + u * kRowsPerPass;
-    const int h = hh[u], t = tt[u], b = bb[u];
+    const int r = r0 + u * kRowsPerPass;
+    const int h = hh[u], t = tt[u];
     float dsum = 0.f;
-    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov[u]);
-    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv[u]);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 a = __bfloat1622float2(o2[e]), c = __bfloat1622float2(g2[e]);
-      dsum = fmaf(a.x, c.x, fmaf(a.y, c.y, dsum));
+    for (int e = 0; e < 2; ++e) {
+      dsum = fma_bf16x2_f32(ov[u][e].x, gv[u][e].x, dsum);
+      dsum = fma_bf16x2_f32(ov[u][e].y, gv[u][e].y, dsum);
+      dsum = fma_bf16x2_f32(ov[u][e].z, gv[u][e].z, dsum);
+      dsum = fma_bf16x2_f32(ov[u][e].w, gv[u][e].w, dsum);
     }
 #pragma unroll
     for (int sh = LK / 2; sh >= 1; sh >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, sh);
-    if (row < rows && lr == 0) {
+    if (r < rows && lr == 0) {
       // clamped to stay finite in bf16 (a huge 1/scale must not turn x into -inf)
       const float x = real[u] ? fminf(fmaxf(-p.lse[((size_t)b * Hq + h) * T + t] * p.inv_scale, -3.0e38f), 3.0e38f)
                               : -1e30f;

@@ -338,9 +338,10 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
     pp.Tpad = Tpad;
     pp.Hq = Hq;
     pp.inv_scale = 1.f / scale;
-    // 256 threads take 2 * 256 / (D / 8) rows (D / 8 lanes per row, two rows per lane)
-    const long long rows = (long long)B * Tpad * Hq, per_block = 2 * 256 / (D / 8);
-    attn_bwd_prep_kernel<D><<<(unsigned)((rows + per_block - 1) / per_block), 256, 0, st>>>(pp);
+    // per batch, 256 threads take 2 * 256 / (D / 16) rows (D / 16 lanes per row, two rows
+    // per lane)
+    const long long rows = (long long)Tpad * Hq, per_block = 2 * 256 / (D / 16);
+    attn_bwd_prep_kernel<D><<<dim3((unsigned)((rows + per_block - 1) / per_block), (unsigned)B), 256, 0, st>>>(pp);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
   }
   BwdParams p{};
@@ -445,11 +446,10 @@ attn_status_t bwd_common(const void* q, const void* k, const void* v, const void
       ws_bytes < bwd_ws_parts(B, T, Hq, window, nullptr, nullptr))
     return ATTN_ERR_INVALID_ARG;
   if (Hq > 65535 || B > 65535 || tiles128(T) > 65535) return ATTN_ERR_INVALID_ARG;
-  // stored dS^T tile rows, the dQ kernel's work items and the prep kernel's blocks are
-  // counted in 32 bits
+  // stored dS^T tile rows, the dQ kernel's work items and the prep kernel's rows per batch
+  // (Tpad * Hq, no more than the tile rows) are counted in 32 bits
   const int nt = tiles128(T);
-  if ((long long)B * Hq * ds_tiles_before(nt, nt, bwd_span(nt, eff_window(window, T))) * 128 >= (1ll << 31) ||
-      (long long)B * nt * 128 * Hq * (D / 8) / 256 >= (1ll << 31))
+  if ((long long)B * Hq * ds_tiles_before(nt, nt, bwd_span(nt, eff_window(window, T))) * 128 >= (1ll << 31))
     return ATTN_ERR_UNSUPPORTED;
   cudaStream_t st = as_stream(stream);
   return D == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, workspace, B, T, Hq, Hkv, window, scale, rb, st)

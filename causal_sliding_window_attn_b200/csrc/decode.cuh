@@ -58,15 +58,6 @@ __device__ __forceinline__ uint4 ld_stream(const __nv_bfloat16* p) {
   return v;
 }
 
-// d += a.lo * b.lo + a.hi * b.hi for packed bf16 pairs, accumulated in fp32 (the
-// products of two bf16 values are exact in fp32): no conversion instructions.
-__device__ __forceinline__ float fma_bf16x2_f32(uint32_t a, uint32_t b, float d) {
-  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
-      "fma.rn.f32.bf16 %0, al, bl, %0;\n\tfma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
-      : "+f"(d)
-      : "r"(a), "r"(b));
-  return d;
-}
 // d_lo += p * b.lo, d_hi += p * b.hi with p a bf16 value (in the low half of pp)
 __device__ __forceinline__ void fma_bf16_pair_f32(uint32_t pp, uint32_t b, float& lo, float& hi) {
   asm("{\n\t.reg .b16 p, x, bl, bh;\n\tmov.b32 {p, x}, %2;\n\tmov.b32 {bl, bh}, %3;\n\t"
