@@ -27,7 +27,7 @@ import torch
 
 __all__ = [
     "AttnError", "lib", "attn_rope_qknorm", "attn_rope_qknorm_bwd", "attn_fwd", "attn_bwd",
-    "attn_bwd_workspace_bytes", "attn_block_bwd", "attn_block_bwd_workspace_bytes", "attn_quantize_fp8",
+    "attn_bwd_workspace_bytes", "attn_bwd_workspace_min_bytes", "attn_block_bwd", "attn_block_bwd_workspace_bytes", "attn_quantize_fp8",
     "attn_fwd_fp8", "attn_decode", "attn_decode_workspace_bytes", "attn_prefill", "attn_layer_window",
     "layer_windows", "attn_kv_replicate", "attn_get_status", "attn_debug_set_wait_limit",
     "attn_status_string", "LIB_PATH",
@@ -45,6 +45,7 @@ _SIGS = {
     "attn_rope_qknorm_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _f, _vp]),
     "attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "attn_bwd_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "attn_bwd_workspace_min_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "attn_bwd": (_i, [_vp] * 9 + [_vp, _sz, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "attn_block_bwd_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "attn_block_bwd": (_i, [_vp] * 12 + [_sz, _i, _i, _i, _i, _i, _i, _f, _f, _f, _vp]),
@@ -204,9 +205,14 @@ def attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, window=-1):
     return int(lib().attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, int(window)))
 
 
+def attn_bwd_workspace_min_bytes(B, T, Hq, Hkv, D, window=-1):
+    return int(lib().attn_bwd_workspace_min_bytes(B, T, Hq, Hkv, D, int(window)))
+
+
 def attn_bwd(q, k, v, o, dout, lse, window=-1, scale=None, dq=None, dk=None, dv=None, workspace=None,
              stream=None):
-    """dq, dk, dv of sum(dout * o) for o = attn_fwd(q, k, v)."""
+    """dq, dk, dv of sum(dout * o) for o = attn_fwd(q, k, v). A workspace smaller than
+    attn_bwd_workspace_bytes (down to attn_bwd_workspace_min_bytes) runs in passes."""
     B, T, Hq, D = _bf16("q", q).shape
     Hkv = _bf16("k", k).shape[2]
     for name, t in (("v", v), ("o", o), ("dout", dout)):

@@ -71,6 +71,10 @@ struct BwdParams {
   int* item_counter;   // [2] next work item of the main and dQ kernels (zeroed by the prep kernel)
   int T, Tpad, Hq, G, window, n_tiles, span;  // tiles of 128 rows; span = query tiles per key tile
   long long tiles_per_bh;                     // stored dS^T tiles per (batch, query head)
+  // the call may run in passes over the (batch, KV head) blocks, blk = b * Hkv + hk: this
+  // launch covers blocks blk0 .. blk0 + n_items / n_tiles - 1, and the stored dS^T tiles of
+  // block blk0 start at the beginning of p.ds
+  int blk0;
   float scale, scale_log2;
   // fused prologue backward (attn_block_bwd): dk and dq with respect to the raw k and
   // q (whose tensor maps the kernels take), the RMS-norm eps and the turns of rotary
@@ -222,6 +226,7 @@ __global__ void __launch_bounds__(384, 1)
     Item it;
     int blk;
     sb_order(item, p.n_tiles, n_items / p.n_tiles, it.n, blk);
+    blk += p.blk0;
     it.hk = blk % (p.Hq / G);
     it.b = blk / (p.Hq / G);
     it.m_cnt = min(p.n_tiles - it.n, p.span);
@@ -542,7 +547,8 @@ __global__ void __launch_bounds__(384, 1)
       const int k0 = I.n * 128;
       const int j = k0 + r;
       // the item's first stored dS^T tile (key tile n of batch b, query head 0)
-      const long long tile0 = ((long long)I.b * p.Hq) * p.tiles_per_bh + ds_tiles_before(I.n, p.n_tiles, p.span);
+      const long long tile0 = ((long long)I.b * p.Hq - (long long)p.blk0 * G) * p.tiles_per_bh +
+                              ds_tiles_before(I.n, p.n_tiles, p.span);
       for (int it = 0; it < I.n_iters; ++it) {
         const int g = g0 + it;
         const int q0 = (I.n + it % I.m_cnt) * 128 + 64 * half;  // first query of this thread's columns
@@ -812,6 +818,7 @@ __global__ void __launch_bounds__(256, 1)
   auto item_of = [&](int item, int& m, int& h, int& b, int& n_lo, int& steps) {
     int t, blk;
     sb_order(item, p.n_tiles, n_items / p.n_tiles, t, blk);
+    blk += p.blk0 * p.G;  // the pass's query-head blocks: G per KV block
     m = p.n_tiles - 1 - t;
     h = blk % p.Hq;
     b = blk / p.Hq;
@@ -867,7 +874,7 @@ __global__ void __launch_bounds__(256, 1)
       if (lane == 0) {
         int m, h, b, n_lo, steps;
         item_of(item, m, h, b, n_lo, steps);
-        const long long bh_base = ((long long)b * p.Hq + h) * p.tiles_per_bh;
+        const long long bh_base = ((long long)b * p.Hq + h - (long long)p.blk0 * p.G) * p.tiles_per_bh;
         for (int i = 0; i < steps; ++i, ++g) {
           const int st = g % L::kStages;
           const int n = n_lo + i;

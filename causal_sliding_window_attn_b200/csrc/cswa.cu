@@ -265,7 +265,10 @@ struct BwdWorkspace {
   int span;
 };
 int eff_window(int window, int T) { return (window >= T) ? -1 : window; }
-size_t bwd_ws_parts(int B, int T, int Hq, int window, BwdWorkspace* w, void* base) {
+// Layout: the two row-extension arrays, the counters, then the dS^T tiles of as many
+// (batch, KV head) blocks as one pass covers (kv_blocks; all B * Hkv of them when the
+// caller's workspace allows a single pass).
+size_t bwd_ws_parts(int B, int T, int Hq, int Hkv, int window, long long kv_blocks, BwdWorkspace* w, void* base) {
   const int nt = tiles128(T);
   const size_t Tpad = (size_t)nt * 128;
   const int span = bwd_span(nt, eff_window(window, T));
@@ -279,8 +282,8 @@ size_t bwd_ws_parts(int B, int T, int Hq, int window, BwdWorkspace* w, void* bas
   };
   uint8_t* e1 = take((size_t)B * Hq * Tpad * 4);
   uint8_t* e2 = take((size_t)B * Hq * Tpad * 4);
-  uint8_t* ds = take((size_t)B * Hq * tiles * 32768);
   uint8_t* cnt = take(256);
+  uint8_t* ds = take((size_t)kv_blocks * (Hq / Hkv) * tiles * 32768);
   if (w) {
     w->ext_lse = e1;
     w->ext_delta = e2;
@@ -290,6 +293,20 @@ size_t bwd_ws_parts(int B, int T, int Hq, int window, BwdWorkspace* w, void* bas
     w->span = span;
   }
   return off;
+}
+// (batch, KV head) blocks per pass that a workspace of ws_bytes holds, at most all of them
+// and at most what keeps a pass's stored tile rows below 2^31; 0 if not even one fits
+long long bwd_blocks_per_pass(int B, int T, int Hq, int Hkv, int window, size_t ws_bytes) {
+  const long long total = (long long)B * Hkv;
+  const size_t fixed = bwd_ws_parts(B, T, Hq, Hkv, window, 0, nullptr, nullptr);
+  const int nt = tiles128(T);
+  const long long per_block = (long long)(Hq / Hkv) * ds_tiles_before(nt, nt, bwd_span(nt, eff_window(window, T)));
+  if (ws_bytes < fixed) return 0;
+  long long n = std::min<long long>(total, (long long)((ws_bytes - fixed) / ((size_t)per_block * 32768)));
+  n = std::min<long long>(n, ((1ll << 31) - 1) / (per_block * 128));
+  // a partial pass must still fit its rounding to 256 bytes
+  while (n > 0 && bwd_ws_parts(B, T, Hq, Hkv, window, n, nullptr, nullptr) > ws_bytes) --n;
+  return n;
 }
 
 // The fused prologue backward of the block variant: raw q and k, and the rotary
@@ -302,13 +319,16 @@ struct RopeBwd {
 
 template <int D>
 attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
-                         const float* lse, void* dq, void* dk, void* dv, void* ws, int B, int T, int Hq, int Hkv,
-                         int window, float scale, const RopeBwd& rb, cudaStream_t st) {
+                         const float* lse, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, int B, int T,
+                         int Hq, int Hkv, int window, float scale, const RopeBwd& rb, cudaStream_t st) {
   const int nt = tiles128(T);
   const int Tpad = nt * 128;
   const bool rope = rb.q_raw != nullptr;
+  const long long total_blocks = (long long)B * Hkv;
+  const long long nblk = bwd_blocks_per_pass(B, T, Hq, Hkv, window, ws_bytes);
+  if (nblk <= 0) return ATTN_ERR_INVALID_ARG;
   BwdWorkspace w;
-  bwd_ws_parts(B, T, Hq, window, &w, ws);
+  bwd_ws_parts(B, T, Hq, Hkv, window, nblk, &w, ws);
   // operands (128-row boxes), the outputs (32-row boxes: one per epilogue warp), and
   // for the block backward the raw k (128 rows, one load per tile) and q (32 rows)
   CUtensorMap tq, tk, tv, tdo, tdk, tdv, tdq, tkr, tqr;
@@ -362,17 +382,23 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
   p.rope = rope ? 1 : 0;
   p.eps = rb.eps;
   if (rope) rope_turns(D, rb.base, p.turns);
-  {
-    // persistent: one CTA per SM walks the (key tile, KV head, batch) items
-    const long long kv_items = (long long)nt * Hkv * B;
+  // One pass (a main and a dQ launch) per nblk (batch, KV head) blocks; the prep kernel
+  // zeroed the work counters for the first, a memset does it for the others.
+  for (long long blk0 = 0; blk0 < total_blocks; blk0 += nblk) {
+    const long long n = std::min(nblk, total_blocks - blk0);
+    if (blk0 > 0 && cudaMemsetAsync(w.counter, 0, 2 * sizeof(int), st) != cudaSuccess) return ATTN_ERR_LAUNCH;
+    p.blk0 = (int)blk0;
+    // persistent: one CTA per SM walks the pass's (key tile, KV head, batch) items
+    const long long kv_items = (long long)nt * n;
     const int kv_grid = (int)std::min<long long>(kv_items, sm_count());
     attn_bwd_kernel<D><<<kv_grid, 384, BwdLayout<D>::kBytes, st>>>(tq, tk, tv, tdo, tkr, tdk, tdv, p,
                                                                     (int)kv_items);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
+    const long long items = kv_items * p.G;
+    const int grid = (int)std::min<long long>(items, sm_count());
+    attn_bwd_dq_kernel<D><<<grid, 256, DqLayout<D>::kBytes, st>>>(tk, tqr, tdq, p, (int)items);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
   }
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
-  const long long items = (long long)nt * Hq * B;
-  const int grid = (int)std::min<long long>(items, sm_count());
-  attn_bwd_dq_kernel<D><<<grid, 256, DqLayout<D>::kBytes, st>>>(tk, tqr, tdq, p, (int)items);
   return launched();
 }
 
@@ -442,18 +468,21 @@ attn_status_t bwd_common(const void* q, const void* k, const void* v, const void
   if (rope && (!rb.k_raw || !aligned16(rb.q_raw) || !aligned16(rb.k_raw) || !(rb.base > 1.f) ||
                !std::isfinite(rb.base) || !(rb.eps >= 0.f) || !std::isfinite(rb.eps)))
     return ATTN_ERR_INVALID_ARG;
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
-      ws_bytes < bwd_ws_parts(B, T, Hq, window, nullptr, nullptr))
-    return ATTN_ERR_INVALID_ARG;
   if (Hq > 65535 || B > 65535 || tiles128(T) > 65535) return ATTN_ERR_INVALID_ARG;
-  // stored dS^T tile rows, the dQ kernel's work items and the prep kernel's rows per batch
-  // (Tpad * Hq, no more than the tile rows) are counted in 32 bits
+  // a pass's stored dS^T tile rows (one (batch, KV head) block at least), its work items
+  // and the prep kernel's rows per batch (Tpad * Hq) are counted in 32 bits
   const int nt = tiles128(T);
-  if ((long long)B * Hq * ds_tiles_before(nt, nt, bwd_span(nt, eff_window(window, T))) * 128 >= (1ll << 31))
+  if ((long long)(Hq / Hkv) * ds_tiles_before(nt, nt, bwd_span(nt, eff_window(window, T))) * 128 >= (1ll << 31) ||
+      (long long)nt * 128 * Hq >= (1ll << 31))
     return ATTN_ERR_UNSUPPORTED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      bwd_blocks_per_pass(B, T, Hq, Hkv, window, ws_bytes) <= 0)
+    return ATTN_ERR_INVALID_ARG;
   cudaStream_t st = as_stream(stream);
-  return D == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, workspace, B, T, Hq, Hkv, window, scale, rb, st)
-                 : launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, workspace, B, T, Hq, Hkv, window, scale, rb, st);
+  return D == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, workspace, ws_bytes, B, T, Hq, Hkv, window, scale,
+                                  rb, st)
+                 : launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, workspace, ws_bytes, B, T, Hq, Hkv, window, scale,
+                                   rb, st);
 }
 }  // namespace
 
@@ -485,12 +514,16 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
 
 size_t attn_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int window) {
   if (!dims_ok(B, T, Hq, Hkv) || (D != 64 && D != 128)) return 0;
-  return bwd_ws_parts(B, T, Hq, window, nullptr, nullptr);
+  return bwd_ws_parts(B, T, Hq, Hkv, window, (long long)B * Hkv, nullptr, nullptr);
+}
+
+size_t attn_bwd_workspace_min_bytes(int B, int T, int Hq, int Hkv, int D, int window) {
+  if (!dims_ok(B, T, Hq, Hkv) || (D != 64 && D != 128)) return 0;
+  return bwd_ws_parts(B, T, Hq, Hkv, window, 1, nullptr, nullptr);
 }
 
 size_t attn_block_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int window) {
-  if (!dims_ok(B, T, Hq, Hkv) || (D != 64 && D != 128)) return 0;
-  return bwd_ws_parts(B, T, Hq, window, nullptr, nullptr);
+  return attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, window);
 }
 
 

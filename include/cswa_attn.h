@@ -91,6 +91,13 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
  * rounded up to 256 bytes. Nothing in it needs to be initialised. */
 size_t attn_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int window);
 
+/* The least workspace attn_bwd and attn_block_bwd accept: the row extensions, the
+ * counters and the dS^T tiles of ONE (batch, KV head) block, i.e. about
+ * (Hq/Hkv)*T*min(T, W+128)*2 bytes plus O(B*Hq*T). With a workspace between this and
+ * attn_bwd_workspace_bytes the call runs in passes, each over as many (batch, KV head)
+ * blocks as the workspace holds (a main and a dQ launch per pass), with the same results. */
+size_t attn_bwd_workspace_min_bytes(int B, int T, int Hq, int Hkv, int D, int window);
+
 /*
  * attn_bwd -- gradients of sum(dO * o) for o = attn_fwd(q, k, v):
  *   Delta_i = dO_i . o_i,  P = exp(scale q k^T - lse),  dV = P^T dO,
@@ -99,11 +106,12 @@ size_t attn_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int window
  * Inputs: q, k, v, o, dO (bf16) and lse (fp32) exactly as attn_fwd produced
  * them. Outputs dq (B,T,Hq,D), dk, dv (B,T,Hkv,D) bf16, fully overwritten.
  * workspace: device memory, 256-byte aligned, of ws_bytes >=
- * attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, window). Three launches: a per-row
- * preparation, the tensor-core main kernel (dK and dV complete per key tile, the
- * dS^T tiles stored to the workspace) and the tensor-core dQ kernel (dQ = scale dS K
- * from the stored tiles). Calls whose stored dS^T tiles would exceed 2^31 rows return
- * ATTN_ERR_UNSUPPORTED.
+ * attn_bwd_workspace_min_bytes(B, T, Hq, Hkv, D, window); attn_bwd_workspace_bytes
+ * (or more) runs the call in one pass. Launches: a per-row preparation, then per pass
+ * the tensor-core main kernel (dK and dV complete per key tile, the dS^T tiles stored
+ * to the workspace) and the tensor-core dQ kernel (dQ = scale dS K from the stored
+ * tiles); passes after the first start with a memset of the two work counters. Calls where one (batch, KV head) block's stored dS^T
+ * tiles would exceed 2^31 rows, or T_pad * Hq reaches 2^31, return ATTN_ERR_UNSUPPORTED.
  */
 attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                        const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B,
@@ -126,7 +134,8 @@ size_t attn_block_bwd_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int 
  *   q (B,T,Hq,D), k (B,T,Hkv,D): the raw inputs of the prologue.
  *   q_hat, k_hat: the prologue's outputs for them (rope_base, eps as given here).
  *   v, o, dO, lse: as for attn_bwd. Outputs dq, dk (raw-input gradients) and dv.
- *   workspace: 256-byte aligned, >= attn_block_bwd_workspace_bytes(...).
+ *   workspace: 256-byte aligned, >= attn_bwd_workspace_min_bytes(...); as for attn_bwd,
+ *   less than attn_block_bwd_workspace_bytes(...) runs in passes.
  * Same checks, errors and launches as attn_bwd; rope_base > 1 and eps >= 0.
  */
 attn_status_t attn_block_bwd(const void* q, const void* k, const void* q_hat, const void* k_hat, const void* v,

@@ -53,6 +53,10 @@ def test_bwd_workspace_size(L):
     assert L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, 2048) == full
     # the block backward needs no more (its rotary angles are computed in the kernels)
     assert L.attn_block_bwd_workspace_bytes(B, T, Hq, Hkv, D, -1) == full
+    # the least workspace holds one (batch, KV head) block's tiles (G = 1 here; G = 4 and
+    # 70 tiles at W = 512 below); workspaces between it and the full size run in passes
+    assert L.attn_bwd_workspace_min_bytes(B, T, Hq, Hkv, D, 1024) == 2 * rows + 256 + 108 * 32768
+    assert L.attn_bwd_workspace_min_bytes(8, 2048, 16, 4, 128, 512) == 2 * 8 * 16 * 2048 * 4 + 256 + 4 * 70 * 32768
     # ragged T pads the per-row arrays to whole 128-row tiles; window 0 keeps the diagonal only
     assert L.attn_bwd_workspace_bytes(1, 130, 2, 1, 64, 0) == 2 * 2048 + 2 * 2 * 32768 + 256
     assert L.attn_block_bwd_workspace_bytes(1, 3, 1, 1, 64, -1) == 2 * 512 + 32768 + 256
@@ -96,7 +100,8 @@ def test_bwd_rejects_bad_args(L):
         a = list(base)
         a[i] = v
         return L.attn_bwd(*a)
-    assert call(10, ws - 1) == INVALID                # workspace too small
+    # a byte less than one (batch, KV head) block's share (less than the full size runs in passes)
+    assert call(10, L.attn_bwd_workspace_min_bytes(1, 128, 4, 2, 128, 64) - 1) == INVALID
     assert call(9, ctypes.c_void_p(0x10010)) == INVALID  # workspace not 256-aligned
     assert call(6, None) == INVALID                   # null dq
     assert call(15, 96) == UNSUPPORTED                # head dim
@@ -110,7 +115,7 @@ def test_block_bwd_rejects_bad_args(L):
         a = list(base)
         a[i] = v
         return L.attn_block_bwd(*a)
-    assert call(12, ws - 1) == INVALID                # workspace too small
+    assert call(12, L.attn_bwd_workspace_min_bytes(1, 128, 4, 2, 128, 64) - 1) == INVALID  # too small
     assert call(0, None) == INVALID                   # null raw q
     assert call(1, MIS) == INVALID                    # misaligned raw k
     assert call(20, f(1.0)) == INVALID                # rope base
@@ -200,12 +205,13 @@ def test_size_limits_rejected_before_launch(L):
     ws = L.attn_decode_workspace_bytes(1, 1, 128, Tmax, -1)
     assert ws > 0
     assert L.attn_decode(P, P, P, None, None, P, P, P, 1, Tmax, 1, 1, 128, -1, f, P, ws, None) == UNSUPPORTED
-    # backward: stored dS^T tiles beyond 2^31 rows (B * Hq * tiles * 128)
-    B, T, H = 64, 65536, 64
-    ws = L.attn_bwd_workspace_bytes(B, T, H, H, 128, -1)
+    # backward: one (batch, KV head) block's stored dS^T tiles beyond 2^31 rows
+    # (G * tiles * 128: 256 * 131328 * 128)
+    B, T, Hq, Hkv = 1, 65536, 256, 1
+    ws = L.attn_bwd_workspace_bytes(B, T, Hq, Hkv, 128, -1)
     big = ctypes.c_void_p(0x100000000)
     assert ws > 0
-    assert L.attn_bwd(*([P] * 9), big, ws, B, T, H, H, 128, -1, f, None) == UNSUPPORTED
+    assert L.attn_bwd(*([P] * 9), big, ws, B, T, Hq, Hkv, 128, -1, f, None) == UNSUPPORTED
     # grid limits: 65535 sequences or query heads at most
     assert L.attn_fwd(P, P, P, P, P, 65536, 16, 1, 1, 128, -1, f, None) == INVALID
     assert L.attn_fwd(P, P, P, P, P, 1, 16, 65536, 1, 128, -1, f, None) == INVALID

@@ -140,6 +140,38 @@ def test_gqa_matches_repeated_kv_on_gpu(cswa):
     check_grad("dv", f64(dv), f64(dvm).reshape(B, T, Hkv, G, D).sum(3), 5e-3)
 
 
+@pytest.mark.parametrize("B,T,Hq,Hkv,D,W", [(2, 700, 4, 2, 128, 200), (3, 300, 6, 3, 64, -1)])
+def test_bwd_in_passes_matches_one_pass(cswa, B, T, Hq, Hkv, D, W):
+    """A workspace below attn_bwd_workspace_bytes runs the backward in passes over the
+    (batch, KV head) blocks; every gradient must equal the one-pass result bit for bit
+    (each key tile's dK/dV and each query tile's dQ are computed the same way), down to
+    one block per pass, and the one-pass result is checked against the oracle elsewhere.
+    The workspaces start out filled with garbage."""
+    scale = workloads.default_scale(D)
+    q, k, v, do = (t.cuda() for t in workloads.training_inputs(B, T, Hq, Hkv, D, seed=31 + T))
+    qh, kh = cswa.attn_rope_qknorm(q, k, rope_base=ROPE_BASE, eps=EPS)
+    o, lse = cswa.attn_fwd(qh, kh, v, W, scale)
+    full = cswa.attn_bwd_workspace_bytes(B, T, Hq, Hkv, D, W)
+    least = cswa.attn_bwd_workspace_min_bytes(B, T, Hq, Hkv, D, W)
+    assert 0 < least < full
+    ref = cswa.attn_bwd(qh, kh, v, o, do, lse, W, scale)
+    ref_f = cswa.attn_block_bwd(q, k, qh, kh, v, o, do, lse, W, scale, rope_base=ROPE_BASE, eps=EPS)
+    per_block = (full - least) // (B * Hkv - 1)
+    for nbytes in (least, least + per_block, least + 2 * per_block + 1000, full - 256):
+        ws = torch.randint(0, 256, (nbytes,), dtype=torch.uint8, device="cuda")
+        got = cswa.attn_bwd(qh, kh, v, o, do, lse, W, scale, workspace=ws)
+        ws.random_(0, 256)
+        got_f = cswa.attn_block_bwd(q, k, qh, kh, v, o, do, lse, W, scale, workspace=ws, rope_base=ROPE_BASE,
+                                    eps=EPS)
+        torch.cuda.synchronize()
+        assert cswa.attn_get_status() == 0
+        for a, b in zip(got + got_f, ref + ref_f):
+            assert torch.equal(a, b), nbytes
+    small = torch.empty(least - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(RuntimeError):
+        cswa.attn_bwd(qh, kh, v, o, do, lse, W, scale, workspace=small)
+
+
 def test_T1_W0_return_v(cswa):
     B, T, Hq, Hkv, D = 2, 200, 4, 2, 64
     q, k, v, _ = workloads.training_inputs(B, T, Hq, Hkv, D, seed=13)
