@@ -41,6 +41,7 @@ CASES = [
     (2, 1, 2, 1, 128, -1),       # T = 1
     (1, 640, 8, 2, 128, 1000),   # window >= T: plain causal
     (1, 384, 2, 1, 128, 127),    # window one short of a tile
+    (1, 300, 16, 1, 128, 100),   # G = 16: one KV head walked by 16 query heads per key tile
 ]
 
 
