@@ -572,9 +572,20 @@ __global__ void __launch_bounds__(384, 1)
         // dV starts on the first while the rest is computed. Chunk c's bf16 pairs land in
         // columns 8c..8c+7, whose fp32 S^T (queries <= 16c+15) is already in registers.
         const float2 sl2v = make_float2(sl2, sl2);
+        // Chunk c+1's exponentials are computed while chunk c's TMEM store completes: the
+        // wait for a chunk's store, and its publication, come after the next chunk's math.
+        uint32_t pkb[2][8];
+        auto publish = [&](int c) {
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&p_chunk[c]);
+          if (tracer && c == 0) CSWA_MARK(trole, g, 3);
+          if (ds_dst) store_ds_units(2 * c, 2 * c + 2);
+          if (lent_stage >= 0 && c == (half ? 0 : 3)) return_stage();
+        };
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t pk[8];
+          uint32_t(&pk)[8] = pkb[c & 1];
 #pragma unroll
           for (int c2 = 8 * c; c2 < 8 * c + 8; ++c2) {
             const float2 e = __fmul2_rn(make_float2(__uint_as_float(sr[2 * c2]), __uint_as_float(sr[2 * c2 + 1])), sl2v);
@@ -590,14 +601,10 @@ __global__ void __launch_bounds__(384, 1)
             sr[2 * c2 + 1] = __float_as_uint(y[1]);
             pk[c2 - 8 * c] = pack_bf16x2(y[0], y[1]);
           }
+          if (c > 0) publish(c - 1);
           tmem_st8(tR0 + cols + 8 * c, pk);
-          tmem_st_wait();
-          tc_fence_before();
-          mbar_arrive(&p_chunk[c]);
-          if (tracer && c == 0) CSWA_MARK(trole, g, 3);
-          if (ds_dst) store_ds_units(2 * c, 2 * c + 2);
-          if (lent_stage >= 0 && c == (half ? 0 : 3)) return_stage();
         }
+        publish(3);
         const float* pf = reinterpret_cast<const float*>(sr);
         if (tracer) CSWA_MARK(trole, g, 4);
 
