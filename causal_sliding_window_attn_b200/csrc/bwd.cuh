@@ -148,6 +148,12 @@ __host__ __device__ inline void sb_order(int item, int n_tiles, int n_blocks, in
   blk = kSB * s + r % w;
 }
 
+// P/dS warps of the main kernel, in groups of 4 (one per TMEM lane quarter), each group
+// taking 128 / (kBwdSoftmaxWarps / 4) query columns of the step. 16 (four per SM
+// sub-partition, 32 columns each, 96 registers a thread) measured slower than 8.
+constexpr int kBwdSoftmaxWarps = 8;
+constexpr int kBwdThreads = (4 + kBwdSoftmaxWarps) * 32;
+
 template <int D>
 struct BwdLayout {
   static constexpr int kQStages = 3, kDOStages = 2;
@@ -172,13 +178,17 @@ struct BwdLayout {
 
 // tm_kr: the raw k (block backward only); tm_dk, tm_dv: the outputs, 32-row boxes.
 template <int D>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_kr, const __grid_constant__ CUtensorMap tm_dk,
                     const __grid_constant__ CUtensorMap tm_dv, const __grid_constant__ BwdParams p, int n_items) {
   using L = BwdLayout<D>;
   constexpr int QS = L::kQStages, DS = L::kDOStages;
+  // query columns of a step: kSGroups groups of kSCols, each group's P^T (and dS^T) packed
+  // as bf16 pairs into the first kSCols / 2 of its own columns, published in kPChunks
+  // chunks of 16 queries (one MMA K step each)
+  constexpr int kSGroups = kBwdSoftmaxWarps / 4, kSCols = 128 / kSGroups, kPChunks = kSCols / 16;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // the layout needs a 1024-byte aligned base: report (never overrun) if the slack is too small
@@ -248,13 +258,13 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&do_borrow[s], 4);  // the four dV epilogue warps
     }
     mbar_init(s_full, 1);
-    for (int c = 0; c < 4; ++c) mbar_init(&p_chunk[c], 256);
+    for (int c = 0; c < 4; ++c) mbar_init(&p_chunk[c], kBwdSoftmaxWarps * 32);
     mbar_init(dp_full, 1);
-    mbar_init(ds_full, 256);
+    mbar_init(ds_full, kBwdSoftmaxWarps * 32);
     mbar_init(final_bar, 1);
     mbar_init(acc_free, 256);
     mbar_init(item_full, 1);
-    mbar_init(item_empty, 11);  // warps 0, 1, 3 and the eight P/dS warps
+    mbar_init(item_empty, 3 + kBwdSoftmaxWarps);  // warps 0, 1, 3 and the P/dS warps
     mbar_init(kr_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -407,7 +417,7 @@ __global__ void __launch_bounds__(384, 1)
     auto issue_acc = [&](uint32_t dst, uint32_t a_tmem, uint64_t dB, uint32_t boff, bool first) {
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        mma_ts(dst, a_tmem + (kk >> 2) * 64 + (kk & 3) * 8, dB + ((boff + kk * 2048) >> 4), idKV,
+        mma_ts(dst, a_tmem + (kk / kPChunks) * kSCols + (kk % kPChunks) * 8, dB + ((boff + kk * 2048) >> 4), idKV,
                (!first || kk > 0), leader);
     };
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
@@ -443,14 +453,14 @@ __global__ void __launch_bounds__(384, 1)
         if (it == 0 && !(ok = wait_all(acc_free, (k & 1) ^ 1))) break;
         // dV(it) chunk by chunk as the P/dS warps publish P^T: chunk c holds queries
         // 16c..16c+15 of each half, i.e. the K steps c and 4 + c
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < kPChunks; ++c) {
           if (!(ok = wait_all(&p_chunk[c], g & 1))) break;
           if (tracer && c == 0) CSWA_MARK(0, g, 1);
           tc_fence_after();
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int kk = c + 4 * u;
-            mma_ts(tdV, tR0 + u * 64 + c * 8, dDO_mn + ((ds * L::kTile + kk * 2048) >> 4), idKV,
+          for (int u = 0; u < kSGroups; ++u) {
+            const int kk = kPChunks * u + c;
+            mma_ts(tdV, tR0 + u * kSCols + c * 8, dDO_mn + ((ds * L::kTile + kk * 2048) >> 4), idKV,
                    (it > 0 || kk > 0), leader);
           }
         }
@@ -503,11 +513,11 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp >= 4) {
     // ------------------------------------------------------------ P and dS (thread = key row)
     // warps 4-7 take query columns 0-63, warps 8-11 columns 64-127 (warp 2 only allocates TMEM)
-    const int half = (warp >= 8) ? 1 : 0;
+    const int half = (warp - 4) >> 2;  // column group; groups 0 and 1 also run the dK / dV epilogue
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t cols = lane_off + 64 * half;  // this thread's S^T / dP^T columns
+    const uint32_t cols = lane_off + kSCols * half;  // this thread's S^T / dP^T columns
     const float sl2 = p.scale_log2;
     const bool tracer = ((warp == 4 || warp == 8) && lane == 0);
     const int trole = 1 + half;
@@ -518,7 +528,7 @@ __global__ void __launch_bounds__(384, 1)
     // phase, whose exp2 work leaves the load/store unit idle (an item's last one before
     // its epilogue). The tile is written as 16-byte units (8 queries of one key) ordered
     // so that every warp store covers 512 contiguous bytes (see ds_unit_offset).
-    uint32_t dsk[32];
+    uint32_t dsk[kSCols / 2];
     uint8_t* ds_dst = nullptr;
     auto store_ds_units = [&](int u0, int u1) {
 #pragma unroll
@@ -551,20 +561,20 @@ __global__ void __launch_bounds__(384, 1)
                               ds_tiles_before(I.n, p.n_tiles, p.span);
       for (int it = 0; it < I.n_iters; ++it) {
         const int g = g0 + it;
-        const int q0 = (I.n + it % I.m_cnt) * 128 + 64 * half;  // first query of this thread's columns
+        const int q0 = (I.n + it % I.m_cnt) * 128 + kSCols * half;  // first query of this thread's columns
         if (tracer) CSWA_MARK(trole, g, 0);
         ok = __all_sync(0xffffffffu, mbar_wait(s_full, g & 1, abort_flag));
         if (tracer) CSWA_MARK(trole, g, 1);
         if (!ok) break;
         tc_fence_after();
-        uint32_t sr[64];
-        tmem_ld32(tR0 + cols + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(tR0 + cols + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        uint32_t sr[kSCols];
+#pragma unroll
+        for (int h32 = 0; h32 < kSCols; h32 += 32) tmem_ld32(tR0 + cols + h32, *reinterpret_cast<uint32_t(*)[32]>(&sr[h32]));
         tmem_ld_wait();
         if (tracer) CSWA_MARK(trole, g, 2);
-        const bool full = (k0 + 127 <= q0) && (W < 0 || q0 + 63 - k0 <= W);
-        const int c_lo = j - q0;                      // query q0 + c sees key j iff c >= c_lo
-        const int c_hi = (W < 0) ? 63 : j + W - q0;   //   and c <= c_hi
+        const bool full = (k0 + 127 <= q0) && (W < 0 || q0 + kSCols - 1 - k0 <= W);
+        const int c_lo = j - q0;                              // query q0 + c sees key j iff c >= c_lo
+        const int c_hi = (W < 0) ? kSCols - 1 : j + W - q0;   //   and c <= c_hi
         // P = exp2(scale log2e (S - lse/scale)): the MMA has already added -lse/scale, so
         // one packed multiply per two columns; masked entries are set to 0 after the exp2,
         // tiles inside the band skip the mask (a warp-uniform branch). P^T goes back to
@@ -581,10 +591,10 @@ __global__ void __launch_bounds__(384, 1)
           mbar_arrive(&p_chunk[c]);
           if (tracer && c == 0) CSWA_MARK(trole, g, 3);
           if (ds_dst) store_ds_units(2 * c, 2 * c + 2);
-          if (lent_stage >= 0 && c == (half ? 0 : 3)) return_stage();
+          if (lent_stage >= 0 && c == (half ? 0 : kPChunks - 1)) return_stage();
         };
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < kPChunks; ++c) {
           uint32_t(&pk)[8] = pkb[c & 1];
 #pragma unroll
           for (int c2 = 8 * c; c2 < 8 * c + 8; ++c2) {
@@ -604,7 +614,7 @@ __global__ void __launch_bounds__(384, 1)
           if (c > 0) publish(c - 1);
           tmem_st8(tR0 + cols + 8 * c, pk);
         }
-        publish(3);
+        publish(kPChunks - 1);
         const float* pf = reinterpret_cast<const float*>(sr);
         if (tracer) CSWA_MARK(trole, g, 4);
 
@@ -615,7 +625,7 @@ __global__ void __launch_bounds__(384, 1)
         // dS = P * (dP - Delta): the MMA has already subtracted Delta; one packed multiply
         // per two columns, 32 columns at a time
 #pragma unroll
-        for (int hc = 0; hc < 2; ++hc) {
+        for (int hc = 0; hc < kSCols / 32; ++hc) {
           uint32_t dp[32];
           tmem_ld32(tR1 + cols + 32 * hc, dp);
           tmem_ld_wait();
@@ -628,18 +638,27 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         if (tracer) CSWA_MARK(trole, g, 6);
-        tmem_st32(tR1 + cols, dsk);  // over this thread's own (already read) dP^T columns
+        // over this thread's own (already read) dP^T columns
+        if constexpr (kSCols == 64)
+          tmem_st32(tR1 + cols, *reinterpret_cast<uint32_t(*)[32]>(dsk));
+        else
+          tmem_st16(tR1 + cols, *reinterpret_cast<uint32_t(*)[16]>(dsk));
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(ds_full);
         if (tracer) CSWA_MARK(trole, g, 7);
         const long long tile = tile0 + (long long)(I.hk * G + it / I.m_cnt) * p.tiles_per_bh + it % I.m_cnt;
-        ds_dst = reinterpret_cast<uint8_t*>(p.ds) + (size_t)tile * 32768 + ds_unit_offset(r, 8 * half);
+        ds_dst = reinterpret_cast<uint8_t*>(p.ds) + (size_t)tile * 32768 + ds_unit_offset(r, (kSCols / 8) * half);
       }
       if (!ok) break;
       // the item's last dS^T now: the epilogue needs the registers
-      store_ds_units(0, 8);
+      store_ds_units(0, kSCols / 8);
       ds_dst = nullptr;
+      // column groups past the first two have no epilogue: on to the next item
+      if (half >= 2) {
+        g0 += I.n_iters;
+        continue;
+      }
       // ------------------------------------------------------ dK (warps 4-7) / dV (8-11) epilogue
       // Thread = key row j of the tile. The accumulator goes to bf16 in the ring stage
       // of the item's last step (the Q stage for dK, the dO stage for dV: lent by the

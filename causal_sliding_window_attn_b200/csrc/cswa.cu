@@ -391,7 +391,7 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
     // persistent: one CTA per SM walks the pass's (key tile, KV head, batch) items
     const long long kv_items = (long long)nt * n;
     const int kv_grid = (int)std::min<long long>(kv_items, sm_count());
-    attn_bwd_kernel<D><<<kv_grid, 384, BwdLayout<D>::kBytes, st>>>(tq, tk, tv, tdo, tkr, tdk, tdv, p,
+    attn_bwd_kernel<D><<<kv_grid, kBwdThreads, BwdLayout<D>::kBytes, st>>>(tq, tk, tv, tdo, tkr, tdk, tdv, p,
                                                                     (int)kv_items);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
     const long long items = kv_items * p.G;
