@@ -206,7 +206,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* do_empty = do_full + DS;           // [DS]  dV has read the dO tile
   uint64_t* do_borrow = do_empty + DS;         // [DS]  the dV epilogue is done with a lent stage
   uint64_t* s_full = do_borrow + DS;           // S^T in TMEM
-  uint64_t* p_chunk = s_full + 1;              // [4] P^T of queries 16c..16c+15 of each half written
+  uint64_t* p_chunk = s_full + 1;              // [4] P^T chunk c of every column group written
   uint64_t* dp_full = p_chunk + 4;             // dP^T in TMEM
   uint64_t* ds_full = dp_full + 1;             // dS^T written over dP^T
   uint64_t* final_bar = ds_full + 1;           // the item's dK and dV are complete in TMEM
@@ -412,8 +412,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mma_ss(dst, dOnes, dX + ((xslot * 512) >> 4), idX, 1, leader);
       mma_commit(done, leader);
     };
-    // dK += dS^T Q: A = the bf16 pairs packed over dP^T (queries 0-63 in columns 0-31,
-    // 64-127 in columns 64-95), B = Q, MN-major
+    // dK += dS^T Q: A = the bf16 pairs packed over dP^T (column group u's queries in its
+    // first kSCols / 2 columns; K step kk = group kk / kPChunks, chunk kk % kPChunks), B = Q,
+    // MN-major
     auto issue_acc = [&](uint32_t dst, uint32_t a_tmem, uint64_t dB, uint32_t boff, bool first) {
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
@@ -452,7 +453,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // the accumulators are free once the epilogue has read the previous item's
         if (it == 0 && !(ok = wait_all(acc_free, (k & 1) ^ 1))) break;
         // dV(it) chunk by chunk as the P/dS warps publish P^T: chunk c holds queries
-        // 16c..16c+15 of each half, i.e. the K steps c and 4 + c
+        // 16c..16c+15 of each column group u, i.e. the K steps kPChunks * u + c
         for (int c = 0; c < kPChunks; ++c) {
           if (!(ok = wait_all(&p_chunk[c], g & 1))) break;
           if (tracer && c == 0) CSWA_MARK(0, g, 1);
@@ -512,7 +513,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ P and dS (thread = key row)
-    // warps 4-7 take query columns 0-63, warps 8-11 columns 64-127 (warp 2 only allocates TMEM)
+    // warps 4-7 take query columns 0 .. kSCols-1, warps 8-11 the next kSCols (warp 2 only
+    // allocates TMEM and schedules)
     const int half = (warp - 4) >> 2;  // column group; groups 0 and 1 also run the dK / dV epilogue
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
@@ -578,9 +580,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // P = exp2(scale log2e (S - lse/scale)): the MMA has already added -lse/scale, so
         // one packed multiply per two columns; masked entries are set to 0 after the exp2,
         // tiles inside the band skip the mask (a warp-uniform branch). P^T goes back to
-        // TMEM in four chunks of 16 queries, each published on its own barrier so that
+        // TMEM in kPChunks chunks of 16 queries, each published on its own barrier so that
         // dV starts on the first while the rest is computed. Chunk c's bf16 pairs land in
-        // columns 8c..8c+7, whose fp32 S^T (queries <= 16c+15) is already in registers.
+        // the group's columns 8c..8c+7, whose fp32 S^T (queries <= 16c+15) is already in
+        // registers.
         const float2 sl2v = make_float2(sl2, sl2);
         // Chunk c+1's exponentials are computed while chunk c's TMEM store completes: the
         // wait for a chunk's store, and its publication, come after the next chunk's math.
