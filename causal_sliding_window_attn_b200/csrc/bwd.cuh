@@ -843,11 +843,14 @@ __global__ void __launch_bounds__(256, 1)
   const int warp = warp_id(), lane = lane_id();
   // item -> (query tile m, head h, batch b) in super-block order with the heaviest
   // query tiles (the most key tiles) first, and the key tiles n whose query range
-  // [n, n + span - 1] holds m; items are handed out first come first served
+  // [n, n + span - 1] holds m; items are handed out first come first served. The blocks
+  // go in the reverse of the main kernel's order: the dS^T tiles it wrote last are the
+  // ones still in L2 when this kernel starts.
   auto item_of = [&](int item, int& m, int& h, int& b, int& n_lo, int& steps) {
     int t, blk;
-    sb_order(item, p.n_tiles, n_items / p.n_tiles, t, blk);
-    blk += p.blk0 * p.G;  // the pass's query-head blocks: G per KV block
+    const int n_blocks = n_items / p.n_tiles;
+    sb_order(item, p.n_tiles, n_blocks, t, blk);
+    blk = n_blocks - 1 - blk + p.blk0 * p.G;  // the pass's query-head blocks: G per KV block
     m = p.n_tiles - 1 - t;
     h = blk % p.Hq;
     b = blk / p.Hq;

@@ -114,6 +114,37 @@ def test_prologue_positions_and_inplace(cswa):
     check_grad("dq", f64(dq), oracle.prologue_bwd(f64(q), f64(dy), positions, ROPE_BASE, EPS))
 
 
+@pytest.mark.parametrize("B,T,Hq,Hkv,D", [(3, 3333, 4, 2, 128), (2, 4801, 6, 3, 64)])
+def test_prologue_large_calls(cswa, B, T, Hq, Hkv, D):
+    """Large calls (thousands of blocks, a partial last block of positions) with
+    position offsets: q and k together, q alone, k alone and in place, all against the
+    oracle."""
+    q, k, _, _ = workloads.training_inputs(B, T, Hq, Hkv, D, seed=11)
+    pos = torch.tensor([5, 1234, 40000][:B], dtype=torch.int32)
+    qd, kd = q.cuda(), k.cuda()
+    positions = oracle.row_positions(B, T, pos.numpy())
+    qh, kh = cswa.attn_rope_qknorm(qd, kd, pos=pos.cuda())
+    check_bf16("q_hat", f64(qh), oracle.prologue(f64(q), positions, ROPE_BASE, EPS))
+    check_bf16("k_hat", f64(kh), oracle.prologue(f64(k), positions, ROPE_BASE, EPS))
+    qa, _ = cswa.attn_rope_qknorm(qd, None, pos=pos.cuda())
+    _, ka = cswa.attn_rope_qknorm(None, kd, pos=pos.cuda())
+    assert torch.equal(qa, qh) and torch.equal(ka, kh)
+    k2 = kd.clone()
+    cswa.attn_rope_qknorm(None, k2, k_out=k2, pos=pos.cuda())
+    assert torch.equal(k2, kh)
+
+
+def test_prologue_wide_positions(cswa):
+    """Positions with many head rows (160 q heads and 40 k heads): the block's row to
+    (operand, position) mapping over long row ranges, against the oracle."""
+    B, T, Hq, Hkv, D = 1, 40, 160, 40, 128
+    q, k, _, _ = workloads.training_inputs(B, T, Hq, Hkv, D, seed=12)
+    qh, kh = cswa.attn_rope_qknorm(q.cuda(), k.cuda())
+    positions = oracle.row_positions(B, T, None)
+    check_bf16("q_hat", f64(qh), oracle.prologue(f64(q), positions, ROPE_BASE, EPS))
+    check_bf16("k_hat", f64(kh), oracle.prologue(f64(k), positions, ROPE_BASE, EPS))
+
+
 def test_window_ge_T_is_causal_on_gpu(cswa):
     B, T, Hq, Hkv, D = 1, 400, 2, 1, 128
     q, k, v, _ = workloads.training_inputs(B, T, Hq, Hkv, D, seed=11)
