@@ -1117,25 +1117,29 @@ struct PrepParams {
   uint8_t* ext_delta;
   int* item_counter;
   int B, T, Tpad, Hq;
+  int chunks;  // chunks of 2 * 256 / (D / 16) rows per batch
   float inv_scale;
 };
 
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __grid_constant__ PrepParams p) {
-  // blockIdx.y = batch b; the block's rows are (t, h) rows of that batch, t over the
-  // padded length. LK lanes per row, 16 elements each; every thread takes kRows rows
-  // (r0 + u * kRowsPerPass) with all their loads in flight before the sums, and forms
-  // o . dO with mixed bf16 x bf16 -> fp32 FMAs (no conversions).
+  // A chunk is kRows * kRowsPerPass consecutive (t, h) rows of one batch, t over the
+  // padded length; the blocks (a few per SM, resident together) take the B * chunks
+  // chunks in turn, so that no partial last wave of short blocks is left. LK lanes per
+  // row, 16 elements each; every thread takes kRows rows (r0 + u * kRowsPerPass) of a
+  // chunk with all their loads in flight before the sums, and forms o . dO with mixed
+  // bf16 x bf16 -> fp32 FMAs (no conversions).
   constexpr int LK = D / 16;
   constexpr int kRows = 2, kRowsPerPass = 256 / LK;
   // the main and dQ kernels that follow on the stream hand out their work items from
   // these two counters
-  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 2) p.item_counter[threadIdx.x] = 0;
-  const int b = blockIdx.y;
+  if (blockIdx.x == 0 && threadIdx.x < 2) p.item_counter[threadIdx.x] = 0;
   const int T = p.T, Tpad = p.Tpad, Hq = p.Hq;
   const int rows = Tpad * Hq;  // < 2^31 (the host checks the stored tile rows, which bound it)
-  const int r0 = blockIdx.x * (kRows * kRowsPerPass) + (int)threadIdx.x / LK;
   const int lr = (int)threadIdx.x % LK;
+  for (long long ch = blockIdx.x; ch < (long long)p.B * p.chunks; ch += gridDim.x) {
+  const int b = (int)(ch / p.chunks);
+  const int r0 = (int)(ch - (long long)b * p.chunks) * (kRows * kRowsPerPass) + (int)threadIdx.x / LK;
   int hh[kRows], tt[kRows];
   bool real[kRows];
   uint4 ov[kRows][2], gv[kRows][2];
@@ -1183,6 +1187,7 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __grid_constan
       *reinterpret_cast<__nv_bfloat16*>(p.ext_delta + at) = yh;
       *reinterpret_cast<__nv_bfloat16*>(p.ext_delta + at + 16) = __float2bfloat16_rn(y - __bfloat162float(yh));
     }
+  }
   }
 }
 

@@ -358,10 +358,17 @@ attn_status_t launch_bwd(const void* q, const void* k, const void* v, const void
     pp.Tpad = Tpad;
     pp.Hq = Hq;
     pp.inv_scale = 1.f / scale;
-    // per batch, 256 threads take 2 * 256 / (D / 16) rows (D / 16 lanes per row, two rows
-    // per lane)
-    const long long rows = (long long)Tpad * Hq, per_block = 2 * 256 / (D / 16);
-    attn_bwd_prep_kernel<D><<<dim3((unsigned)((rows + per_block - 1) / per_block), (unsigned)B), 256, 0, st>>>(pp);
+    // chunks of 2 * 256 / (D / 16) rows (D / 16 lanes per row, two rows per lane), taken
+    // in turn by as many blocks as are resident at once
+    const long long rows = (long long)Tpad * Hq, per_chunk = 2 * 256 / (D / 16);
+    pp.chunks = (int)((rows + per_chunk - 1) / per_chunk);
+    const long long n_chunks = (long long)B * pp.chunks;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_bwd_prep_kernel<D>, 256, 0) != cudaSuccess ||
+        per_sm < 1)
+      per_sm = 1;
+    const unsigned blocks = (unsigned)std::min<long long>(n_chunks, (long long)per_sm * sm_count());
+    attn_bwd_prep_kernel<D><<<blocks, 256, 0, st>>>(pp);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_LAUNCH;
   }
   BwdParams p{};
