@@ -1138,56 +1138,56 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __grid_constan
   const int rows = Tpad * Hq;  // < 2^31 (the host checks the stored tile rows, which bound it)
   const int lr = (int)threadIdx.x % LK;
   for (long long ch = blockIdx.x; ch < (long long)p.B * p.chunks; ch += gridDim.x) {
-  const int b = (int)(ch / p.chunks);
-  const int r0 = (int)(ch - (long long)b * p.chunks) * (kRows * kRowsPerPass) + (int)threadIdx.x / LK;
-  int hh[kRows], tt[kRows];
-  bool real[kRows];
-  uint4 ov[kRows][2], gv[kRows][2];
+    const int b = (int)(ch / p.chunks);
+    const int r0 = (int)(ch - (long long)b * p.chunks) * (kRows * kRowsPerPass) + (int)threadIdx.x / LK;
+    int hh[kRows], tt[kRows];
+    bool real[kRows];
+    uint4 ov[kRows][2], gv[kRows][2];
 #pragma unroll
-  for (int u = 0; u < kRows; ++u) {
-    const int r = r0 + u * kRowsPerPass;
-    tt[u] = r / Hq;
-    hh[u] = r - tt[u] * Hq;
-    real[u] = r < rows && tt[u] < T;
+    for (int u = 0; u < kRows; ++u) {
+      const int r = r0 + u * kRowsPerPass;
+      tt[u] = r / Hq;
+      hh[u] = r - tt[u] * Hq;
+      real[u] = r < rows && tt[u] < T;
 #pragma unroll
-    for (int e = 0; e < 2; ++e) ov[u][e] = gv[u][e] = make_uint4(0, 0, 0, 0);
-    if (real[u]) {
-      const size_t off = ((size_t)((size_t)b * T + tt[u]) * Hq + hh[u]) * D + lr * 16;
+      for (int e = 0; e < 2; ++e) ov[u][e] = gv[u][e] = make_uint4(0, 0, 0, 0);
+      if (real[u]) {
+        const size_t off = ((size_t)((size_t)b * T + tt[u]) * Hq + hh[u]) * D + lr * 16;
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        ov[u][e] = *reinterpret_cast<const uint4*>(p.o + off + 8 * e);
-        gv[u][e] = *reinterpret_cast<const uint4*>(p.dout + off + 8 * e);
+        for (int e = 0; e < 2; ++e) {
+          ov[u][e] = *reinterpret_cast<const uint4*>(p.o + off + 8 * e);
+          gv[u][e] = *reinterpret_cast<const uint4*>(p.dout + off + 8 * e);
+        }
       }
     }
-  }
 #pragma unroll
-  for (int u = 0; u < kRows; ++u) {
-    const int r = r0 + u * kRowsPerPass;
-    const int h = hh[u], t = tt[u];
-    float dsum = 0.f;
+    for (int u = 0; u < kRows; ++u) {
+      const int r = r0 + u * kRowsPerPass;
+      const int h = hh[u], t = tt[u];
+      float dsum = 0.f;
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      dsum = fma_bf16x2_f32(ov[u][e].x, gv[u][e].x, dsum);
-      dsum = fma_bf16x2_f32(ov[u][e].y, gv[u][e].y, dsum);
-      dsum = fma_bf16x2_f32(ov[u][e].z, gv[u][e].z, dsum);
-      dsum = fma_bf16x2_f32(ov[u][e].w, gv[u][e].w, dsum);
+      for (int e = 0; e < 2; ++e) {
+        dsum = fma_bf16x2_f32(ov[u][e].x, gv[u][e].x, dsum);
+        dsum = fma_bf16x2_f32(ov[u][e].y, gv[u][e].y, dsum);
+        dsum = fma_bf16x2_f32(ov[u][e].z, gv[u][e].z, dsum);
+        dsum = fma_bf16x2_f32(ov[u][e].w, gv[u][e].w, dsum);
+      }
+#pragma unroll
+      for (int sh = LK / 2; sh >= 1; sh >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, sh);
+      if (r < rows && lr == 0) {
+        // clamped to stay finite in bf16 (a huge 1/scale must not turn x into -inf)
+        const float x = real[u] ? fminf(fmaxf(-p.lse[((size_t)b * Hq + h) * T + t] * p.inv_scale, -3.0e38f), 3.0e38f)
+                                : -1e30f;
+        const float y = real[u] ? -dsum : 0.f;
+        const int i = t & 127;
+        const size_t at = (((size_t)b * Hq + h) * (Tpad / 128) + t / 128) * 512 + (i >> 3) * 32 + (i & 7) * 2;
+        const __nv_bfloat16 xh = __float2bfloat16_rn(x), yh = __float2bfloat16_rn(y);
+        *reinterpret_cast<__nv_bfloat16*>(p.ext_lse + at) = xh;
+        *reinterpret_cast<__nv_bfloat16*>(p.ext_lse + at + 16) = __float2bfloat16_rn(x - __bfloat162float(xh));
+        *reinterpret_cast<__nv_bfloat16*>(p.ext_delta + at) = yh;
+        *reinterpret_cast<__nv_bfloat16*>(p.ext_delta + at + 16) = __float2bfloat16_rn(y - __bfloat162float(yh));
+      }
     }
-#pragma unroll
-    for (int sh = LK / 2; sh >= 1; sh >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, sh);
-    if (r < rows && lr == 0) {
-      // clamped to stay finite in bf16 (a huge 1/scale must not turn x into -inf)
-      const float x = real[u] ? fminf(fmaxf(-p.lse[((size_t)b * Hq + h) * T + t] * p.inv_scale, -3.0e38f), 3.0e38f)
-                              : -1e30f;
-      const float y = real[u] ? -dsum : 0.f;
-      const int i = t & 127;
-      const size_t at = (((size_t)b * Hq + h) * (Tpad / 128) + t / 128) * 512 + (i >> 3) * 32 + (i & 7) * 2;
-      const __nv_bfloat16 xh = __float2bfloat16_rn(x), yh = __float2bfloat16_rn(y);
-      *reinterpret_cast<__nv_bfloat16*>(p.ext_lse + at) = xh;
-      *reinterpret_cast<__nv_bfloat16*>(p.ext_lse + at + 16) = __float2bfloat16_rn(x - __bfloat162float(xh));
-      *reinterpret_cast<__nv_bfloat16*>(p.ext_delta + at) = yh;
-      *reinterpret_cast<__nv_bfloat16*>(p.ext_delta + at + 16) = __float2bfloat16_rn(y - __bfloat162float(yh));
-    }
-  }
   }
 }
 
