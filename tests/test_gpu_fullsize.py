@@ -40,8 +40,25 @@ def sample_rows(T, W, seed):
 def test_fullsize_sampled(cswa, name, W):
     c = workloads.CONFIGS[name]
     B, T, Hq, Hkv, D = c["B"], c["T"], c["Hq"], c["Hkv"], c["D"]
+    _sampled_check(cswa, name, B, T, Hq, Hkv, D, W, workloads.config_inputs(name))
+
+
+# the longest sequences: 512 and 256 query tiles per head, window and full causal, both head dims
+LONG_CASES = [(1, 65536, 2, 1, 128, 8192), (1, 32768, 4, 2, 64, -1)]
+
+
+@pytest.mark.parametrize("case", LONG_CASES, ids=lambda c: "B{}_T{}_Hq{}_Hkv{}_D{}_W{}".format(*c))
+def test_long_sequence_sampled(cswa, case):
+    B, T, Hq, Hkv, D, W = case
+    # dk/dv at keys near the end only: a key near the start is seen by W or more query rows,
+    # each of which the oracle expands over the whole sequence
+    _sampled_check(cswa, f"T{T}", B, T, Hq, Hkv, D, W, workloads.training_inputs(B, T, Hq, Hkv, D, seed=T + 7),
+                   early_keys=False)
+
+
+def _sampled_check(cswa, name, B, T, Hq, Hkv, D, W, inputs, early_keys=True):
     scale = workloads.default_scale(D)
-    q, k, v, do = workloads.config_inputs(name)
+    q, k, v, do = inputs
     g = run_block(cswa, q, k, v, do, W, scale)
     qh, kh = f64(g["qh"]), f64(g["kh"])
     vf, dof = f64(v), f64(do)
@@ -70,7 +87,7 @@ def test_fullsize_sampled(cswa, name, W):
     check_grad(f"{name} dq_hat rows", f64(g["dqh"])[bs][:, rows], dq_ref)
 
     clusters = [np.arange(T - 12, T)]
-    clusters.append(np.arange(100, 104) if W >= 0 else np.arange(T - 300, T - 296))
+    clusters.append(np.arange(100, 104) if W >= 0 and early_keys else np.arange(T - 300, T - 296))
     for keys in clusters:
         dk_ref, dv_ref = oracle.attention_bwd_keys(qh[:1], kh[:1], vf[:1], dof[:1], W, scale, keys)
         check_grad(f"{name} dk_hat keys {keys[0]}..", f64(g["dkh"])[:1, keys], dk_ref)
