@@ -270,6 +270,13 @@ def test_decode_wide_groups(cswa, Hq, Hkv, D):
     _decode_case(cswa, 3, 900, Hq, Hkv, D, 700, [899, 0, 431], seed=24, append=True)
 
 
+@pytest.mark.parametrize("W", [-1, 20000])
+def test_decode_long_cache(cswa, W):
+    """Up to 547 chunks of one sequence merged (more than the merging CTA takes in one
+    round of weights), next to a short sequence in the same batch."""
+    _decode_case(cswa, 3, 70000, 4, 2, 128, W, [69999, 40000, 130], seed=25, append=True)
+
+
 def test_decode_repeated_calls_share_a_workspace(cswa):
     """The arrival counters in the workspace are tagged per call: a workspace reused
     across calls (and one that starts out holding garbage) gives the same results."""

@@ -83,6 +83,8 @@ CASES = [
     (2, 1, 300, 8, 2, 64, 100, [0, 77]),               # one-token chunk, G = 4, D = 64
     (1, 517, 2000, 6, 3, 64, 1023, [1483]),            # window shorter than the cache
     (2, 640, 640, 2, 1, 128, 2000, [0, 0]),            # window beyond every position: plain causal
+    (2, 300, 70000, 4, 2, 128, -1, [69700, 40000]),    # long caches, full causal: ~545 key tiles
+    (1, 200, 70000, 2, 1, 64, 8000, [65000]),          # long cache, window of 63 tiles
 ]
 
 
