@@ -525,18 +525,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int trole = 1 + half;
     (void)tracer;
     (void)trole;
-    // dS^T of the previous step (this warp's 32 keys x 64 queries) and where it goes in
-    // the workspace tile the dQ kernel reads; it is stored during the next step's P
-    // phase, whose exp2 work leaves the load/store unit idle (an item's last one before
-    // its epilogue). The tile is written as 16-byte units (8 queries of one key) ordered
-    // so that every warp store covers 512 contiguous bytes (see ds_unit_offset).
+    // dS^T of the step (this warp's 32 keys x 64 queries) and where it goes in the
+    // workspace tile the dQ kernel reads. It is stored right after the dS phase, while the
+    // warp waits for the next S^T (the stores drain while nothing else runs on the warp,
+    // and the registers are free again for the P phase). The tile is written as 16-byte
+    // units (8 queries of one key) ordered so that every warp store covers 512 contiguous
+    // bytes (see ds_unit_offset).
     uint32_t dsk[kSCols / 2];
-    uint8_t* ds_dst = nullptr;
-    auto store_ds_units = [&](int u0, int u1) {
-#pragma unroll
-      for (int u = u0; u < u1; ++u)
-        *reinterpret_cast<uint4*>(ds_dst + u * 512) = make_uint4(dsk[4 * u], dsk[4 * u + 1], dsk[4 * u + 2], dsk[4 * u + 3]);
-    };
     bool ok = true;
     int g0 = 0, k = 0;
     int kr_pending = -1;  // warp 4, lane 0: the item whose raw k load nobody has waited for yet
@@ -593,7 +588,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_fence_before();
           mbar_arrive(&p_chunk[c]);
           if (tracer && c == 0) CSWA_MARK(trole, g, 3);
-          if (ds_dst) store_ds_units(2 * c, 2 * c + 2);
           if (lent_stage >= 0 && c == (half ? 0 : kPChunks - 1)) return_stage();
         };
 #pragma unroll
@@ -651,12 +645,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_arrive(ds_full);
         if (tracer) CSWA_MARK(trole, g, 7);
         const long long tile = tile0 + (long long)(I.hk * G + it / I.m_cnt) * p.tiles_per_bh + it % I.m_cnt;
-        ds_dst = reinterpret_cast<uint8_t*>(p.ds) + (size_t)tile * 32768 + ds_unit_offset(r, (kSCols / 8) * half);
+        uint8_t* const ds_dst =
+            reinterpret_cast<uint8_t*>(p.ds) + (size_t)tile * 32768 + ds_unit_offset(r, (kSCols / 8) * half);
+#pragma unroll
+        for (int u = 0; u < kSCols / 8; ++u)
+          *reinterpret_cast<uint4*>(ds_dst + u * 512) = make_uint4(dsk[4 * u], dsk[4 * u + 1], dsk[4 * u + 2], dsk[4 * u + 3]);
       }
       if (!ok) break;
-      // the item's last dS^T now: the epilogue needs the registers
-      store_ds_units(0, kSCols / 8);
-      ds_dst = nullptr;
       // column groups past the first two have no epilogue: on to the next item
       if (half >= 2) {
         g0 += I.n_iters;
