@@ -12,8 +12,8 @@
 //   bwd_prep     per query row, -lse_i/scale and -Delta_i as bf16 hi + lo pairs,
 //                laid out as one extra K = 16 step of an MMA (padded rows: a
 //                large negative lse term, so P = 0 there).
-//   bwd_main     persistent, one CTA per SM, walking (128-key tile, KV head,
-//                batch) items round-robin. For an item, K and V stay in shared
+//   bwd_main     persistent, one CTA per SM, taking (128-key tile, KV head,
+//                batch) items from a global counter. For an item, K and V stay in shared
 //                memory and the CTA walks every (query head of the group, 128-row
 //                query tile) that sees the key tile, with Q and dO in rings of 3
 //                and 2 stages that run on across items; the next item's K and V
@@ -38,7 +38,7 @@
 //                the Q or dO ring stage of the item's last step (lent to the
 //                epilogue until its TMA stores have read it) and leaves as TMA
 //                stores of 32-row boxes.
-//   bwd_dq       one CTA per (128-row query tile, query head, batch):
+//   bwd_dq       persistent, (128-row query tile, query head, batch) items:
 //                dQ = scale * sum over key tiles of dS K, accumulated in TMEM
 //                from the stored dS^T tiles (one bulk copy each) and K tiles,
 //                written once as bf16 through a staging tile and TMA stores.
