@@ -177,8 +177,10 @@ attn_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, f
   p.window = (window >= T) ? -1 : window;
   p.scale_log2 = scale * kLog2e;
   p.nq_tiles = tiles128(T);
-  p.n_pairs = (p.nq_tiles + 1) / 2;
-  dim3 grid(Hq, B, p.n_pairs);
+  // G even: the slots are two query heads of one KV group at one query tile
+  p.head_pairs = (p.G % 2 == 0) ? 1 : 0;
+  p.n_pairs = p.head_pairs ? p.nq_tiles : (p.nq_tiles + 1) / 2;
+  dim3 grid(p.head_pairs ? Hq / 2 : Hq, B, p.n_pairs);
   // the two chunk maps are unused in training: q's map stands in for them
   attn_fwd_kernel<D><<<grid, 384, FwdLayout<D>::kBytes, st>>>(tq, tk, tv, tq, tq, to, p);
   return launched();

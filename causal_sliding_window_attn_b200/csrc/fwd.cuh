@@ -9,7 +9,10 @@
 //
 // One CTA owns two 128-row query tiles ("slots") of one (b, h): tiles 2p and
 // 2p+1. It walks the union of their key-tile ranges inside the causal/window
-// band; key tiles outside the band are never loaded.
+// band; key tiles outside the band are never loaded. With an even group size G
+// the training forward pairs two query heads of one KV group at the same query
+// tile instead: both slots then see the same key tiles, and no key tile is
+// walked by one slot alone (the first and last tiles of a tile pair are).
 //   warp 0      TMA producer: Q once, then K and V tiles into 2-stage rings
 //   warp 1      MMA issuer (whole warp, one elected lane issues): S_s = Q_s K^T (SS),
 //               O_s += P_s V (TS)
@@ -65,6 +68,10 @@ struct FwdParams {
   uint4* vc;
   // fp8 forward only: the dequantization factors of q, k, v (device memory, 3 floats)
   const float* descale;
+  // training forward with G even: the two slots are query heads 2x and 2x + 1 (one KV
+  // group) at the same query tile, so that both walk the same key tiles (0: the slots
+  // are query tiles 2p and 2p + 1 of one head)
+  int head_pairs;
 };
 
 constexpr int kMaxRankedItems = 256;  // prefill items ranked by weight (more: pair order)
@@ -110,7 +117,9 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* p_chunk = bars + 18;  // [2][4] P_s of keys 32c .. 32c+31 written over S_s
 
   const int warp = warp_id(), lane = lane_id();
-  const int h = blockIdx.x;
+  const int hp = p.head_pairs;
+  const int h = hp ? 2 * blockIdx.x : blockIdx.x;  // the first slot's query head
+  auto head_of = [&](int s) { return h + (hp ? s : 0); };
   int b = blockIdx.y;
   int pair = p.n_pairs - 1 - blockIdx.z;  // heaviest tiles first
   const int hk = h / p.G;
@@ -168,7 +177,7 @@ __global__ void __launch_bounds__(384, 1)
   bool has[2];
 #pragma unroll
   for (int s = 0; s < 2; ++s) {
-    qt[s] = 2 * pair + s;
+    qt[s] = hp ? pair : 2 * pair + s;
     has[s] = qt[s] < p.nq_tiles;
     hi[s] = qt[s];
     lo[s] = lo_of(qt[s]);
@@ -219,7 +228,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int s = 0; s < 2; ++s)
         if (has[s])
           for (int pn = 0; pn < L::kPanels; ++pn)
-            tma_load_4d(smem + (s ? L::kQ1 : L::kQ0) + pn * 16384, &tm_q, q_full, pn * kPanelElems, h,
+            tma_load_4d(smem + (s ? L::kQ1 : L::kQ0) + pn * 16384, &tm_q, q_full, pn * kPanelElems, head_of(s),
                         qt[s] * 128 - shift, b);
       // K and V stages are released separately (K once the S products have read it, V
       // once the PV products have), so K of the next tile loads a whole tile ahead
@@ -392,7 +401,8 @@ __global__ void __launch_bounds__(384, 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const int my_qt = 2 * pair + s;
+    const int my_qt = hp ? pair : 2 * pair + s;
+    const int my_h = head_of(s);
     const int my_hi = my_qt;
     const int my_lo = lo_of(my_qt);
     const uint32_t tSs = tS(s) + lane_off, tOs = tO(s) + lane_off;
@@ -540,17 +550,17 @@ __global__ void __launch_bounds__(384, 1)
         __syncwarp();
         if (lane == 0) {
           for (int pn = 0; pn < D / 64; ++pn)
-            tma_store_4d(&tm_o, stg + pn * 16384 + quarter * 4096, pn * 64, h, my_qt * 128 + 32 * quarter, b);
+            tma_store_4d(&tm_o, stg + pn * 16384 + quarter * 4096, pn * 64, my_h, my_qt * 128 + 32 * quarter, b);
           bulk_commit();
         }
-        if (cr < p.T) p.lse[((size_t)b * p.Hq + h) * p.T + cr] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+        if (cr < p.T) p.lse[((size_t)b * p.Hq + my_h) * p.T + cr] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
       } else if (ok) {
         // tcgen05.ld is warp-collective: every lane loads, only rows of [0, T) store
         const int cr = my_qt * 128 - shift + row;  // output row (chunk row in kCache)
         const bool store = (cr < p.T) && (!kCache || cr >= 0);
         // fp8: O and l both carry P's 2^8, and O the quantization scale of v
         const float inv_l = (kFp8 ? p.descale[2] : 1.f) / l_run;
-        __nv_bfloat16* dst = p.o + ((size_t)((size_t)b * p.T + cr) * p.Hq + h) * D;
+        __nv_bfloat16* dst = p.o + ((size_t)((size_t)b * p.T + cr) * p.Hq + my_h) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -568,7 +578,7 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         if (store && (!kCache || p.lse))
-          p.lse[((size_t)b * p.Hq + h) * p.T + cr] = (m_run + __log2f(l_run) - kPBias) * 0.69314718055994531f;
+          p.lse[((size_t)b * p.Hq + my_h) * p.T + cr] = (m_run + __log2f(l_run) - kPBias) * 0.69314718055994531f;
       }
     }
   }
